@@ -1,0 +1,137 @@
+"""Oracle for the fused linear cross-entropy forward (fp64, CPU).
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` are the only callers.  The product package
+never imports this module, and this module never imports the product package.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64, OpenMP over rows).  It
+writes out the definition from D. Ineshin, "Een gefuseerde forward-kernel voor
+lineaire cross-entropy op Apple-GPU's" (2026), section 1:
+Z = H W^T and loss_i = logsumexp(Z_i) - Z_{i, y_i}.  This wrapper only builds
+the shared object, marshals numpy arrays and raises on error codes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+BF16 = 0
+FP32 = 1
+
+_ERRORS = {-1: "invalid argument", -2: "target outside [0, V)", -3: "out of memory"}
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` into ``liboracle.so`` (no fast-math: fp64 sums stay in order)."""
+    stale = (not os.path.exists(_LIB_PATH)) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared",
+                               "-std=c11", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            vp, i64, dp = ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p
+            lib.oracle_forward_rows.argtypes = [vp, vp, ctypes.c_int, vp, i64, i64, i64,
+                                                vp, i64, dp, dp, dp, dp, ctypes.c_int]
+            lib.oracle_forward_rows.restype = ctypes.c_int
+            lib.oracle_logits_row.argtypes = [vp, vp, ctypes.c_int, i64, i64, i64, dp]
+            lib.oracle_logits_row.restype = ctypes.c_int
+            lib.oracle_mean.argtypes = [dp, i64]
+            lib.oracle_mean.restype = ctypes.c_double
+            lib.oracle_max_threads.argtypes = []
+            lib.oracle_max_threads.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _as_storage(a: np.ndarray):
+    """Return (contiguous array, dtype code): uint16 holds bf16 bit patterns."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return a, BF16
+    if a.dtype == np.float32:
+        return a, FP32
+    raise TypeError(f"oracle takes bf16 bits (uint16) or float32, got {a.dtype}")
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def forward(H: np.ndarray, W: np.ndarray, y: np.ndarray, rows=None, nthreads: int = 0):
+    """Per-token loss, lse, target logit and row max for ``rows`` (default: all).
+
+    H is (N, D) and W is (V, D), both uint16 bf16 bit patterns or both float32;
+    y is int64 of length N.  Returns a dict of float64 arrays indexed like ``rows``.
+    """
+    lib = _load()
+    H, dt_h = _as_storage(H)
+    W, dt_w = _as_storage(W)
+    if dt_h != dt_w:
+        raise TypeError("H and W must share one storage type")
+    if H.ndim != 2 or W.ndim != 2 or H.shape[1] != W.shape[1]:
+        raise ValueError("H must be (N, D) and W (V, D)")
+    y = np.ascontiguousarray(y, dtype=np.int64)
+    N, D = H.shape
+    V = W.shape[0]
+    if y.shape != (N,):
+        raise ValueError("y must have length N")
+    if rows is None:
+        rows_arr, n = None, N
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        n = rows_arr.shape[0]
+    out = {k: np.empty(n, dtype=np.float64) for k in ("loss", "lse", "target", "max")}
+    rc = lib.oracle_forward_rows(_ptr(H), _ptr(W), dt_h, _ptr(y), N, V, D,
+                                 _ptr(rows_arr), n, _ptr(out["loss"]), _ptr(out["lse"]),
+                                 _ptr(out["target"]), _ptr(out["max"]), int(nthreads))
+    if rc != 0:
+        raise OracleError(_ERRORS.get(rc, f"oracle error {rc}"))
+    return out
+
+
+def logits_row(H: np.ndarray, W: np.ndarray, i: int) -> np.ndarray:
+    """The full fp64 logits row Z_i (only for small V: it is V doubles)."""
+    lib = _load()
+    H, dt = _as_storage(H)
+    W, _ = _as_storage(W)
+    V, D = W.shape
+    z = np.empty(V, dtype=np.float64)
+    rc = lib.oracle_logits_row(_ptr(H), _ptr(W), dt, int(i), V, D, _ptr(z))
+    if rc != 0:
+        raise OracleError(_ERRORS.get(rc, f"oracle error {rc}"))
+    return z
+
+
+def mean(loss: np.ndarray) -> float:
+    """Mean loss over the given per-token losses (sequential fp64 sum / n)."""
+    lib = _load()
+    loss = np.ascontiguousarray(loss, dtype=np.float64)
+    return float(lib.oracle_mean(_ptr(loss), loss.shape[0]))
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())

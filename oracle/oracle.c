@@ -1,0 +1,160 @@
+/*
+ * Oracle for the fused linear cross-entropy forward: plain, slow, fp64, CPU.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may include, link or
+ * call this file; only the test suite, the smoke check and the CPU-baseline leg
+ * of the benchmark use it.  It shares no code, header or constant with the CUDA
+ * library.
+ *
+ * Source: D. Ineshin, "Een gefuseerde forward-kernel voor lineaire
+ * cross-entropy op Apple-GPU's" (2026), section 1 ("De loss streamen zonder
+ * volledige logits"):
+ *   - the logits are Z = H W^T, with H an (N, D) matrix of hidden states and
+ *     W the (V, D) output projection;
+ *   - the per-token loss is loss_i = logsumexp(Z_i) - Z_{i, y_i};
+ *   - the loss needs just two statistics of each row: its log-sum-exp and
+ *     its target logit.
+ * The method reaches this plain definition exactly (up to rounding order), so
+ * the oracle is that definition written out: it materialises one full logits
+ * row in fp64 and does a two-pass log-sum-exp (max pass, then sum of exp).
+ * It deliberately does NOT stream vocab tiles or use the online (m, s)
+ * recurrence; that is the thing under test.
+ *
+ * Readings of points the page leaves open:
+ *   - log is the natural logarithm;
+ *   - inputs are converted exactly to fp64 from their stored type (bf16 bit
+ *     patterns or fp32), and every dot product is a sequential fp64 sum over
+ *     k = 0..D-1;
+ *   - a target outside [0, V) is invalid input: the call fails with
+ *     ORACLE_ERR_TARGET and writes nothing for that row;
+ *   - the mean loss is the plain sum of the per-token losses divided by N,
+ *     summed sequentially in fp64.
+ *
+ * Parity is pinned for every function here (closed forms, invariants, a
+ * library cross-entropy on fp64 logits and exact brute force; see the tests).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG (-1)
+#define ORACLE_ERR_TARGET (-2)
+#define ORACLE_ERR_NOMEM (-3)
+
+/* dtype codes for the stored element type of H and W */
+#define ORACLE_BF16 0
+#define ORACLE_FP32 1
+
+/* Exact conversion of one stored element to double.  A bf16 value is the
+ * upper 16 bits of the fp32 with the same sign, exponent and leading mantissa
+ * bits, so widening the bit pattern by 16 zero bits gives the fp32 exactly. */
+static double load_elem(const void *base, int dtype, int64_t idx) {
+    if (dtype == ORACLE_BF16) {
+        uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]) << 16;
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        return (double)f;
+    }
+    return (double)((const float *)base)[idx];
+}
+
+/* One logit z_{ij} = sum_k H_ik W_jk in fp64, k in order (definition Z = H W^T). */
+static double logit(const void *H, const void *W, int dtype, int64_t i,
+                    int64_t j, int64_t D) {
+    double acc = 0.0;
+    for (int64_t k = 0; k < D; ++k)
+        acc += load_elem(H, dtype, i * D + k) * load_elem(W, dtype, j * D + k);
+    return acc;
+}
+
+/* Full logits row i into z[0..V). */
+int oracle_logits_row(const void *H, const void *W, int dtype, int64_t i,
+                      int64_t V, int64_t D, double *z) {
+    if (!H || !W || !z || V < 1 || D < 1 || i < 0) return ORACLE_ERR_ARG;
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP32) return ORACLE_ERR_ARG;
+    for (int64_t j = 0; j < V; ++j) z[j] = logit(H, W, dtype, i, j, D);
+    return ORACLE_OK;
+}
+
+/*
+ * Per-token outputs for a subset of rows.
+ *   rows[t] (t < nrows) is the row index into H / y; rows == NULL means all N
+ *   rows in order (nrows must then equal N).
+ *   out_*[t] receive loss, lse, target logit and the row maximum max_j z_ij.
+ *   Any out_* pointer may be NULL.
+ * Returns ORACLE_OK, ORACLE_ERR_ARG, ORACLE_ERR_TARGET (some selected row has
+ * y outside [0, V)) or ORACLE_ERR_NOMEM.
+ */
+int oracle_forward_rows(const void *H, const void *W, int dtype,
+                        const int64_t *y, int64_t N, int64_t V, int64_t D,
+                        const int64_t *rows, int64_t nrows, double *out_loss,
+                        double *out_lse, double *out_target, double *out_max,
+                        int nthreads) {
+    if (!H || !W || !y || N < 0 || V < 1 || D < 1 || nrows < 0)
+        return ORACLE_ERR_ARG;
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP32) return ORACLE_ERR_ARG;
+    if (!rows && nrows != N) return ORACLE_ERR_ARG;
+    for (int64_t t = 0; t < nrows; ++t) {
+        int64_t i = rows ? rows[t] : t;
+        if (i < 0 || i >= N) return ORACLE_ERR_ARG;
+        if (y[i] < 0 || y[i] >= V) return ORACLE_ERR_TARGET;
+    }
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int status = ORACLE_OK;
+#pragma omp parallel
+    {
+        double *z = (double *)malloc((size_t)V * sizeof(double));
+        if (!z) {
+#pragma omp atomic write
+            status = ORACLE_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < nrows; ++t) {
+            if (!z) continue;
+            int64_t i = rows ? rows[t] : t;
+            /* Z_i: the full logits row, materialised */
+            for (int64_t j = 0; j < V; ++j) z[j] = logit(H, W, dtype, i, j, D);
+            /* pass 1: M = max_j z_ij */
+            double M = z[0];
+            for (int64_t j = 1; j < V; ++j)
+                if (z[j] > M) M = z[j];
+            /* pass 2: S = sum_j exp(z_ij - M); logsumexp = M + log S */
+            double S = 0.0;
+            for (int64_t j = 0; j < V; ++j) S += exp(z[j] - M);
+            double lse = M + log(S);
+            double tgt = z[y[i]];
+            if (out_loss) out_loss[t] = lse - tgt;
+            if (out_lse) out_lse[t] = lse;
+            if (out_target) out_target[t] = tgt;
+            if (out_max) out_max[t] = M;
+        }
+        free(z);
+    }
+    return status;
+}
+
+/* Mean loss: (sum_i loss_i) / n, summed sequentially in fp64.  n == 0 gives NaN. */
+double oracle_mean(const double *loss, int64_t n) {
+    if (!loss || n <= 0) return NAN;
+    double acc = 0.0;
+    for (int64_t i = 0; i < n; ++i) acc += loss[i];
+    return acc / (double)n;
+}
+
+/* Threads the OpenMP runtime would use (for reporting the CPU baseline). */
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
