@@ -1,0 +1,171 @@
+/*
+ * flce.h — C ABI of libflce.so: the fused linear cross-entropy forward on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (D. Ineshin, "Een gefuseerde forward-kernel voor lineaire
+ * cross-entropy op Apple-GPU's", 2026, section 1): for hidden states H (N, D),
+ * an output projection W (V, D) and targets y (N),
+ *     Z = H W^T,    loss_i = logsumexp(Z_i) - Z_{i, y_i},
+ * computed by streaming vocabulary tiles through the online log-sum-exp
+ *     m' = max(m, m_t),   s' = s * exp(m - m') + sum_j exp(z_j - m'),
+ *     logsumexp = m + log(s) after the last tile,
+ * and capturing the target logit in whichever tile holds it, so the (N, V)
+ * logits matrix never exists (same section).  log is the natural logarithm.
+ * The mean loss is the plain average of the N per-token losses.
+ *
+ * General contract of every entry point:
+ *   - Pointers named H, W, y, out_*, workspace are DEVICE pointers on the
+ *     current CUDA device, allocated and owned by the caller.  The library
+ *     allocates no device or pinned memory and keeps no per-call state.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued asynchronously; the call returns before the GPU finishes.
+ *   - Host-detectable problems are returned synchronously and nothing is
+ *     enqueued.  Problems found on the device (a target outside [0, V), a
+ *     bounded wait that ran out) are recorded in the workspace status word
+ *     and reported by flce_check().
+ *   - Thread safety: calls on different workspaces may run concurrently.
+ *     Calls that share one workspace must be ordered on one stream.
+ */
+#ifndef FLCE_H_
+#define FLCE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FLCE_API __attribute__((visibility("default")))
+#else
+#define FLCE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of H and W.  bf16 runs on the tcgen05 tensor-core path
+ * (fp32 accumulation in TMEM); fp32 runs on an fp32 FFMA path. */
+typedef enum { FLCE_BF16 = 0, FLCE_FP32 = 1 } flce_dtype;
+
+typedef enum {
+  FLCE_OK = 0,
+  FLCE_ERR_INVALID_ARG = 1,          /* null pointer, negative size, bad workspace, ... */
+  FLCE_ERR_UNSUPPORTED = 2,          /* device is not sm_100, D % 8 != 0 or a pointer is
+                                        not 16-byte aligned for bf16, sizes beyond int32 */
+  FLCE_ERR_WORKSPACE_TOO_SMALL = 3,  /* workspace_bytes < flce_workspace_size(...) */
+  FLCE_ERR_CUDA = 4,                 /* a CUDA runtime/driver call or launch failed */
+  FLCE_ERR_TARGET_OUT_OF_RANGE = 5,  /* (flce_check) some y_i outside [0, V) */
+  FLCE_ERR_TIMEOUT = 6               /* (flce_check) a bounded device wait ran out */
+} flce_status;
+
+/* Schedule the library uses for one problem (host-side, informational).
+ * The contraction is cut into work units of `block_rows` tokens by one vocab
+ * slab; a slab is a run of consecutive `tile_cols`-column vocab tiles.  The
+ * first `slab_rem` slabs hold slab_base + 1 tiles, the others slab_base. */
+typedef struct {
+  int64_t N, V, D;
+  int32_t dtype;           /* flce_dtype */
+  int32_t block_rows;      /* tokens per work unit (TMEM lanes on the bf16 path) */
+  int32_t tile_cols;       /* vocab columns per tile */
+  int32_t k_block;         /* D elements per pipeline stage */
+  int64_t token_blocks;    /* ceil(N / block_rows) */
+  int64_t vocab_tiles;     /* ceil(V / tile_cols) */
+  int32_t slabs;           /* P: partial (m, s) states per token */
+  int32_t slab_base;       /* vocab_tiles / slabs */
+  int32_t slab_rem;        /* vocab_tiles % slabs */
+  int32_t grid;            /* CTAs launched for the contraction kernel */
+  int64_t units;           /* token_blocks * slabs */
+  int64_t makespan_tiles;  /* tiles processed by the busiest CTA */
+  size_t workspace_bytes;  /* == flce_workspace_size(N, V, D, dtype) */
+} flce_plan_t;
+
+/* Bytes of device workspace that flce_forward / flce_partials need for this
+ * problem: a 256-byte header, the per-(slab, token) partial states (8 bytes
+ * each, at most 512 slabs per token, so O(N), never O(N*V)), and one fp64
+ * per 256 tokens for the mean.  Depends only on its arguments (not on the
+ * device).  Returns 0 for invalid arguments (N < 0, V < 1, D < 1, unknown
+ * dtype).  Host only; never touches the GPU. */
+FLCE_API size_t flce_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype dtype);
+
+/* The schedule for a device with `sm_count` SMs (host only, no GPU call).
+ * Returns FLCE_ERR_INVALID_ARG for invalid sizes, sm_count < 1 or plan NULL. */
+FLCE_API flce_status flce_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int32_t sm_count,
+                      flce_plan_t* plan);
+
+/*
+ * The full forward: per-token loss, log-sum-exp and target logit, and the
+ * mean loss.  Section 1 of the page: loss_i = logsumexp(Z_i) - Z_{i, y_i}.
+ *
+ *   H            (N, D) row-major, dtype elements, contiguous (row stride D)
+ *   W            (V, D) row-major, dtype elements, contiguous (row stride D)
+ *   y            (N) int64 targets; each must lie in [0, V)
+ *   N >= 0, V >= 1, D >= 1; N, V < 2^31.  bf16 also needs D % 8 == 0 and
+ *                16-byte-aligned H and W (tensor-memory-access strides).
+ *   out_loss, out_lse, out_target_logit   (N) fp32 each, written for every row
+ *   out_mean     (1) fp32 or NULL; mean of out_loss computed in fp64
+ *   workspace    >= flce_workspace_size(N, V, D, dtype) bytes, 256-byte aligned;
+ *                contents on entry are ignored; it holds the status word that
+ *                flce_check() reads until the next call that uses it
+ *   stream       cudaStream_t
+ * A row whose target is out of range gets NaN loss and NaN target logit and
+ * sets FLCE_ERR_TARGET_OUT_OF_RANGE for flce_check().  N == 0 is a no-op that
+ * returns FLCE_OK and writes nothing (out_mean untouched).
+ * Results are bitwise deterministic run to run on the same device.
+ */
+FLCE_API flce_status flce_forward(const void* H, const void* W, const int64_t* y,
+                         int64_t N, int64_t V, int64_t D, flce_dtype dtype,
+                         float* out_loss, float* out_lse, float* out_target_logit,
+                         float* out_mean, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/*
+ * First stage of flce_forward, on its own: the contraction Z = H W^T tile by
+ * tile with the online (m, s) update of section 1 of the page, leaving one
+ * partial state per (vocab slab, token) in the workspace and writing the
+ * target logit of every row whose target is in range (from the tile that
+ * holds it).  Arguments as for flce_forward.  Resets the workspace status
+ * word.  Must be followed by flce_merge on the same workspace and stream.
+ */
+FLCE_API flce_status flce_partials(const void* H, const void* W, const int64_t* y,
+                          int64_t N, int64_t V, int64_t D, flce_dtype dtype,
+                          float* out_target_logit, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/*
+ * Second stage: combines the partial states left by flce_partials in a fixed
+ * order (m = max_p m_p, s = sum_p s_p exp(m_p - m), logsumexp = m + log s:
+ * the same recurrence applied to whole slabs), then writes loss = lse -
+ * target logit, and the mean if out_mean is not NULL.  N, V and y must be
+ * those given to flce_partials; out_target_logit is read (and set to NaN for
+ * out-of-range targets).
+ */
+FLCE_API flce_status flce_merge(const int64_t* y, int64_t N, int64_t V,
+                       float* out_loss, float* out_lse, float* out_target_logit,
+                       float* out_mean, const void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/* Waits for `stream`, then reads the workspace status word left by the last
+ * flce_forward / flce_partials + flce_merge that used this workspace.
+ * Returns FLCE_OK, FLCE_ERR_TARGET_OUT_OF_RANGE, FLCE_ERR_TIMEOUT,
+ * FLCE_ERR_INVALID_ARG (merge saw a workspace flce_partials did not prepare)
+ * or FLCE_ERR_CUDA. */
+FLCE_API flce_status flce_check(const void* workspace, void* stream);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+FLCE_API const char* flce_status_string(flce_status status);
+
+/*
+ * Self-test of the bounded device waits.  Launches one CTA whose thread
+ * waits on a shared-memory barrier that nothing completes, with a limit of
+ * `limit_ns` nanoseconds (1000 <= limit_ns <= 10^9); the wait gives up,
+ * records FLCE_ERR_TIMEOUT in the workspace status word and the kernel
+ * returns normally.  `workspace` needs 256 bytes.  Use flce_check() to read
+ * the result.  No GPU fault, trap or hang is involved.
+ */
+FLCE_API flce_status flce_selftest_wait_timeout(void* workspace, size_t workspace_bytes,
+                                       uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLCE_H_ */

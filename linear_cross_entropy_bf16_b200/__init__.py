@@ -1,1 +1,253 @@
-"""Fused linear cross-entropy forward for NVIDIA B200 (sm_100a)."""
+"""Fused linear cross-entropy forward for NVIDIA B200 (sm_100a).
+
+For hidden states H (N, D), an output projection W (V, D) and targets y (N),
+computes loss_i = logsumexp(H_i W^T) - H_i . W_{y_i}, the log-sum-exp, the
+target logit and the mean loss without ever forming the (N, V) logits
+(D. Ineshin, "Een gefuseerde forward-kernel voor lineaire cross-entropy op
+Apple-GPU's", 2026, section 1).
+
+This module is a thin ctypes binding over ``libflce.so`` (C ABI in
+``include/flce.h``): it checks and marshals torch tensors, allocates outputs
+and workspace with torch on the current stream, and calls the library.  All
+arithmetic runs in the library's CUDA kernels; there is no fallback.  If the
+library is missing, calls raise ``FlceError`` (build it with
+``python -m linear_cross_entropy_bf16_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "FlceError", "forward", "partials", "merge", "workspace_size", "plan", "check",
+    "status_string", "selftest_wait_timeout", "library_path", "load_library",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libflce.so")
+_lock = threading.RLock()
+_lib = None
+
+# flce_dtype
+BF16 = 0
+FP32 = 1
+# flce_status
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE_TOO_SMALL, ERR_CUDA, \
+    ERR_TARGET_OUT_OF_RANGE, ERR_TIMEOUT = range(7)
+
+
+_STATUS_NAMES = ("ok", "invalid argument", "unsupported device, shape or alignment",
+                 "workspace too small", "CUDA error", "target outside [0, V)",
+                 "bounded device wait timed out")
+
+
+class FlceError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        name = _STATUS_NAMES[status] if 0 <= status < len(_STATUS_NAMES) else "unknown status"
+        super().__init__(f"{what}: {name} (status {status})")
+
+
+class Plan(ctypes.Structure):
+    """Mirror of flce_plan_t."""
+    _fields_ = [
+        ("N", ctypes.c_int64), ("V", ctypes.c_int64), ("D", ctypes.c_int64),
+        ("dtype", ctypes.c_int32), ("block_rows", ctypes.c_int32),
+        ("tile_cols", ctypes.c_int32), ("k_block", ctypes.c_int32),
+        ("token_blocks", ctypes.c_int64), ("vocab_tiles", ctypes.c_int64),
+        ("slabs", ctypes.c_int32), ("slab_base", ctypes.c_int32),
+        ("slab_rem", ctypes.c_int32), ("grid", ctypes.c_int32),
+        ("units", ctypes.c_int64), ("makespan_tiles", ctypes.c_int64),
+        ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libflce.so (once).  Raises FlceError if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise FlceError(ERR_UNSUPPORTED, f"{_LIB_PATH} is missing; build it with "
+                            "`python -m linear_cross_entropy_bf16_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        vp, i64, sz, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+        lib.flce_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int]
+        lib.flce_workspace_size.restype = sz
+        lib.flce_plan.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int32, ctypes.POINTER(Plan)]
+        lib.flce_plan.restype = st
+        lib.flce_forward.argtypes = [vp, vp, vp, i64, i64, i64, ctypes.c_int, vp, vp, vp, vp, vp, sz, vp]
+        lib.flce_forward.restype = st
+        lib.flce_partials.argtypes = [vp, vp, vp, i64, i64, i64, ctypes.c_int, vp, vp, sz, vp]
+        lib.flce_partials.restype = st
+        lib.flce_merge.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp, sz, vp]
+        lib.flce_merge.restype = st
+        lib.flce_check.argtypes = [vp, vp]
+        lib.flce_check.restype = st
+        lib.flce_status_string.argtypes = [ctypes.c_int]
+        lib.flce_status_string.restype = ctypes.c_char_p
+        lib.flce_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint64, vp]
+        lib.flce_selftest_wait_timeout.restype = st
+        _lib = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return load_library().flce_status_string(int(status)).decode()
+    except FlceError:
+        return f"status {status}"
+
+
+def _raise_on(status: int, what: str):
+    if status != OK:
+        raise FlceError(status, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"H and W must be bfloat16 or float32, got {t.dtype}")
+
+
+def workspace_size(N: int, V: int, D: int, dtype=torch.bfloat16) -> int:
+    code = dtype if isinstance(dtype, int) else (BF16 if dtype == torch.bfloat16 else FP32)
+    n = load_library().flce_workspace_size(int(N), int(V), int(D), code)
+    if n == 0:
+        raise FlceError(ERR_INVALID_ARG, "workspace_size")
+    return int(n)
+
+
+def plan(N: int, V: int, D: int, dtype=torch.bfloat16, sm_count: int = 148) -> dict:
+    """The work decomposition the library uses on a device with ``sm_count`` SMs."""
+    code = dtype if isinstance(dtype, int) else (BF16 if dtype == torch.bfloat16 else FP32)
+    p = Plan()
+    _raise_on(load_library().flce_plan(int(N), int(V), int(D), code, int(sm_count), ctypes.byref(p)),
+              "plan")
+    return p.as_dict()
+
+
+def _stream_ptr(stream, device) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return int(s.cuda_stream)
+
+
+def _check_inputs(H, W, y):
+    for name, t in (("H", H), ("W", W), ("y", y)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if H.dim() != 2 or W.dim() != 2 or H.shape[1] != W.shape[1]:
+        raise ValueError(f"H must be (N, D) and W (V, D); got {tuple(H.shape)} and {tuple(W.shape)}")
+    if H.dtype != W.dtype:
+        raise TypeError("H and W must have the same dtype")
+    if y.dtype != torch.int64 or y.dim() != 1 or y.shape[0] != H.shape[0]:
+        raise ValueError("y must be int64 of shape (N,)")
+    if H.device != W.device or H.device != y.device:
+        raise ValueError("H, W and y must be on one device")
+    return H.shape[0], W.shape[0], H.shape[1], _dtype_code(H)
+
+
+def _alloc_outputs(N, device, out):
+    if out is None:
+        out = {}
+    f32 = dict(dtype=torch.float32, device=device)
+    loss = out.get("loss") if out.get("loss") is not None else torch.empty(N, **f32)
+    lse = out.get("lse") if out.get("lse") is not None else torch.empty(N, **f32)
+    tgt = out.get("target_logit") if out.get("target_logit") is not None else torch.empty(N, **f32)
+    mean = out.get("mean") if out.get("mean") is not None else torch.full((), float("nan"), **f32)
+    for t in (loss, lse, tgt, mean):
+        if t.dtype != torch.float32 or t.device != device or not t.is_contiguous():
+            raise ValueError("outputs must be contiguous float32 tensors on the input device")
+    return loss, lse, tgt, mean
+
+
+def _workspace(N, V, D, code, device, workspace):
+    need = load_library().flce_workspace_size(int(N), int(V), int(D), code)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    if workspace.device != device or workspace.numel() * workspace.element_size() < need:
+        raise FlceError(ERR_WORKSPACE_TOO_SMALL, "forward")
+    return workspace
+
+
+def forward(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, *, out: dict | None = None,
+            workspace: torch.Tensor | None = None, stream=None, check: bool = False):
+    """Per-token loss, lse and target logit, and the mean loss.
+
+    H (N, D) and W (V, D) are contiguous CUDA tensors, both bfloat16 or both
+    float32; y is int64 (N,).  Returns (loss, lse, target_logit, mean) as fp32
+    CUDA tensors (mean is 0-d).  ``out`` may supply any of the output tensors
+    by name and ``workspace`` a uint8 tensor of at least ``workspace_size``
+    bytes.  The call is asynchronous on ``stream`` (default: current stream);
+    ``check=True`` synchronises and raises on device-side errors.
+    """
+    N, V, D, code = _check_inputs(H, W, y)
+    dev = H.device
+    loss, lse, tgt, mean = _alloc_outputs(N, dev, out)
+    if N == 0:
+        return loss, lse, tgt, mean
+    ws = _workspace(N, V, D, code, dev, workspace)
+    sp = _stream_ptr(stream, dev)
+    lib = load_library()
+    st = lib.flce_forward(H.data_ptr(), W.data_ptr(), y.data_ptr(), N, V, D, code,
+                          loss.data_ptr(), lse.data_ptr(), tgt.data_ptr(), mean.data_ptr(),
+                          ws.data_ptr(), ws.numel() * ws.element_size(), sp)
+    _raise_on(st, "flce_forward")
+    if check:
+        _raise_on(lib.flce_check(ws.data_ptr(), sp), "flce_forward (device)")
+    return loss, lse, tgt, mean
+
+
+def partials(H, W, y, target_logit, workspace, stream=None):
+    """First stage only (contraction + online (m, s) per vocab slab); see flce_partials."""
+    N, V, D, code = _check_inputs(H, W, y)
+    if N == 0:
+        return
+    sp = _stream_ptr(stream, H.device)
+    _raise_on(load_library().flce_partials(H.data_ptr(), W.data_ptr(), y.data_ptr(), N, V, D, code,
+                                           target_logit.data_ptr(), workspace.data_ptr(),
+                                           workspace.numel() * workspace.element_size(), sp),
+              "flce_partials")
+
+
+def merge(y, V, loss, lse, target_logit, mean, workspace, stream=None):
+    """Second stage only (combine slab states, loss, mean); see flce_merge."""
+    N = y.shape[0]
+    if N == 0:
+        return
+    sp = _stream_ptr(stream, y.device)
+    _raise_on(load_library().flce_merge(y.data_ptr(), N, int(V), loss.data_ptr(), lse.data_ptr(),
+                                        target_logit.data_ptr(),
+                                        mean.data_ptr() if mean is not None else None,
+                                        workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(), sp),
+              "flce_merge")
+
+
+def check(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise ``stream`` and return the status of the last call on ``workspace``."""
+    return int(load_library().flce_check(workspace.data_ptr(), _stream_ptr(stream, workspace.device)))
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int = 1_000_000, stream=None) -> int:
+    """Run the bounded-wait self-test kernel; returns the launch status (read the result with check)."""
+    return int(load_library().flce_selftest_wait_timeout(
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(), int(limit_ns),
+        _stream_ptr(stream, workspace.device)))

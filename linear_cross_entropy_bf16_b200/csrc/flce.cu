@@ -1,0 +1,345 @@
+// libflce.so: host side of the C ABI declared in include/flce.h.
+//
+// Argument validation, the split-V schedule, TMA tensor maps and the kernel
+// launches for the fused linear cross-entropy forward (D. Ineshin, "Een
+// gefuseerde forward-kernel voor lineaire cross-entropy op Apple-GPU's",
+// 2026, section 1).  Every launch is asynchronous on the caller's stream; the
+// library allocates nothing.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "flce.h"
+#include "flce_kernels.cuh"
+
+namespace {
+
+using namespace flce;
+
+constexpr uint64_t kDefaultWaitLimitNs = 4000000000ull;  // 4 s in one wait: far beyond any real stage
+constexpr int kSimtBlocksPerSm = 4;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+bool sizes_ok(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
+  if (N < 0 || V < 1 || D < 1) return false;
+  if (dtype != FLCE_BF16 && dtype != FLCE_FP32) return false;
+  return true;
+}
+
+int64_t slab_capacity(int64_t V) { return std::min<int64_t>(cdiv(V, kTileCols), kMaxSlabs); }
+
+size_t workspace_bytes_for(int64_t N, int64_t V) {
+  const size_t part = align256(size_t(8) * size_t(N) * size_t(slab_capacity(V)));
+  const size_t sums = align256(size_t(8) * size_t(std::max<int64_t>(1, cdiv(N, kMergeThreads))));
+  return kHeaderBytes + part + sums;
+}
+
+// Choose P (slabs per token block) for `tb` token blocks, `nt` vocab tiles and
+// `g` concurrent CTAs.  Units are handed out round-robin (CTA c takes units
+// c, c+g, ...), slab-major, so the CTAs running at the same time share the
+// same W tiles.  CTA 0 is then the busiest: it takes ceil(U/g) units, of
+// which ceil(R/g) are the longer ones (R = rem * tb units in the first `rem`
+// slabs).  Minimise that makespan in tiles plus a small per-unit cost.
+void choose_slabs(int64_t tb, int64_t nt, int64_t g, int64_t pcap, int32_t& P_out,
+                  int64_t& makespan_out) {
+  double best = 1e300;
+  int32_t bestP = 1;
+  int64_t best_ms = 0;
+  for (int64_t P = 1; P <= std::min(nt, pcap); ++P) {
+    const int64_t U = tb * P;
+    const int64_t base = nt / P, rem = nt % P;
+    const int64_t waves = cdiv(U, g);
+    const int64_t ms = waves * base + cdiv(rem * tb, g);
+    const double cost = double(ms) + 0.05 * double(waves);
+    if (cost < best - 1e-9) {
+      best = cost;
+      bestP = int32_t(P);
+      best_ms = ms;
+    }
+  }
+  P_out = bestP;
+  makespan_out = best_ms;
+}
+
+flce_status make_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int32_t sms,
+                      flce_plan_t* p) {
+  std::memset(p, 0, sizeof(*p));
+  p->N = N;
+  p->V = V;
+  p->D = D;
+  p->dtype = int32_t(dtype);
+  p->tile_cols = kTileCols;
+  const bool tc = dtype == FLCE_BF16;
+  p->block_rows = tc ? tc::BM : simt::BM;
+  p->k_block = tc ? tc::BK : simt::BK;
+  p->token_blocks = cdiv(std::max<int64_t>(N, 1), p->block_rows);
+  p->vocab_tiles = cdiv(V, kTileCols);
+  const int64_t g = tc ? int64_t(sms) : int64_t(sms) * kSimtBlocksPerSm;
+  int64_t ms = 0;
+  choose_slabs(p->token_blocks, p->vocab_tiles, g, slab_capacity(V), p->slabs, ms);
+  p->slab_base = int32_t(p->vocab_tiles / p->slabs);
+  p->slab_rem = int32_t(p->vocab_tiles % p->slabs);
+  p->units = p->token_blocks * p->slabs;
+  p->grid = int32_t(tc ? std::min<int64_t>(sms, p->units) : p->units);
+  p->makespan_tiles = ms;
+  p->workspace_bytes = workspace_bytes_for(N, V);
+  return FLCE_OK;
+}
+
+// ---------------------------------------------------------------- driver entry point
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool load_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// Row-major (rows, D) bf16 matrix, boxes of 64 x box_rows, 128-byte swizzle,
+// zero fill outside the matrix (ragged N, V and D).
+bool encode_bf16_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t D, int box_rows) {
+  cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(D) * 2};
+  cuuint32_t box[2] = {cuuint32_t(tc::BK), cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0, minor = 0;
+};
+
+flce_status device_info(DeviceInfo& di) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&di.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&di.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  // The kernels are built for sm_100a only (B200).
+  if (di.major != 10 || di.minor != 0) return FLCE_ERR_UNSUPPORTED;
+  return FLCE_OK;
+}
+
+flce_status set_smem_attr_once() {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    err = cudaFuncSetAttribute(tc::flce_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tc::SMEM_BYTES);
+  });
+  return err == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+flce_status check_forward_args(const void* H, const void* W, const int64_t* y, int64_t N,
+                               int64_t V, int64_t D, flce_dtype dtype, const void* ws,
+                               size_t ws_bytes) {
+  if (!sizes_ok(N, V, D, dtype)) return FLCE_ERR_INVALID_ARG;
+  if (N == 0) return FLCE_OK;
+  if (!H || !W || !y || !ws) return FLCE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FLCE_ERR_INVALID_ARG;
+  if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31) || D >= (int64_t(1) << 31))
+    return FLCE_ERR_UNSUPPORTED;
+  if (dtype == FLCE_BF16 && (D % 8 != 0 || !aligned16(H) || !aligned16(W)))
+    return FLCE_ERR_UNSUPPORTED;
+  if (dtype == FLCE_FP32 && ((reinterpret_cast<uintptr_t>(H) | reinterpret_cast<uintptr_t>(W)) & 3u))
+    return FLCE_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes_for(N, V)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  return FLCE_OK;
+}
+
+flce_status launch_partials(const void* H, const void* W, const int64_t* y, int64_t N, int64_t V,
+                            int64_t D, flce_dtype dtype, float* out_target, void* ws,
+                            cudaStream_t st) {
+  DeviceInfo di;
+  flce_status s = device_info(di);
+  if (s != FLCE_OK) return s;
+  flce_plan_t plan;
+  make_plan(N, V, D, dtype, di.sms, &plan);
+
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
+  float2* part = reinterpret_cast<float2*>(wsb + kHeaderBytes);
+  if (cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
+
+  Schedule sch;
+  sch.token_blocks = int32_t(plan.token_blocks);
+  sch.slabs = plan.slabs;
+  sch.slab_base = plan.slab_base;
+  sch.slab_rem = plan.slab_rem;
+  sch.units = int32_t(plan.units);
+
+  if (dtype == FLCE_BF16) {
+    if (!load_encoder()) return FLCE_ERR_CUDA;
+    if ((s = set_smem_attr_once()) != FLCE_OK) return s;
+    CUtensorMap tmH, tmW;
+    if (!encode_bf16_rows(&tmH, H, N, D, tc::BM) || !encode_bf16_rows(&tmW, W, V, D, tc::BN))
+      return FLCE_ERR_UNSUPPORTED;
+    tc::Args a;
+    a.y = y;
+    a.part = part;
+    a.target_logit = out_target;
+    a.hdr = hdr;
+    a.N = int32_t(N);
+    a.V = int32_t(V);
+    a.D = int32_t(D);
+    a.kblocks = int32_t(cdiv(D, tc::BK));
+    a.sch = sch;
+    a.wait_limit_ns = kDefaultWaitLimitNs;
+    tc::flce_tc_kernel<<<plan.grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(tmH, tmW, a);
+  } else {
+    simt::Args a;
+    a.H = H;
+    a.W = W;
+    a.y = y;
+    a.part = part;
+    a.target_logit = out_target;
+    a.hdr = hdr;
+    a.N = int32_t(N);
+    a.V = int32_t(V);
+    a.D = int32_t(D);
+    a.sch = sch;
+    simt::flce_simt_kernel<float><<<plan.grid, simt::NUM_THREADS, 0, st>>>(a);
+  }
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+flce_status launch_merge(const int64_t* y, int64_t N, int64_t V, float* out_loss, float* out_lse,
+                         float* out_target, float* out_mean, const void* ws, size_t ws_bytes,
+                         cudaStream_t st) {
+  uint8_t* wsb = static_cast<uint8_t*>(const_cast<void*>(ws));
+  MergeArgs m;
+  m.hdr = reinterpret_cast<WsHeader*>(wsb);
+  m.part = reinterpret_cast<const float2*>(wsb + kHeaderBytes);
+  m.block_sums = reinterpret_cast<double*>(
+      wsb + kHeaderBytes + align256(size_t(8) * size_t(N) * size_t(slab_capacity(V))));
+  m.y = y;
+  m.target_logit = out_target;
+  m.loss = out_loss;
+  m.lse = out_lse;
+  m.mean = out_mean;
+  m.N = int32_t(N);
+  m.V = int32_t(V);
+  m.max_slabs = int32_t(slab_capacity(V));
+  (void)ws_bytes;
+  const int blocks = int(cdiv(N, kMergeThreads));
+  flce_merge_kernel<<<blocks, kMergeThreads, 0, st>>>(m);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t flce_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
+  if (!sizes_ok(N, V, D, dtype)) return 0;
+  return workspace_bytes_for(N, V);
+}
+
+flce_status flce_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int32_t sm_count,
+                      flce_plan_t* plan) {
+  if (!plan || sm_count < 1 || !sizes_ok(N, V, D, dtype)) return FLCE_ERR_INVALID_ARG;
+  return make_plan(N, V, D, dtype, sm_count, plan);
+}
+
+flce_status flce_partials(const void* H, const void* W, const int64_t* y, int64_t N, int64_t V,
+                          int64_t D, flce_dtype dtype, float* out_target_logit, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  flce_status s = check_forward_args(H, W, y, N, V, D, dtype, workspace, workspace_bytes);
+  if (s != FLCE_OK || N == 0) return s;
+  if (!out_target_logit) return FLCE_ERR_INVALID_ARG;
+  return launch_partials(H, W, y, N, V, D, dtype, out_target_logit, workspace,
+                         static_cast<cudaStream_t>(stream));
+}
+
+flce_status flce_merge(const int64_t* y, int64_t N, int64_t V, float* out_loss, float* out_lse,
+                       float* out_target_logit, float* out_mean, const void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (N < 0 || V < 1) return FLCE_ERR_INVALID_ARG;
+  if (N == 0) return FLCE_OK;
+  if (!y || !out_loss || !out_lse || !out_target_logit || !workspace) return FLCE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FLCE_ERR_INVALID_ARG;
+  if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
+  if (workspace_bytes < workspace_bytes_for(N, V)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  return launch_merge(y, N, V, out_loss, out_lse, out_target_logit, out_mean, workspace,
+                      workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+flce_status flce_forward(const void* H, const void* W, const int64_t* y, int64_t N, int64_t V,
+                         int64_t D, flce_dtype dtype, float* out_loss, float* out_lse,
+                         float* out_target_logit, float* out_mean, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  flce_status s = check_forward_args(H, W, y, N, V, D, dtype, workspace, workspace_bytes);
+  if (s != FLCE_OK || N == 0) return s;
+  if (!out_loss || !out_lse || !out_target_logit) return FLCE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = launch_partials(H, W, y, N, V, D, dtype, out_target_logit, workspace, st);
+  if (s != FLCE_OK) return s;
+  return launch_merge(y, N, V, out_loss, out_lse, out_target_logit, out_mean, workspace,
+                      workspace_bytes, st);
+}
+
+flce_status flce_check(const void* workspace, void* stream) {
+  if (!workspace) return FLCE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FLCE_ERR_CUDA;
+  uint32_t status = 0;
+  if (cudaMemcpy(&status, workspace, sizeof(status), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  if (status & kStatTimeout) return FLCE_ERR_TIMEOUT;
+  if (status & kStatTarget) return FLCE_ERR_TARGET_OUT_OF_RANGE;
+  if (status & kStatBadWs) return FLCE_ERR_INVALID_ARG;
+  return FLCE_OK;
+}
+
+const char* flce_status_string(flce_status status) {
+  switch (status) {
+    case FLCE_OK: return "ok";
+    case FLCE_ERR_INVALID_ARG: return "invalid argument";
+    case FLCE_ERR_UNSUPPORTED: return "unsupported device, shape or alignment";
+    case FLCE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case FLCE_ERR_CUDA: return "CUDA error";
+    case FLCE_ERR_TARGET_OUT_OF_RANGE: return "target outside [0, V)";
+    case FLCE_ERR_TIMEOUT: return "bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+flce_status flce_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint64_t limit_ns,
+                                       void* stream) {
+  if (!workspace || workspace_bytes < kHeaderBytes) return FLCE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FLCE_ERR_INVALID_ARG;
+  if (limit_ns < 1000 || limit_ns > 1000000000ull) return FLCE_ERR_INVALID_ARG;
+  DeviceInfo di;
+  flce_status s = device_info(di);
+  if (s != FLCE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
+  flce_wait_probe_kernel<<<1, 32, 0, st>>>(static_cast<WsHeader*>(workspace), limit_ns);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+}  // extern "C"

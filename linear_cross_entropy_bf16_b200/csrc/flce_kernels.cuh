@@ -1,0 +1,640 @@
+// Device code of the fused linear cross-entropy forward (sm_100a).
+//
+// Operation: D. Ineshin, "Een gefuseerde forward-kernel voor lineaire
+// cross-entropy op Apple-GPU's" (2026), section 1.  Z = H W^T; each vocab tile
+// is folded into a running online log-sum-exp state (m, s) with
+//   m' = max(m, m_t),  s' = s exp(m - m') + sum_j exp(z_j - m'),
+// the target logit is captured from the tile that holds it, and after the last
+// tile logsumexp = m + log s and loss = logsumexp - z_target.
+//
+// B200 design (not the page's one-dispatch-per-tile chain):
+//   * flce_tc_kernel: a persistent, warp-specialised tcgen05 GEMM.  One CTA
+//     per SM walks work units (128 tokens x one vocab slab of 256-column
+//     tiles).  Warp 0 streams H and W K-blocks with TMA into a 4-stage
+//     shared-memory ring, warp 1 issues 128x256x16 bf16 MMAs into a
+//     double-buffered fp32 TMEM accumulator, and warps 2-5 (one TMEM lane,
+//     i.e. one token, per thread) fold each finished tile into (m, s) and
+//     capture the target logit.  Logits never leave TMEM/registers.
+//   * flce_simt_kernel: the same decomposition with fp32 FFMA tiles, for fp32
+//     inputs (bf16 tensor cores cannot honour fp32 inputs).
+//   * flce_merge_kernel: combines the P slab states of each token in a fixed
+//     order (the recurrence of section 1 applied to whole slabs), writes
+//     lse/loss, and reduces the mean deterministically in fp64.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ptx_sm100.cuh"
+
+namespace flce {
+
+// ----------------------------------------------------------------- constants
+
+constexpr int kTileCols = 256;   // vocab columns per tile (UMMA N, TMEM columns)
+constexpr int kMaxSlabs = 512;   // partial states per token, at most
+
+// workspace layout: [header 256 B][partials float2[P][N]][block sums double[ceil(N/256)]]
+constexpr size_t kHeaderBytes = 256;
+constexpr uint32_t kWsMagic = 0x464C4345u;  // "FLCE"
+
+// device status bits (workspace header word 0)
+constexpr uint32_t kStatTarget = 1u;    // some y_i outside [0, V)
+constexpr uint32_t kStatTimeout = 2u;   // a bounded wait ran out
+constexpr uint32_t kStatBadWs = 4u;     // merge found a workspace not prepared by partials
+
+struct WsHeader {
+  uint32_t status;    // OR of kStat* bits for the current call
+  uint32_t counter;   // merge blocks finished (last one computes the mean)
+  uint32_t magic;     // kWsMagic once the partials stage has run
+  int32_t slabs;      // P used by the partials stage
+  int64_t N;
+  int64_t V;
+};
+static_assert(sizeof(WsHeader) <= kHeaderBytes, "header");
+
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e): exp(x) = 2^(x log2 e)
+
+// ----------------------------------------------------------------- schedule
+
+struct Schedule {
+  int32_t token_blocks;  // TB
+  int32_t slabs;         // P
+  int32_t slab_base;     // tiles per slab (NT / P)
+  int32_t slab_rem;      // the first slab_rem slabs hold one more tile
+  int32_t units;         // TB * P; unit u -> slab u / TB, token block u % TB
+};
+
+__device__ __forceinline__ void unit_coords(const Schedule& s, int u, int& slab, int& tblock,
+                                            int& tile0, int& ntiles) {
+  slab = u / s.token_blocks;
+  tblock = u - slab * s.token_blocks;
+  tile0 = slab * s.slab_base + min(slab, s.slab_rem);
+  ntiles = s.slab_base + (slab < s.slab_rem ? 1 : 0);
+}
+
+// ----------------------------------------------------------------- bounded waits
+
+// Bounded mbarrier waits.  `flag` is the CTA's shared abort flag: once any
+// role of the CTA gives up, the others stop waiting too.  `status` is the
+// workspace status word in global memory.
+
+// Wait for phase `parity` of the mbarrier at `bar`, for at most limit_ns.
+// Returns false (after recording kStatTimeout and raising the CTA abort flag)
+// when the limit runs out, or when another role of this CTA has aborted
+// (flag == nullptr: ignore other roles, only the time limit applies).
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int* flag,
+                                       uint32_t* status, uint64_t limit_ns) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((n & 31u) == 0) {
+      if (flag != nullptr && *flag) return false;
+      if (ptx::globaltimer_ns() - t0 > limit_ns) {
+        if (flag != nullptr) *flag = 1;
+        atomicOr(status, kStatTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* flag,
+                                             uint32_t* status, uint64_t limit_ns) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, flag, status, limit_ns);
+}
+
+// z[idx] for a register array and a runtime idx in [0, 32), as a five-level
+// select tree with compile-time indices (an indexed read would move the whole
+// array to local memory).
+__device__ __forceinline__ float pick32(const float (&z)[32], int idx) {
+  float a[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) a[j] = (idx & 16) ? z[j + 16] : z[j];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = (idx & 8) ? a[j + 8] : a[j];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) a[j] = (idx & 4) ? a[j + 4] : a[j];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) a[j] = (idx & 2) ? a[j + 2] : a[j];
+  return (idx & 1) ? a[1] : a[0];
+}
+
+// ----------------------------------------------------------------- tcgen05 kernel
+
+namespace tc {
+
+constexpr int BM = 128;                      // tokens per tile (UMMA M, TMEM lanes)
+constexpr int BN = kTileCols;                // vocab columns per tile (UMMA N)
+constexpr int BK = 64;                       // bf16 per K block = 128 B = one swizzle row
+constexpr int UMMA_K = 16;                   // K per tcgen05.mma (32 bytes)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;         // 16 KiB
+constexpr int B_BYTES = BN * BK * 2;         // 32 KiB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;             // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int EPI_WARPS = 4;
+constexpr uint32_t TMEM_COLS = 512;          // two BN-column fp32 accumulators
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+// Instruction descriptor of tcgen05.mma kind::f16: D fp32 (bits 4-5 = 1),
+// A and B bf16 (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0),
+// N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
+                            (uint32_t(BM >> 4) << 24);
+
+// Shared-memory matrix descriptor for a K-major operand tile written by TMA
+// with 128-byte swizzling: rows of 128 B, 8-row swizzle atoms of 1024 B
+// (stride byte offset 1024), version 1 (bit 46), swizzle mode 2 (bits 61-63).
+// `addr` is the shared address of the first element used by this MMA; moving
+// along K inside the 128-byte row is a plain +32 B per 16 bf16.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+  return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
+struct Args {
+  const int64_t* y;
+  float2* part;            // [P][N] (m, s) per slab and token
+  float* target_logit;     // [N]
+  WsHeader* hdr;
+  int32_t N, V, D;
+  int32_t kblocks;         // ceil(D / BK)
+  Schedule sch;
+  uint64_t wait_limit_ns;
+};
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW,
+               const Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzle atoms
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full_bar = bars;                  // [STAGES] TMA landed
+  uint64_t* empty_bar = bars + STAGES;        // [STAGES] MMAs done reading the slot
+  uint64_t* tfull_bar = bars + 2 * STAGES;    // [2] accumulator ready
+  uint64_t* tempty_bar = bars + 2 * STAGES + 2;  // [2] accumulator drained
+  uint64_t* done_bar = bars + 2 * STAGES + 4;    // all MMAs retired
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(ptx::smem_addr(&full_bar[s]), 1);
+      ptx::mbar_init(ptx::smem_addr(&empty_bar[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(ptx::smem_addr(&tfull_bar[b]), 1);
+      ptx::mbar_init(ptx::smem_addr(&tempty_bar[b]), EPI_WARPS);
+    }
+    ptx::mbar_init(ptx::smem_addr(done_bar), 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+    ptx::fence_proxy_async_smem();
+    ptx::prefetch_tensormap(&tmH);
+    ptx::prefetch_tensormap(&tmW);
+    if (blockIdx.x == 0) {
+      a.hdr->slabs = a.sch.slabs;
+      a.hdr->N = a.N;
+      a.hdr->V = a.V;
+      a.hdr->magic = kWsMagic;
+    }
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_addr(tmem_slot), TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before_sync();
+  __syncthreads();
+  ptx::tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  uint32_t* status = &a.hdr->status;
+  const uint64_t lim = a.wait_limit_ns;
+  const Schedule& sch = a.sch;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_h = ptx::policy_evict_last();    // H is re-read for every tile
+      const uint64_t pol_w = ptx::policy_evict_normal();  // W tiles are shared by concurrent CTAs
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t used = 0, last_parity = 0;  // per stage: ever issued / parity of last issue
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < sch.units; u += gridDim.x) {
+        int slab, tb, t0, nt;
+        unit_coords(sch, u, slab, tb, t0, nt);
+        for (int t = t0; ok && t < t0 + nt; ++t) {
+          for (int kb = 0; kb < a.kblocks; ++kb) {
+            if (!wait_bounded(ptx::smem_addr(&empty_bar[stage]), phase ^ 1u, abort_flag, status, lim)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = ptx::smem_addr(&full_bar[stage]);
+            const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
+            ptx::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+            ptx::tma_load_2d(sa, &tmH, fb, kb * BK, tb * BM, pol_h);
+            ptx::tma_load_2d(sa + A_BYTES, &tmW, fb, kb * BK, t * BN, pol_w);
+            used |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+      // Every issued copy must land before the CTA may exit.  On the normal
+      // path each of these waits returns at once.
+      for (int s = 0; s < STAGES; ++s)
+        if (used & (1u << s))
+          wait_bounded(ptx::smem_addr(&full_bar[s]), (last_parity >> s) & 1u, nullptr, status, lim);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < sch.units; u += gridDim.x) {
+        int slab, tb, t0, nt;
+        unit_coords(sch, u, slab, tb, t0, nt);
+        for (int t = 0; ok && t < nt; ++t) {
+          if (!wait_bounded(ptx::smem_addr(&tempty_bar[acc]), acc_phase ^ 1u, abort_flag, status, lim)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after_sync();
+          const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+          for (int kb = 0; kb < a.kblocks; ++kb) {
+            if (!wait_bounded(ptx::smem_addr(&full_bar[stage]), phase, abort_flag, status, lim)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after_sync();
+            const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              const uint64_t ad = sw128_desc(sa + k * UMMA_K * 2);
+              const uint64_t bd = sw128_desc(sa + A_BYTES + k * UMMA_K * 2);
+              ptx::mma_bf16(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+            }
+            ptx::mma_commit(ptx::smem_addr(&empty_bar[stage]));  // slot free once read
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          ptx::mma_commit(ptx::smem_addr(&tfull_bar[acc]));  // accumulator complete
+          if (++acc == 2) {
+            acc = 0;
+            acc_phase ^= 1u;
+          }
+        }
+      }
+      // Retire every MMA this thread issued before TMEM is released.
+      ptx::mma_commit(ptx::smem_addr(done_bar));
+      wait_bounded(ptx::smem_addr(done_bar), 0, nullptr, status, lim);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
+    const int row_in_tile = quad * 32 + lane;  // token row of this thread inside the tile
+    const uint32_t lane_addr = uint32_t(quad * 32) << 16;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < sch.units; u += gridDim.x) {
+      int slab, tb, t0, nt;
+      unit_coords(sch, u, slab, tb, t0, nt);
+      const int row = tb * BM + row_in_tile;
+      const bool valid = row < a.N;
+      const int64_t yi = valid ? a.y[row] : -1;
+      float m = -INFINITY, s = 0.f, zt = 0.f;
+      bool got = false;
+      for (int t = t0; t < t0 + nt; ++t) {
+        bool w = wait_bounded(ptx::smem_addr(&tfull_bar[acc]), acc_phase, abort_flag, status, lim);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after_sync();
+        const int v0 = t * BN;
+        const int ncols = min(BN, a.V - v0);
+        const int64_t rel = yi - v0;  // target column inside this tile, if in [0, BN)
+        const uint32_t taddr = tmem_base + lane_addr + uint32_t(acc * BN);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          if (c * 32 >= ncols) break;  // warp-uniform: the rest of the tile is past V
+          uint32_t u32[32];
+          ptx::tmem_ld32_wait(taddr + uint32_t(c * 32), u32);
+          float z[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) z[j] = __uint_as_float(u32[j]);
+          if (ncols - c * 32 < 32) {  // ragged last tile: columns >= V do not exist
+            const int lim = ncols - c * 32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j >= lim) z[j] = -INFINITY;
+          }
+          // target capture: the tile holding y_i records z_{i, y_i}
+          const int64_t rc = rel - c * 32;
+          if (rc >= 0 && rc < 32) {
+            zt = pick32(z, int(rc));
+            got = true;
+          }
+          // m_t = max_j z_j over this chunk, tree-reduced
+          float mx[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) mx[j] = fmaxf(z[j], z[j + 16]);
+#pragma unroll
+          for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+            for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
+          const float m_new = fmaxf(m, mx[0]);
+          const float ms = m_new * kLog2e;
+          // sum_j exp(z_j - m') as 2^(z_j log2 e - m' log2 e)
+          float e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int j = 0; j < 32; ++j) e[j & 3] += ptx::ex2(fmaf(z[j], kLog2e, -ms));
+          // s' = s exp(m - m') + sum; m = -inf on the first chunk gives exp(-inf) = 0
+          s = fmaf(s, ptx::ex2((m - m_new) * kLog2e), (e[0] + e[1]) + (e[2] + e[3]));
+          m = m_new;
+        }
+        ptx::tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&tempty_bar[acc]));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (valid) {
+        a.part[size_t(slab) * size_t(a.N) + size_t(row)] = make_float2(m, s);
+        if (got) a.target_logit[row] = zt;
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  __syncwarp();  // lanes 1..31 of warps 0 and 1 wait here for their lane 0
+  ptx::tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after_sync();
+    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace tc
+
+// ----------------------------------------------------------------- fp32 FFMA kernel
+
+namespace simt {
+
+constexpr int BM = 64;           // tokens per work unit
+constexpr int BNS = 64;          // vocab columns per sub-tile (4 per 256-column tile)
+constexpr int BK = 32;
+constexpr int NUM_THREADS = 256; // 16 x 16 threads, 4 x 4 outputs each
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+struct Args {
+  const void* H;
+  const void* W;
+  const int64_t* y;
+  float2* part;
+  float* target_logit;
+  WsHeader* hdr;
+  int32_t N, V, D;
+  Schedule sch;
+};
+
+// One CTA per work unit (slab, token block).  Thread (ty, tx) owns rows
+// ty*4 + i and columns tx + 16 j of each 64 x 64 sub-tile.  The 16 threads
+// sharing a row sit in one half-warp, so each row's tile max and exp-sum are
+// reduced with xor shuffles over 16 lanes.
+template <typename T>
+__global__ void __launch_bounds__(NUM_THREADS) flce_simt_kernel(const Args a) {
+  __shared__ float sH[BK][BM + 4];
+  __shared__ float sW[BK][BNS + 4];
+  const T* H = static_cast<const T*>(a.H);
+  const T* W = static_cast<const T*>(a.W);
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+
+  if (blockIdx.x == 0 && tid == 0) {
+    a.hdr->slabs = a.sch.slabs;
+    a.hdr->N = a.N;
+    a.hdr->V = a.V;
+    a.hdr->magic = kWsMagic;
+  }
+
+  int slab, tb, t0, nt;
+  unit_coords(a.sch, blockIdx.x, slab, tb, t0, nt);
+  const int row0 = tb * BM;
+
+  float m[4], s[4], zt[4];
+  bool got[4];
+  int64_t yrow[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m[i] = -INFINITY;
+    s[i] = 0.f;
+    zt[i] = 0.f;
+    got[i] = false;
+    const int r = row0 + ty * 4 + i;
+    yrow[i] = r < a.N ? a.y[r] : -1;
+  }
+
+  const int c_begin = t0 * kTileCols;
+  const int c_end = min(a.V, (t0 + nt) * kTileCols);
+  for (int c0 = c_begin; c0 < c_end; c0 += BNS) {
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+    for (int k0 = 0; k0 < a.D; k0 += BK) {
+      // stage a 64 x 32 block of H and of W, transposed to [k][row]; zeros off the edges
+      for (int e = tid; e < BM * BK; e += NUM_THREADS) {
+        const int r = e / BK, k = e % BK;
+        const int gr = row0 + r, gk = k0 + k;
+        sH[k][r] = (gr < a.N && gk < a.D) ? to_f32<T>(H[size_t(gr) * a.D + gk]) : 0.f;
+        const int gc = c0 + r;
+        sW[k][r] = (gc < a.V && gk < a.D) ? to_f32<T>(W[size_t(gc) * a.D + gk]) : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int k = 0; k < BK; ++k) {
+        float hv[4], wv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) hv[i] = sH[k][ty * 4 + i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) wv[j] = sW[k][tx + 16 * j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(hv[i], wv[j], acc[i][j]);
+      }
+      __syncthreads();
+    }
+
+    // online update of each owned row with this 64-column sub-tile
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float z[4];
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int col = c0 + tx + 16 * j;
+        z[j] = col < a.V ? acc[i][j] : -INFINITY;
+        if (int64_t(col) == yrow[i]) {
+          zt[i] = acc[i][j];
+          got[i] = true;
+        }
+        tmax = fmaxf(tmax, z[j]);
+      }
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1)
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
+      const float m_new = fmaxf(m[i], tmax);
+      const float ms = m_new * kLog2e;
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sum += ptx::ex2(fmaf(z[j], kLog2e, -ms));
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      s[i] = fmaf(s[i], ptx::ex2((m[i] - m_new) * kLog2e), sum);
+      m[i] = m_new;
+    }
+  }
+
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = row0 + ty * 4 + i;
+    if (r < a.N) {
+      if (tx == 0) a.part[size_t(slab) * size_t(a.N) + size_t(r)] = make_float2(m[i], s[i]);
+      if (got[i]) a.target_logit[r] = zt[i];
+    }
+  }
+}
+
+}  // namespace simt
+
+// ----------------------------------------------------------------- merge + mean
+
+constexpr int kMergeThreads = 256;
+
+struct MergeArgs {
+  const float2* part;
+  const int64_t* y;
+  float* target_logit;
+  float* loss;
+  float* lse;
+  float* mean;          // may be null
+  double* block_sums;   // [gridDim.x]
+  WsHeader* hdr;
+  int32_t N, V;
+  int32_t max_slabs;    // capacity of the partial array in this workspace
+};
+
+// One thread per token: m = max_p m_p, s = sum_p s_p exp(m_p - m) over the P
+// slab states in slab order (fp64), lse = m + log s, loss = lse - z_target.
+// The mean is a fixed-order fp64 reduction: a shuffle tree per block, then the
+// last block to finish sums the block results in block order.
+__global__ void __launch_bounds__(kMergeThreads) flce_merge_kernel(const MergeArgs a) {
+  __shared__ double warp_sums[kMergeThreads / 32];
+  __shared__ bool is_last;
+  const int i = blockIdx.x * kMergeThreads + threadIdx.x;
+  const WsHeader h = *a.hdr;
+  const bool ws_ok = h.magic == kWsMagic && h.N == a.N && h.V == a.V && h.slabs >= 1 &&
+                     h.slabs <= a.max_slabs;
+  double l = 0.0;
+  if (i < a.N) {
+    float loss_f, lse_f;
+    if (!ws_ok) {
+      loss_f = lse_f = __int_as_float(0x7fc00000);
+      if (i == 0) atomicOr(&a.hdr->status, kStatBadWs);
+    } else {
+      const int P = h.slabs;
+      float M = -INFINITY;
+      for (int p = 0; p < P; ++p) M = fmaxf(M, a.part[size_t(p) * a.N + i].x);
+      double S = 0.0;
+      for (int p = 0; p < P; ++p) {
+        const float2 st = a.part[size_t(p) * a.N + i];
+        S += double(st.y) * exp(double(st.x) - double(M));
+      }
+      const double lse = double(M) + log(S);
+      const int64_t yi = a.y[i];
+      lse_f = float(lse);
+      if (yi < 0 || yi >= a.V) {
+        loss_f = __int_as_float(0x7fc00000);
+        a.target_logit[i] = loss_f;
+        atomicOr(&a.hdr->status, kStatTarget);
+      } else {
+        loss_f = float(lse - double(a.target_logit[i]));
+      }
+    }
+    a.loss[i] = loss_f;
+    a.lse[i] = lse_f;
+    l = double(loss_f);
+  }
+  if (a.mean == nullptr) return;
+  // fixed-order block reduction
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) l += __shfl_down_sync(0xffffffffu, l, off);
+  if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = l;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double b = 0.0;
+    for (int w = 0; w < kMergeThreads / 32; ++w) b += warp_sums[w];
+    a.block_sums[blockIdx.x] = b;
+    __threadfence();
+    const uint32_t ticket = atomicAdd(&a.hdr->counter, 1u);
+    is_last = ticket == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (is_last && threadIdx.x == 0) {
+    __threadfence();
+    const volatile double* bs = a.block_sums;
+    double total = 0.0;
+    for (int b = 0; b < int(gridDim.x); ++b) total += bs[b];
+    *a.mean = float(total / double(a.N));
+    a.hdr->counter = 0;
+  }
+}
+
+// ----------------------------------------------------------------- self-test
+
+// One thread waits on a barrier that nothing will complete; the bounded wait
+// gives up after limit_ns, records kStatTimeout and the kernel returns.
+__global__ void flce_wait_probe_kernel(WsHeader* hdr, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int flag;
+  if (threadIdx.x != 0) return;
+  flag = 0;
+  ptx::mbar_init(ptx::smem_addr(&bar), 1);
+  ptx::fence_barrier_init();
+  wait_bounded(ptx::smem_addr(&bar), 0, &flag, &hdr->status, limit_ns);
+}
+
+}  // namespace flce

@@ -1,0 +1,164 @@
+"""The C ABI on the host (no GPU): exports, sizes, schedule and argument checks.
+
+Nothing here launches a kernel: every call below returns before any CUDA API
+is reached (argument checks) or is host-only by contract (workspace size,
+plan, status strings).
+"""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import linear_cross_entropy_bf16_b200 as flce
+from linear_cross_entropy_bf16_b200 import build as flce_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flce.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    flce_build.build()
+    return flce.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"FLCE_API\s+[\w\s\*]+?\b(flce_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    assert {"flce_workspace_size", "flce_forward", "flce_check", "flce_status_string",
+            "flce_partials", "flce_merge", "flce_plan"} <= names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert getattr(lib, name) is not None
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert flce.status_string(s) and flce.status_string(s) != "unknown status"
+    assert flce.status_string(99) == "unknown status"
+
+
+def test_workspace_is_O_N_not_O_NV(lib):
+    for N, V, D in [(8192, 151936, 4096), (16384, 262144, 2048), (1, 1, 8), (4096, 128256, 4096)]:
+        ws = flce.workspace_size(N, V, D)
+        slabs = min(math.ceil(V / 256), 512)
+        assert ws >= 256 + 8 * N * slabs
+        assert ws <= 256 + 8 * N * 512 + 256 + 8 * (N // 256 + 1) + 512
+        if V >= 100000:
+            assert ws < 4 * N * V / 50        # the logits it replaces are 4 N V bytes
+    assert lib.flce_workspace_size(-1, 10, 8, 0) == 0
+    assert lib.flce_workspace_size(4, 0, 8, 0) == 0
+    assert lib.flce_workspace_size(4, 10, 0, 0) == 0
+    assert lib.flce_workspace_size(4, 10, 8, 7) == 0
+    # independent of dtype and D
+    assert flce.workspace_size(100, 5000, 64) == flce.workspace_size(100, 5000, 4096, 1)
+
+
+def simulate_makespan(p):
+    tb, P, base, rem, grid = p["token_blocks"], p["slabs"], p["slab_base"], p["slab_rem"], p["grid"]
+    units = tb * P
+    load = [0] * grid
+    for u in range(units):
+        slab = u // tb
+        load[u % grid] += base + (1 if slab < rem else 0)
+    return max(load)
+
+
+@pytest.mark.parametrize("N,V,D,dtype,sms", [
+    (8192, 151936, 4096, 0, 148), (4096, 128256, 4096, 0, 148), (16384, 262144, 2048, 0, 148),
+    (1024, 32000, 1024, 0, 148), (256, 2048, 256, 1, 148), (1, 1, 8, 0, 148), (7, 257, 8, 0, 148),
+    (129, 1000, 64, 0, 132), (300, 151936, 128, 0, 148), (2048, 500, 16, 1, 148)])
+def test_plan_covers_every_tile_once_and_balances(lib, N, V, D, dtype, sms):
+    p = flce.plan(N, V, D, dtype, sm_count=sms)
+    assert p["vocab_tiles"] == math.ceil(V / 256)
+    assert p["token_blocks"] == math.ceil(N / p["block_rows"])
+    assert 1 <= p["slabs"] <= min(p["vocab_tiles"], 512)
+    # the slabs partition the vocab tiles
+    sizes = [p["slab_base"] + (1 if s < p["slab_rem"] else 0) for s in range(p["slabs"])]
+    assert sum(sizes) == p["vocab_tiles"] and min(sizes) >= 1
+    assert p["units"] == p["token_blocks"] * p["slabs"]
+    assert p["workspace_bytes"] == flce.workspace_size(N, V, D, dtype)
+    if dtype == 0:
+        assert p["grid"] == min(sms, p["units"])
+        assert simulate_makespan(p) == p["makespan_tiles"]
+        total = p["token_blocks"] * p["vocab_tiles"]
+        # within one tile per CTA of the perfect split, whenever every CTA has work
+        if total >= sms:
+            assert p["makespan_tiles"] <= math.ceil(total / sms) + 1
+
+
+def test_headline_plan(lib):
+    p = flce.plan(8192, 151936, 4096, 0, sm_count=148)
+    assert p["block_rows"] == 128 and p["tile_cols"] == 256 and p["k_block"] == 64
+    assert p["token_blocks"] == 64 and p["vocab_tiles"] == 594
+    assert p["makespan_tiles"] == 257          # ceil(64 * 594 / 148)
+
+
+def test_plan_rejects_bad_args(lib):
+    p = flce.Plan()
+    assert lib.flce_plan(4, 10, 8, 0, 0, ctypes.byref(p)) == flce.ERR_INVALID_ARG
+    assert lib.flce_plan(-4, 10, 8, 0, 148, ctypes.byref(p)) == flce.ERR_INVALID_ARG
+    assert lib.flce_plan(4, 10, 8, 0, 148, None) == flce.ERR_INVALID_ARG
+
+
+FAKE = 0x10000          # 64 KiB-aligned, never dereferenced: the checks return first
+
+
+def fwd(lib, H=FAKE, W=FAKE, y=FAKE, N=16, V=100, D=64, dtype=0, loss=FAKE, lse=FAKE, tgt=FAKE,
+        mean=None, ws=FAKE, ws_bytes=1 << 30):
+    return lib.flce_forward(H, W, y, N, V, D, dtype, loss, lse, tgt, mean, ws, ws_bytes, None)
+
+
+def test_forward_argument_checks_need_no_gpu(lib):
+    assert fwd(lib, N=-1) == flce.ERR_INVALID_ARG
+    assert fwd(lib, V=0) == flce.ERR_INVALID_ARG
+    assert fwd(lib, D=0) == flce.ERR_INVALID_ARG
+    assert fwd(lib, dtype=5) == flce.ERR_INVALID_ARG
+    assert fwd(lib, H=None) == flce.ERR_INVALID_ARG
+    assert fwd(lib, W=None) == flce.ERR_INVALID_ARG
+    assert fwd(lib, y=None) == flce.ERR_INVALID_ARG
+    assert fwd(lib, ws=None) == flce.ERR_INVALID_ARG
+    assert fwd(lib, loss=None) == flce.ERR_INVALID_ARG
+    assert fwd(lib, tgt=None) == flce.ERR_INVALID_ARG
+    assert fwd(lib, ws=FAKE + 128) == flce.ERR_INVALID_ARG          # workspace not 256-aligned
+    assert fwd(lib, D=60) == flce.ERR_UNSUPPORTED                   # bf16 rows must be 16-byte strided
+    assert fwd(lib, H=FAKE + 8) == flce.ERR_UNSUPPORTED             # bf16 base must be 16-byte aligned
+    assert fwd(lib, N=1 << 31) == flce.ERR_UNSUPPORTED
+    assert fwd(lib, ws_bytes=767) == flce.ERR_WORKSPACE_TOO_SMALL      # needs 768 here
+    assert fwd(lib, N=0) == flce.OK                                  # no-op
+    assert fwd(lib, N=0, H=None, W=None, y=None, ws=None) == flce.OK
+
+
+def test_merge_and_partials_argument_checks_need_no_gpu(lib):
+    m = lib.flce_merge
+    assert m(FAKE, -1, 10, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None) == flce.ERR_INVALID_ARG
+    assert m(None, 4, 10, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None) == flce.ERR_INVALID_ARG
+    assert m(FAKE, 4, 10, FAKE, FAKE, FAKE, None, FAKE, 10, None) == flce.ERR_WORKSPACE_TOO_SMALL
+    assert m(FAKE, 0, 10, None, None, None, None, None, 0, None) == flce.OK
+    p = lib.flce_partials
+    assert p(FAKE, FAKE, FAKE, 4, 10, 64, 0, None, FAKE, 1 << 30, None) == flce.ERR_INVALID_ARG
+    assert p(FAKE, FAKE, FAKE, 4, 10, 64, 0, FAKE, FAKE, 10, None) == flce.ERR_WORKSPACE_TOO_SMALL
+
+
+def test_selftest_argument_checks_need_no_gpu(lib):
+    s = lib.flce_selftest_wait_timeout
+    assert s(None, 256, 10000, None) == flce.ERR_INVALID_ARG
+    assert s(FAKE, 100, 10000, None) == flce.ERR_INVALID_ARG
+    assert s(FAKE, 256, 10, None) == flce.ERR_INVALID_ARG
+    assert s(FAKE, 256, 10 ** 10, None) == flce.ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(flce, "_lib", None)
+    monkeypatch.setattr(flce, "_LIB_PATH", str(tmp_path / "nope.so"))
+    with pytest.raises(flce.FlceError):
+        flce.load_library()

@@ -1,0 +1,189 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small shapes are compared on every row; they span several 128-token blocks,
+several 256-column vocab tiles and slabs, and ragged N, V and D tails.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_cross_entropy_bf16_b200 import synth
+from tests.flce_testing import LOSS_TOL, compare, check_properties, run, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from linear_cross_entropy_bf16_b200 import build
+    build.build()
+    oracle.build()
+
+
+SHAPES = [
+    # N, V, D
+    (1, 1, 8), (7, 2, 16), (129, 127, 64), (255, 129, 72), (128, 255, 64), (200, 257, 128),
+    (300, 1000, 256), (129, 2047, 64), (513, 3000, 8), (64, 4097, 136), (1000, 600, 1024),
+    (257, 20000, 64),
+]
+
+
+@pytest.mark.parametrize("N,V,D", SHAPES)
+def test_bf16_shapes_every_row(N, V, D):
+    H, W, y = synth.random_inputs(N, V, D, seed=N * 7 + V + D)
+    gpu = run(H, W, y)
+    ref = oracle.forward(H, W, y)
+    compare(gpu, ref, mean_ref=oracle.mean(ref["loss"]))
+
+
+@pytest.mark.parametrize("N,V,D", [(1, 1, 1), (5, 3, 7), (130, 300, 33), (256, 2048, 256), (70, 5000, 100)])
+def test_fp32_shapes_every_row(N, V, D):
+    H, W, y = synth.random_inputs(N, V, D, seed=N + V + D, dtype="fp32")
+    gpu = run(H, W, y)
+    ref = oracle.forward(H, W, y)
+    compare(gpu, ref, mean_ref=oracle.mean(ref["loss"]))
+
+
+@pytest.mark.parametrize("where", ["first", "last", "last_ragged_tile", "one_column"])
+def test_target_positions(where):
+    N, V, D = 300, 1100, 64          # 5 tiles, the last holds 76 columns
+    H, W, y = synth.random_inputs(N, V, D, seed=3)
+    y = {"first": np.zeros(N), "last": np.full(N, V - 1),
+         "last_ragged_tile": np.random.default_rng(0).integers(1024, V, N),
+         "one_column": np.full(N, 517)}[where].astype(np.int64)
+    gpu = run(H, W, y)
+    ref = oracle.forward(H, W, y)
+    compare(gpu, ref, mean_ref=oracle.mean(ref["loss"]))
+
+
+def test_stress_scale_logits():
+    """Row scales log-uniform in [0.1, 10]/sqrt(D): logits up to ~+-50 stress the online max."""
+    H, W, y = synth.generate("stress_n16384_v262144_d2048", N=384, V=9000, D=256)
+    gpu = run(H, W, y)
+    ref = oracle.forward(H, W, y)
+    compare(gpu, ref, mean_ref=oracle.mean(ref["loss"]))
+
+
+def test_zero_weights_give_log_V():
+    N, V, D = 130, 3000, 64
+    H, _, y = synth.random_inputs(N, V, D, seed=5)
+    W = np.zeros((V, D), dtype=np.uint16)
+    gpu = run(H, W, y)
+    assert np.all(gpu["target"] == 0.0)
+    np.testing.assert_allclose(gpu["loss"], math.log(V), atol=1e-5)
+
+
+def test_dominant_target():
+    V, D = 700, 64
+    rng = np.random.default_rng(1)
+    W = synth.round_to_bf16_bits(np.sign(rng.standard_normal((V, D))).astype(np.float32))
+    y = rng.integers(0, V, 200)
+    H = synth.round_to_bf16_bits(0.5 * synth.bf16_bits_to_f32(W[y]))
+    gpu = run(H, W, y)
+    ref = oracle.forward(H, W, y)
+    compare(gpu, ref)
+    assert np.all(gpu["loss"] < 1e-3)
+
+
+def test_deterministic_bitwise():
+    import linear_cross_entropy_bf16_b200 as flce
+    H, W, y = synth.random_inputs(700, 40000, 256, seed=11)
+    Hd, Wd, yd = to_device(H, W, y)
+    a = [t.clone() for t in flce.forward(Hd, Wd, yd)]
+    b = flce.forward(Hd, Wd, yd)
+    for x, z in zip(a, b):
+        assert torch.equal(x, z)
+
+
+def test_partials_then_merge_equals_forward():
+    import linear_cross_entropy_bf16_b200 as flce
+    H, W, y = synth.random_inputs(333, 5000, 128, seed=12)
+    Hd, Wd, yd = to_device(H, W, y)
+    ref = flce.forward(Hd, Wd, yd)
+    N = 333
+    ws = torch.empty(flce.workspace_size(N, 5000, 128), dtype=torch.uint8, device="cuda")
+    loss, lse, tgt = (torch.empty(N, device="cuda") for _ in range(3))
+    mean = torch.empty((), device="cuda")
+    flce.partials(Hd, Wd, yd, tgt, ws)
+    flce.merge(yd, 5000, loss, lse, tgt, mean, ws)
+    assert flce.check(ws) == flce.OK
+    for x, z in zip(ref, (loss, lse, tgt, mean)):
+        assert torch.equal(x, z)
+
+
+def test_out_of_range_targets_flagged():
+    import linear_cross_entropy_bf16_b200 as flce
+    N, V, D = 200, 1000, 64
+    H, W, y = synth.random_inputs(N, V, D, seed=13)
+    y[[3, 150]] = [-1, V]
+    Hd, Wd, yd = to_device(H, W, y)
+    ws = torch.empty(flce.workspace_size(N, V, D), dtype=torch.uint8, device="cuda")
+    loss, lse, tgt, mean = flce.forward(Hd, Wd, yd, workspace=ws)
+    assert flce.check(ws) == flce.ERR_TARGET_OUT_OF_RANGE
+    loss = loss.cpu().numpy()
+    assert np.isnan(loss[3]) and np.isnan(loss[150]) and math.isnan(mean.item())
+    good = np.setdiff1d(np.arange(N), [3, 150])
+    yv = y.copy()
+    yv[[3, 150]] = 0
+    ref = oracle.forward(H, W, yv, rows=good)
+    assert np.abs(loss[good] - ref["loss"]).max() <= LOSS_TOL
+    # the status clears on the next good call with the same workspace
+    y2 = torch.from_numpy(yv).cuda()
+    flce.forward(Hd, Wd, y2, workspace=ws)
+    assert flce.check(ws) == flce.OK
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    import linear_cross_entropy_bf16_b200 as flce
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    assert flce.selftest_wait_timeout(ws, limit_ns=2_000_000) == flce.OK
+    assert flce.check(ws) == flce.ERR_TIMEOUT
+    H, W, y = synth.random_inputs(64, 500, 64, seed=14)
+    gpu = run(H, W, y)
+    compare(gpu, oracle.forward(H, W, y))
+
+
+def test_host_errors_raise():
+    import linear_cross_entropy_bf16_b200 as flce
+    H = torch.zeros(4, 60, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros(10, 60, dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros(4, dtype=torch.int64, device="cuda")
+    with pytest.raises(flce.FlceError) as e:
+        flce.forward(H, W, y)
+    assert e.value.status == flce.ERR_UNSUPPORTED
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(flce.FlceError):
+        flce.forward(H[:, :56].contiguous(), W[:, :56].contiguous(), y, workspace=ws)
+
+
+def test_empty_batch_is_a_noop():
+    import linear_cross_entropy_bf16_b200 as flce
+    H = torch.zeros(0, 64, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros(10, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros(0, dtype=torch.int64, device="cuda")
+    loss, lse, tgt, mean = flce.forward(H, W, y)
+    assert loss.numel() == 0 and math.isnan(mean.item())
+
+
+def test_no_N_by_V_allocation():
+    """With outputs and workspace supplied, the call allocates nothing on the device."""
+    import linear_cross_entropy_bf16_b200 as flce
+    N, V, D = 2048, 64000, 512
+    H, W, y = synth.random_inputs(N, V, D, seed=15)
+    Hd, Wd, yd = to_device(H, W, y)
+    ws = torch.empty(flce.workspace_size(N, V, D), dtype=torch.uint8, device="cuda")
+    out = {k: torch.empty(N, device="cuda") for k in ("loss", "lse", "target_logit")}
+    out["mean"] = torch.empty((), device="cuda")
+    flce.forward(Hd, Wd, yd, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    base = torch.cuda.memory_allocated()
+    flce.forward(Hd, Wd, yd, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.cuda.max_memory_allocated() == base
+    assert ws.numel() < 4 * N * V / 30
