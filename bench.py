@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Benchmark of the fused linear cross-entropy forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one full forward (contraction with online log-sum-exp, merge, mean)
+over one batch of synthetic input already resident in HBM.  Rank 0 prints one
+JSON line.  Under torchrun (N > 1) every rank runs its own batch of N tokens
+against the same W (data-parallel, no collective on the data path; scaling is
+weak) and the step time is the maximum over ranks.
+
+Also measured: the contraction kernel's own duration (CUDA events around
+flce_partials on the launching stream) for the roofline, an end-to-end leg
+through the public API from pinned host buffers, SM clocks during the timed
+region, and the CPU oracle on a bounded sample of the same workload.
+
+``--impl reference`` times the fp64 CPU oracle instead (the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import shutil
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_cross_entropy_bf16_b200 import synth  # noqa: E402
+
+METRIC = "LCE fwd tokens/s & % bf16 tensor peak at N=8192 V=151936 D=4096"
+# The page's fused forward at N=8192, V=151936, D=4096 took 2.105 s on an Apple
+# M1 Max under MLX/Metal (D. Ineshin, "Een gefuseerde forward-kernel voor
+# lineaire cross-entropy op Apple-GPU's", 2026, introduction): 8192 / 2.105 s.
+PAGES_TOKENS_PER_S = 8192 / 2.105
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+PROFILE = os.path.join(ROOT, "profiles", "flce_tc_kernel_n8192_v151936_d4096.md")
+KERNEL_SOURCES = ["linear_cross_entropy_bf16_b200/csrc/flce.cu",
+                  "linear_cross_entropy_bf16_b200/csrc/flce_kernels.cuh",
+                  "linear_cross_entropy_bf16_b200/csrc/ptx_sm100.cuh"]
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def kernel_sources_sha256() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current sources."""
+    if workload != synth.HEADLINE or not os.path.exists(PROFILE):
+        return None
+    text = open(PROFILE).read()
+    m_sha = re.search(r"kernel_sources_sha256:\s*([0-9a-f]{64})", text)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != kernel_sources_sha256():
+        return None
+    return float(m_tr.group(1))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv") \
+            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/flce_clocks_{os.getpid()}.csv"
+        self.gpu_index = gpu_index
+
+    def start(self):
+        if shutil.which("nvidia-smi") is None:
+            return
+        self.f = open(self.path, "w")
+        self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits", "-lms", "100"],
+                                     stdout=self.f, stderr=subprocess.DEVNULL)
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        sm = [r[0] for r in rows]
+        loaded = [r for r in rows if r[2] > 300] or rows     # samples drawing real power
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3][1:]) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[0] for r in loaded])), "sm_max_mhz": max(r[1] for r in rows),
+                "sm_mhz_min": min(sm), "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r[2] for r in rows), "reasons": reasons}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(H, W, y, seconds: float, seed: int, max_rows: int = 4096):
+    """Time the oracle on growing batches of seeded rows until `seconds` have passed."""
+    import oracle
+    oracle.build()
+    cores = oracle.max_threads()
+    order = np.random.default_rng([seed, 99]).permutation(H.shape[0])
+    done, t_total = 0, 0.0
+    while t_total < seconds and done < min(max_rows, H.shape[0]):
+        rows = order[done:done + cores]
+        t0 = time.perf_counter()
+        oracle.forward(H, W, y, rows=rows)
+        t_total += time.perf_counter() - t0
+        done += len(rows)
+    return done, t_total, cores
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, w, rank, world):
+    """The fp64 CPU oracle as the reference implementation (rank 0 only)."""
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    H, W, y = synth.generate(w)
+    cores = oracle.max_threads()
+    order = np.random.default_rng([w.seed, 98]).permutation(w.N)
+    per_step = cores
+    pos = 0
+
+    def step():
+        nonlocal pos
+        rows = order[pos % w.N: pos % w.N + per_step]
+        pos += per_step
+        oracle.forward(H, W, y, rows=rows)
+        return len(rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    rows = sum(step() for _ in range(args.steps))
+    dt = time.perf_counter() - t0
+    value = rows / dt
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": value / PAGES_TOKENS_PER_S, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": w.name, "N": w.N, "V": w.V, "D": w.D, "input_dtype": w.dtype,
+                   "targets": w.targets, "seed": w.seed, "global_batch": w.N, "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{per_step} seeded rows per step of the {w.name} workload "
+                                   f"({rows} rows over {args.steps} steps); fp64, logits materialised per row"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import linear_cross_entropy_bf16_b200 as flce
+    from linear_cross_entropy_bf16_b200 import build as lib_build
+
+    if rank == 0:
+        lib_build.build()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    flce.load_library()
+
+    # inputs: W is the shared projection; each rank has its own tokens and targets
+    t0 = time.perf_counter()
+    Hn, Wn, yn = synth.generate(w, token_stream=rank)
+    log(f"[rank {rank}] generated inputs in {time.perf_counter() - t0:.1f} s")
+
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def host_tensor(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return t.view(torch.bfloat16) if a.dtype == np.uint16 else t
+
+    H_h = host_tensor(Hn).pin_memory()
+    W_h = host_tensor(Wn).pin_memory()
+    y_h = torch.from_numpy(yn).pin_memory()
+    H = H_h.to(dev)
+    W = W_h.to(dev)
+    y = y_h.to(dev)
+    N, V, D = w.N, w.V, w.D
+    ws = torch.empty(flce.workspace_size(N, V, D, tdt), dtype=torch.uint8, device=dev)
+    loss = torch.empty(N, device=dev)
+    lse = torch.empty(N, device=dev)
+    tgt = torch.empty(N, device=dev)
+    mean = torch.empty((), device=dev)
+    out = {"loss": loss, "lse": lse, "target_logit": tgt, "mean": mean}
+    stream = torch.cuda.Stream(dev)
+
+    def step():
+        flce.forward(H, W, y, out=out, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    stream.synchronize()
+    st = flce.check(ws, stream)
+    if st != flce.OK:
+        raise flce.FlceError(st, "warm-up")
+
+    # ---- timed region: K steps, per-kernel events on the launching stream
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for k in range(K):
+            ev[k][0].record(stream)
+            flce.partials(H, W, y, tgt, ws, stream=stream)
+            ev[k][1].record(stream)
+            flce.merge(y, V, loss, lse, tgt, mean, ws, stream=stream)
+            ev[k][2].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
+    part_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
+    merge_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+    st = flce.check(ws, stream)
+    if st != flce.OK:
+        raise flce.FlceError(st, "timed region")
+    mean_loss = float(mean.item())
+
+    # ---- end to end through the public API from pinned host memory
+    H_d2 = torch.empty_like(H)
+    W_d2 = torch.empty_like(W)
+    y_d2 = torch.empty_like(y)
+    loss_h = torch.empty(N, pin_memory=True)
+    mean_h = torch.empty((), pin_memory=True)
+    out2 = {"loss": torch.empty(N, device=dev), "lse": torch.empty(N, device=dev),
+            "target_logit": torch.empty(N, device=dev), "mean": torch.empty((), device=dev)}
+
+    def e2e_step():
+        H_d2.copy_(H_h, non_blocking=True)
+        W_d2.copy_(W_h, non_blocking=True)
+        y_d2.copy_(y_h, non_blocking=True)
+        flce.forward(H_d2, W_d2, y_d2, out=out2, workspace=ws, stream=stream)
+        loss_h.copy_(out2["loss"], non_blocking=True)
+        mean_h.copy_(out2["mean"], non_blocking=True)
+
+    Ke = max(3, min(K, args.e2e_steps))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            e2e_step()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / Ke
+    assert abs(float(mean_h.item()) - mean_loss) <= 1e-6 * abs(mean_loss)
+    h2d = H_h.numel() * H_h.element_size() + W_h.numel() * W_h.element_size() + y_h.numel() * 8
+    d2h = N * 4 + 4
+
+    # ---- max over ranks
+    vals = torch.tensor([total_ms, float(np.mean(part_ms)), e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, part_avg_ms, e2e_ms = (float(v) for v in vals.tolist())
+
+    if rank != 0:
+        return 0
+
+    ms_step = total_ms / K
+    tokens_per_s = world * N / (ms_step / 1e3)
+    flops = w.flops
+    peaks, peak_kind = measured_peaks()
+    achieved = flops / (part_avg_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": tokens_per_s,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": tokens_per_s / PAGES_TOKENS_PER_S,
+        "vs_baseline_note": "divides by the page's fused forward on an Apple M1 Max (8192 tokens / 2.105 s): context, other hardware",
+        "dtype": "bf16" if w.dtype == "bf16" else "fp32",
+        "data": "synthetic (seeded numpy: H~N(0,1), W~N(0,1/D), targets per workload)",
+        "config": {"workload": w.name, "N": N, "V": V, "D": D, "input_dtype": w.dtype,
+                   "targets": w.targets, "seed": w.seed, "global_batch": world * N,
+                   "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs larger than L2 (W is {Wn.nbytes / 1e9:.2f} GB), no flush",
+                   "tflops_per_gpu": flops / (ms_step / 1e3) / 1e12,
+                   "frac_of_bf16_peak_per_gpu": flops / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"],
+                   "mean_loss": mean_loss},
+        "roofline": {"bound": "tensor", "kernel": "flce_tc_kernel" if w.dtype == "bf16" else "flce_simt_kernel",
+                     "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"],
+                     "peak_kind": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json bf16_tflops)",
+                     "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                     "kernel_ms": part_avg_ms, "merge_ms": float(np.mean(merge_ms)),
+                     "flops_per_launch": flops,
+                     "traffic": profiled_traffic(w.name)},
+        "e2e": {"value": world * N / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rows, secs, cores = oracle_sample(Hn, Wn, yn, args.cpu_seconds, w.seed)
+        line["cpu_baseline"] = {"value": rows / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": f"{rows} seeded rows of {w.name} (full V and D per row), {secs:.1f} s"}
+    if world == 1 and args.context:
+        line["context"] = torch_materialised(H, W, y, dev)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def torch_materialised(H, W, y, dev):
+    """The materialising forward (cuBLAS logits + logsumexp) timed the same way, for context."""
+    import torch
+    try:
+        def f():
+            Z = torch.matmul(H, W.t())                     # (N, V) bf16 logits
+            lse = torch.logsumexp(Z.float(), dim=1)
+            return lse - Z.gather(1, y[:, None]).float().squeeze(1)
+        for _ in range(2):
+            f()
+        torch.cuda.synchronize(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(5):
+            f()
+        e.record()
+        torch.cuda.synchronize(dev)
+        return {"torch_materialised_ms": s.elapsed_time(e) / 5,
+                "torch_materialised_extra_gib": (torch.cuda.max_memory_allocated(dev) - base) / 2 ** 30}
+    except RuntimeError as ex:  # out of memory on very large shapes
+        return {"torch_materialised_error": str(ex)[:200]}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=synth.HEADLINE, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--context", action="store_true", help="also time the materialising torch forward")
+    ap.add_argument("--shape", default=None,
+                    help="N,V,D: a custom shape with the chosen workload's distributions "
+                         "(used for small profiling captures; not a reported workload)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = synth.WORKLOADS[args.workload]
+    if args.shape:
+        n, v, d = (int(x) for x in args.shape.split(","))
+        w = synth.Workload(f"custom_n{n}_v{v}_d{d}", n, v, d, w.dtype, w.targets, w.w_scale, w.seed)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        log(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE")
+
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -131,19 +131,22 @@ def targets(N: int, V: int, seed: int, kind: str) -> np.ndarray:
 
 
 def generate(w: Workload | str, N: int | None = None, V: int | None = None,
-             D: int | None = None):
+             D: int | None = None, token_stream: int = 0):
     """Return (H, W, y) numpy arrays for workload ``w`` (optionally reshaped).
 
     H and W are uint16 bf16 bit patterns for bf16 workloads, float32 otherwise.
+    ``token_stream`` > 0 draws a different, equally distributed batch of tokens
+    and targets (one per data-parallel rank) against the same W.
     """
     if isinstance(w, str):
         w = WORKLOADS[w]
     N = w.N if N is None else N
     V = w.V if V is None else V
     D = w.D if D is None else D
-    H = _fill_rows(N, D, w.seed, _S_H, w.dtype, None)
+    tseed = w.seed if token_stream == 0 else w.seed * 1000003 + token_stream
+    H = _fill_rows(N, D, tseed, _S_H, w.dtype, None)
     W = _fill_rows(V, D, w.seed, _S_W, w.dtype, row_scales(V, D, w.seed, w.w_scale))
-    y = targets(N, V, w.seed, w.targets)
+    y = targets(N, V, tseed, w.targets)
     return H, W, y
 
 
