@@ -164,6 +164,43 @@ FLCE_API const char* flce_status_string(flce_status status);
 FLCE_API flce_status flce_selftest_wait_timeout(void* workspace, size_t workspace_bytes,
                                        uint64_t limit_ns, void* stream);
 
+/*
+ * flce_forward without a caller-supplied workspace, for callers that cannot
+ * allocate device memory when they need the loss: code that runs inside an
+ * allocator or memory-pool callback, runtimes that forbid cudaMalloc while
+ * they own the device memory budget, or hosts with no spare buffer to pass.
+ * The page has no counterpart to this entry point; it only changes where the
+ * workspace lives.
+ *
+ * The scratch is a fixed device array of FLCE_NOALLOC_SCRATCH_BYTES (64 MiB)
+ * inside the library's CUDA module.  Every GPU on which the library's kernels
+ * are loaded holds it until the process exits.  The call allocates nothing:
+ * no cudaMalloc, cudaFree or allocating library routine.
+ *   - Arguments, results and errors are those of flce_forward, except that
+ *     there is no workspace argument.
+ *   - A problem whose flce_workspace_size(N, V, D, dtype) exceeds
+ *     FLCE_NOALLOC_SCRATCH_BYTES is rejected with FLCE_ERR_WORKSPACE_TOO_SMALL
+ *     and nothing is enqueued.  With V >= 131072 (512 slab states per token)
+ *     that means N <= 16383.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current.  Make that first call
+ *     before any stream capture on that device.
+ *   - All calls on one device share the array, and it keeps the contents of
+ *     the last call.  Each call resets the header words it needs before its
+ *     kernels run.  Calls whose work overlaps on the GPU (different streams,
+ *     or threads without ordering) race on the array and give wrong results:
+ *     order them on one stream.
+ *   - The device status word lives in the shared array, so flce_check() does
+ *     not apply.  An out-of-range target still gives a NaN loss and target
+ *     logit for its row.
+ */
+#define FLCE_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+FLCE_API flce_status flce_forward_noalloc(const void* H, const void* W, const int64_t* y,
+                                          int64_t N, int64_t V, int64_t D, flce_dtype dtype,
+                                          float* out_loss, float* out_lse, float* out_target_logit,
+                                          float* out_mean, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

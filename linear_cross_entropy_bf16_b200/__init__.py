@@ -251,3 +251,32 @@ def selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int = 1_000_000, st
     return int(load_library().flce_selftest_wait_timeout(
         workspace.data_ptr(), workspace.numel() * workspace.element_size(), int(limit_ns),
         _stream_ptr(stream, workspace.device)))
+
+
+# Built-in scratch size of flce_forward_noalloc (FLCE_NOALLOC_SCRATCH_BYTES in include/flce.h).
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+
+def forward_noalloc(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, out: dict, stream=None):
+    """flce_forward_noalloc: the forward with the library's built-in scratch.
+
+    For callers that cannot allocate device memory at call time (allocator
+    callbacks, runtimes that own the device memory budget): no workspace is
+    passed, and the library allocates nothing.  ``out`` must supply all four
+    output tensors ("loss", "lse", "target_logit", "mean").  The scratch is
+    shared by every call on the device, so calls must be ordered on one stream.
+    Raises FlceError(ERR_WORKSPACE_TOO_SMALL) for problems beyond the scratch.
+    """
+    N, V, D, code = _check_inputs(H, W, y)
+    tensors = [out[k] for k in ("loss", "lse", "target_logit", "mean")]
+    for t in tensors:
+        if t.dtype != torch.float32 or t.device != H.device or not t.is_contiguous():
+            raise ValueError("outputs must be contiguous float32 tensors on the input device")
+    lib = load_library()
+    fn = lib.flce_forward_noalloc
+    fn.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 3 + [ctypes.c_int] + [ctypes.c_void_p] * 5
+    fn.restype = ctypes.c_int
+    st = fn(H.data_ptr(), W.data_ptr(), y.data_ptr(), N, V, D, code,
+            *(t.data_ptr() for t in tensors), _stream_ptr(stream, H.device))
+    _raise_on(st, "flce_forward_noalloc")
+    return tuple(tensors)

@@ -343,3 +343,62 @@ flce_status flce_selftest_wait_timeout(void* workspace, size_t workspace_bytes, 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation entry point
+//
+// Some callers cannot allocate device memory at the point where they need the
+// loss: code running inside an allocator or memory-pool callback, a runtime
+// that forbids cudaMalloc while it owns the device memory budget, or a host
+// that has no workspace to hand over.  flce_forward_noalloc serves them: its
+// scratch (the workspace of flce_forward) is one file-scope device array
+// that the CUDA module carries, so the call itself allocates nothing.
+
+namespace {
+
+// Every GPU on which this library's module is loaded holds this array until
+// the process exits.  In host code the name is only a stand-in: the device
+// address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FLCE_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on the
+// first call for that device, with that device current).
+flce_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FLCE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return FLCE_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FLCE_OK;
+}
+
+}  // namespace
+
+extern "C" flce_status flce_forward_noalloc(const void* H, const void* W, const int64_t* y,
+                                            int64_t N, int64_t V, int64_t D, flce_dtype dtype,
+                                            float* out_loss, float* out_lse,
+                                            float* out_target_logit, float* out_mean,
+                                            void* stream) {
+  if (!sizes_ok(N, V, D, dtype)) return FLCE_ERR_INVALID_ARG;
+  if (N == 0) return FLCE_OK;
+  // The problem must fit the built-in scratch; nothing larger is ever allocated.
+  if (workspace_bytes_for(N, V) > size_t(FLCE_NOALLOC_SCRATCH_BYTES))
+    return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  flce_status s = noalloc_scratch(&scratch);
+  if (s != FLCE_OK) return s;
+  // flce_forward checks the remaining arguments; it clears the scratch header
+  // (status word and merge counter) on the stream before its kernels run, and
+  // every other scratch byte it reads is written earlier in the same call.
+  return flce_forward(H, W, y, N, V, D, dtype, out_loss, out_lse, out_target_logit, out_mean,
+                      scratch, size_t(FLCE_NOALLOC_SCRATCH_BYTES), stream);
+}
