@@ -74,8 +74,11 @@ typedef struct {
   int32_t slab_rem;        /* vocab_tiles % slabs */
   int32_t grid;            /* CTAs launched for the contraction kernel */
   int64_t units;           /* token_blocks * slabs */
-  int64_t makespan_tiles;  /* tiles processed by the busiest CTA */
+  int64_t makespan_tiles;  /* tiles processed by the busiest CTA (or CTA pair) */
   size_t workspace_bytes;  /* == flce_workspace_size(N, V, D, dtype) */
+  int32_t ctas_per_unit;   /* 2: a CTA pair shares each 256-token tile (bf16, N > 128);
+                              1: one CTA per tile */
+  int32_t reserved;
 } flce_plan_t;
 
 /* Bytes of device workspace that flce_forward / flce_partials need for this
@@ -86,7 +89,9 @@ typedef struct {
  * dtype).  Host only; never touches the GPU. */
 FLCE_API size_t flce_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype dtype);
 
-/* The schedule for a device with `sm_count` SMs (host only, no GPU call).
+/* The schedule for a device with `sm_count` SMs, assuming every SM pair can
+ * hold a CTA pair (host only, no GPU call; at launch the library sizes the
+ * grid from the device's actual cluster occupancy).
  * Returns FLCE_ERR_INVALID_ARG for invalid sizes, sm_count < 1 or plan NULL. */
 FLCE_API flce_status flce_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int32_t sm_count,
                       flce_plan_t* plan);

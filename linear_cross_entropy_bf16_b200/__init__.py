@@ -61,7 +61,8 @@ class Plan(ctypes.Structure):
         ("slabs", ctypes.c_int32), ("slab_base", ctypes.c_int32),
         ("slab_rem", ctypes.c_int32), ("grid", ctypes.c_int32),
         ("units", ctypes.c_int64), ("makespan_tiles", ctypes.c_int64),
-        ("workspace_bytes", ctypes.c_size_t),
+        ("workspace_bytes", ctypes.c_size_t), ("ctas_per_unit", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
     ]
 
     def as_dict(self):

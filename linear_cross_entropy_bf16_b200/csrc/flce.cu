@@ -69,7 +69,12 @@ void choose_slabs(int64_t tb, int64_t nt, int64_t g, int64_t pcap, int32_t& P_ou
   makespan_out = best_ms;
 }
 
-flce_status make_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int32_t sms,
+// The bf16 path runs on CTA pairs (256-token tiles) unless the batch fits one
+// 128-token tile, where half of every pair tile would be padding.
+bool use_pair_kernel(int64_t N, flce_dtype dtype) { return dtype == FLCE_BF16 && N > tc::BM; }
+
+// `workers`: CTAs (single-CTA kernels) or CTA pairs (pair kernel) that run at once.
+flce_status make_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int64_t workers,
                       flce_plan_t* p) {
   std::memset(p, 0, sizeof(*p));
   p->N = N;
@@ -78,20 +83,27 @@ flce_status make_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int32_t
   p->dtype = int32_t(dtype);
   p->tile_cols = kTileCols;
   const bool tc = dtype == FLCE_BF16;
-  p->block_rows = tc ? tc::BM : simt::BM;
+  const bool pair = use_pair_kernel(N, dtype);
+  p->ctas_per_unit = pair ? 2 : 1;
+  p->block_rows = pair ? tc2::PAIR_M : (tc ? tc::BM : simt::BM);
   p->k_block = tc ? tc::BK : simt::BK;
   p->token_blocks = cdiv(std::max<int64_t>(N, 1), p->block_rows);
   p->vocab_tiles = cdiv(V, kTileCols);
-  const int64_t g = tc ? int64_t(sms) : int64_t(sms) * kSimtBlocksPerSm;
+  const int64_t g = std::max<int64_t>(1, workers);
   int64_t ms = 0;
   choose_slabs(p->token_blocks, p->vocab_tiles, g, slab_capacity(V), p->slabs, ms);
   p->slab_base = int32_t(p->vocab_tiles / p->slabs);
   p->slab_rem = int32_t(p->vocab_tiles % p->slabs);
   p->units = p->token_blocks * p->slabs;
-  p->grid = int32_t(tc ? std::min<int64_t>(sms, p->units) : p->units);
+  p->grid = int32_t(tc ? std::min<int64_t>(g, p->units) * p->ctas_per_unit : p->units);
   p->makespan_tiles = ms;
   p->workspace_bytes = workspace_bytes_for(N, V);
   return FLCE_OK;
+}
+
+int64_t nominal_workers(int32_t sms, int64_t N, flce_dtype dtype) {
+  if (dtype != FLCE_BF16) return int64_t(sms) * kSimtBlocksPerSm;
+  return use_pair_kernel(N, dtype) ? std::max<int64_t>(1, sms / 2) : int64_t(sms);
 }
 
 // ---------------------------------------------------------------- driver entry point
@@ -148,8 +160,32 @@ flce_status set_smem_attr_once() {
   std::call_once(once, [] {
     err = cudaFuncSetAttribute(tc::flce_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                tc::SMEM_BYTES);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(tc2::flce_tc2_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, tc2::SMEM_BYTES);
   });
   return err == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+// CTA pairs of the pair kernel that can be resident at once on the current
+// device (queried once per device; SM count / 2 if the query is unavailable).
+int64_t resident_pairs(int dev, int sms) {
+  static std::mutex mu;
+  static int cached[64] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(sms & ~1), 1, 1);
+  cfg.blockDim = dim3(tc2::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = tc2::SMEM_BYTES;
+  if (cudaOccupancyMaxActiveClusters(&n, tc2::flce_tc2_kernel, &cfg) != cudaSuccess || n < 1) {
+    (void)cudaGetLastError();
+    n = sms / 2;
+  }
+  n = std::min(n, sms / 2);
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -177,8 +213,15 @@ flce_status launch_partials(const void* H, const void* W, const int64_t* y, int6
   DeviceInfo di;
   flce_status s = device_info(di);
   if (s != FLCE_OK) return s;
+  if (dtype == FLCE_BF16 && (s = set_smem_attr_once()) != FLCE_OK) return s;
+  int64_t workers = nominal_workers(di.sms, N, dtype);
+  if (use_pair_kernel(N, dtype)) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+    workers = resident_pairs(dev, di.sms);
+  }
   flce_plan_t plan;
-  make_plan(N, V, D, dtype, di.sms, &plan);
+  make_plan(N, V, D, dtype, workers, &plan);
 
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
@@ -194,9 +237,10 @@ flce_status launch_partials(const void* H, const void* W, const int64_t* y, int6
 
   if (dtype == FLCE_BF16) {
     if (!load_encoder()) return FLCE_ERR_CUDA;
-    if ((s = set_smem_attr_once()) != FLCE_OK) return s;
+    const bool pair = plan.ctas_per_unit == 2;
     CUtensorMap tmH, tmW;
-    if (!encode_bf16_rows(&tmH, H, N, D, tc::BM) || !encode_bf16_rows(&tmW, W, V, D, tc::BN))
+    if (!encode_bf16_rows(&tmH, H, N, D, tc::BM) ||
+        !encode_bf16_rows(&tmW, W, V, D, pair ? tc2::HALF_N : tc::BN))
       return FLCE_ERR_UNSUPPORTED;
     tc::Args a;
     a.y = y;
@@ -209,7 +253,10 @@ flce_status launch_partials(const void* H, const void* W, const int64_t* y, int6
     a.kblocks = int32_t(cdiv(D, tc::BK));
     a.sch = sch;
     a.wait_limit_ns = kDefaultWaitLimitNs;
-    tc::flce_tc_kernel<<<plan.grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(tmH, tmW, a);
+    if (pair)
+      tc2::flce_tc2_kernel<<<plan.grid, tc2::NUM_THREADS, tc2::SMEM_BYTES, st>>>(tmH, tmW, a);
+    else
+      tc::flce_tc_kernel<<<plan.grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(tmH, tmW, a);
   } else {
     simt::Args a;
     a.H = H;
@@ -262,7 +309,7 @@ size_t flce_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
 flce_status flce_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int32_t sm_count,
                       flce_plan_t* plan) {
   if (!plan || sm_count < 1 || !sizes_ok(N, V, D, dtype)) return FLCE_ERR_INVALID_ARG;
-  return make_plan(N, V, D, dtype, sm_count, plan);
+  return make_plan(N, V, D, dtype, nominal_workers(sm_count, N, dtype), plan);
 }
 
 flce_status flce_partials(const void* H, const void* W, const int64_t* y, int64_t N, int64_t V,

@@ -122,6 +122,58 @@ __device__ __forceinline__ float pick32(const float (&z)[32], int idx) {
   return (idx & 1) ? a[1] : a[0];
 }
 
+// ----------------------------------------------------------------- epilogue
+
+// Fold one finished accumulator tile into this thread's running state.  The
+// thread owns one TMEM lane (one token); `taddr` addresses that lane at
+// column 0 of the tile, `ncols` columns exist (the rest of the tile lies past
+// V), and `rel` is the target's column inside the tile (any value outside
+// [0, ncols) means the target is elsewhere).  Per 32-column chunk:
+//   m_t = max_j z_j,  m' = max(m, m_t),
+//   s'  = s * exp(m - m') + sum_j exp(z_j - m')     (the page, section 1)
+// with exp(x) evaluated as 2^(x log2 e).  Must be called by all 32 lanes.
+__device__ __forceinline__ void fold_tile(uint32_t taddr, int ncols, int64_t rel, float& m, float& s,
+                                          float& zt, bool& got) {
+#pragma unroll 1
+  for (int c = 0; c < kTileCols / 32; ++c) {
+    if (c * 32 >= ncols) break;  // warp-uniform: the rest of the tile is past V
+    uint32_t u32[32];
+    ptx::tmem_ld32_wait(taddr + uint32_t(c * 32), u32);
+    float z[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) z[j] = __uint_as_float(u32[j]);
+    if (ncols - c * 32 < 32) {  // ragged last tile: columns >= V do not exist
+      const int lim = ncols - c * 32;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j >= lim) z[j] = -INFINITY;
+    }
+    // target capture: the tile holding y_i records z_{i, y_i}
+    const int64_t rc = rel - c * 32;
+    if (rc >= 0 && rc < 32) {
+      zt = pick32(z, int(rc));
+      got = true;
+    }
+    // m_t = max_j z_j over this chunk, tree-reduced
+    float mx[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) mx[j] = fmaxf(z[j], z[j + 16]);
+#pragma unroll
+    for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+      for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
+    const float m_new = fmaxf(m, mx[0]);
+    const float ms = m_new * kLog2e;
+    // sum_j exp(z_j - m') as 2^(z_j log2 e - m' log2 e)
+    float e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) e[j & 3] += ptx::ex2(fmaf(z[j], kLog2e, -ms));
+    // s' = s exp(m - m') + sum; m = -inf on the first chunk gives exp(-inf) = 0
+    s = fmaf(s, ptx::ex2((m - m_new) * kLog2e), (e[0] + e[1]) + (e[2] + e[3]));
+    m = m_new;
+  }
+}
+
 // ----------------------------------------------------------------- tcgen05 kernel
 
 namespace tc {
@@ -331,47 +383,8 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
         }
         ptx::tc_fence_after_sync();
         const int v0 = t * BN;
-        const int ncols = min(BN, a.V - v0);
-        const int64_t rel = yi - v0;  // target column inside this tile, if in [0, BN)
-        const uint32_t taddr = tmem_base + lane_addr + uint32_t(acc * BN);
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          if (c * 32 >= ncols) break;  // warp-uniform: the rest of the tile is past V
-          uint32_t u32[32];
-          ptx::tmem_ld32_wait(taddr + uint32_t(c * 32), u32);
-          float z[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) z[j] = __uint_as_float(u32[j]);
-          if (ncols - c * 32 < 32) {  // ragged last tile: columns >= V do not exist
-            const int lim = ncols - c * 32;
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j >= lim) z[j] = -INFINITY;
-          }
-          // target capture: the tile holding y_i records z_{i, y_i}
-          const int64_t rc = rel - c * 32;
-          if (rc >= 0 && rc < 32) {
-            zt = pick32(z, int(rc));
-            got = true;
-          }
-          // m_t = max_j z_j over this chunk, tree-reduced
-          float mx[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) mx[j] = fmaxf(z[j], z[j + 16]);
-#pragma unroll
-          for (int w2 = 8; w2 >= 1; w2 >>= 1)
-#pragma unroll
-            for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
-          const float m_new = fmaxf(m, mx[0]);
-          const float ms = m_new * kLog2e;
-          // sum_j exp(z_j - m') as 2^(z_j log2 e - m' log2 e)
-          float e[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int j = 0; j < 32; ++j) e[j & 3] += ptx::ex2(fmaf(z[j], kLog2e, -ms));
-          // s' = s exp(m - m') + sum; m = -inf on the first chunk gives exp(-inf) = 0
-          s = fmaf(s, ptx::ex2((m - m_new) * kLog2e), (e[0] + e[1]) + (e[2] + e[3]));
-          m = m_new;
-        }
+        fold_tile(tmem_base + lane_addr + uint32_t(acc * BN), min(BN, a.V - v0), yi - v0, m, s,
+                  zt, got);
         ptx::tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&tempty_bar[acc]));
@@ -399,6 +412,245 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
 }
 
 }  // namespace tc
+
+// ----------------------------------------------------------------- tcgen05 pair kernel
+
+// The same contraction with 256 x 256 tiles computed by a CTA pair
+// (cta_group::2).  Each CTA stages its own 128 token rows of H and its own
+// 128 vocab rows of W per K block (no multicast); the even CTA issues
+// 256x256x16 MMAs that read both CTAs' shared memory and write 128 rows x 256
+// columns into each CTA's TMEM.  Per unit of work a pair reads 2 MB of H and
+// 2 MB of W (D = 4096) where two single-CTA 128x256 tiles read 6 MB, and the
+// smaller per-CTA stage (32 KB) affords a 6-deep ring.
+namespace tc2 {
+
+constexpr int BM = 128;                      // token rows per CTA
+constexpr int PAIR_M = 2 * BM;               // token rows per pair tile (UMMA M)
+constexpr int BN = kTileCols;                // vocab columns per tile (UMMA N)
+constexpr int HALF_N = BN / 2;               // W rows staged by each CTA
+constexpr int BK = 64;
+constexpr int UMMA_K = 16;
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BK * 2;         // 16 KiB
+constexpr int B_BYTES = HALF_N * BK * 2;     // 16 KiB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t PAIR_TX_BYTES = 2 * STAGE_BYTES;  // both CTAs' copies complete on the even CTA
+constexpr int NUM_THREADS = 192;             // warp 0 TMA, warp 1 MMA (even CTA), warps 2..5 epilogue
+constexpr int EPI_WARPS = 4;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr uint16_t kPairMask = 0x3;
+
+// kind::f16 descriptor as in the single-CTA kernel, with M = 256 (bits 24-28).
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
+                            (uint32_t(PAIR_M >> 4) << 24);
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW,
+                const tc::Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full_bar = bars;                     // [STAGES] (even CTA) both CTAs' copies landed
+  uint64_t* empty_bar = bars + STAGES;           // [STAGES] MMAs done reading the slot
+  uint64_t* tfull_bar = bars + 2 * STAGES;       // [2] accumulator ready
+  uint64_t* tempty_bar = bars + 2 * STAGES + 2;  // [2] (even CTA) drained by both CTAs
+  uint64_t* done_bar = bars + 2 * STAGES + 4;    // (even CTA) all MMAs retired
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();    // 0 = even CTA (issues the MMAs)
+  const int pair = int(ptx::cluster_id_x());
+  const int npairs = int(ptx::cluster_count_x());
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(ptx::smem_addr(&full_bar[s]), 1);
+      ptx::mbar_init(ptx::smem_addr(&empty_bar[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(ptx::smem_addr(&tfull_bar[b]), 1);
+      ptx::mbar_init(ptx::smem_addr(&tempty_bar[b]), 2 * EPI_WARPS);
+    }
+    ptx::mbar_init(ptx::smem_addr(done_bar), 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+    ptx::fence_proxy_async_smem();
+    ptx::prefetch_tensormap(&tmH);
+    ptx::prefetch_tensormap(&tmW);
+    if (blockIdx.x == 0) {
+      a.hdr->slabs = a.sch.slabs;
+      a.hdr->N = a.N;
+      a.hdr->V = a.V;
+      a.hdr->magic = kWsMagic;
+    }
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(ptx::smem_addr(tmem_slot), TMEM_COLS);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before_sync();
+  ptx::cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
+  ptx::tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  uint32_t* status = &a.hdr->status;
+  const uint64_t lim = a.wait_limit_ns;
+  const Schedule& sch = a.sch;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      const uint64_t pol_h = ptx::policy_evict_last();
+      const uint64_t pol_w = ptx::policy_evict_normal();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t used = 0, last_parity = 0;
+      bool ok = true;
+      for (int u = pair; ok && u < sch.units; u += npairs) {
+        int slab, tb, t0, nt;
+        unit_coords(sch, u, slab, tb, t0, nt);
+        const int hrow = tb * PAIR_M + int(rank) * BM;
+        for (int t = t0; ok && t < t0 + nt; ++t) {
+          const int wrow = t * BN + int(rank) * HALF_N;
+          for (int kb = 0; kb < a.kblocks; ++kb) {
+            if (!wait_bounded(ptx::smem_addr(&empty_bar[stage]), phase ^ 1u, abort_flag, status,
+                              lim)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb_local = ptx::smem_addr(&full_bar[stage]);
+            const uint32_t fb_even = ptx::map_to_cta(fb_local, 0);
+            const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
+            if (rank == 0) ptx::mbar_arrive_expect_tx(fb_local, PAIR_TX_BYTES);
+            ptx::tma_load_2d_pair(sa, &tmH, fb_even, kb * BK, hrow, pol_h);
+            ptx::tma_load_2d_pair(sa + A_BYTES, &tmW, fb_even, kb * BK, wrow, pol_w);
+            used |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+      // The even CTA's full barriers count both CTAs' bytes: once its last
+      // phase on each slot has completed, no copy of this pair is in flight.
+      if (rank == 0)
+        for (int s = 0; s < STAGES; ++s)
+          if (used & (1u << s))
+            wait_bounded(ptx::smem_addr(&full_bar[s]), (last_parity >> s) & 1u, nullptr, status,
+                         lim);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = pair; ok && u < sch.units; u += npairs) {
+        int slab, tb, t0, nt;
+        unit_coords(sch, u, slab, tb, t0, nt);
+        for (int t = 0; ok && t < nt; ++t) {
+          if (!wait_bounded(ptx::smem_addr(&tempty_bar[acc]), acc_phase ^ 1u, abort_flag, status,
+                            lim)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after_sync();
+          const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+          for (int kb = 0; kb < a.kblocks; ++kb) {
+            if (!wait_bounded(ptx::smem_addr(&full_bar[stage]), phase, abort_flag, status, lim)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after_sync();
+            const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              const uint64_t ad = tc::sw128_desc(sa + k * UMMA_K * 2);
+              const uint64_t bd = tc::sw128_desc(sa + A_BYTES + k * UMMA_K * 2);
+              ptx::mma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+            }
+            ptx::mma_commit_pair_mc(ptx::smem_addr(&empty_bar[stage]), kPairMask);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          ptx::mma_commit_pair_mc(ptx::smem_addr(&tfull_bar[acc]), kPairMask);
+          if (++acc == 2) {
+            acc = 0;
+            acc_phase ^= 1u;
+          }
+        }
+      }
+      ptx::mma_commit_pair(ptx::smem_addr(done_bar));
+      wait_bounded(ptx::smem_addr(done_bar), 0, nullptr, status, lim);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quad = warp & 3;
+    const int row_in_tile = quad * 32 + lane;
+    const uint32_t lane_addr = uint32_t(quad * 32) << 16;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int u = pair; ok && u < sch.units; u += npairs) {
+      int slab, tb, t0, nt;
+      unit_coords(sch, u, slab, tb, t0, nt);
+      const int row = tb * PAIR_M + int(rank) * BM + row_in_tile;
+      const bool valid = row < a.N;
+      const int64_t yi = valid ? a.y[row] : -1;
+      float m = -INFINITY, s = 0.f, zt = 0.f;
+      bool got = false;
+      for (int t = t0; t < t0 + nt; ++t) {
+        bool w = wait_bounded(ptx::smem_addr(&tfull_bar[acc]), acc_phase, abort_flag, status, lim);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after_sync();
+        const int v0 = t * BN;
+        fold_tile(tmem_base + lane_addr + uint32_t(acc * BN), min(BN, a.V - v0), yi - v0, m, s,
+                  zt, got);
+        ptx::tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0)
+          ptx::mbar_arrive_cluster(ptx::map_to_cta(ptx::smem_addr(&tempty_bar[acc]), 0));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (valid) {
+        a.part[size_t(slab) * size_t(a.N) + size_t(row)] = make_float2(m, s);
+        if (got) a.target_logit[row] = zt;
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  __syncwarp();
+  ptx::tc_fence_before_sync();
+  __syncthreads();
+  // Neither CTA leaves while the other may still read its shared memory or
+  // signal its barriers; the even CTA's MMAs have retired (done_bar).
+  ptx::cluster_sync();
+  if (warp == 1) {
+    ptx::tc_fence_after_sync();
+    ptx::tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace tc2
 
 // ----------------------------------------------------------------- fp32 FFMA kernel
 

@@ -64,12 +64,13 @@ def test_workspace_is_O_N_not_O_NV(lib):
 
 
 def simulate_makespan(p):
-    tb, P, base, rem, grid = p["token_blocks"], p["slabs"], p["slab_base"], p["slab_rem"], p["grid"]
+    tb, P, base, rem = p["token_blocks"], p["slabs"], p["slab_base"], p["slab_rem"]
+    workers = p["grid"] // p["ctas_per_unit"]          # CTAs, or CTA pairs
     units = tb * P
-    load = [0] * grid
+    load = [0] * workers
     for u in range(units):
         slab = u // tb
-        load[u % grid] += base + (1 if slab < rem else 0)
+        load[u % workers] += base + (1 if slab < rem else 0)
     return max(load)
 
 
@@ -88,19 +89,24 @@ def test_plan_covers_every_tile_once_and_balances(lib, N, V, D, dtype, sms):
     assert p["units"] == p["token_blocks"] * p["slabs"]
     assert p["workspace_bytes"] == flce.workspace_size(N, V, D, dtype)
     if dtype == 0:
-        assert p["grid"] == min(sms, p["units"])
+        pair = N > 128
+        assert p["ctas_per_unit"] == (2 if pair else 1)
+        assert p["block_rows"] == (256 if pair else 128)
+        workers = sms // 2 if pair else sms
+        assert p["grid"] == min(workers, p["units"]) * p["ctas_per_unit"]
         assert simulate_makespan(p) == p["makespan_tiles"]
         total = p["token_blocks"] * p["vocab_tiles"]
-        # within one tile per CTA of the perfect split, whenever every CTA has work
-        if total >= sms:
-            assert p["makespan_tiles"] <= math.ceil(total / sms) + 1
+        # within one tile per worker of the perfect split, whenever every worker has work
+        if total >= workers:
+            assert p["makespan_tiles"] <= math.ceil(total / workers) + 1
 
 
 def test_headline_plan(lib):
     p = flce.plan(8192, 151936, 4096, 0, sm_count=148)
-    assert p["block_rows"] == 128 and p["tile_cols"] == 256 and p["k_block"] == 64
-    assert p["token_blocks"] == 64 and p["vocab_tiles"] == 594
-    assert p["makespan_tiles"] == 257          # ceil(64 * 594 / 148)
+    assert p["ctas_per_unit"] == 2 and p["grid"] == 148
+    assert p["block_rows"] == 256 and p["tile_cols"] == 256 and p["k_block"] == 64
+    assert p["token_blocks"] == 32 and p["vocab_tiles"] == 594
+    assert p["makespan_tiles"] == 257          # ceil(32 * 594 / 74) pair tiles
 
 
 def test_plan_rejects_bad_args(lib):
