@@ -42,7 +42,7 @@ METRIC = "LCE fwd tokens/s & % bf16 tensor peak at N=8192 V=151936 D=4096"
 # lineaire cross-entropy op Apple-GPU's", 2026, introduction): 8192 / 2.105 s.
 PAGES_TOKENS_PER_S = 8192 / 2.105
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
-PROFILE = os.path.join(ROOT, "profiles", "flce_tc_kernel_n8192_v151936_d4096.md")
+PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = ["linear_cross_entropy_bf16_b200/csrc/flce.cu",
                   "linear_cross_entropy_bf16_b200/csrc/flce_kernels.cuh",
                   "linear_cross_entropy_bf16_b200/csrc/ptx_sm100.cuh"]
@@ -60,11 +60,12 @@ def kernel_sources_sha256() -> str:
     return h.hexdigest()
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, kernel: str):
     """DRAM bytes per launch from the committed ncu summary, if it matches the current sources."""
-    if workload != synth.HEADLINE or not os.path.exists(PROFILE):
+    path = os.path.join(PROFILE_DIR, f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
         return None
-    text = open(PROFILE).read()
+    text = open(path).read()
     m_sha = re.search(r"kernel_sources_sha256:\s*([0-9a-f]{64})", text)
     m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     if not m_sha or not m_tr or m_sha.group(1) != kernel_sources_sha256():
@@ -131,6 +132,28 @@ class ClockSampler:
         return {"sm_mhz": float(np.median([r[0] for r in loaded])), "sm_max_mhz": max(r[1] for r in rows),
                 "sm_mhz_min": min(sm), "samples": len(rows), "samples_under_load": len(loaded),
                 "power_w_max": max(r[2] for r in rows), "reasons": reasons}
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def rank_inputs(w, rank: int):
+    """Inputs of one data-parallel rank: its own tokens and targets, the shared W."""
+    return synth.generate(w, token_stream=rank)
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise maximum of a list of floats over all ranks (identity when world == 1)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def weak_scaling_tokens_per_s(world: int, n_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes n_per_rank tokens per step."""
+    return world * n_per_rank / (ms_per_step / 1e3)
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -214,7 +237,7 @@ def run_ours(args, w, rank, world, local_rank):
 
     # inputs: W is the shared projection; each rank has its own tokens and targets
     t0 = time.perf_counter()
-    Hn, Wn, yn = synth.generate(w, token_stream=rank)
+    Hn, Wn, yn = rank_inputs(w, rank)
     log(f"[rank {rank}] generated inputs in {time.perf_counter() - t0:.1f} s")
 
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
@@ -312,19 +335,22 @@ def run_ours(args, w, rank, world, local_rank):
     d2h = N * 4 + 4
 
     # ---- max over ranks
-    vals = torch.tensor([total_ms, float(np.mean(part_ms)), e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, part_avg_ms, e2e_ms = (float(v) for v in vals.tolist())
+    total_ms, part_avg_ms, e2e_ms = max_over_ranks([total_ms, float(np.mean(part_ms)), e2e_ms],
+                                                   world, device=dev)
 
     if rank != 0:
         return 0
 
     ms_step = total_ms / K
-    tokens_per_s = world * N / (ms_step / 1e3)
+    tokens_per_s = weak_scaling_tokens_per_s(world, N, ms_step)
     flops = w.flops
     peaks, peak_kind = measured_peaks()
     achieved = flops / (part_avg_ms * 1e-3) / 1e12
+    p = flce.plan(N, V, D, tdt)
+    if w.dtype != "bf16":
+        kernel = "flce_simt_kernel"
+    else:
+        kernel = "flce_tc2_kernel" if p["ctas_per_unit"] == 2 else "flce_tc_kernel"
     line = {
         "metric": METRIC,
         "value": tokens_per_s,
@@ -346,15 +372,15 @@ def run_ours(args, w, rank, world, local_rank):
                    "tflops_per_gpu": flops / (ms_step / 1e3) / 1e12,
                    "frac_of_bf16_peak_per_gpu": flops / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"],
                    "mean_loss": mean_loss},
-        "roofline": {"bound": "tensor", "kernel": "flce_tc_kernel" if w.dtype == "bf16" else "flce_simt_kernel",
+        "roofline": {"bound": "tensor", "kernel": kernel,
                      "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops"],
                      "peak_kind": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json bf16_tflops)",
                      "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                      "kernel_ms": part_avg_ms, "merge_ms": float(np.mean(merge_ms)),
                      "flops_per_launch": flops,
-                     "traffic": profiled_traffic(w.name)},
-        "e2e": {"value": world * N / (e2e_ms / 1e3), "unit": "tokens/s",
+                     "traffic": profiled_traffic(w.name, kernel)},
+        "e2e": {"value": weak_scaling_tokens_per_s(world, N, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
         "gpu_launches": 2 * K,
         "clocks": clocks,

@@ -1,0 +1,86 @@
+"""The multi-rank (N > 1) benchmark path on CPU: two gloo ranks.
+
+Each rank runs its own batch of tokens against the same W (data-parallel,
+weak scaling, no collective on the data path); timings are combined as the
+maximum over ranks.  Nothing here touches a GPU.
+"""
+import hashlib
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        from linear_cross_entropy_bf16_b200 import synth
+        w = synth.Workload("t", 300, 1000, 64, "bf16", "uniform", "inv_sqrt_d", 9)
+        H, W, y = bench.rank_inputs(w, rank)
+        digests = [hashlib.sha256(a.tobytes()).hexdigest() for a in (H, W, y)]
+        gathered = [None] * world
+        dist.all_gather_object(gathered, digests)
+        mx = bench.max_over_ranks([rank + 1.0, 10.0 * (world - rank), -1.0], world)
+        dist.barrier()
+        q.put((rank, gathered, mx))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_share_W_and_reduce_max():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=240) for _ in procs]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    for rank, gathered, mx in out:
+        (h0, w0, y0), (h1, w1, y1) = gathered
+        assert w0 == w1                 # the projection is replicated
+        assert h0 != h1 and y0 != y1    # each rank has its own tokens and targets
+        assert mx == [2.0, 20.0, -1.0]  # element-wise max over ranks
+
+
+def test_weak_scaling_value_counts_all_ranks():
+    import bench
+    assert bench.weak_scaling_tokens_per_s(1, 8192, 8.0) == pytest.approx(1.024e6)
+    assert bench.weak_scaling_tokens_per_s(8, 8192, 8.0) == pytest.approx(8.192e6)
+    assert bench.max_over_ranks([1.5, 2.5], 1) == [1.5, 2.5]
+
+
+def test_reference_arm_under_torchrun_prints_one_line():
+    """`--impl reference` under torchrun: rank 0 prints one JSON line, the other rank exits 0."""
+    env = dict(os.environ, OMP_NUM_THREADS="2")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr=127.0.0.1", f"--master-port={free_port()}", "bench.py", "--gpus", "2",
+           "--impl", "reference", "--workload", "tiny_n256_v2048_d256_fp32", "--steps", "2",
+           "--warmup", "3"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    import json
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["e2e"]["h2d_bytes_per_step"] == 0
