@@ -78,7 +78,8 @@ typedef struct {
   size_t workspace_bytes;  /* == flce_workspace_size(N, V, D, dtype) */
   int32_t ctas_per_unit;   /* 2: a CTA pair shares each 256-token tile (bf16, N > 128);
                               1: one CTA per tile */
-  int32_t reserved;
+  int32_t group_blocks;    /* token blocks per raster group: units are ordered group by
+                              group, slab-major inside a group, and handed out round-robin */
 } flce_plan_t;
 
 /* Bytes of device workspace that flce_forward / flce_partials need for this

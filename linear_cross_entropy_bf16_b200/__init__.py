@@ -62,7 +62,7 @@ class Plan(ctypes.Structure):
         ("slab_rem", ctypes.c_int32), ("grid", ctypes.c_int32),
         ("units", ctypes.c_int64), ("makespan_tiles", ctypes.c_int64),
         ("workspace_bytes", ctypes.c_size_t), ("ctas_per_unit", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("group_blocks", ctypes.c_int32),
     ]
 
     def as_dict(self):

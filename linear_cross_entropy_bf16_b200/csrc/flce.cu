@@ -14,6 +14,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "flce.h"
 #include "flce_kernels.cuh"
@@ -42,23 +43,54 @@ size_t workspace_bytes_for(int64_t N, int64_t V) {
   return kHeaderBytes + part + sums;
 }
 
-// Choose P (slabs per token block) for `tb` token blocks, `nt` vocab tiles and
-// `g` concurrent CTAs.  Units are handed out round-robin (CTA c takes units
-// c, c+g, ...), slab-major, so the CTAs running at the same time share the
-// same W tiles.  CTA 0 is then the busiest: it takes ceil(U/g) units, of
-// which ceil(R/g) are the longer ones (R = rem * tb units in the first `rem`
-// slabs).  Minimise that makespan in tiles plus a small per-unit cost.
-void choose_slabs(int64_t tb, int64_t nt, int64_t g, int64_t pcap, int32_t& P_out,
+// Makespan, in tiles, of the busiest worker when the units of a schedule are
+// handed out round-robin (worker c takes units c, c + g, c + 2g, ...) in the
+// grouped order of unit_coords.  Unit sizes are base + 1 tiles for slabs
+// < rem and base otherwise.  In group k the long units form one contiguous
+// run of rem * gt_k units starting at k * gt * P; a run of L units gives every
+// worker floor(L / g) of them plus one more to L mod g consecutive workers
+// (mod g), which a circular difference array accumulates.
+int64_t grouped_makespan(int64_t tb, int64_t gt, int64_t P, int64_t base, int64_t rem, int64_t g,
+                         std::vector<int64_t>& diff) {
+  const int64_t U = tb * P;
+  diff.assign(size_t(g) + 1, 0);
+  int64_t every = 0;
+  for (int64_t k = 0; k * gt < tb; ++k) {
+    const int64_t gk = std::min(gt, tb - k * gt);
+    const int64_t L = rem * gk;
+    every += L / g;
+    const int64_t r = L % g, a = (k * gt * P) % g;
+    if (r == 0) continue;
+    diff[size_t(a)] += 1;
+    if (a + r <= g) {
+      diff[size_t(a + r)] -= 1;
+    } else {
+      diff[size_t(g)] -= 1;
+      diff[0] += 1;
+      diff[size_t(a + r - g)] -= 1;
+    }
+  }
+  int64_t best = 0, run = 0;
+  for (int64_t c = 0; c < g; ++c) {
+    run += diff[size_t(c)];
+    const int64_t units_c = U / g + (c < U % g ? 1 : 0);
+    best = std::max(best, units_c * base + every + run);
+  }
+  return best;
+}
+
+// Choose P (slabs per token block) for `tb` token blocks in groups of `gt`,
+// `nt` vocab tiles and `g` concurrent workers: the smallest makespan, plus a
+// small per-unit cost (a partial state write and a pipeline restart).
+void choose_slabs(int64_t tb, int64_t gt, int64_t nt, int64_t g, int64_t pcap, int32_t& P_out,
                   int64_t& makespan_out) {
   double best = 1e300;
   int32_t bestP = 1;
   int64_t best_ms = 0;
+  std::vector<int64_t> diff;
   for (int64_t P = 1; P <= std::min(nt, pcap); ++P) {
-    const int64_t U = tb * P;
-    const int64_t base = nt / P, rem = nt % P;
-    const int64_t waves = cdiv(U, g);
-    const int64_t ms = waves * base + cdiv(rem * tb, g);
-    const double cost = double(ms) + 0.05 * double(waves);
+    const int64_t ms = grouped_makespan(tb, gt, P, nt / P, nt % P, g, diff);
+    const double cost = double(ms) + 0.05 * double(cdiv(tb * P, g));
     if (cost < best - 1e-9) {
       best = cost;
       bestP = int32_t(P);
@@ -67,6 +99,16 @@ void choose_slabs(int64_t tb, int64_t nt, int64_t g, int64_t pcap, int32_t& P_ou
   }
   P_out = bestP;
   makespan_out = best_ms;
+}
+
+// Token blocks per raster group: as many as keep the live part of H within
+// kGroupHBytes, so that it and the W tiles in flight stay in one die's L2
+// partition.
+constexpr int64_t kGroupHBytes = 32ll << 20;
+
+int64_t group_blocks_for(int64_t tb, int64_t block_rows, int64_t D, int64_t elem_bytes) {
+  const int64_t per_block = std::max<int64_t>(1, block_rows * D * elem_bytes);
+  return std::max<int64_t>(1, std::min(tb, kGroupHBytes / per_block));
 }
 
 // The bf16 path runs on CTA pairs (256-token tiles) unless the batch fits one
@@ -90,8 +132,10 @@ flce_status make_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int64_t
   p->token_blocks = cdiv(std::max<int64_t>(N, 1), p->block_rows);
   p->vocab_tiles = cdiv(V, kTileCols);
   const int64_t g = std::max<int64_t>(1, workers);
+  p->group_blocks = int32_t(group_blocks_for(p->token_blocks, p->block_rows, D, tc ? 2 : 4));
   int64_t ms = 0;
-  choose_slabs(p->token_blocks, p->vocab_tiles, g, slab_capacity(V), p->slabs, ms);
+  choose_slabs(p->token_blocks, p->group_blocks, p->vocab_tiles, g, slab_capacity(V), p->slabs,
+               ms);
   p->slab_base = int32_t(p->vocab_tiles / p->slabs);
   p->slab_rem = int32_t(p->vocab_tiles % p->slabs);
   p->units = p->token_blocks * p->slabs;
@@ -234,6 +278,7 @@ flce_status launch_partials(const void* H, const void* W, const int64_t* y, int6
   sch.slab_base = plan.slab_base;
   sch.slab_rem = plan.slab_rem;
   sch.units = int32_t(plan.units);
+  sch.group_blocks = plan.group_blocks;
 
   if (dtype == FLCE_BF16) {
     if (!load_encoder()) return FLCE_ERR_CUDA;

@@ -63,13 +63,23 @@ struct Schedule {
   int32_t slabs;         // P
   int32_t slab_base;     // tiles per slab (NT / P)
   int32_t slab_rem;      // the first slab_rem slabs hold one more tile
-  int32_t units;         // TB * P; unit u -> slab u / TB, token block u % TB
+  int32_t units;         // TB * P
+  int32_t group_blocks;  // GT: token blocks per raster group
 };
 
+// Work-unit order.  Token blocks are taken in groups of GT; inside a group the
+// order is slab-major (all GT token blocks of slab 0, then of slab 1, ...).
+// Units handed out round-robin therefore run, at any moment, over a few
+// consecutive slabs of one group: each W tile is read by GT token blocks close
+// together in time, and only GT blocks of H are live in L2.
 __device__ __forceinline__ void unit_coords(const Schedule& s, int u, int& slab, int& tblock,
                                             int& tile0, int& ntiles) {
-  slab = u / s.token_blocks;
-  tblock = u - slab * s.token_blocks;
+  const int per_group = s.group_blocks * s.slabs;
+  const int g = u / per_group;
+  const int l = u - g * per_group;
+  const int gt = min(s.group_blocks, s.token_blocks - g * s.group_blocks);  // last group may be short
+  slab = l / gt;
+  tblock = g * s.group_blocks + (l - slab * gt);
   tile0 = slab * s.slab_base + min(slab, s.slab_rem);
   ntiles = s.slab_base + (slab < s.slab_rem ? 1 : 0);
 }
@@ -275,8 +285,6 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint64_t pol_h = ptx::policy_evict_last();    // H is re-read for every tile
-      const uint64_t pol_w = ptx::policy_evict_normal();  // W tiles are shared by concurrent CTAs
       int stage = 0;
       uint32_t phase = 0;
       uint32_t used = 0, last_parity = 0;  // per stage: ever issued / parity of last issue
@@ -293,8 +301,8 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
             const uint32_t fb = ptx::smem_addr(&full_bar[stage]);
             const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
             ptx::mbar_arrive_expect_tx(fb, STAGE_BYTES);
-            ptx::tma_load_2d(sa, &tmH, fb, kb * BK, tb * BM, pol_h);
-            ptx::tma_load_2d(sa + A_BYTES, &tmW, fb, kb * BK, t * BN, pol_w);
+            ptx::tma_load_2d(sa, &tmH, fb, kb * BK, tb * BM);
+            ptx::tma_load_2d(sa + A_BYTES, &tmW, fb, kb * BK, t * BN);
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) {
@@ -504,8 +512,6 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
-      const uint64_t pol_h = ptx::policy_evict_last();
-      const uint64_t pol_w = ptx::policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t used = 0, last_parity = 0;
@@ -526,8 +532,8 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
             const uint32_t fb_even = ptx::map_to_cta(fb_local, 0);
             const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
             if (rank == 0) ptx::mbar_arrive_expect_tx(fb_local, PAIR_TX_BYTES);
-            ptx::tma_load_2d_pair(sa, &tmH, fb_even, kb * BK, hrow, pol_h);
-            ptx::tma_load_2d_pair(sa + A_BYTES, &tmW, fb_even, kb * BK, wrow, pol_w);
+            ptx::tma_load_2d_pair(sa, &tmH, fb_even, kb * BK, hrow);
+            ptx::tma_load_2d_pair(sa + A_BYTES, &tmW, fb_even, kb * BK, wrow);
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) {

@@ -63,13 +63,21 @@ def test_workspace_is_O_N_not_O_NV(lib):
     assert flce.workspace_size(100, 5000, 64) == flce.workspace_size(100, 5000, 4096, 1)
 
 
+def unit_order(p):
+    """(slab, token block) of each unit, in the documented grouped order."""
+    tb, P, gt = p["token_blocks"], p["slabs"], p["group_blocks"]
+    order = []
+    for g0 in range(0, tb, gt):
+        blocks = list(range(g0, min(tb, g0 + gt)))
+        order += [(slab, b) for slab in range(P) for b in blocks]
+    return order
+
+
 def simulate_makespan(p):
-    tb, P, base, rem = p["token_blocks"], p["slabs"], p["slab_base"], p["slab_rem"]
+    base, rem = p["slab_base"], p["slab_rem"]
     workers = p["grid"] // p["ctas_per_unit"]          # CTAs, or CTA pairs
-    units = tb * P
     load = [0] * workers
-    for u in range(units):
-        slab = u // tb
+    for u, (slab, _) in enumerate(unit_order(p)):
         load[u % workers] += base + (1 if slab < rem else 0)
     return max(load)
 
@@ -87,6 +95,9 @@ def test_plan_covers_every_tile_once_and_balances(lib, N, V, D, dtype, sms):
     sizes = [p["slab_base"] + (1 if s < p["slab_rem"] else 0) for s in range(p["slabs"])]
     assert sum(sizes) == p["vocab_tiles"] and min(sizes) >= 1
     assert p["units"] == p["token_blocks"] * p["slabs"]
+    order = unit_order(p)
+    assert len(order) == p["units"] and len(set(order)) == p["units"]   # each unit exactly once
+    assert 1 <= p["group_blocks"] <= p["token_blocks"]
     assert p["workspace_bytes"] == flce.workspace_size(N, V, D, dtype)
     if dtype == 0:
         pair = N > 128
@@ -101,12 +112,27 @@ def test_plan_covers_every_tile_once_and_balances(lib, N, V, D, dtype, sms):
             assert p["makespan_tiles"] <= math.ceil(total / workers) + 1
 
 
+def test_grouped_makespan_matches_simulation_on_random_shapes(lib):
+    import random
+    rnd = random.Random(7)
+    for _ in range(60):
+        N = rnd.choice([rnd.randint(1, 5000), rnd.randint(5000, 70000)])
+        V = rnd.randint(1, 300000)
+        D = 8 * rnd.randint(1, 1024)
+        sms = rnd.choice([148, 132, 120, 16, 2, 1])
+        p = flce.plan(N, V, D, 0, sm_count=sms)
+        assert simulate_makespan(p) == p["makespan_tiles"], (N, V, D, sms, p)
+        order = unit_order(p)
+        assert len(set(order)) == p["units"] == len(order)
+
+
 def test_headline_plan(lib):
     p = flce.plan(8192, 151936, 4096, 0, sm_count=148)
     assert p["ctas_per_unit"] == 2 and p["grid"] == 148
     assert p["block_rows"] == 256 and p["tile_cols"] == 256 and p["k_block"] == 64
     assert p["token_blocks"] == 32 and p["vocab_tiles"] == 594
-    assert p["makespan_tiles"] == 257          # ceil(32 * 594 / 74) pair tiles
+    assert p["group_blocks"] == 16             # 16 x 2 MB of H live at a time
+    assert p["makespan_tiles"] <= 258          # ceil(32 * 594 / 74) = 257 pair tiles
 
 
 def test_plan_rejects_bad_args(lib):
