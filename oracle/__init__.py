@@ -27,6 +27,7 @@ _lib = None
 
 BF16 = 0
 FP32 = 1
+FP64 = 2   # only for the oracle's own finite-difference pins
 
 _ERRORS = {-1: "invalid argument", -2: "target outside [0, V)", -3: "out of memory"}
 
@@ -63,6 +64,12 @@ def _load():
             lib.oracle_mean.restype = ctypes.c_double
             lib.oracle_max_threads.argtypes = []
             lib.oracle_max_threads.restype = ctypes.c_int
+            lib.oracle_backward.argtypes = [vp, vp, ctypes.c_int, vp, dp, i64, i64, i64,
+                                            dp, dp, dp, dp, ctypes.c_int]
+            lib.oracle_backward.restype = ctypes.c_int
+            lib.oracle_grad_logits_row.argtypes = [vp, vp, ctypes.c_int, vp, ctypes.c_double,
+                                                   i64, i64, i64, dp]
+            lib.oracle_grad_logits_row.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -74,7 +81,9 @@ def _as_storage(a: np.ndarray):
         return a, BF16
     if a.dtype == np.float32:
         return a, FP32
-    raise TypeError(f"oracle takes bf16 bits (uint16) or float32, got {a.dtype}")
+    if a.dtype == np.float64:
+        return a, FP64
+    raise TypeError(f"oracle takes bf16 bits (uint16), float32 or float64, got {a.dtype}")
 
 
 def _ptr(a):
@@ -135,3 +144,46 @@ def mean(loss: np.ndarray) -> float:
 
 def max_threads() -> int:
     return int(_load().oracle_max_threads())
+
+
+def backward(H: np.ndarray, W: np.ndarray, y: np.ndarray, g, bounds: bool = False,
+             want_dW: bool = True, nthreads: int = 0):
+    """Gradients of sum_i g_i loss_i with respect to H and W (fp64).
+
+    g is a per-token array of upstream gradients or a scalar (1/N gives the
+    mean loss).  Returns dict with dH (N, D), dW (V, D) and, with bounds=True,
+    bH = |dZ| |W| and bW = |dZ|^T |H| (elementwise magnitudes of the sums).
+    """
+    lib = _load()
+    H, dt = _as_storage(H)
+    W, dt_w = _as_storage(W)
+    if dt != dt_w:
+        raise TypeError("H and W must share one storage type")
+    N, D = H.shape
+    V = W.shape[0]
+    y = np.ascontiguousarray(y, dtype=np.int64)
+    gv = np.ascontiguousarray(np.broadcast_to(np.asarray(g, dtype=np.float64), (N,)))
+    out = {"dH": np.empty((N, D)), "dW": np.empty((V, D)) if want_dW else None}
+    if bounds:
+        out["bH"] = np.empty((N, D))
+        out["bW"] = np.empty((V, D)) if want_dW else None
+    rc = lib.oracle_backward(_ptr(H), _ptr(W), dt, _ptr(y), _ptr(gv), N, V, D,
+                             _ptr(out["dH"]), _ptr(out["dW"]), _ptr(out.get("bH")),
+                             _ptr(out.get("bW")), int(nthreads))
+    if rc != 0:
+        raise OracleError(_ERRORS.get(rc, f"oracle error {rc}"))
+    return out
+
+
+def grad_logits_row(H: np.ndarray, W: np.ndarray, y: np.ndarray, g_i: float, i: int) -> np.ndarray:
+    """dL/dZ_i. for one row (V values)."""
+    lib = _load()
+    H, dt = _as_storage(H)
+    W, _ = _as_storage(W)
+    V, D = W.shape
+    y = np.ascontiguousarray(y, dtype=np.int64)
+    dz = np.empty(V, dtype=np.float64)
+    rc = lib.oracle_grad_logits_row(_ptr(H), _ptr(W), dt, _ptr(y), float(g_i), int(i), V, D, _ptr(dz))
+    if rc != 0:
+        raise OracleError(_ERRORS.get(rc, f"oracle error {rc}"))
+    return dz

@@ -30,8 +30,12 @@
  *   - the mean loss is the plain sum of the per-token losses divided by N,
  *     summed sequentially in fp64.
  *
+ * The backward (oracle_backward) differentiates that definition; see its
+ * comment.
+ *
  * Parity is pinned for every function here (closed forms, invariants, a
- * library cross-entropy on fp64 logits and exact brute force; see the tests).
+ * library cross-entropy and autograd on fp64 logits, finite differences and
+ * exact brute force; see the tests).
  */
 #include <math.h>
 #include <stdint.h>
@@ -49,6 +53,7 @@
 /* dtype codes for the stored element type of H and W */
 #define ORACLE_BF16 0
 #define ORACLE_FP32 1
+#define ORACLE_FP64 2   /* only for the oracle's own finite-difference pins */
 
 /* Exact conversion of one stored element to double.  A bf16 value is the
  * upper 16 bits of the fp32 with the same sign, exponent and leading mantissa
@@ -60,6 +65,7 @@ static double load_elem(const void *base, int dtype, int64_t idx) {
         memcpy(&f, &bits, sizeof f);
         return (double)f;
     }
+    if (dtype == ORACLE_FP64) return ((const double *)base)[idx];
     return (double)((const float *)base)[idx];
 }
 
@@ -76,7 +82,7 @@ static double logit(const void *H, const void *W, int dtype, int64_t i,
 int oracle_logits_row(const void *H, const void *W, int dtype, int64_t i,
                       int64_t V, int64_t D, double *z) {
     if (!H || !W || !z || V < 1 || D < 1 || i < 0) return ORACLE_ERR_ARG;
-    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP32) return ORACLE_ERR_ARG;
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP32 && dtype != ORACLE_FP64) return ORACLE_ERR_ARG;
     for (int64_t j = 0; j < V; ++j) z[j] = logit(H, W, dtype, i, j, D);
     return ORACLE_OK;
 }
@@ -97,7 +103,7 @@ int oracle_forward_rows(const void *H, const void *W, int dtype,
                         int nthreads) {
     if (!H || !W || !y || N < 0 || V < 1 || D < 1 || nrows < 0)
         return ORACLE_ERR_ARG;
-    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP32) return ORACLE_ERR_ARG;
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP32 && dtype != ORACLE_FP64) return ORACLE_ERR_ARG;
     if (!rows && nrows != N) return ORACLE_ERR_ARG;
     for (int64_t t = 0; t < nrows; ++t) {
         int64_t i = rows ? rows[t] : t;
@@ -140,6 +146,123 @@ int oracle_forward_rows(const void *H, const void *W, int dtype,
         free(z);
     }
     return status;
+}
+
+/*
+ * Backward of the weighted loss sum_i g_i loss_i (g_i = dL/dloss_i; g_i = 1/N
+ * for the mean loss).  Differentiating loss_i = logsumexp(Z_i) - Z_{i,y_i}
+ * (the page, section 1) gives
+ *     dL/dZ_ij = g_i (softmax(Z_i)_j - [j == y_i]),  softmax(Z_i)_j = exp(z_ij - lse_i),
+ * and through Z = H W^T
+ *     dH = (dL/dZ) W        (N x D),     dW = (dL/dZ)^T H      (V x D).
+ * Written out directly: pass 1 computes each row's logits and lse and its dH
+ * row; pass 2 forms each dW row by recomputing the logits column it needs.
+ * Optionally also returns the elementwise magnitudes
+ *     bH_ik = sum_j |dZ_ij| |W_jk|,   bW_jk = sum_i |dZ_ij| |H_ik|
+ * (the scale that rounding dZ to a narrower type multiplies), for tests.
+ * Any of dH, dW, bH, bW may be NULL.  y must lie in [0, V).
+ */
+int oracle_backward(const void *H, const void *W, int dtype, const int64_t *y,
+                    const double *g, int64_t N, int64_t V, int64_t D,
+                    double *dH, double *dW, double *bH, double *bW, int nthreads) {
+    if (!H || !W || !y || !g || N < 1 || V < 1 || D < 1) return ORACLE_ERR_ARG;
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP32 && dtype != ORACLE_FP64) return ORACLE_ERR_ARG;
+    for (int64_t i = 0; i < N; ++i)
+        if (y[i] < 0 || y[i] >= V) return ORACLE_ERR_TARGET;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    double *lse = (double *)malloc((size_t)N * sizeof(double));
+    if (!lse) return ORACLE_ERR_NOMEM;
+    int status = ORACLE_OK;
+    /* pass 1: per row, logits, lse, and the dH row */
+#pragma omp parallel
+    {
+        double *z = (double *)malloc((size_t)V * sizeof(double));
+        if (!z) {
+#pragma omp atomic write
+            status = ORACLE_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < N; ++i) {
+            if (!z) continue;
+            for (int64_t j = 0; j < V; ++j) z[j] = logit(H, W, dtype, i, j, D);
+            double M = z[0];
+            for (int64_t j = 1; j < V; ++j)
+                if (z[j] > M) M = z[j];
+            double S = 0.0;
+            for (int64_t j = 0; j < V; ++j) S += exp(z[j] - M);
+            lse[i] = M + log(S);
+            for (int64_t j = 0; j < V; ++j)  /* z[j] becomes dL/dZ_ij */
+                z[j] = g[i] * (exp(z[j] - lse[i]) - (j == y[i] ? 1.0 : 0.0));
+            for (int64_t k = 0; k < D; ++k) {
+                double acc = 0.0, mag = 0.0;
+                for (int64_t j = 0; j < V; ++j) {
+                    double w = load_elem(W, dtype, j * D + k);
+                    acc += z[j] * w;
+                    mag += fabs(z[j]) * fabs(w);
+                }
+                if (dH) dH[i * D + k] = acc;
+                if (bH) bH[i * D + k] = mag;
+            }
+        }
+        free(z);
+    }
+    if (status != ORACLE_OK) {
+        free(lse);
+        return status;
+    }
+    /* pass 2: per vocab row, the dW row (the logits column recomputed) */
+    if (dW || bW) {
+#pragma omp parallel
+        {
+            double *dz = (double *)malloc((size_t)N * sizeof(double));
+            if (!dz) {
+#pragma omp atomic write
+                status = ORACLE_ERR_NOMEM;
+            }
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t j = 0; j < V; ++j) {
+                if (!dz) continue;
+                for (int64_t i = 0; i < N; ++i)
+                    dz[i] = g[i] * (exp(logit(H, W, dtype, i, j, D) - lse[i]) -
+                                    (j == y[i] ? 1.0 : 0.0));
+                for (int64_t k = 0; k < D; ++k) {
+                    double acc = 0.0, mag = 0.0;
+                    for (int64_t i = 0; i < N; ++i) {
+                        double h = load_elem(H, dtype, i * D + k);
+                        acc += dz[i] * h;
+                        mag += fabs(dz[i]) * fabs(h);
+                    }
+                    if (dW) dW[j * D + k] = acc;
+                    if (bW) bW[j * D + k] = mag;
+                }
+            }
+            free(dz);
+        }
+    }
+    free(lse);
+    return status;
+}
+
+/* dL/dZ for one row i (V values), given upstream gradient g_i: the vector the
+ * backward contracts with W and H.  For tests of the gradient definition. */
+int oracle_grad_logits_row(const void *H, const void *W, int dtype, const int64_t *y, double g_i,
+                           int64_t i, int64_t V, int64_t D, double *dz) {
+    if (!H || !W || !y || !dz || V < 1 || D < 1 || i < 0) return ORACLE_ERR_ARG;
+    if (y[i] < 0 || y[i] >= V) return ORACLE_ERR_TARGET;
+    int rc = oracle_logits_row(H, W, dtype, i, V, D, dz);
+    if (rc != ORACLE_OK) return rc;
+    double M = dz[0];
+    for (int64_t j = 1; j < V; ++j)
+        if (dz[j] > M) M = dz[j];
+    double S = 0.0;
+    for (int64_t j = 0; j < V; ++j) S += exp(dz[j] - M);
+    double lse = M + log(S);
+    for (int64_t j = 0; j < V; ++j) dz[j] = g_i * (exp(dz[j] - lse) - (j == y[i] ? 1.0 : 0.0));
+    return ORACLE_OK;
 }
 
 /* Mean loss: (sum_i loss_i) / n, summed sequentially in fp64.  n == 0 gives NaN. */
