@@ -149,6 +149,38 @@ FLCE_API flce_status flce_merge(const int64_t* y, int64_t N, int64_t V,
                        float* out_mean, const void* workspace, size_t workspace_bytes,
                        void* stream);
 
+/*
+ * Backward of the weighted loss sum_i g_i loss_i (g_i = grad_scale *
+ * grad_loss[i], or grad_scale when grad_loss is NULL; g_i = 1/N for the mean
+ * loss).  Differentiating section 1 of the page:
+ *     dZ_ij = g_i (exp(z_ij - lse_i) - [j == y_i]),   dH = dZ W,   dW = dZ^T H.
+ * As on the page, the forward's log-sum-exp is kept and the logits are
+ * regenerated tile by tile; vocabulary chunks of up to 16384 rows bound the
+ * working slice of dZ to O(N * chunk) (never O(N * V)).
+ *
+ *   H, W, y, N, V, D, dtype   as for flce_forward (bf16 only for now:
+ *                             FLCE_FP32 returns FLCE_ERR_UNSUPPORTED)
+ *   lse          (N) fp32: out_lse of the forward on the same H, W
+ *   grad_loss    (N) fp32 upstream gradient dL/dloss_i, or NULL
+ *   dH           (N, D) fp32 row-major, overwritten
+ *   dW           (V, D) fp32 row-major, overwritten
+ *   workspace    >= flce_backward_workspace_size(N, V, D, dtype) bytes,
+ *                256-byte aligned (holds W^T, H^T, two chunk slices of dZ in
+ *                bf16, and the status word read by flce_check)
+ * dZ is rounded to bf16 before the two gradient contractions (fp32
+ * accumulation), so each gradient entry carries an error of at most about
+ * 2^-8 times sum_j |dZ_ij| |W_jk| (resp. sum_i |dZ_ij| |H_ik|).
+ * A target outside [0, V) sets FLCE_ERR_TARGET_OUT_OF_RANGE for flce_check.
+ * Deterministic run to run.
+ */
+FLCE_API size_t flce_backward_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype dtype);
+
+FLCE_API flce_status flce_backward(const void* H, const void* W, const int64_t* y,
+                                   const float* lse, const float* grad_loss, float grad_scale,
+                                   int64_t N, int64_t V, int64_t D, flce_dtype dtype, float* dH,
+                                   float* dW, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
 /* Waits for `stream`, then reads the workspace status word left by the last
  * flce_forward / flce_partials + flce_merge that used this workspace.
  * Returns FLCE_OK, FLCE_ERR_TARGET_OUT_OF_RANGE, FLCE_ERR_TIMEOUT,

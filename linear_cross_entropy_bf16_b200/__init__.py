@@ -22,7 +22,8 @@ import threading
 import torch
 
 __all__ = [
-    "FlceError", "forward", "partials", "merge", "workspace_size", "plan", "check",
+    "FlceError", "forward", "backward", "partials", "merge", "workspace_size",
+    "backward_workspace_size", "plan", "check",
     "status_string", "selftest_wait_timeout", "library_path", "load_library",
 ]
 
@@ -100,6 +101,11 @@ def load_library():
         lib.flce_status_string.restype = ctypes.c_char_p
         lib.flce_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint64, vp]
         lib.flce_selftest_wait_timeout.restype = st
+        lib.flce_backward_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int]
+        lib.flce_backward_workspace_size.restype = sz
+        lib.flce_backward.argtypes = [vp, vp, vp, vp, vp, ctypes.c_float, i64, i64, i64,
+                                      ctypes.c_int, vp, vp, vp, sz, vp]
+        lib.flce_backward.restype = st
         _lib = lib
         return lib
 
@@ -214,6 +220,57 @@ def forward(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, *, out: dict | No
     if check:
         _raise_on(lib.flce_check(ws.data_ptr(), sp), "flce_forward (device)")
     return loss, lse, tgt, mean
+
+
+def backward_workspace_size(N: int, V: int, D: int, dtype=torch.bfloat16) -> int:
+    code = dtype if isinstance(dtype, int) else (BF16 if dtype == torch.bfloat16 else FP32)
+    n = load_library().flce_backward_workspace_size(int(N), int(V), int(D), code)
+    if n == 0:
+        raise FlceError(ERR_INVALID_ARG, "backward_workspace_size")
+    return int(n)
+
+
+def backward(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, lse: torch.Tensor,
+             grad: torch.Tensor | None = None, grad_scale: float = 1.0, *,
+             out: dict | None = None, workspace: torch.Tensor | None = None, stream=None,
+             check: bool = False):
+    """Gradients (dH, dW) of sum_i g_i loss_i, g_i = grad_scale * grad[i] (or grad_scale).
+
+    ``lse`` is the forward's log-sum-exp for the same H and W.  Returns fp32
+    tensors dH (N, D) and dW (V, D); ``out`` may supply them as "dH" / "dW".
+    Use grad_scale = 1/N with grad = None for the mean loss.
+    """
+    N, V, D, code = _check_inputs(H, W, y)
+    dev = H.device
+    out = out or {}
+    dH = out.get("dH") if out.get("dH") is not None else torch.empty(N, D, dtype=torch.float32, device=dev)
+    dW = out.get("dW") if out.get("dW") is not None else torch.empty(V, D, dtype=torch.float32, device=dev)
+    for t, shape in ((dH, (N, D)), (dW, (V, D))):
+        if t.dtype != torch.float32 or t.device != dev or not t.is_contiguous() or tuple(t.shape) != shape:
+            raise ValueError("dH and dW must be contiguous float32 (N, D) and (V, D) tensors")
+    if lse.dtype != torch.float32 or lse.shape != (N,) or not lse.is_contiguous() or lse.device != dev:
+        raise ValueError("lse must be a contiguous float32 (N,) tensor on the input device")
+    if grad is not None and (grad.dtype != torch.float32 or grad.shape != (N,) or not grad.is_contiguous()
+                             or grad.device != dev):
+        raise ValueError("grad must be a contiguous float32 (N,) tensor on the input device")
+    if N == 0:
+        dW.zero_()
+        return dH, dW
+    lib = load_library()
+    need = lib.flce_backward_workspace_size(N, V, D, code)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace.numel() * workspace.element_size() < need:
+        raise FlceError(ERR_WORKSPACE_TOO_SMALL, "backward")
+    sp = _stream_ptr(stream, dev)
+    st = lib.flce_backward(H.data_ptr(), W.data_ptr(), y.data_ptr(), lse.data_ptr(),
+                           grad.data_ptr() if grad is not None else None, float(grad_scale),
+                           N, V, D, code, dH.data_ptr(), dW.data_ptr(), workspace.data_ptr(),
+                           workspace.numel() * workspace.element_size(), sp)
+    _raise_on(st, "flce_backward")
+    if check:
+        _raise_on(lib.flce_check(workspace.data_ptr(), sp), "flce_backward (device)")
+    return dH, dW
 
 
 def partials(H, W, y, target_logit, workspace, stream=None):

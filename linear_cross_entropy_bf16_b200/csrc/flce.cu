@@ -17,6 +17,7 @@
 #include <vector>
 
 #include "flce.h"
+#include "flce_backward.cuh"
 #include "flce_kernels.cuh"
 
 namespace {
@@ -435,6 +436,187 @@ flce_status flce_selftest_wait_timeout(void* workspace, size_t workspace_bytes, 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- backward
+
+namespace {
+
+constexpr int64_t kBwdChunkCols = 16384;  // vocabulary rows per backward chunk
+
+inline int64_t round_up(int64_t x, int64_t m) { return cdiv(x, m) * m; }
+
+struct BwdLayout {
+  int64_t chunk, Vp, Np;
+  size_t off_wt, off_ht, off_dz, off_dzt, total;
+};
+
+BwdLayout bwd_layout(int64_t N, int64_t V, int64_t D) {
+  BwdLayout L;
+  L.chunk = std::min(round_up(V, kTileCols), kBwdChunkCols);
+  L.Vp = round_up(V, 8);
+  L.Np = round_up(N, 8);
+  size_t off = kHeaderBytes;
+  L.off_wt = off;
+  off += align256(size_t(D) * size_t(L.Vp) * 2);
+  L.off_ht = off;
+  off += align256(size_t(D) * size_t(L.Np) * 2);
+  L.off_dz = off;
+  off += align256(size_t(N) * size_t(L.chunk) * 2);
+  L.off_dzt = off;
+  off += align256(size_t(L.chunk) * size_t(L.Np) * 2);
+  L.total = off;
+  return L;
+}
+
+// Row-major bf16 matrix (rows x cols, row stride ld elements) as a TMA map
+// with 64 x box_rows boxes, 128-byte swizzle and zero fill outside.
+bool encode_bf16_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                    int box_rows) {
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(ld) * 2};
+  cuuint32_t box[2] = {cuuint32_t(bwd::BK), cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bwd::GemmShape gemm_shape(int64_t M, int64_t Nc, int64_t K) {
+  bwd::GemmShape g;
+  g.M = int32_t(M);
+  g.N = int32_t(Nc);
+  g.K = int32_t(K);
+  g.tiles_m = int32_t(cdiv(M, bwd::PAIR_M));
+  g.tiles_n = int32_t(cdiv(Nc, bwd::BN));
+  // keep about 32 MB of A live per raster group
+  g.group_m = int32_t(std::max<int64_t>(
+      1, std::min<int64_t>(g.tiles_m, kGroupHBytes / std::max<int64_t>(1, bwd::PAIR_M * K * 2))));
+  g.tiles = g.tiles_m * g.tiles_n;
+  g.kblocks = int32_t(cdiv(K, bwd::BK));
+  return g;
+}
+
+template <class Epi>
+flce_status launch_gemm(const CUtensorMap& A, const CUtensorMap& B, const bwd::GemmShape& g,
+                        const Epi& epi, uint32_t* status, int64_t pairs, cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [] {
+    attr = cudaFuncSetAttribute(bwd::gemm_pair_kernel<Epi>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::SMEM_BYTES);
+  });
+  if (attr != cudaSuccess) return FLCE_ERR_CUDA;
+  const int grid = int(2 * std::min<int64_t>(pairs, g.tiles));
+  bwd::gemm_pair_kernel<Epi><<<grid, bwd::NUM_THREADS, bwd::SMEM_BYTES, st>>>(
+      A, B, g, epi, status, kDefaultWaitLimitNs);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+flce_status launch_transpose(const void* in, int64_t rows, int64_t cols, void* out, int64_t ld_out,
+                             cudaStream_t st) {
+  dim3 grid(unsigned(cdiv(rows, bwd::kTrTile)), unsigned(cdiv(cols, bwd::kTrTile)));
+  bwd::transpose_bf16_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in), rows,
+                                                   cols, cols,
+                                                   static_cast<__nv_bfloat16*>(out), ld_out);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" size_t flce_backward_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
+  if (!sizes_ok(N, V, D, dtype) || N < 1) return 0;
+  return bwd_layout(N, V, D).total;
+}
+
+extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t* y,
+                                     const float* lse, const float* grad_loss, float grad_scale,
+                                     int64_t N, int64_t V, int64_t D, flce_dtype dtype, float* dH,
+                                     float* dW, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  if (!sizes_ok(N, V, D, dtype)) return FLCE_ERR_INVALID_ARG;
+  if (N == 0) return FLCE_OK;
+  if (!H || !W || !y || !lse || !dH || !dW || !workspace) return FLCE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FLCE_ERR_INVALID_ARG;
+  if (dtype != FLCE_BF16) return FLCE_ERR_UNSUPPORTED;
+  if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31) || D >= (int64_t(1) << 31))
+    return FLCE_ERR_UNSUPPORTED;
+  if (D % 8 != 0 || !aligned16(H) || !aligned16(W)) return FLCE_ERR_UNSUPPORTED;
+  const BwdLayout L = bwd_layout(N, V, D);
+  if (workspace_bytes < L.total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+
+  DeviceInfo di;
+  flce_status s = device_info(di);
+  if (s != FLCE_OK) return s;
+  if (!load_encoder()) return FLCE_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if ((s = set_smem_attr_once()) != FLCE_OK) return s;
+  const int64_t pairs = resident_pairs(dev, di.sms);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+  __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(ws + L.off_wt);    // (D x Vp)
+  __nv_bfloat16* ht = reinterpret_cast<__nv_bfloat16*>(ws + L.off_ht);    // (D x Np)
+  __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dz);    // (N x chunk)
+  __nv_bfloat16* dzt = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dzt);  // (chunk x Np)
+  if (cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
+  if ((s = launch_transpose(W, V, D, wt, L.Vp, st)) != FLCE_OK) return s;
+  if ((s = launch_transpose(H, N, D, ht, L.Np, st)) != FLCE_OK) return s;
+
+  CUtensorMap mH, mHt;
+  if (!encode_bf16_2d(&mH, H, N, D, D, bwd::BM) || !encode_bf16_2d(&mHt, ht, D, N, L.Np, bwd::HALF_N))
+    return FLCE_ERR_UNSUPPORTED;
+  for (int64_t c0 = 0; c0 < V; c0 += L.chunk) {
+    const int64_t clen = std::min(L.chunk, V - c0);
+    CUtensorMap mW, mDz, mWt, mDzt;
+    if (!encode_bf16_2d(&mW, static_cast<const __nv_bfloat16*>(W) + c0 * D, clen, D, D,
+                        bwd::HALF_N) ||
+        !encode_bf16_2d(&mDz, dz, N, clen, L.chunk, bwd::BM) ||
+        !encode_bf16_2d(&mWt, wt + c0, D, clen, L.Vp, bwd::HALF_N) ||
+        !encode_bf16_2d(&mDzt, dzt, clen, N, L.Np, bwd::BM))
+      return FLCE_ERR_UNSUPPORTED;
+    // K1: dZ for this chunk from the regenerated logits
+    bwd::EpiGradLogits e1;
+    e1.lse = lse;
+    e1.y = y;
+    e1.grad = grad_loss;
+    e1.grad_scale = grad_scale;
+    e1.N = int32_t(N);
+    e1.V = int32_t(V);
+    e1.c0 = int32_t(c0);
+    e1.clen = int32_t(clen);
+    e1.dz = dz;
+    e1.ldz = int32_t(L.chunk);
+    e1.dzt = dzt;
+    e1.ldzt = int32_t(L.Np);
+    e1.status = &hdr->status;
+    if ((s = launch_gemm(mH, mW, gemm_shape(N, clen, D), e1, &hdr->status, pairs, st)) != FLCE_OK)
+      return s;
+    // K2: dH (+)= dZ_C W_C
+    bwd::EpiStoreF32 e2;
+    e2.out = dH;
+    e2.ld = int32_t(D);
+    e2.rows = int32_t(N);
+    e2.cols = int32_t(D);
+    e2.row_base = 0;
+    e2.accumulate = c0 > 0 ? 1 : 0;
+    if ((s = launch_gemm(mDz, mWt, gemm_shape(N, D, clen), e2, &hdr->status, pairs, st)) != FLCE_OK)
+      return s;
+    // K3: dW_C = dZ_C^T H
+    bwd::EpiStoreF32 e3;
+    e3.out = dW;
+    e3.ld = int32_t(D);
+    e3.rows = int32_t(clen);
+    e3.cols = int32_t(D);
+    e3.row_base = int32_t(c0);
+    e3.accumulate = 0;
+    if ((s = launch_gemm(mDzt, mHt, gemm_shape(clen, D, N), e3, &hdr->status, pairs, st)) != FLCE_OK)
+      return s;
+  }
+  return FLCE_OK;
+}
 
 // ---------------------------------------------------------------- no-allocation entry point
 //

@@ -1,0 +1,112 @@
+"""GPU parity of the backward (dH, dW) against the fp64 oracle, through the C ABI.
+
+Tolerance, derived from the arithmetic: dZ is rounded to bf16 (relative
+error <= 2^-9) before the two contractions, which accumulate in fp32 over at
+most K = 16384 (chunk) or N terms (error <= K 2^-24 of the magnitude), so
+each entry satisfies |d dH_ik| <= 2^-8 sum_j |dZ_ij||W_jk| (the oracle's bH)
+and |d dW_jk| <= 2^-8 sum_i |dZ_ij||H_ik| (bW) for the shapes below, plus a
+tiny absolute floor for entries whose magnitude is zero.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_cross_entropy_bf16_b200 import synth
+from tests.flce_testing import to_device
+
+pytestmark = pytest.mark.gpu
+REL = 2.0 ** -8
+FLOOR = 1e-7
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from linear_cross_entropy_bf16_b200 import build
+    build.build()
+    oracle.build()
+
+
+def run_backward(H, W, y, g=None, scale=1.0):
+    import linear_cross_entropy_bf16_b200 as flce
+    Hd, Wd, yd = to_device(H, W, y)
+    _, lse, _, _ = flce.forward(Hd, Wd, yd, check=True)
+    gd = torch.from_numpy(np.asarray(g, dtype=np.float32)).cuda() if g is not None else None
+    dH, dW = flce.backward(Hd, Wd, yd, lse, gd, scale, check=True)
+    torch.cuda.synchronize()
+    return dH.cpu().double().numpy(), dW.cpu().double().numpy()
+
+
+def compare(got, ref, bound, name):
+    err = np.abs(got - ref)
+    lim = REL * bound + FLOOR
+    worst = np.unravel_index(np.argmax(err - lim), err.shape)
+    assert np.all(np.isfinite(got)), name
+    assert np.all(err <= lim), (f"{name}: |diff| {err[worst]:.3e} > {lim[worst]:.3e} at {worst} "
+                                f"(gpu {got[worst]!r}, oracle {ref[worst]!r})")
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert rel < 3e-3, f"{name}: relative Frobenius error {rel:.2e}"
+    return rel
+
+
+SHAPES = [(1, 1, 8), (7, 3, 16), (130, 300, 64), (256, 1000, 128), (300, 2047, 72), (513, 777, 136),
+          (64, 20000, 64), (1000, 600, 264)]
+
+
+@pytest.mark.parametrize("N,V,D", SHAPES)
+def test_backward_every_element(N, V, D):
+    H, W, y = synth.random_inputs(N, V, D, seed=N + 3 * V + 7 * D)
+    g = np.random.default_rng(N).uniform(-1, 1, N)
+    dH, dW = run_backward(H, W, y, g)
+    gf = g.astype(np.float32).astype(np.float64)       # the GPU receives fp32 g
+    ref = oracle.backward(H, W, y, gf, bounds=True)
+    compare(dH, ref["dH"], ref["bH"], "dH")
+    compare(dW, ref["dW"], ref["bW"], "dW")
+
+
+def test_backward_mean_loss_scale_and_multi_chunk():
+    """V > 16384 spans several vocabulary chunks; g = 1/N (mean loss) via grad_scale."""
+    N, V, D = 200, 40000, 64
+    H, W, y = synth.random_inputs(N, V, D, seed=41)
+    dH, dW = run_backward(H, W, y, None, 1.0 / N)
+    ref = oracle.backward(H, W, y, np.float64(np.float32(1.0 / N)), bounds=True)
+    compare(dH, ref["dH"], ref["bH"], "dH")
+    compare(dW, ref["dW"], ref["bW"], "dW")
+
+
+def test_backward_matches_torch_autograd_fp32():
+    """Against torch autograd on the same bf16 values in fp32 (relative Frobenius)."""
+    N, V, D = 384, 5000, 256
+    H, W, y = synth.random_inputs(N, V, D, seed=42)
+    dH, dW = run_backward(H, W, y, None, 1.0 / N)
+    Ht = torch.tensor(synth.bf16_bits_to_f32(H), requires_grad=True)
+    Wt = torch.tensor(synth.bf16_bits_to_f32(W), requires_grad=True)
+    torch.nn.functional.cross_entropy(Ht @ Wt.T, torch.from_numpy(y)).backward()
+    for got, ref in ((dH, Ht.grad.double().numpy()), (dW, Wt.grad.double().numpy())):
+        assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 3e-3
+
+
+def test_backward_vocab_gradient_sums_to_zero():
+    N, V, D = 256, 3000, 128
+    H, W, y = synth.random_inputs(N, V, D, seed=43)
+    _, dW = run_backward(H, W, y, None, 1.0)
+    col = np.abs(dW.sum(axis=0))
+    assert col.max() <= 2.0 ** -7 * np.abs(dW).sum(axis=0).max()
+
+
+def test_backward_deterministic_and_flags_bad_targets():
+    import linear_cross_entropy_bf16_b200 as flce
+    N, V, D = 300, 2000, 64
+    H, W, y = synth.random_inputs(N, V, D, seed=44)
+    Hd, Wd, yd = to_device(H, W, y)
+    _, lse, _, _ = flce.forward(Hd, Wd, yd)
+    a = [t.clone() for t in flce.backward(Hd, Wd, yd, lse)]
+    b = flce.backward(Hd, Wd, yd, lse)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    yb = yd.clone()
+    yb[5] = V + 3
+    ws = torch.empty(flce.backward_workspace_size(N, V, D), dtype=torch.uint8, device="cuda")
+    flce.backward(Hd, Wd, yb, lse, workspace=ws)
+    assert flce.check(ws) == flce.ERR_TARGET_OUT_OF_RANGE
