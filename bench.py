@@ -385,6 +385,9 @@ def run_ours(args, w, rank, world, local_rank):
         "gpu_launches": 2 * K,
         "clocks": clocks,
     }
+    if args.backward and w.dtype == "bf16":
+        line["backward"] = time_backward(flce, H, W, y, lse, N, V, D, tdt, dev, stream, args,
+                                         peaks["bf16_tflops"], world)
     if world == 1 and not args.no_cpu_baseline:
         rows, secs, cores = oracle_sample(Hn, Wn, yn, args.cpu_seconds, w.seed)
         line["cpu_baseline"] = {"value": rows / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -393,6 +396,38 @@ def run_ours(args, w, rank, world, local_rank):
         line["context"] = torch_materialised(H, W, y, dev)
     print(json.dumps(line), flush=True)
     return 0
+
+
+def time_backward(flce, H, W, y, lse, N, V, D, tdt, dev, stream, args, peak, world):
+    """The backward (dH, dW of the mean loss) on the same inputs, timed like the forward."""
+    import torch
+    out = {"dH": torch.empty(N, D, device=dev), "dW": torch.empty(V, D, device=dev)}
+    ws = torch.empty(flce.backward_workspace_size(N, V, D, tdt), dtype=torch.uint8, device=dev)
+
+    def step():
+        flce.backward(H, W, y, lse, None, 1.0 / N, out=out, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+    stream.synchronize()
+    if flce.check(ws, stream) != flce.OK:
+        raise flce.FlceError(flce.check(ws, stream), "backward")
+    Kb = max(3, args.backward_steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(Kb):
+            step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks([e0.elapsed_time(e1) / Kb], world, device=dev)[0]
+    flops = 3 * 2 * N * V * D          # logits regenerated, dH, dW
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"ms_per_step": ms, "steps": Kb, "tokens_per_s": weak_scaling_tokens_per_s(world, N, ms),
+            "flops_per_step": flops, "tflops": tflops, "frac_of_bf16_peak": tflops / peak,
+            "workspace_bytes": int(ws.numel()),
+            "what": "dH and dW of the mean loss from the forward's lse (3 contractions per step)"}
 
 
 def torch_materialised(H, W, y, dev):
@@ -430,6 +465,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the backward (dH, dW) and add a 'backward' object to the line")
+    ap.add_argument("--backward-steps", type=int, default=10)
     ap.add_argument("--context", action="store_true", help="also time the materialising torch forward")
     ap.add_argument("--shape", default=None,
                     help="N,V,D: a custom shape with the chosen workload's distributions "

@@ -165,8 +165,9 @@ FLCE_API flce_status flce_merge(const int64_t* y, int64_t N, int64_t V,
  *   dH           (N, D) fp32 row-major, overwritten
  *   dW           (V, D) fp32 row-major, overwritten
  *   workspace    >= flce_backward_workspace_size(N, V, D, dtype) bytes,
- *                256-byte aligned (holds W^T, H^T, two chunk slices of dZ in
- *                bf16, and the status word read by flce_check)
+ *                256-byte aligned (the status word read by flce_check and one
+ *                N x chunk slice of dZ in bf16: 256 B + 2 N min(V, 16384) B,
+ *                rounded up)
  * dZ is rounded to bf16 before the two gradient contractions (fp32
  * accumulation), so each gradient entry carries an error of at most about
  * 2^-8 times sum_j |dZ_ij| |W_jk| (resp. sum_i |dZ_ij| |H_ik|).

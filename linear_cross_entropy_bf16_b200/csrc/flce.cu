@@ -446,30 +446,24 @@ constexpr int64_t kBwdChunkCols = 16384;  // vocabulary rows per backward chunk
 inline int64_t round_up(int64_t x, int64_t m) { return cdiv(x, m) * m; }
 
 struct BwdLayout {
-  int64_t chunk, Vp, Np;
-  size_t off_wt, off_ht, off_dz, off_dzt, total;
+  int64_t chunk;
+  size_t off_dz, total;
 };
 
+// [256 B header][dZ slice: N x chunk bf16]
 BwdLayout bwd_layout(int64_t N, int64_t V, int64_t D) {
+  (void)D;
   BwdLayout L;
   L.chunk = std::min(round_up(V, kTileCols), kBwdChunkCols);
-  L.Vp = round_up(V, 8);
-  L.Np = round_up(N, 8);
-  size_t off = kHeaderBytes;
-  L.off_wt = off;
-  off += align256(size_t(D) * size_t(L.Vp) * 2);
-  L.off_ht = off;
-  off += align256(size_t(D) * size_t(L.Np) * 2);
-  L.off_dz = off;
-  off += align256(size_t(N) * size_t(L.chunk) * 2);
-  L.off_dzt = off;
-  off += align256(size_t(L.chunk) * size_t(L.Np) * 2);
-  L.total = off;
+  L.off_dz = kHeaderBytes;
+  L.total = L.off_dz + align256(size_t(N) * size_t(L.chunk) * 2);
   return L;
 }
 
 // Row-major bf16 matrix (rows x cols, row stride ld elements) as a TMA map
-// with 64 x box_rows boxes, 128-byte swizzle and zero fill outside.
+// with 64 (cols) x box_rows boxes, 128-byte swizzle and zero fill outside.
+// K-major operands use box_rows = 128 (operand rows per CTA); MN-major
+// operands use box_rows = 64 (K rows per stage).
 bool encode_bf16_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
                     int box_rows) {
   cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
@@ -497,28 +491,19 @@ bwd::GemmShape gemm_shape(int64_t M, int64_t Nc, int64_t K) {
   return g;
 }
 
-template <class Epi>
+template <class Epi, bool kAmn, bool kBmn>
 flce_status launch_gemm(const CUtensorMap& A, const CUtensorMap& B, const bwd::GemmShape& g,
                         const Epi& epi, uint32_t* status, int64_t pairs, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(bwd::gemm_pair_kernel<Epi>,
+    attr = cudaFuncSetAttribute(bwd::gemm_pair_kernel<Epi, kAmn, kBmn>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::SMEM_BYTES);
   });
   if (attr != cudaSuccess) return FLCE_ERR_CUDA;
   const int grid = int(2 * std::min<int64_t>(pairs, g.tiles));
-  bwd::gemm_pair_kernel<Epi><<<grid, bwd::NUM_THREADS, bwd::SMEM_BYTES, st>>>(
+  bwd::gemm_pair_kernel<Epi, kAmn, kBmn><<<grid, bwd::NUM_THREADS, bwd::SMEM_BYTES, st>>>(
       A, B, g, epi, status, kDefaultWaitLimitNs);
-  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
-}
-
-flce_status launch_transpose(const void* in, int64_t rows, int64_t cols, void* out, int64_t ld_out,
-                             cudaStream_t st) {
-  dim3 grid(unsigned(cdiv(rows, bwd::kTrTile)), unsigned(cdiv(cols, bwd::kTrTile)));
-  bwd::transpose_bf16_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in), rows,
-                                                   cols, cols,
-                                                   static_cast<__nv_bfloat16*>(out), ld_out);
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
@@ -557,25 +542,21 @@ extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
-  __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(ws + L.off_wt);    // (D x Vp)
-  __nv_bfloat16* ht = reinterpret_cast<__nv_bfloat16*>(ws + L.off_ht);    // (D x Np)
-  __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dz);    // (N x chunk)
-  __nv_bfloat16* dzt = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dzt);  // (chunk x Np)
+  __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dz);  // (N x chunk)
   if (cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
-  if ((s = launch_transpose(W, V, D, wt, L.Vp, st)) != FLCE_OK) return s;
-  if ((s = launch_transpose(H, N, D, ht, L.Np, st)) != FLCE_OK) return s;
 
-  CUtensorMap mH, mHt;
-  if (!encode_bf16_2d(&mH, H, N, D, D, bwd::BM) || !encode_bf16_2d(&mHt, ht, D, N, L.Np, bwd::HALF_N))
+  const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(W);
+  CUtensorMap mH_k, mH_mn;
+  if (!encode_bf16_2d(&mH_k, H, N, D, D, bwd::BM) ||     // K1 A: (N, D), K = D
+      !encode_bf16_2d(&mH_mn, H, N, D, D, bwd::BK))      // K3 B: d contiguous, K = N
     return FLCE_ERR_UNSUPPORTED;
   for (int64_t c0 = 0; c0 < V; c0 += L.chunk) {
     const int64_t clen = std::min(L.chunk, V - c0);
-    CUtensorMap mW, mDz, mWt, mDzt;
-    if (!encode_bf16_2d(&mW, static_cast<const __nv_bfloat16*>(W) + c0 * D, clen, D, D,
-                        bwd::HALF_N) ||
-        !encode_bf16_2d(&mDz, dz, N, clen, L.chunk, bwd::BM) ||
-        !encode_bf16_2d(&mWt, wt + c0, D, clen, L.Vp, bwd::HALF_N) ||
-        !encode_bf16_2d(&mDzt, dzt, clen, N, L.Np, bwd::BM))
+    CUtensorMap mW_k, mW_mn, mDz_k, mDz_mn;
+    if (!encode_bf16_2d(&mW_k, Wb + c0 * D, clen, D, D, bwd::HALF_N) ||  // K1 B: (clen, D)
+        !encode_bf16_2d(&mW_mn, Wb + c0 * D, clen, D, D, bwd::BK) ||     // K2 B: d contiguous
+        !encode_bf16_2d(&mDz_k, dz, N, clen, L.chunk, bwd::BM) ||        // K2 A: K = vocab
+        !encode_bf16_2d(&mDz_mn, dz, N, clen, L.chunk, bwd::BK))         // K3 A: vocab contiguous
       return FLCE_ERR_UNSUPPORTED;
     // K1: dZ for this chunk from the regenerated logits
     bwd::EpiGradLogits e1;
@@ -589,11 +570,10 @@ extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t
     e1.clen = int32_t(clen);
     e1.dz = dz;
     e1.ldz = int32_t(L.chunk);
-    e1.dzt = dzt;
-    e1.ldzt = int32_t(L.Np);
     e1.status = &hdr->status;
-    if ((s = launch_gemm(mH, mW, gemm_shape(N, clen, D), e1, &hdr->status, pairs, st)) != FLCE_OK)
-      return s;
+    s = launch_gemm<bwd::EpiGradLogits, false, false>(mH_k, mW_k, gemm_shape(N, clen, D), e1,
+                                                      &hdr->status, pairs, st);
+    if (s != FLCE_OK) return s;
     // K2: dH (+)= dZ_C W_C
     bwd::EpiStoreF32 e2;
     e2.out = dH;
@@ -602,8 +582,9 @@ extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t
     e2.cols = int32_t(D);
     e2.row_base = 0;
     e2.accumulate = c0 > 0 ? 1 : 0;
-    if ((s = launch_gemm(mDz, mWt, gemm_shape(N, D, clen), e2, &hdr->status, pairs, st)) != FLCE_OK)
-      return s;
+    s = launch_gemm<bwd::EpiStoreF32, false, true>(mDz_k, mW_mn, gemm_shape(N, D, clen), e2,
+                                                   &hdr->status, pairs, st);
+    if (s != FLCE_OK) return s;
     // K3: dW_C = dZ_C^T H
     bwd::EpiStoreF32 e3;
     e3.out = dW;
@@ -612,8 +593,9 @@ extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t
     e3.cols = int32_t(D);
     e3.row_base = int32_t(c0);
     e3.accumulate = 0;
-    if ((s = launch_gemm(mDzt, mHt, gemm_shape(clen, D, N), e3, &hdr->status, pairs, st)) != FLCE_OK)
-      return s;
+    s = launch_gemm<bwd::EpiStoreF32, true, true>(mDz_mn, mH_mn, gemm_shape(clen, D, N), e3,
+                                                  &hdr->status, pairs, st);
+    if (s != FLCE_OK) return s;
   }
   return FLCE_OK;
 }

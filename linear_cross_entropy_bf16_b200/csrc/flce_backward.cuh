@@ -8,13 +8,17 @@
 // and regenerates the logits tile by tile, one vocabulary chunk at a time, so
 // only an (N x chunk) slice of dZ ever exists.  Per chunk C of W's rows:
 //   K1  Z_C = H W_C^T on the tensor cores; the epilogue turns each tile into
-//       dZ_C (bf16) and writes it twice, token-major and vocab-major;
-//   K2  dH (+)= dZ_C W_C           (A = dZ_C, B = (W^T)_C: both K-major)
-//   K3  dW_C  = dZ_C^T H           (A = dZ_C^T, B = H^T: both K-major)
-// All three are one CTA-pair GEMM kernel (C = A B^T with A, B K-major,
-// 256 x 256 pair tiles, 6-stage TMA ring, double-buffered TMEM accumulators)
-// with different epilogues.  W^T and H^T are written once per call by a
-// tiled transpose so that every operand is K-major.
+//       dZ_C (bf16, token-major);
+//   K2  dH (+)= dZ_C W_C     A = dZ_C (K = vocab, contiguous: K-major),
+//                            B = W_C read as (d, vocab) with d contiguous
+//                            (MN-major);
+//   K3  dW_C  = dZ_C^T H     A = dZ_C read as (vocab, token) with vocab
+//                            contiguous (MN-major), B = H read as (d, token)
+//                            with d contiguous (MN-major).
+// All three are one CTA-pair GEMM kernel (C = A B^T, 256 x 256 pair tiles,
+// 6-stage TMA ring, double-buffered TMEM accumulators) with different
+// epilogues and operand orders; the tensor cores read MN-major operands
+// directly, so nothing is transposed in memory.
 #pragma once
 
 #include <cstdint>
@@ -26,31 +30,6 @@
 
 namespace flce {
 namespace bwd {
-
-// ----------------------------------------------------------------- transpose
-
-constexpr int kTrTile = 64;
-
-// out[c][r] = in[r][c] for a (rows x cols) bf16 matrix with row stride ld_in;
-// out has row stride ld_out.  Columns of out past `rows` are not written.
-__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16* __restrict__ in,
-                                                             int64_t rows, int64_t cols,
-                                                             int64_t ld_in,
-                                                             __nv_bfloat16* __restrict__ out,
-                                                             int64_t ld_out) {
-  __shared__ __nv_bfloat16 tile[kTrTile][kTrTile + 2];
-  const int64_t r0 = int64_t(blockIdx.x) * kTrTile, c0 = int64_t(blockIdx.y) * kTrTile;
-  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 x 4 threads
-  for (int r = ty; r < kTrTile; r += 4) {
-    const int64_t gr = r0 + r, gc = c0 + tx;
-    tile[r][tx] = (gr < rows && gc < cols) ? in[gr * ld_in + gc] : __float2bfloat16(0.f);
-  }
-  __syncthreads();
-  for (int c = ty; c < kTrTile; c += 4) {
-    const int64_t gc = c0 + c, gr = r0 + tx;
-    if (gc < cols && gr < rows) out[gc * ld_out + gr] = tile[tx][c];
-  }
-}
 
 // ----------------------------------------------------------------- tile schedule
 
@@ -92,8 +71,6 @@ struct EpiGradLogits {
   int32_t clen;              // vocabulary rows in this chunk
   __nv_bfloat16* dz;         // (N x ldz) token-major slice, columns = chunk vocab
   int32_t ldz;
-  __nv_bfloat16* dzt;        // (clen x ldzt) vocab-major slice, columns = tokens
-  int32_t ldzt;
   uint32_t* status;
 
   __device__ __forceinline__ void operator()(int row, int n0, uint32_t taddr) const {
@@ -137,11 +114,6 @@ struct EpiGradLogits {
         for (int j = 0; j < 32; ++j)
           if (col0 + j < clen) dst[j] = __float2bfloat16_rn(d[j]);
       }
-      // vocab-major: lanes hold consecutive tokens, so each column is one
-      // coalesced 64-byte row segment of dZ^T
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (col0 + j < clen) dzt[size_t(col0 + j) * size_t(ldzt) + row] = __float2bfloat16_rn(d[j]);
     }
   }
 };
@@ -207,18 +179,33 @@ constexpr int EPI_WARPS = 4;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr uint16_t kPairMask = 0x3;
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
-                            (uint32_t(PAIR_M >> 4) << 24);
+constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
+                                (uint32_t(PAIR_M >> 4) << 24);
+constexpr int MN_CHUNK = 64;                 // MN elements per 128-byte swizzle row
+constexpr int MN_BOX_BYTES = MN_CHUNK * BK * 2;  // one 64 (MN) x 64 (K) box: 8 KiB
+
+// Shared-memory descriptor of an MN-major operand staged as 64 (MN) x 64 (K)
+// TMA boxes with 128-byte swizzling: each K row holds 64 MN elements (128 B),
+// 8-row K groups are 1024 B apart (stride byte offset) and consecutive
+// 64-element MN chunks are one box, 8 KiB, apart (leading byte offset).  One
+// K = 16 step of the MMA covers 16 rows, i.e. +2048 B.
+__device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t addr) {
+  return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t(MN_BOX_BYTES >> 4) << 16) |
+         (uint64_t(1024 >> 4) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
 
 // C = A B^T on CTA pairs, C tiles handed to `epi`.  Same pipeline and
 // barrier protocol as the forward's pair kernel (see tc2::flce_tc2_kernel):
 // warp 0 of each CTA streams its A rows and its half of the B rows by TMA,
 // warp 1 of the even CTA issues the pair MMAs, warps 2-5 of both CTAs run the
 // epilogue on their own TMEM rows.  Bounded waits throughout.
-template <class Epi>
+// kAmn / kBmn: the operand is MN-major (its tensor map's inner dimension is
+// M resp. N, the outer one K); otherwise K-major (inner dimension K).
+template <class Epi, bool kAmn, bool kBmn>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const GemmShape shape, const Epi epi, uint32_t* status, uint64_t wait_limit_ns) {
+  constexpr uint32_t kIdesc = kIdescBase | (kAmn ? (1u << 15) : 0u) | (kBmn ? (1u << 16) : 0u);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -284,8 +271,19 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           const uint32_t fb_even = ptx::map_to_cta(fb_local, 0);
           const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
           if (rank == 0) ptx::mbar_arrive_expect_tx(fb_local, PAIR_TX_BYTES);
-          ptx::tma_load_2d_pair(sa, &tmA, fb_even, kb * BK, arow);
-          ptx::tma_load_2d_pair(sa + A_BYTES, &tmB, fb_even, kb * BK, brow);
+          if (kAmn) {  // two 64 (M) x 64 (K) boxes
+            ptx::tma_load_2d_pair(sa, &tmA, fb_even, arow, kb * BK);
+            ptx::tma_load_2d_pair(sa + MN_BOX_BYTES, &tmA, fb_even, arow + MN_CHUNK, kb * BK);
+          } else {     // one 64 (K) x 128 (M) box
+            ptx::tma_load_2d_pair(sa, &tmA, fb_even, kb * BK, arow);
+          }
+          if (kBmn) {
+            ptx::tma_load_2d_pair(sa + A_BYTES, &tmB, fb_even, brow, kb * BK);
+            ptx::tma_load_2d_pair(sa + A_BYTES + MN_BOX_BYTES, &tmB, fb_even, brow + MN_CHUNK,
+                                  kb * BK);
+          } else {
+            ptx::tma_load_2d_pair(sa + A_BYTES, &tmB, fb_even, kb * BK, brow);
+          }
           used |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -324,8 +322,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
-            const uint64_t ad = tc::sw128_desc(sa + k * UMMA_K * 2);
-            const uint64_t bd = tc::sw128_desc(sa + A_BYTES + k * UMMA_K * 2);
+            // K-major: +32 B along the 128-byte row; MN-major: +16 rows of 128 B
+            const uint64_t ad = kAmn ? sw128_desc_mn(sa + k * UMMA_K * 128)
+                                     : tc::sw128_desc(sa + k * UMMA_K * 2);
+            const uint64_t bd = kBmn ? sw128_desc_mn(sa + A_BYTES + k * UMMA_K * 128)
+                                     : tc::sw128_desc(sa + A_BYTES + k * UMMA_K * 2);
             ptx::mma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
           }
           ptx::mma_commit_pair_mc(ptx::smem_addr(&empty_bar[stage]), kPairMask);
