@@ -70,6 +70,9 @@ def _load():
             lib.oracle_grad_logits_row.argtypes = [vp, vp, ctypes.c_int, vp, ctypes.c_double,
                                                    i64, i64, i64, dp]
             lib.oracle_grad_logits_row.restype = ctypes.c_int
+            lib.oracle_grad_hidden_rows.argtypes = [vp, vp, ctypes.c_int, vp, dp, i64, i64, i64,
+                                                    vp, i64, dp, dp, ctypes.c_int]
+            lib.oracle_grad_hidden_rows.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -187,3 +190,22 @@ def grad_logits_row(H: np.ndarray, W: np.ndarray, y: np.ndarray, g_i: float, i: 
     if rc != 0:
         raise OracleError(_ERRORS.get(rc, f"oracle error {rc}"))
     return dz
+
+
+def grad_hidden_rows(H: np.ndarray, W: np.ndarray, y: np.ndarray, g, rows, nthreads: int = 0):
+    """dH (and its magnitude bound bH) for the selected rows only."""
+    lib = _load()
+    H, dt = _as_storage(H)
+    W, _ = _as_storage(W)
+    N, D = H.shape
+    V = W.shape[0]
+    y = np.ascontiguousarray(y, dtype=np.int64)
+    gv = np.ascontiguousarray(np.broadcast_to(np.asarray(g, dtype=np.float64), (N,)))
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    dH = np.empty((rows.shape[0], D))
+    bH = np.empty((rows.shape[0], D))
+    rc = lib.oracle_grad_hidden_rows(_ptr(H), _ptr(W), dt, _ptr(y), _ptr(gv), N, V, D, _ptr(rows),
+                                     rows.shape[0], _ptr(dH), _ptr(bH), int(nthreads))
+    if rc != 0:
+        raise OracleError(_ERRORS.get(rc, f"oracle error {rc}"))
+    return {"dH": dH, "bH": bH}

@@ -247,6 +247,61 @@ int oracle_backward(const void *H, const void *W, int dtype, const int64_t *y,
     return status;
 }
 
+/* dH rows only (rows[t], t < nrows), with their magnitudes bH: row i of dH
+ * depends on row i of the logits alone, so this is cheap for a row sample.
+ * Same arithmetic as pass 1 of oracle_backward.  g is indexed by token. */
+int oracle_grad_hidden_rows(const void *H, const void *W, int dtype, const int64_t *y,
+                            const double *g, int64_t N, int64_t V, int64_t D, const int64_t *rows,
+                            int64_t nrows, double *dH, double *bH, int nthreads) {
+    if (!H || !W || !y || !g || !rows || !dH || N < 1 || V < 1 || D < 1 || nrows < 0)
+        return ORACLE_ERR_ARG;
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP32 && dtype != ORACLE_FP64) return ORACLE_ERR_ARG;
+    for (int64_t t = 0; t < nrows; ++t) {
+        if (rows[t] < 0 || rows[t] >= N) return ORACLE_ERR_ARG;
+        if (y[rows[t]] < 0 || y[rows[t]] >= V) return ORACLE_ERR_TARGET;
+    }
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int status = ORACLE_OK;
+#pragma omp parallel
+    {
+        double *z = (double *)malloc((size_t)V * sizeof(double));
+        if (!z) {
+#pragma omp atomic write
+            status = ORACLE_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < nrows; ++t) {
+            if (!z) continue;
+            const int64_t i = rows[t];
+            for (int64_t j = 0; j < V; ++j) z[j] = logit(H, W, dtype, i, j, D);
+            double M = z[0];
+            for (int64_t j = 1; j < V; ++j)
+                if (z[j] > M) M = z[j];
+            double S = 0.0;
+            for (int64_t j = 0; j < V; ++j) S += exp(z[j] - M);
+            const double lse = M + log(S);
+            for (int64_t j = 0; j < V; ++j)
+                z[j] = g[i] * (exp(z[j] - lse) - (j == y[i] ? 1.0 : 0.0));
+            for (int64_t k = 0; k < D; ++k) {
+                double acc = 0.0, mag = 0.0;
+                for (int64_t j = 0; j < V; ++j) {
+                    double w = load_elem(W, dtype, j * D + k);
+                    acc += z[j] * w;
+                    mag += fabs(z[j]) * fabs(w);
+                }
+                dH[t * D + k] = acc;
+                if (bH) bH[t * D + k] = mag;
+            }
+        }
+        free(z);
+    }
+    return status;
+}
+
 /* dL/dZ for one row i (V values), given upstream gradient g_i: the vector the
  * backward contracts with W and H.  For tests of the gradient definition. */
 int oracle_grad_logits_row(const void *H, const void *W, int dtype, const int64_t *y, double g_i,

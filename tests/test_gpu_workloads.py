@@ -58,3 +58,47 @@ def test_large_workload_sampled_rows(name):
     rows = synth.sample_rows(w.N, SAMPLE_ROWS, w.seed)
     ref = oracle.forward(H, W, y, rows=rows)
     compare(gpu, ref, rows=rows)
+
+
+# ----------------------------------------------------------------------------- backward
+
+def _backward(name, N=None, V=None, D=None):
+    """dH and dW of the mean loss (device tensors), after checking bitwise repeatability."""
+    import linear_cross_entropy_bf16_b200 as flce
+    H, W, y = synth.generate(name, N=N, V=V, D=D)
+    Hd, Wd, yd = to_device(H, W, y)
+    _, lse, _, _ = flce.forward(Hd, Wd, yd, check=True)
+    n = H.shape[0]
+    dH, dW = flce.backward(Hd, Wd, yd, lse, None, 1.0 / n, check=True)
+    again = flce.backward(Hd, Wd, yd, lse, None, 1.0 / n)
+    assert torch.equal(dH, again[0]) and torch.equal(dW, again[1])
+    return H, W, y, dH, dW
+
+
+def _within(got, ref, bound):
+    err = np.abs(got - ref)
+    assert np.all(err <= 2.0 ** -8 * bound + 1e-7), float((err - 2.0 ** -8 * bound).max())
+
+
+def test_backward_workload_n1024_every_element():
+    """The N=1024, V=32000, D=1024 workload: every element of dH and dW (mean loss)."""
+    H, W, y, dH, dW = _backward("n1024_v32000_d1024")
+    g = np.float64(np.float32(1.0 / H.shape[0]))
+    ref = oracle.backward(H, W, y, g, bounds=True)
+    _within(dH.cpu().double().numpy(), ref["dH"], ref["bH"])
+    _within(dW.cpu().double().numpy(), ref["dW"], ref["bW"])
+
+
+def test_backward_headline_sampled_rows_and_properties():
+    """The page's shape: sampled dH rows against the oracle; dW by its exact zero-sum."""
+    H, W, y, dH, dW = _backward(synth.HEADLINE)
+    w = synth.WORKLOADS[synth.HEADLINE]
+    assert bool(torch.isfinite(dH).all()) and bool(torch.isfinite(dW).all())
+    rows = synth.sample_rows(w.N, 16, w.seed)
+    ref = oracle.grad_hidden_rows(H, W, y, np.float64(np.float32(1.0 / w.N)), rows)
+    _within(dH[torch.from_numpy(rows).cuda()].cpu().double().numpy(), ref["dH"], ref["bH"])
+    # sum_j dL/dZ_ij = 0 exactly, so the vocabulary rows of dW sum to zero up to the
+    # bf16 rounding of dZ (relative 2^-9 per term); reduced on the device in fp64
+    colsum = dW.double().sum(dim=0).abs().max().item()
+    scale = dW.double().abs().sum(dim=0).max().item()
+    assert colsum <= 2.0 ** -8 * scale

@@ -147,3 +147,13 @@ def test_gradient_is_linear_in_g(oracle_mod):
     c = oracle_mod.backward(H, W, y, 2 * g1 - g2)
     np.testing.assert_allclose(c["dH"], 2 * a["dH"] - b["dH"], rtol=1e-11, atol=1e-13)
     np.testing.assert_allclose(c["dW"], 2 * a["dW"] - b["dW"], rtol=1e-11, atol=1e-13)
+
+
+def test_hidden_rows_match_full_backward(oracle_mod):
+    H, W, y = synth.random_inputs(40, 300, 24, seed=38)
+    g = np.random.default_rng(39).uniform(-1, 1, 40)
+    full = oracle_mod.backward(H, W, y, g, bounds=True, want_dW=False)
+    rows = np.array([39, 0, 7, 7])
+    sub = oracle_mod.grad_hidden_rows(H, W, y, g, rows)
+    np.testing.assert_array_equal(sub["dH"], full["dH"][rows])
+    np.testing.assert_array_equal(sub["bH"], full["bH"][rows])
