@@ -182,6 +182,53 @@ FLCE_API flce_status flce_backward(const void* H, const void* W, const int64_t* 
                                    float* dW, void* workspace, size_t workspace_bytes,
                                    void* stream);
 
+/*
+ * Vocabulary-parallel forward (W split by rows over G ranks or devices).
+ * The recurrence of section 1 of the page is associative over any split of
+ * the vocabulary, so each shard can fold its own columns and the shards'
+ * states merge exactly like the tiles of one device:
+ *   1. each shard r: flce_partials_shard on its rows W[v_offset, v_offset + V_shard)
+ *      (y holds global vocabulary ids), then flce_shard_state -> one
+ *      {m, s, target logit, owned} float4 per token;
+ *   2. gather the G state arrays in shard order (e.g. one all-gather of
+ *      16 N bytes per rank);
+ *   3. flce_merge_shards -> loss, lse, target logit and mean for the whole
+ *      vocabulary.
+ * Workspaces and scratch are caller-owned device memory, as elsewhere.
+ */
+
+/* flce_partials on the vocabulary shard W_shard = W[v_offset, v_offset +
+ * V_shard): writes the target logit only for rows whose target lies in the
+ * shard; other rows of out_target_logit are left as they were.  Sizes and
+ * workspace as for flce_partials with V = V_shard; v_offset >= 0. */
+FLCE_API flce_status flce_partials_shard(const void* H, const void* W_shard, const int64_t* y,
+                                         int64_t N, int64_t V_shard, int64_t v_offset, int64_t D,
+                                         flce_dtype dtype, float* out_target_logit, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+
+/* After flce_partials_shard on `workspace`: out_state (N float4, 16-byte
+ * aligned) = {m, s, target logit, owned} per token, where (m, s) folds the
+ * shard's slab states and owned = 1 iff v_offset <= y_i < v_offset + V_shard
+ * (target is then the shard's target logit, else 0). */
+FLCE_API flce_status flce_shard_state(const int64_t* y, int64_t N, int64_t V_shard,
+                                      int64_t v_offset, const float* target_logit,
+                                      const void* workspace, size_t workspace_bytes,
+                                      float* out_state, void* stream);
+
+/* Bytes of scratch flce_merge_shards needs: 256 + 8 ceil(N / 256), rounded. */
+FLCE_API size_t flce_merge_shards_scratch_size(int64_t N);
+
+/* Merges G shard states, laid out [G][N] float4 in shard order (any order
+ * gives the same lse up to rounding; a fixed order makes it deterministic),
+ * into per-token loss, lse and target logit and the mean (out_mean may be
+ * NULL).  A token whose target is outside [0, V_total) or is held by no
+ * shard or by more than one gets NaN and sets FLCE_ERR_TARGET_OUT_OF_RANGE
+ * in the scratch status word (read with flce_check(scratch, stream)). */
+FLCE_API flce_status flce_merge_shards(const float* states, int32_t G, const int64_t* y, int64_t N,
+                                       int64_t V_total, float* out_loss, float* out_lse,
+                                       float* out_target_logit, float* out_mean, void* scratch,
+                                       size_t scratch_bytes, void* stream);
+
 /* Waits for `stream`, then reads the workspace status word left by the last
  * flce_forward / flce_partials + flce_merge that used this workspace.
  * Returns FLCE_OK, FLCE_ERR_TARGET_OUT_OF_RANGE, FLCE_ERR_TIMEOUT,

@@ -23,6 +23,7 @@ import torch
 
 __all__ = [
     "FlceError", "forward", "backward", "partials", "merge", "workspace_size",
+    "shard_state", "merge_shards", "forward_vocab_parallel",
     "backward_workspace_size", "plan", "check",
     "status_string", "selftest_wait_timeout", "library_path", "load_library",
 ]
@@ -106,6 +107,14 @@ def load_library():
         lib.flce_backward.argtypes = [vp, vp, vp, vp, vp, ctypes.c_float, i64, i64, i64,
                                       ctypes.c_int, vp, vp, vp, sz, vp]
         lib.flce_backward.restype = st
+        lib.flce_partials_shard.argtypes = [vp, vp, vp, i64, i64, i64, i64, ctypes.c_int, vp, vp, sz, vp]
+        lib.flce_partials_shard.restype = st
+        lib.flce_shard_state.argtypes = [vp, i64, i64, i64, vp, vp, sz, vp, vp]
+        lib.flce_shard_state.restype = st
+        lib.flce_merge_shards_scratch_size.argtypes = [i64]
+        lib.flce_merge_shards_scratch_size.restype = sz
+        lib.flce_merge_shards.argtypes = [vp, ctypes.c_int32, vp, i64, i64, vp, vp, vp, vp, vp, sz, vp]
+        lib.flce_merge_shards.restype = st
         _lib = lib
         return lib
 
@@ -271,6 +280,78 @@ def backward(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, lse: torch.Tenso
     if check:
         _raise_on(lib.flce_check(workspace.data_ptr(), sp), "flce_backward (device)")
     return dH, dW
+
+
+def shard_state(H: torch.Tensor, W_shard: torch.Tensor, y: torch.Tensor, v_offset: int, *,
+                workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """This vocabulary shard's per-token state (N, 4) fp32 {m, s, target logit, owned}.
+
+    W_shard holds rows [v_offset, v_offset + V_shard) of the full W; y holds
+    global vocabulary ids.  Steps 1 of the vocabulary-parallel forward
+    (flce_partials_shard, then flce_shard_state).
+    """
+    N, Vs, D, code = _check_inputs(H, W_shard, y)
+    dev = H.device
+    state = torch.zeros(N, 4, dtype=torch.float32, device=dev)
+    if N == 0:
+        return state
+    ws = _workspace(N, Vs, D, code, dev, workspace)
+    wsb = ws.numel() * ws.element_size()
+    tgt = torch.zeros(N, dtype=torch.float32, device=dev)
+    sp = _stream_ptr(stream, dev)
+    lib = load_library()
+    _raise_on(lib.flce_partials_shard(H.data_ptr(), W_shard.data_ptr(), y.data_ptr(), N, Vs,
+                                      int(v_offset), D, code, tgt.data_ptr(), ws.data_ptr(), wsb, sp),
+              "flce_partials_shard")
+    _raise_on(lib.flce_shard_state(y.data_ptr(), N, Vs, int(v_offset), tgt.data_ptr(),
+                                   ws.data_ptr(), wsb, state.data_ptr(), sp), "flce_shard_state")
+    return state
+
+
+def merge_shards(states: torch.Tensor, y: torch.Tensor, V_total: int, *, stream=None,
+                 check: bool = False):
+    """Merge (G, N, 4) shard states (in shard order) into (loss, lse, target_logit, mean)."""
+    if states.dim() != 3 or states.shape[2] != 4 or states.dtype != torch.float32 or not states.is_contiguous():
+        raise ValueError("states must be a contiguous float32 (G, N, 4) tensor")
+    G, N = states.shape[0], states.shape[1]
+    dev = states.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    loss, lse, tgt = (torch.empty(N, **f32) for _ in range(3))
+    mean = torch.full((), float("nan"), **f32)
+    if N == 0:
+        return loss, lse, tgt, mean
+    lib = load_library()
+    scratch = torch.empty(lib.flce_merge_shards_scratch_size(N), dtype=torch.uint8, device=dev)
+    sp = _stream_ptr(stream, dev)
+    _raise_on(lib.flce_merge_shards(states.data_ptr(), G, y.data_ptr(), N, int(V_total),
+                                    loss.data_ptr(), lse.data_ptr(), tgt.data_ptr(), mean.data_ptr(),
+                                    scratch.data_ptr(), scratch.numel(), sp), "flce_merge_shards")
+    if check:
+        _raise_on(lib.flce_check(scratch.data_ptr(), sp), "flce_merge_shards (device)")
+    return loss, lse, tgt, mean
+
+
+def forward_vocab_parallel(H: torch.Tensor, W_shard: torch.Tensor, y: torch.Tensor, v_offset: int,
+                           V_total: int, group=None, check: bool = False):
+    """Vocabulary-parallel forward: this rank holds W rows [v_offset, v_offset + V_shard).
+
+    Every rank of `group` passes the same H and y.  The only exchange is one
+    all-gather of the (N, 4) shard states over torch.distributed (NCCL on
+    GPUs); shards must be ordered by rank.  Returns (loss, lse, target_logit,
+    mean) for the full vocabulary on every rank.
+    """
+    import torch.distributed as dist
+    state = shard_state(H, W_shard, y, v_offset)
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    if world > 1:
+        # concatenated along dim 0 (accepted by every backend), then viewed as (G, N, 4)
+        flat = torch.empty((world * state.shape[0],) + tuple(state.shape[1:]), dtype=state.dtype,
+                           device=state.device)
+        dist.all_gather_into_tensor(flat, state, group=group)
+        gathered = flat.view((world,) + tuple(state.shape))
+    else:
+        gathered = state.unsqueeze(0)
+    return merge_shards(gathered, y, V_total, check=check)
 
 
 def partials(H, W, y, target_logit, workspace, stream=None):

@@ -252,9 +252,9 @@ flce_status check_forward_args(const void* H, const void* W, const int64_t* y, i
   return FLCE_OK;
 }
 
-flce_status launch_partials(const void* H, const void* W, const int64_t* y, int64_t N, int64_t V,
-                            int64_t D, flce_dtype dtype, float* out_target, void* ws,
-                            cudaStream_t st) {
+flce_status launch_partials(const void* H, const void* W, const int64_t* y, int64_t y_offset,
+                            int64_t N, int64_t V, int64_t D, flce_dtype dtype, float* out_target,
+                            void* ws, cudaStream_t st) {
   DeviceInfo di;
   flce_status s = device_info(di);
   if (s != FLCE_OK) return s;
@@ -290,6 +290,7 @@ flce_status launch_partials(const void* H, const void* W, const int64_t* y, int6
       return FLCE_ERR_UNSUPPORTED;
     tc::Args a;
     a.y = y;
+    a.y_offset = y_offset;
     a.part = part;
     a.target_logit = out_target;
     a.hdr = hdr;
@@ -308,6 +309,7 @@ flce_status launch_partials(const void* H, const void* W, const int64_t* y, int6
     a.H = H;
     a.W = W;
     a.y = y;
+    a.y_offset = y_offset;
     a.part = part;
     a.target_logit = out_target;
     a.hdr = hdr;
@@ -364,7 +366,7 @@ flce_status flce_partials(const void* H, const void* W, const int64_t* y, int64_
   flce_status s = check_forward_args(H, W, y, N, V, D, dtype, workspace, workspace_bytes);
   if (s != FLCE_OK || N == 0) return s;
   if (!out_target_logit) return FLCE_ERR_INVALID_ARG;
-  return launch_partials(H, W, y, N, V, D, dtype, out_target_logit, workspace,
+  return launch_partials(H, W, y, 0, N, V, D, dtype, out_target_logit, workspace,
                          static_cast<cudaStream_t>(stream));
 }
 
@@ -389,10 +391,72 @@ flce_status flce_forward(const void* H, const void* W, const int64_t* y, int64_t
   if (s != FLCE_OK || N == 0) return s;
   if (!out_loss || !out_lse || !out_target_logit) return FLCE_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = launch_partials(H, W, y, N, V, D, dtype, out_target_logit, workspace, st);
+  s = launch_partials(H, W, y, 0, N, V, D, dtype, out_target_logit, workspace, st);
   if (s != FLCE_OK) return s;
   return launch_merge(y, N, V, out_loss, out_lse, out_target_logit, out_mean, workspace,
                       workspace_bytes, st);
+}
+
+flce_status flce_partials_shard(const void* H, const void* W_shard, const int64_t* y, int64_t N,
+                                int64_t V_shard, int64_t v_offset, int64_t D, flce_dtype dtype,
+                                float* out_target_logit, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  if (v_offset < 0) return FLCE_ERR_INVALID_ARG;
+  flce_status s =
+      check_forward_args(H, W_shard, y, N, V_shard, D, dtype, workspace, workspace_bytes);
+  if (s != FLCE_OK || N == 0) return s;
+  if (!out_target_logit) return FLCE_ERR_INVALID_ARG;
+  return launch_partials(H, W_shard, y, v_offset, N, V_shard, D, dtype, out_target_logit,
+                         workspace, static_cast<cudaStream_t>(stream));
+}
+
+flce_status flce_shard_state(const int64_t* y, int64_t N, int64_t V_shard, int64_t v_offset,
+                             const float* target_logit, const void* workspace,
+                             size_t workspace_bytes, float* out_state, void* stream) {
+  if (N < 0 || V_shard < 1 || v_offset < 0) return FLCE_ERR_INVALID_ARG;
+  if (N == 0) return FLCE_OK;
+  if (!y || !target_logit || !workspace || !out_state) return FLCE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      (reinterpret_cast<uintptr_t>(out_state) & 15u) != 0)
+    return FLCE_ERR_INVALID_ARG;
+  if (N >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
+  if (workspace_bytes < workspace_bytes_for(N, V_shard)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  const uint8_t* wsb = static_cast<const uint8_t*>(workspace);
+  const WsHeader* hdr = reinterpret_cast<const WsHeader*>(wsb);
+  flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0,
+                            static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const float2*>(wsb + kHeaderBytes), hdr, y, int32_t(N), v_offset, V_shard,
+      int32_t(slab_capacity(V_shard)), target_logit, reinterpret_cast<float4*>(out_state),
+      const_cast<uint32_t*>(&hdr->status));
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+size_t flce_merge_shards_scratch_size(int64_t N) {
+  if (N < 0) return 0;
+  return kHeaderBytes + align256(size_t(8) * size_t(std::max<int64_t>(1, cdiv(N, kMergeThreads))));
+}
+
+flce_status flce_merge_shards(const float* states, int32_t G, const int64_t* y, int64_t N,
+                              int64_t V_total, float* out_loss, float* out_lse,
+                              float* out_target_logit, float* out_mean, void* scratch,
+                              size_t scratch_bytes, void* stream) {
+  if (G < 1 || N < 0 || V_total < 1) return FLCE_ERR_INVALID_ARG;
+  if (N == 0) return FLCE_OK;
+  if (!states || !y || !out_loss || !out_lse || !out_target_logit || !scratch)
+    return FLCE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0 ||
+      (reinterpret_cast<uintptr_t>(states) & 15u) != 0)
+    return FLCE_ERR_INVALID_ARG;
+  if (N >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
+  if (scratch_bytes < flce_merge_shards_scratch_size(N)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* sb = static_cast<uint8_t*>(scratch);
+  if (cudaMemsetAsync(sb, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
+  flce_merge_shards_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
+      reinterpret_cast<const float4*>(states), G, y, int32_t(N), V_total, out_loss, out_lse,
+      out_target_logit, out_mean, reinterpret_cast<double*>(sb + kHeaderBytes),
+      reinterpret_cast<WsHeader*>(sb));
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
 flce_status flce_check(const void* workspace, void* stream) {

@@ -219,6 +219,7 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
 
 struct Args {
   const int64_t* y;
+  int64_t y_offset;        // first vocabulary id of W's rows (a vocabulary shard); 0 otherwise
   float2* part;            // [P][N] (m, s) per slab and token
   float* target_logit;     // [N]
   WsHeader* hdr;
@@ -380,7 +381,7 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
       unit_coords(sch, u, slab, tb, t0, nt);
       const int row = tb * BM + row_in_tile;
       const bool valid = row < a.N;
-      const int64_t yi = valid ? a.y[row] : -1;
+      const int64_t yi = valid ? a.y[row] - a.y_offset : -1;  // target column within W
       float m = -INFINITY, s = 0.f, zt = 0.f;
       bool got = false;
       for (int t = t0; t < t0 + nt; ++t) {
@@ -613,7 +614,7 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
       unit_coords(sch, u, slab, tb, t0, nt);
       const int row = tb * PAIR_M + int(rank) * BM + row_in_tile;
       const bool valid = row < a.N;
-      const int64_t yi = valid ? a.y[row] : -1;
+      const int64_t yi = valid ? a.y[row] - a.y_offset : -1;  // target column within W
       float m = -INFINITY, s = 0.f, zt = 0.f;
       bool got = false;
       for (int t = t0; t < t0 + nt; ++t) {
@@ -678,6 +679,7 @@ struct Args {
   const void* H;
   const void* W;
   const int64_t* y;
+  int64_t y_offset;
   float2* part;
   float* target_logit;
   WsHeader* hdr;
@@ -719,7 +721,7 @@ __global__ void __launch_bounds__(NUM_THREADS) flce_simt_kernel(const Args a) {
     zt[i] = 0.f;
     got[i] = false;
     const int r = row0 + ty * 4 + i;
-    yrow[i] = r < a.N ? a.y[r] : -1;
+    yrow[i] = r < a.N ? a.y[r] - a.y_offset : -1;
   }
 
   const int c_begin = t0 * kTileCols;
@@ -878,6 +880,101 @@ __global__ void __launch_bounds__(kMergeThreads) flce_merge_kernel(const MergeAr
     for (int b = 0; b < int(gridDim.x); ++b) total += bs[b];
     *a.mean = float(total / double(a.N));
     a.hdr->counter = 0;
+  }
+}
+
+// ----------------------------------------------------------------- vocabulary shards
+
+// One vocabulary shard's contribution per token, after flce_partials on the
+// shard: its slab states folded into one (m, s) (the section-1 recurrence
+// over slabs), the target logit if the shard holds the target, and 1/0 for
+// "holds it".  Layout: float4 {m, s, target, owned}.
+__global__ void __launch_bounds__(kMergeThreads) flce_shard_state_kernel(
+    const float2* part, const WsHeader* hdr, const int64_t* y, int32_t N, int64_t v_offset,
+    int64_t v_count, int32_t max_slabs, const float* target_logit, float4* out,
+    uint32_t* status) {
+  const int i = blockIdx.x * kMergeThreads + threadIdx.x;
+  if (i >= N) return;
+  const WsHeader h = *hdr;
+  float4 r;
+  if (h.magic != kWsMagic || h.N != N || h.V != v_count || h.slabs < 1 || h.slabs > max_slabs) {
+    r = make_float4(__int_as_float(0x7fc00000), 0.f, 0.f, 0.f);
+    if (i == 0) atomicOr(status, kStatBadWs);
+  } else {
+    float M = -INFINITY;
+    for (int p = 0; p < h.slabs; ++p) M = fmaxf(M, part[size_t(p) * N + i].x);
+    double S = 0.0;
+    for (int p = 0; p < h.slabs; ++p) {
+      const float2 st = part[size_t(p) * N + i];
+      S += double(st.y) * exp(double(st.x) - double(M));
+    }
+    const int64_t rel = y[i] - v_offset;
+    const bool owned = rel >= 0 && rel < v_count;
+    r = make_float4(M, float(S), owned ? target_logit[i] : 0.f, owned ? 1.f : 0.f);
+  }
+  out[i] = r;
+}
+
+// Combines the per-token states of G shards (in shard order): m = max_r m_r,
+// s = sum_r s_r exp(m_r - m), lse = m + log s; the target logit comes from
+// the shard that holds it (exactly one for a valid target); loss = lse -
+// target; mean as in flce_merge_kernel.
+__global__ void __launch_bounds__(kMergeThreads) flce_merge_shards_kernel(
+    const float4* states, int32_t G, const int64_t* y, int32_t N, int64_t V_total, float* loss,
+    float* lse, float* target_logit, float* mean, double* block_sums, WsHeader* hdr) {
+  __shared__ double warp_sums[kMergeThreads / 32];
+  __shared__ bool is_last;
+  const int i = blockIdx.x * kMergeThreads + threadIdx.x;
+  double l = 0.0;
+  if (i < N) {
+    float M = -INFINITY;
+    for (int r = 0; r < G; ++r) M = fmaxf(M, states[size_t(r) * N + i].x);
+    double S = 0.0;
+    float t = 0.f;
+    int owners = 0;
+    for (int r = 0; r < G; ++r) {
+      const float4 st = states[size_t(r) * N + i];
+      S += double(st.y) * exp(double(st.x) - double(M));
+      if (st.w != 0.f) {
+        t = st.z;
+        ++owners;
+      }
+    }
+    const double lse_d = double(M) + log(S);
+    const int64_t yi = y[i];
+    float loss_f;
+    if (yi < 0 || yi >= V_total || owners != 1) {
+      loss_f = t = __int_as_float(0x7fc00000);
+      atomicOr(&hdr->status, kStatTarget);
+    } else {
+      loss_f = float(lse_d - double(t));
+    }
+    loss[i] = loss_f;
+    lse[i] = float(lse_d);
+    target_logit[i] = t;
+    l = double(loss_f);
+  }
+  if (mean == nullptr) return;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) l += __shfl_down_sync(0xffffffffu, l, off);
+  if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = l;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double b = 0.0;
+    for (int w = 0; w < kMergeThreads / 32; ++w) b += warp_sums[w];
+    block_sums[blockIdx.x] = b;
+    __threadfence();
+    const uint32_t ticket = atomicAdd(&hdr->counter, 1u);
+    is_last = ticket == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (is_last && threadIdx.x == 0) {
+    __threadfence();
+    const volatile double* bs = block_sums;
+    double total = 0.0;
+    for (int b = 0; b < int(gridDim.x); ++b) total += bs[b];
+    *mean = float(total / double(N));
+    hdr->counter = 0;
   }
 }
 

@@ -1,0 +1,67 @@
+"""Vocabulary-parallel forward on one GPU: G shards run one after another and
+their per-token states are merged, as the ranks of a real run would after
+their all-gather.  Checked against the fp64 oracle on every row."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_cross_entropy_bf16_b200 import synth
+from tests.flce_testing import compare, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from linear_cross_entropy_bf16_b200 import build
+    build.build()
+    oracle.build()
+
+
+def sharded_forward(Hd, Wd, yd, bounds):
+    import linear_cross_entropy_bf16_b200 as flce
+    states = [flce.shard_state(Hd, Wd[a:b].contiguous(), yd, a) for a, b in zip(bounds[:-1], bounds[1:])]
+    loss, lse, tgt, mean = flce.merge_shards(torch.stack(states).contiguous(), yd, Wd.shape[0], check=True)
+    torch.cuda.synchronize()
+    return {"loss": loss.cpu().double().numpy(), "lse": lse.cpu().double().numpy(),
+            "target": tgt.cpu().double().numpy(), "mean": float(mean.item())}
+
+
+@pytest.mark.parametrize("N,V,D,bounds", [
+    (300, 5000, 128, [0, 2000, 2100, 5000]),          # uneven, one shard of 100 rows
+    (129, 70000, 64, [0, 17500, 35000, 52500, 70000]),
+    (1000, 1100, 72, [0, 1, 1100]),                    # a one-row shard
+])
+def test_sharded_matches_oracle(N, V, D, bounds):
+    H, W, y = synth.random_inputs(N, V, D, seed=V + len(bounds))
+    Hd, Wd, yd = to_device(H, W, y)
+    got = sharded_forward(Hd, Wd, yd, bounds)
+    ref = oracle.forward(H, W, y)
+    compare(got, ref, mean_ref=oracle.mean(ref["loss"]))
+
+
+def test_one_shard_agrees_with_the_plain_forward():
+    import linear_cross_entropy_bf16_b200 as flce
+    H, W, y = synth.random_inputs(700, 9000, 256, seed=51)
+    Hd, Wd, yd = to_device(H, W, y)
+    got = sharded_forward(Hd, Wd, yd, [0, 9000])
+    loss, lse, tgt, mean = flce.forward(Hd, Wd, yd)
+    assert np.array_equal(got["target"], tgt.cpu().double().numpy())
+    assert np.abs(got["lse"] - lse.cpu().double().numpy()).max() <= 1e-5
+
+
+def test_target_held_by_no_shard_is_flagged():
+    import linear_cross_entropy_bf16_b200 as flce
+    H, W, y = synth.random_inputs(64, 1000, 64, seed=52)
+    y[10] = 1000                       # outside the vocabulary
+    Hd, Wd, yd = to_device(H, W, y)
+    states = torch.stack([flce.shard_state(Hd, Wd[:600].contiguous(), yd, 0),
+                          flce.shard_state(Hd, Wd[600:].contiguous(), yd, 600)]).contiguous()
+    with pytest.raises(flce.FlceError) as e:
+        flce.merge_shards(states, yd, 1000, check=True)
+    assert e.value.status == flce.ERR_TARGET_OUT_OF_RANGE

@@ -84,3 +84,59 @@ def test_reference_arm_under_torchrun_prints_one_line():
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _vp_worker(rank, world, port, q):
+    """forward_vocab_parallel's exchange on two gloo ranks; the kernel steps are
+    replaced by an fp64 restatement so that only the orchestration is under test."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import linear_cross_entropy_bf16_b200 as flce
+        rng = np.random.default_rng(7)
+        N, V, D = 6, 10, 4
+        H = torch.from_numpy(rng.standard_normal((N, D)))
+        W = torch.from_numpy(rng.standard_normal((V, D)))
+        y = torch.from_numpy(rng.integers(0, V, N))
+        cut = [0, 4, 10]
+        a, b = cut[rank], cut[rank + 1]
+
+        def fake_state(H_, W_shard, y_, v_offset, **kw):
+            z = (H_ @ W_shard.T)
+            m = z.max(dim=1).values
+            s = torch.exp(z - m[:, None]).sum(dim=1)
+            rel = y_ - v_offset
+            own = (rel >= 0) & (rel < W_shard.shape[0])
+            t = torch.where(own, z[torch.arange(z.shape[0]), rel.clamp(0, W_shard.shape[0] - 1)], 0.0)
+            return torch.stack([m, s, t, own.double()], dim=1)
+
+        def fake_merge(states, y_, V_total, **kw):
+            m = states[..., 0].max(dim=0).values
+            s = (states[..., 1] * torch.exp(states[..., 0] - m)).sum(dim=0)
+            lse = m + torch.log(s)
+            t = (states[..., 2] * states[..., 3]).sum(dim=0)
+            return lse - t, lse, t, (lse - t).mean()
+
+        flce.shard_state = fake_state
+        flce.merge_shards = fake_merge
+        loss, lse, t, mean = flce.forward_vocab_parallel(H, W[a:b].contiguous(), y, a, V)
+        ref = torch.nn.functional.cross_entropy(H @ W.T, y, reduction="none")
+        q.put((rank, float((loss - ref).abs().max()), float(mean - ref.mean())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_vocab_parallel_exchange_on_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_vp_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=240) for _ in procs]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    for rank, dloss, dmean in out:
+        assert dloss < 1e-12 and abs(dmean) < 1e-12
