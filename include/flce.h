@@ -123,6 +123,36 @@ FLCE_API flce_status flce_forward(const void* H, const void* W, const int64_t* y
                          float* out_mean, void* workspace, size_t workspace_bytes,
                          void* stream);
 
+/* Element type of the targets y in flce_forward_ex. */
+typedef enum { FLCE_INDEX_INT64 = 0, FLCE_INDEX_INT32 = 1 } flce_index_dtype;
+
+/* Arguments of flce_forward_ex: those of flce_forward plus row strides and
+ * the target type. */
+typedef struct {
+  const void* H;            /* (N, D) rows, row stride ldh elements */
+  int64_t ldh;              /* >= D; 0 means D.  bf16: a multiple of 8 */
+  const void* W;            /* (V, D) rows, row stride ldw elements */
+  int64_t ldw;              /* >= D; 0 means D.  bf16: a multiple of 8 */
+  const void* y;            /* (N) targets of type y_dtype, each in [0, V) */
+  int32_t y_dtype;          /* flce_index_dtype */
+  int32_t dtype;            /* flce_dtype of H and W */
+  int64_t N, V, D;
+  float* out_loss;          /* (N) */
+  float* out_lse;           /* (N) */
+  float* out_target_logit;  /* (N) */
+  float* out_mean;          /* (1) or NULL */
+} flce_forward_args;
+
+/*
+ * flce_forward with strided H and W (for example slices of larger buffers)
+ * and int32 or int64 targets.  Same operation, workspace (sized by
+ * flce_workspace_size(N, V, D, dtype)), results and error behaviour as
+ * flce_forward; FLCE_ERR_INVALID_ARG for a bad stride or index type,
+ * FLCE_ERR_UNSUPPORTED for a bf16 stride that is not a multiple of 8.
+ */
+FLCE_API flce_status flce_forward_ex(const flce_forward_args* args, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
 /*
  * First stage of flce_forward, on its own: the contraction Z = H W^T tile by
  * tile with the online (m, s) update of section 1 of the page, leaving one

@@ -23,7 +23,7 @@ import torch
 
 __all__ = [
     "FlceError", "forward", "backward", "partials", "merge", "workspace_size",
-    "shard_state", "merge_shards", "forward_vocab_parallel",
+    "shard_state", "merge_shards", "forward_vocab_parallel", "forward_strided",
     "backward_workspace_size", "plan", "check",
     "status_string", "selftest_wait_timeout", "library_path", "load_library",
 ]
@@ -36,6 +36,9 @@ _lib = None
 # flce_dtype
 BF16 = 0
 FP32 = 1
+# flce_index_dtype
+INDEX_INT64 = 0
+INDEX_INT32 = 1
 # flce_status
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE_TOO_SMALL, ERR_CUDA, \
     ERR_TARGET_OUT_OF_RANGE, ERR_TIMEOUT = range(7)
@@ -51,6 +54,17 @@ class FlceError(RuntimeError):
         self.status = status
         name = _STATUS_NAMES[status] if 0 <= status < len(_STATUS_NAMES) else "unknown status"
         super().__init__(f"{what}: {name} (status {status})")
+
+
+class ForwardArgs(ctypes.Structure):
+    """Mirror of flce_forward_args."""
+    _fields_ = [
+        ("H", ctypes.c_void_p), ("ldh", ctypes.c_int64), ("W", ctypes.c_void_p),
+        ("ldw", ctypes.c_int64), ("y", ctypes.c_void_p), ("y_dtype", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("N", ctypes.c_int64), ("V", ctypes.c_int64),
+        ("D", ctypes.c_int64), ("out_loss", ctypes.c_void_p), ("out_lse", ctypes.c_void_p),
+        ("out_target_logit", ctypes.c_void_p), ("out_mean", ctypes.c_void_p),
+    ]
 
 
 class Plan(ctypes.Structure):
@@ -115,6 +129,8 @@ def load_library():
         lib.flce_merge_shards_scratch_size.restype = sz
         lib.flce_merge_shards.argtypes = [vp, ctypes.c_int32, vp, i64, i64, vp, vp, vp, vp, vp, sz, vp]
         lib.flce_merge_shards.restype = st
+        lib.flce_forward_ex.argtypes = [ctypes.POINTER(ForwardArgs), vp, sz, vp]
+        lib.flce_forward_ex.restype = st
         _lib = lib
         return lib
 
@@ -280,6 +296,37 @@ def backward(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, lse: torch.Tenso
     if check:
         _raise_on(lib.flce_check(workspace.data_ptr(), sp), "flce_backward (device)")
     return dH, dW
+
+
+def forward_strided(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, *, out: dict | None = None,
+                    workspace: torch.Tensor | None = None, stream=None, check: bool = False):
+    """flce_forward_ex: like forward(), for H and W whose rows are strided (each row
+    contiguous, row stride >= D) and int32 or int64 targets."""
+    for name, t in (("H", H), ("W", W)):
+        if not t.is_cuda or t.dim() != 2 or t.stride(1) != 1 or t.stride(0) < t.shape[1]:
+            raise ValueError(f"{name} must be a 2-D CUDA tensor with contiguous rows")
+    if y.dtype not in (torch.int64, torch.int32) or y.dim() != 1 or not y.is_contiguous() or not y.is_cuda:
+        raise ValueError("y must be a contiguous int64 or int32 CUDA tensor")
+    if H.dtype != W.dtype or H.shape[1] != W.shape[1] or y.shape[0] != H.shape[0]:
+        raise ValueError("shapes or dtypes of H, W and y do not match")
+    N, D = H.shape
+    V = W.shape[0]
+    code = _dtype_code(H)
+    dev = H.device
+    loss, lse, tgt, mean = _alloc_outputs(N, dev, out)
+    if N == 0:
+        return loss, lse, tgt, mean
+    ws = _workspace(N, V, D, code, dev, workspace)
+    a = ForwardArgs(H.data_ptr(), H.stride(0), W.data_ptr(), W.stride(0), y.data_ptr(),
+                    INDEX_INT32 if y.dtype == torch.int32 else INDEX_INT64, code, N, V, D,
+                    loss.data_ptr(), lse.data_ptr(), tgt.data_ptr(), mean.data_ptr())
+    sp = _stream_ptr(stream, dev)
+    lib = load_library()
+    _raise_on(lib.flce_forward_ex(ctypes.byref(a), ws.data_ptr(), ws.numel() * ws.element_size(), sp),
+              "flce_forward_ex")
+    if check:
+        _raise_on(lib.flce_check(ws.data_ptr(), sp), "flce_forward_ex (device)")
+    return loss, lse, tgt, mean
 
 
 def shard_state(H: torch.Tensor, W_shard: torch.Tensor, y: torch.Tensor, v_offset: int, *,

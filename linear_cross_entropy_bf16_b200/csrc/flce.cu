@@ -168,11 +168,13 @@ bool load_encoder() {
   return g_encode != nullptr;
 }
 
-// Row-major (rows, D) bf16 matrix, boxes of 64 x box_rows, 128-byte swizzle,
-// zero fill outside the matrix (ragged N, V and D).
-bool encode_bf16_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t D, int box_rows) {
+// Row-major (rows, D) bf16 matrix with row stride ld elements, boxes of
+// 64 x box_rows, 128-byte swizzle, zero fill outside the matrix (ragged N, V
+// and D).
+bool encode_bf16_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t D, int64_t ld,
+                      int box_rows) {
   cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(rows)};
-  cuuint64_t strides[1] = {cuuint64_t(D) * 2};
+  cuuint64_t strides[1] = {cuuint64_t(ld) * 2};
   cuuint32_t box[2] = {cuuint32_t(tc::BK), cuuint32_t(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
@@ -252,9 +254,9 @@ flce_status check_forward_args(const void* H, const void* W, const int64_t* y, i
   return FLCE_OK;
 }
 
-flce_status launch_partials(const void* H, const void* W, const int64_t* y, int64_t y_offset,
-                            int64_t N, int64_t V, int64_t D, flce_dtype dtype, float* out_target,
-                            void* ws, cudaStream_t st) {
+flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t ldw, Targets y,
+                            int64_t y_offset, int64_t N, int64_t V, int64_t D, flce_dtype dtype,
+                            float* out_target, void* ws, cudaStream_t st) {
   DeviceInfo di;
   flce_status s = device_info(di);
   if (s != FLCE_OK) return s;
@@ -285,8 +287,8 @@ flce_status launch_partials(const void* H, const void* W, const int64_t* y, int6
     if (!load_encoder()) return FLCE_ERR_CUDA;
     const bool pair = plan.ctas_per_unit == 2;
     CUtensorMap tmH, tmW;
-    if (!encode_bf16_rows(&tmH, H, N, D, tc::BM) ||
-        !encode_bf16_rows(&tmW, W, V, D, pair ? tc2::HALF_N : tc::BN))
+    if (!encode_bf16_rows(&tmH, H, N, D, ldh, tc::BM) ||
+        !encode_bf16_rows(&tmW, W, V, D, ldw, pair ? tc2::HALF_N : tc::BN))
       return FLCE_ERR_UNSUPPORTED;
     tc::Args a;
     a.y = y;
@@ -308,6 +310,8 @@ flce_status launch_partials(const void* H, const void* W, const int64_t* y, int6
     simt::Args a;
     a.H = H;
     a.W = W;
+    a.ldh = ldh;
+    a.ldw = ldw;
     a.y = y;
     a.y_offset = y_offset;
     a.part = part;
@@ -322,7 +326,7 @@ flce_status launch_partials(const void* H, const void* W, const int64_t* y, int6
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
-flce_status launch_merge(const int64_t* y, int64_t N, int64_t V, float* out_loss, float* out_lse,
+flce_status launch_merge(Targets y, int64_t N, int64_t V, float* out_loss, float* out_lse,
                          float* out_target, float* out_mean, const void* ws, size_t ws_bytes,
                          cudaStream_t st) {
   uint8_t* wsb = static_cast<uint8_t*>(const_cast<void*>(ws));
@@ -366,7 +370,7 @@ flce_status flce_partials(const void* H, const void* W, const int64_t* y, int64_
   flce_status s = check_forward_args(H, W, y, N, V, D, dtype, workspace, workspace_bytes);
   if (s != FLCE_OK || N == 0) return s;
   if (!out_target_logit) return FLCE_ERR_INVALID_ARG;
-  return launch_partials(H, W, y, 0, N, V, D, dtype, out_target_logit, workspace,
+  return launch_partials(H, D, W, D, Targets{y, 0}, 0, N, V, D, dtype, out_target_logit, workspace,
                          static_cast<cudaStream_t>(stream));
 }
 
@@ -379,7 +383,7 @@ flce_status flce_merge(const int64_t* y, int64_t N, int64_t V, float* out_loss, 
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FLCE_ERR_INVALID_ARG;
   if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
   if (workspace_bytes < workspace_bytes_for(N, V)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
-  return launch_merge(y, N, V, out_loss, out_lse, out_target_logit, out_mean, workspace,
+  return launch_merge(Targets{y, 0}, N, V, out_loss, out_lse, out_target_logit, out_mean, workspace,
                       workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -391,10 +395,35 @@ flce_status flce_forward(const void* H, const void* W, const int64_t* y, int64_t
   if (s != FLCE_OK || N == 0) return s;
   if (!out_loss || !out_lse || !out_target_logit) return FLCE_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = launch_partials(H, W, y, 0, N, V, D, dtype, out_target_logit, workspace, st);
+  s = launch_partials(H, D, W, D, Targets{y, 0}, 0, N, V, D, dtype, out_target_logit, workspace,
+                      st);
   if (s != FLCE_OK) return s;
-  return launch_merge(y, N, V, out_loss, out_lse, out_target_logit, out_mean, workspace,
+  return launch_merge(Targets{y, 0}, N, V, out_loss, out_lse, out_target_logit, out_mean, workspace,
                       workspace_bytes, st);
+}
+
+flce_status flce_forward_ex(const flce_forward_args* a, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (!a) return FLCE_ERR_INVALID_ARG;
+  const flce_dtype dtype = flce_dtype(a->dtype);
+  if (!sizes_ok(a->N, a->V, a->D, dtype)) return FLCE_ERR_INVALID_ARG;
+  if (a->y_dtype != FLCE_INDEX_INT64 && a->y_dtype != FLCE_INDEX_INT32) return FLCE_ERR_INVALID_ARG;
+  const int64_t ldh = a->ldh == 0 ? a->D : a->ldh;
+  const int64_t ldw = a->ldw == 0 ? a->D : a->ldw;
+  if (ldh < a->D || ldw < a->D) return FLCE_ERR_INVALID_ARG;
+  if (dtype == FLCE_BF16 && (ldh % 8 != 0 || ldw % 8 != 0)) return FLCE_ERR_UNSUPPORTED;
+  flce_status s = check_forward_args(a->H, a->W, static_cast<const int64_t*>(a->y), a->N, a->V,
+                                     a->D, dtype, workspace, workspace_bytes);
+  if (s != FLCE_OK || a->N == 0) return s;
+  if (!a->out_loss || !a->out_lse || !a->out_target_logit) return FLCE_ERR_INVALID_ARG;
+  if (ldh >= (int64_t(1) << 31) || ldw >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Targets y{a->y, a->y_dtype == FLCE_INDEX_INT32 ? 1 : 0};
+  s = launch_partials(a->H, ldh, a->W, ldw, y, 0, a->N, a->V, a->D, dtype, a->out_target_logit,
+                      workspace, st);
+  if (s != FLCE_OK) return s;
+  return launch_merge(y, a->N, a->V, a->out_loss, a->out_lse, a->out_target_logit, a->out_mean,
+                      workspace, workspace_bytes, st);
 }
 
 flce_status flce_partials_shard(const void* H, const void* W_shard, const int64_t* y, int64_t N,
@@ -406,7 +435,8 @@ flce_status flce_partials_shard(const void* H, const void* W_shard, const int64_
       check_forward_args(H, W_shard, y, N, V_shard, D, dtype, workspace, workspace_bytes);
   if (s != FLCE_OK || N == 0) return s;
   if (!out_target_logit) return FLCE_ERR_INVALID_ARG;
-  return launch_partials(H, W_shard, y, v_offset, N, V_shard, D, dtype, out_target_logit,
+  return launch_partials(H, D, W_shard, D, Targets{y, 0}, v_offset, N, V_shard, D, dtype,
+                         out_target_logit,
                          workspace, static_cast<cudaStream_t>(stream));
 }
 

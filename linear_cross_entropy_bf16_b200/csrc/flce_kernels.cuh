@@ -56,6 +56,17 @@ static_assert(sizeof(WsHeader) <= kHeaderBytes, "header");
 
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e): exp(x) = 2^(x log2 e)
 
+// ----------------------------------------------------------------- targets
+
+// Target ids, stored as int64 (the default) or int32.
+struct Targets {
+  const void* p;
+  int32_t is32;
+  __device__ __forceinline__ int64_t operator[](int64_t i) const {
+    return is32 ? int64_t(static_cast<const int32_t*>(p)[i]) : static_cast<const int64_t*>(p)[i];
+  }
+};
+
 // ----------------------------------------------------------------- schedule
 
 struct Schedule {
@@ -218,7 +229,7 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
 }
 
 struct Args {
-  const int64_t* y;
+  Targets y;
   int64_t y_offset;        // first vocabulary id of W's rows (a vocabulary shard); 0 otherwise
   float2* part;            // [P][N] (m, s) per slab and token
   float* target_logit;     // [N]
@@ -678,7 +689,8 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return
 struct Args {
   const void* H;
   const void* W;
-  const int64_t* y;
+  int64_t ldh, ldw;        // row strides of H and W in elements
+  Targets y;
   int64_t y_offset;
   float2* part;
   float* target_logit;
@@ -738,9 +750,9 @@ __global__ void __launch_bounds__(NUM_THREADS) flce_simt_kernel(const Args a) {
       for (int e = tid; e < BM * BK; e += NUM_THREADS) {
         const int r = e / BK, k = e % BK;
         const int gr = row0 + r, gk = k0 + k;
-        sH[k][r] = (gr < a.N && gk < a.D) ? to_f32<T>(H[size_t(gr) * a.D + gk]) : 0.f;
+        sH[k][r] = (gr < a.N && gk < a.D) ? to_f32<T>(H[size_t(gr) * a.ldh + gk]) : 0.f;
         const int gc = c0 + r;
-        sW[k][r] = (gc < a.V && gk < a.D) ? to_f32<T>(W[size_t(gc) * a.D + gk]) : 0.f;
+        sW[k][r] = (gc < a.V && gk < a.D) ? to_f32<T>(W[size_t(gc) * a.ldw + gk]) : 0.f;
       }
       __syncthreads();
 #pragma unroll 8
@@ -806,7 +818,7 @@ constexpr int kMergeThreads = 256;
 
 struct MergeArgs {
   const float2* part;
-  const int64_t* y;
+  Targets y;
   float* target_logit;
   float* loss;
   float* lse;

@@ -194,3 +194,19 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(flce, "_LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(flce.FlceError):
         flce.load_library()
+
+
+def test_forward_ex_argument_checks_need_no_gpu(lib):
+    def call(**kw):
+        a = dict(H=FAKE, ldh=0, W=FAKE, ldw=0, y=FAKE, y_dtype=0, dtype=0, N=16, V=100, D=64,
+                 out_loss=FAKE, out_lse=FAKE, out_target_logit=FAKE, out_mean=None)
+        a.update(kw)
+        args = flce.ForwardArgs(**a)
+        return lib.flce_forward_ex(ctypes.byref(args), kw.get("ws", FAKE), kw.get("ws_bytes", 1 << 30), None)
+    assert lib.flce_forward_ex(None, FAKE, 1 << 30, None) == flce.ERR_INVALID_ARG
+    assert call(y_dtype=2) == flce.ERR_INVALID_ARG
+    assert call(ldh=32) == flce.ERR_INVALID_ARG        # stride below D
+    assert call(ldw=65) == flce.ERR_UNSUPPORTED        # bf16 stride not a multiple of 8
+    assert call(out_lse=None) == flce.ERR_INVALID_ARG
+    assert call(N=0) == flce.OK
+    assert call(dtype=1, ldh=65, ldw=66, ws_bytes=10) == flce.ERR_WORKSPACE_TOO_SMALL   # fp32: any stride

@@ -187,3 +187,25 @@ def test_no_N_by_V_allocation():
     torch.cuda.synchronize()
     assert torch.cuda.max_memory_allocated() == base
     assert ws.numel() < 4 * N * V / 30
+
+
+@pytest.mark.parametrize("dtype,y32", [("bf16", False), ("bf16", True), ("fp32", True)])
+def test_strided_rows_and_int32_targets(dtype, y32):
+    """flce_forward_ex on row slices of wider buffers (row stride > D) with int32/int64 targets."""
+    import linear_cross_entropy_bf16_b200 as flce
+    N, V, D, pad = 300, 3000, 128, 72
+    H, W, y = synth.random_inputs(N, V, D + pad, seed=61, dtype=dtype)
+    Hd, Wd, yd = to_device(H, W, y)
+    Hs, Ws = Hd[:, pad:], Wd[:, 8:8 + D]            # strided views: rows of D, stride D + pad
+    assert Hs.stride(0) == D + pad and not Hs.is_contiguous()
+    yy = yd.to(torch.int32) if y32 else yd
+    loss, lse, tgt, mean = flce.forward_strided(Hs, Ws, yy, check=True)
+    Hc = np.ascontiguousarray(H[:, pad:])
+    Wc = np.ascontiguousarray(W[:, 8:8 + D])
+    ref = oracle.forward(Hc, Wc, y)
+    gpu = {"loss": loss.cpu().double().numpy(), "lse": lse.cpu().double().numpy(),
+           "target": tgt.cpu().double().numpy(), "mean": float(mean.item())}
+    compare(gpu, ref, mean_ref=oracle.mean(ref["loss"]))
+    # identical to the contiguous call on copies
+    ref_gpu = flce.forward(Hs.contiguous(), Ws.contiguous(), yd)
+    assert torch.equal(ref_gpu[0], loss)
