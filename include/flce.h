@@ -43,7 +43,12 @@ extern "C" {
 #endif
 
 /* Element type of H and W.  bf16 runs on the tcgen05 tensor-core path
- * (fp32 accumulation in TMEM); fp32 runs on an fp32 FFMA path. */
+ * (fp32 accumulation in TMEM).  fp32 inputs are first split, value by value,
+ * into two bf16 parts hi = bf16(x), lo = bf16(x - hi) in the workspace, and
+ * the same tensor-core path contracts hi*hi + hi*lo + lo*hi (three bf16
+ * products per fp32 product, each accurate to about 3 * 2^-16 relative;
+ * Henry, Tang and Heinecke, ARITH 2019).  fp32 values must be finite and
+ * below bf16's largest finite value (about 3.39e38) in magnitude. */
 typedef enum { FLCE_BF16 = 0, FLCE_FP32 = 1 } flce_dtype;
 
 typedef enum {
@@ -64,7 +69,7 @@ typedef enum {
 typedef struct {
   int64_t N, V, D;
   int32_t dtype;           /* flce_dtype */
-  int32_t block_rows;      /* tokens per work unit (TMEM lanes on the bf16 path) */
+  int32_t block_rows;      /* tokens per work unit (128 TMEM lanes per CTA) */
   int32_t tile_cols;       /* vocab columns per tile */
   int32_t k_block;         /* D elements per pipeline stage */
   int64_t token_blocks;    /* ceil(N / block_rows) */
@@ -76,7 +81,7 @@ typedef struct {
   int64_t units;           /* token_blocks * slabs */
   int64_t makespan_tiles;  /* tiles processed by the busiest CTA (or CTA pair) */
   size_t workspace_bytes;  /* == flce_workspace_size(N, V, D, dtype) */
-  int32_t ctas_per_unit;   /* 2: a CTA pair shares each 256-token tile (bf16, N > 128);
+  int32_t ctas_per_unit;   /* 2: a CTA pair shares each 256-token tile (N > 128);
                               1: one CTA per tile */
   int32_t group_blocks;    /* token blocks per raster group: units are ordered group by
                               group, slab-major inside a group, and handed out round-robin */
@@ -85,9 +90,11 @@ typedef struct {
 /* Bytes of device workspace that flce_forward / flce_partials need for this
  * problem: a 256-byte header, the per-(slab, token) partial states (8 bytes
  * each, at most 512 slabs per token, so O(N), never O(N*V)), and one fp64
- * per 256 tokens for the mean.  Depends only on its arguments (not on the
- * device).  Returns 0 for invalid arguments (N < 0, V < 1, D < 1, unknown
- * dtype).  Host only; never touches the GPU. */
+ * per 256 tokens for the mean.  fp32 inputs add the bf16 split copies of H
+ * and W, 6 * Dp bytes per row of each (Dp = D rounded up to 8): O((N + V) D),
+ * still never O(N*V).  Depends only on its arguments (not on the device).
+ * Returns 0 for invalid arguments (N < 0, V < 1, D < 1, unknown dtype).  Host
+ * only; never touches the GPU. */
 FLCE_API size_t flce_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype dtype);
 
 /* The schedule for a device with `sm_count` SMs, assuming every SM pair can

@@ -25,7 +25,6 @@ namespace {
 using namespace flce;
 
 constexpr uint64_t kDefaultWaitLimitNs = 4000000000ull;  // 4 s in one wait: far beyond any real stage
-constexpr int kSimtBlocksPerSm = 4;
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -38,10 +37,30 @@ bool sizes_ok(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
 
 int64_t slab_capacity(int64_t V) { return std::min<int64_t>(cdiv(V, kTileCols), kMaxSlabs); }
 
-size_t workspace_bytes_for(int64_t N, int64_t V) {
+// Header, (m, s) partial states and the mean's block sums: what the merge reads.
+size_t state_bytes_for(int64_t N, int64_t V) {
   const size_t part = align256(size_t(8) * size_t(N) * size_t(slab_capacity(V)));
   const size_t sums = align256(size_t(8) * size_t(std::max<int64_t>(1, cdiv(N, kMergeThreads))));
   return kHeaderBytes + part + sums;
+}
+
+// Length of the bf16 K axis the tensor-core kernels contract over: D for bf16
+// inputs; for fp32 inputs three segments (hi / lo parts) of D rounded up to 8.
+int64_t split_segment(int64_t D) { return (D + 7) / 8 * 8; }
+int64_t k_extent(int64_t D, flce_dtype dtype) {
+  return dtype == FLCE_FP32 ? 3 * split_segment(D) : D;
+}
+
+// fp32 inputs: room after the state for the split copies of H and W,
+// (N, 3 Dp) and (V, 3 Dp) bf16, each 256-byte aligned.
+size_t split_bytes_for(int64_t rows, int64_t D) {
+  return align256(size_t(rows) * size_t(3 * split_segment(D)) * 2);
+}
+
+size_t workspace_bytes_for(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
+  size_t b = state_bytes_for(N, V);
+  if (dtype == FLCE_FP32) b += split_bytes_for(N, D) + split_bytes_for(V, D);
+  return b;
 }
 
 // Makespan, in tiles, of the busiest worker when the units of a schedule are
@@ -112,9 +131,9 @@ int64_t group_blocks_for(int64_t tb, int64_t block_rows, int64_t D, int64_t elem
   return std::max<int64_t>(1, std::min(tb, kGroupHBytes / per_block));
 }
 
-// The bf16 path runs on CTA pairs (256-token tiles) unless the batch fits one
-// 128-token tile, where half of every pair tile would be padding.
-bool use_pair_kernel(int64_t N, flce_dtype dtype) { return dtype == FLCE_BF16 && N > tc::BM; }
+// The contraction runs on CTA pairs (256-token tiles) unless the batch fits
+// one 128-token tile, where half of every pair tile would be padding.
+bool use_pair_kernel(int64_t N) { return N > tc::BM; }
 
 // `workers`: CTAs (single-CTA kernels) or CTA pairs (pair kernel) that run at once.
 flce_status make_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int64_t workers,
@@ -125,30 +144,28 @@ flce_status make_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int64_t
   p->D = D;
   p->dtype = int32_t(dtype);
   p->tile_cols = kTileCols;
-  const bool tc = dtype == FLCE_BF16;
-  const bool pair = use_pair_kernel(N, dtype);
+  const bool pair = use_pair_kernel(N);
   p->ctas_per_unit = pair ? 2 : 1;
-  p->block_rows = pair ? tc2::PAIR_M : (tc ? tc::BM : simt::BM);
-  p->k_block = tc ? tc::BK : simt::BK;
+  p->block_rows = pair ? tc2::PAIR_M : tc::BM;
+  p->k_block = tc::BK;
   p->token_blocks = cdiv(std::max<int64_t>(N, 1), p->block_rows);
   p->vocab_tiles = cdiv(V, kTileCols);
   const int64_t g = std::max<int64_t>(1, workers);
-  p->group_blocks = int32_t(group_blocks_for(p->token_blocks, p->block_rows, D, tc ? 2 : 4));
+  p->group_blocks = int32_t(group_blocks_for(p->token_blocks, p->block_rows, k_extent(D, dtype), 2));
   int64_t ms = 0;
   choose_slabs(p->token_blocks, p->group_blocks, p->vocab_tiles, g, slab_capacity(V), p->slabs,
                ms);
   p->slab_base = int32_t(p->vocab_tiles / p->slabs);
   p->slab_rem = int32_t(p->vocab_tiles % p->slabs);
   p->units = p->token_blocks * p->slabs;
-  p->grid = int32_t(tc ? std::min<int64_t>(g, p->units) * p->ctas_per_unit : p->units);
+  p->grid = int32_t(std::min<int64_t>(g, p->units) * p->ctas_per_unit);
   p->makespan_tiles = ms;
-  p->workspace_bytes = workspace_bytes_for(N, V);
+  p->workspace_bytes = workspace_bytes_for(N, V, D, dtype);
   return FLCE_OK;
 }
 
-int64_t nominal_workers(int32_t sms, int64_t N, flce_dtype dtype) {
-  if (dtype != FLCE_BF16) return int64_t(sms) * kSimtBlocksPerSm;
-  return use_pair_kernel(N, dtype) ? std::max<int64_t>(1, sms / 2) : int64_t(sms);
+int64_t nominal_workers(int32_t sms, int64_t N) {
+  return use_pair_kernel(N) ? std::max<int64_t>(1, sms / 2) : int64_t(sms);
 }
 
 // ---------------------------------------------------------------- driver entry point
@@ -250,8 +267,32 @@ flce_status check_forward_args(const void* H, const void* W, const int64_t* y, i
     return FLCE_ERR_UNSUPPORTED;
   if (dtype == FLCE_FP32 && ((reinterpret_cast<uintptr_t>(H) | reinterpret_cast<uintptr_t>(W)) & 3u))
     return FLCE_ERR_INVALID_ARG;
-  if (ws_bytes < workspace_bytes_for(N, V)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  if (dtype == FLCE_FP32 && k_extent(D, dtype) >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
+  if (ws_bytes < workspace_bytes_for(N, V, D, dtype)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
   return FLCE_OK;
+}
+
+// fp32 inputs: split `src` (rows, D; row stride ld) into its bf16 (rows,
+// 3 Dp) copy at `dst` with hi / lo parts in the segments the operand needs.
+flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, int lo_segment,
+                         void* dst, int sms, cudaStream_t st) {
+  split::Args a;
+  a.src = static_cast<const float*>(src);
+  a.ld = ld;
+  a.rows = rows;
+  a.D = int32_t(D);
+  a.Dp = int32_t(split_segment(D));
+  a.lo_segment = lo_segment;
+  a.dst = static_cast<__nv_bfloat16*>(dst);
+  const int64_t warps_per_block = split::NUM_THREADS / 32;
+  const int64_t blocks = std::max<int64_t>(
+      1, std::min<int64_t>(cdiv(rows, warps_per_block), int64_t(sms) * 8));
+  const bool vec = D % 8 == 0 && ld % 4 == 0 && aligned16(src);
+  if (vec)
+    split::flce_split3_kernel<true><<<unsigned(blocks), split::NUM_THREADS, 0, st>>>(a);
+  else
+    split::flce_split3_kernel<false><<<unsigned(blocks), split::NUM_THREADS, 0, st>>>(a);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
 flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t ldw, Targets y,
@@ -260,9 +301,9 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
   DeviceInfo di;
   flce_status s = device_info(di);
   if (s != FLCE_OK) return s;
-  if (dtype == FLCE_BF16 && (s = set_smem_attr_once()) != FLCE_OK) return s;
-  int64_t workers = nominal_workers(di.sms, N, dtype);
-  if (use_pair_kernel(N, dtype)) {
+  if ((s = set_smem_attr_once()) != FLCE_OK) return s;
+  int64_t workers = nominal_workers(di.sms, N);
+  if (use_pair_kernel(N)) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
     workers = resident_pairs(dev, di.sms);
@@ -275,6 +316,23 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
   float2* part = reinterpret_cast<float2*>(wsb + kHeaderBytes);
   if (cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
 
+  // The operands the tensor-core kernels read: H and W themselves (bf16), or
+  // their split copies in the workspace (fp32), K = 3 Dp.
+  const void* opH = H;
+  const void* opW = W;
+  int64_t K = D;
+  if (dtype == FLCE_FP32) {
+    K = k_extent(D, dtype);
+    uint8_t* hs = wsb + state_bytes_for(N, V);
+    uint8_t* wsplit = hs + split_bytes_for(N, D);
+    if ((s = launch_split(H, ldh, N, D, 2, hs, di.sms, st)) != FLCE_OK) return s;
+    if ((s = launch_split(W, ldw, V, D, 1, wsplit, di.sms, st)) != FLCE_OK) return s;
+    opH = hs;
+    opW = wsplit;
+    ldh = K;
+    ldw = K;
+  }
+
   Schedule sch;
   sch.token_blocks = int32_t(plan.token_blocks);
   sch.slabs = plan.slabs;
@@ -283,46 +341,28 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
   sch.units = int32_t(plan.units);
   sch.group_blocks = plan.group_blocks;
 
-  if (dtype == FLCE_BF16) {
-    if (!load_encoder()) return FLCE_ERR_CUDA;
-    const bool pair = plan.ctas_per_unit == 2;
-    CUtensorMap tmH, tmW;
-    if (!encode_bf16_rows(&tmH, H, N, D, ldh, tc::BM) ||
-        !encode_bf16_rows(&tmW, W, V, D, ldw, pair ? tc2::HALF_N : tc::BN))
-      return FLCE_ERR_UNSUPPORTED;
-    tc::Args a;
-    a.y = y;
-    a.y_offset = y_offset;
-    a.part = part;
-    a.target_logit = out_target;
-    a.hdr = hdr;
-    a.N = int32_t(N);
-    a.V = int32_t(V);
-    a.D = int32_t(D);
-    a.kblocks = int32_t(cdiv(D, tc::BK));
-    a.sch = sch;
-    a.wait_limit_ns = kDefaultWaitLimitNs;
-    if (pair)
-      tc2::flce_tc2_kernel<<<plan.grid, tc2::NUM_THREADS, tc2::SMEM_BYTES, st>>>(tmH, tmW, a);
-    else
-      tc::flce_tc_kernel<<<plan.grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(tmH, tmW, a);
-  } else {
-    simt::Args a;
-    a.H = H;
-    a.W = W;
-    a.ldh = ldh;
-    a.ldw = ldw;
-    a.y = y;
-    a.y_offset = y_offset;
-    a.part = part;
-    a.target_logit = out_target;
-    a.hdr = hdr;
-    a.N = int32_t(N);
-    a.V = int32_t(V);
-    a.D = int32_t(D);
-    a.sch = sch;
-    simt::flce_simt_kernel<float><<<plan.grid, simt::NUM_THREADS, 0, st>>>(a);
-  }
+  if (!load_encoder()) return FLCE_ERR_CUDA;
+  const bool pair = plan.ctas_per_unit == 2;
+  CUtensorMap tmH, tmW;
+  if (!encode_bf16_rows(&tmH, opH, N, K, ldh, tc::BM) ||
+      !encode_bf16_rows(&tmW, opW, V, K, ldw, pair ? tc2::HALF_N : tc::BN))
+    return FLCE_ERR_UNSUPPORTED;
+  tc::Args a;
+  a.y = y;
+  a.y_offset = y_offset;
+  a.part = part;
+  a.target_logit = out_target;
+  a.hdr = hdr;
+  a.N = int32_t(N);
+  a.V = int32_t(V);
+  a.D = int32_t(K);
+  a.kblocks = int32_t(cdiv(K, tc::BK));
+  a.sch = sch;
+  a.wait_limit_ns = kDefaultWaitLimitNs;
+  if (pair)
+    tc2::flce_tc2_kernel<<<plan.grid, tc2::NUM_THREADS, tc2::SMEM_BYTES, st>>>(tmH, tmW, a);
+  else
+    tc::flce_tc_kernel<<<plan.grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(tmH, tmW, a);
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
@@ -355,13 +395,13 @@ extern "C" {
 
 size_t flce_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
   if (!sizes_ok(N, V, D, dtype)) return 0;
-  return workspace_bytes_for(N, V);
+  return workspace_bytes_for(N, V, D, dtype);
 }
 
 flce_status flce_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int32_t sm_count,
                       flce_plan_t* plan) {
   if (!plan || sm_count < 1 || !sizes_ok(N, V, D, dtype)) return FLCE_ERR_INVALID_ARG;
-  return make_plan(N, V, D, dtype, nominal_workers(sm_count, N, dtype), plan);
+  return make_plan(N, V, D, dtype, nominal_workers(sm_count, N), plan);
 }
 
 flce_status flce_partials(const void* H, const void* W, const int64_t* y, int64_t N, int64_t V,
@@ -382,7 +422,7 @@ flce_status flce_merge(const int64_t* y, int64_t N, int64_t V, float* out_loss, 
   if (!y || !out_loss || !out_lse || !out_target_logit || !workspace) return FLCE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FLCE_ERR_INVALID_ARG;
   if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
-  if (workspace_bytes < workspace_bytes_for(N, V)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  if (workspace_bytes < state_bytes_for(N, V)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
   return launch_merge(Targets{y, 0}, N, V, out_loss, out_lse, out_target_logit, out_mean, workspace,
                       workspace_bytes, static_cast<cudaStream_t>(stream));
 }
@@ -450,7 +490,7 @@ flce_status flce_shard_state(const int64_t* y, int64_t N, int64_t V_shard, int64
       (reinterpret_cast<uintptr_t>(out_state) & 15u) != 0)
     return FLCE_ERR_INVALID_ARG;
   if (N >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
-  if (workspace_bytes < workspace_bytes_for(N, V_shard)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  if (workspace_bytes < state_bytes_for(N, V_shard)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
   const uint8_t* wsb = static_cast<const uint8_t*>(workspace);
   const WsHeader* hdr = reinterpret_cast<const WsHeader*>(wsb);
   flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0,
@@ -741,7 +781,7 @@ extern "C" flce_status flce_forward_noalloc(const void* H, const void* W, const 
   if (!sizes_ok(N, V, D, dtype)) return FLCE_ERR_INVALID_ARG;
   if (N == 0) return FLCE_OK;
   // The problem must fit the built-in scratch; nothing larger is ever allocated.
-  if (workspace_bytes_for(N, V) > size_t(FLCE_NOALLOC_SCRATCH_BYTES))
+  if (workspace_bytes_for(N, V, D, dtype) > size_t(FLCE_NOALLOC_SCRATCH_BYTES))
     return FLCE_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = nullptr;
   flce_status s = noalloc_scratch(&scratch);

@@ -15,8 +15,10 @@
 //     double-buffered fp32 TMEM accumulator, and warps 2-5 (one TMEM lane,
 //     i.e. one token, per thread) fold each finished tile into (m, s) and
 //     capture the target logit.  Logits never leave TMEM/registers.
-//   * flce_simt_kernel: the same decomposition with fp32 FFMA tiles, for fp32
-//     inputs (bf16 tensor cores cannot honour fp32 inputs).
+//   * flce_split3_kernel: for fp32 inputs, splits H and W into bf16 hi/lo
+//     parts laid out along a tripled K axis, so that the same tensor-core
+//     kernels compute the three-product fp32 emulation Hhi Whi + Hhi Wlo +
+//     Hlo Whi.
 //   * flce_merge_kernel: combines the P slab states of each token in a fixed
 //     order (the recurrence of section 1 applied to whole slabs), writes
 //     lse/loss, and reduces the mean deterministically in fp64.
@@ -670,147 +672,83 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
 
 }  // namespace tc2
 
-// ----------------------------------------------------------------- fp32 FFMA kernel
+// ----------------------------------------------------------------- fp32 inputs
 
-namespace simt {
+// fp32 inputs run on the same bf16 tensor-core kernels after a split of
+// every value into two bf16 values (Henry, Tang and Heinecke, "Leveraging
+// the bfloat16 artificial intelligence datatype for higher-precision
+// computations", ARITH 2019):  hi = bf16(x),  lo = bf16(x - hi),  so that
+// |x - hi - lo| <= 2^-16 |x|.  Laying H out as [hi | hi | lo] and W as
+// [hi | lo | hi] along K (three segments of Dp = D rounded up to 8, zero
+// padded) turns one bf16 contraction over 3 Dp into
+//   Z = Hhi Whi^T + Hhi Wlo^T + Hlo Whi^T
+// with fp32 accumulation in TMEM: each product h w is off by at most about
+// 3 * 2^-16 |h w| (the dropped lo*lo term and the two rounding residues).
+namespace split {
 
-constexpr int BM = 64;           // tokens per work unit
-constexpr int BNS = 64;          // vocab columns per sub-tile (4 per 256-column tile)
-constexpr int BK = 32;
-constexpr int NUM_THREADS = 256; // 16 x 16 threads, 4 x 4 outputs each
-
-template <typename T>
-__device__ __forceinline__ float to_f32(T v);
-template <>
-__device__ __forceinline__ float to_f32<float>(float v) { return v; }
-template <>
-__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+constexpr int NUM_THREADS = 256;   // 8 warps, one row per warp at a time
 
 struct Args {
-  const void* H;
-  const void* W;
-  int64_t ldh, ldw;        // row strides of H and W in elements
-  Targets y;
-  int64_t y_offset;
-  float2* part;
-  float* target_logit;
-  WsHeader* hdr;
-  int32_t N, V, D;
-  Schedule sch;
+  const float* src;       // (rows, D) fp32, row stride ld elements
+  int64_t ld;
+  int64_t rows;
+  int32_t D;
+  int32_t Dp;             // D rounded up to a multiple of 8
+  int32_t lo_segment;     // 1 (W: [hi | lo | hi]) or 2 (H: [hi | hi | lo])
+  __nv_bfloat16* dst;     // (rows, 3 Dp) bf16, contiguous
 };
 
-// One CTA per work unit (slab, token block).  Thread (ty, tx) owns rows
-// ty*4 + i and columns tx + 16 j of each 64 x 64 sub-tile.  The 16 threads
-// sharing a row sit in one half-warp, so each row's tile max and exp-sum are
-// reduced with xor shuffles over 16 lanes.
-template <typename T>
-__global__ void __launch_bounds__(NUM_THREADS) flce_simt_kernel(const Args a) {
-  __shared__ float sH[BK][BM + 4];
-  __shared__ float sW[BK][BNS + 4];
-  const T* H = static_cast<const T*>(a.H);
-  const T* W = static_cast<const T*>(a.W);
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
+__device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 a, __nv_bfloat16 b) {
+  return uint32_t(__bfloat16_as_ushort(a)) | (uint32_t(__bfloat16_as_ushort(b)) << 16);
+}
 
-  if (blockIdx.x == 0 && tid == 0) {
-    a.hdr->slabs = a.sch.slabs;
-    a.hdr->N = a.N;
-    a.hdr->V = a.V;
-    a.hdr->magic = kWsMagic;
-  }
-
-  int slab, tb, t0, nt;
-  unit_coords(a.sch, blockIdx.x, slab, tb, t0, nt);
-  const int row0 = tb * BM;
-
-  float m[4], s[4], zt[4];
-  bool got[4];
-  int64_t yrow[4];
+// Each lane converts groups of 8 consecutive elements of its warp's row: it
+// loads 32 bytes of fp32 (two float4 when `kVec`, i.e. D % 8 == 0, ld % 4 ==
+// 0 and a 16-byte-aligned base) and stores 16 bytes to each of the three
+// segments.  Purely bandwidth-bound: 4 bytes in, 6 bytes out per element.
+template <bool kVec>
+__global__ void __launch_bounds__(NUM_THREADS) flce_split3_kernel(const Args a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = int64_t(gridDim.x) * (NUM_THREADS / 32);
+  const int groups = a.Dp / 8;
+  for (int64_t r = int64_t(blockIdx.x) * (NUM_THREADS / 32) + (threadIdx.x >> 5); r < a.rows;
+       r += warps) {
+    const float* row = a.src + r * a.ld;
+    uint4* out = reinterpret_cast<uint4*>(a.dst + r * 3 * int64_t(a.Dp));
+    for (int g = lane; g < groups; g += 32) {
+      const int k0 = g * 8;
+      float x[8];
+      if (kVec) {
+        const float4 u = __ldg(reinterpret_cast<const float4*>(row + k0));
+        const float4 v = __ldg(reinterpret_cast<const float4*>(row + k0 + 4));
+        x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+        x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+      } else {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    m[i] = -INFINITY;
-    s[i] = 0.f;
-    zt[i] = 0.f;
-    got[i] = false;
-    const int r = row0 + ty * 4 + i;
-    yrow[i] = r < a.N ? a.y[r] - a.y_offset : -1;
-  }
-
-  const int c_begin = t0 * kTileCols;
-  const int c_end = min(a.V, (t0 + nt) * kTileCols);
-  for (int c0 = c_begin; c0 < c_end; c0 += BNS) {
-    float acc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-
-    for (int k0 = 0; k0 < a.D; k0 += BK) {
-      // stage a 64 x 32 block of H and of W, transposed to [k][row]; zeros off the edges
-      for (int e = tid; e < BM * BK; e += NUM_THREADS) {
-        const int r = e / BK, k = e % BK;
-        const int gr = row0 + r, gk = k0 + k;
-        sH[k][r] = (gr < a.N && gk < a.D) ? to_f32<T>(H[size_t(gr) * a.ldh + gk]) : 0.f;
-        const int gc = c0 + r;
-        sW[k][r] = (gc < a.V && gk < a.D) ? to_f32<T>(W[size_t(gc) * a.ldw + gk]) : 0.f;
+        for (int j = 0; j < 8; ++j) x[j] = (k0 + j < a.D) ? __ldg(row + k0 + j) : 0.f;
       }
-      __syncthreads();
-#pragma unroll 8
-      for (int k = 0; k < BK; ++k) {
-        float hv[4], wv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) hv[i] = sH[k][ty * 4 + i];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) wv[j] = sW[k][tx + 16 * j];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(hv[i], wv[j], acc[i][j]);
-      }
-      __syncthreads();
-    }
-
-    // online update of each owned row with this 64-column sub-tile
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float z[4];
-      float tmax = -INFINITY;
+      uint32_t hi[4], lo[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int col = c0 + tx + 16 * j;
-        z[j] = col < a.V ? acc[i][j] : -INFINITY;
-        if (int64_t(col) == yrow[i]) {
-          zt[i] = acc[i][j];
-          got[i] = true;
-        }
-        tmax = fmaxf(tmax, z[j]);
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * j]);
+        const __nv_bfloat16 h1 = __float2bfloat16_rn(x[2 * j + 1]);
+        // hi lies within a factor 2 of x, so x - hi is exact in fp32
+        // (Sterbenz's lemma); its bf16 rounding is the lo part.
+        const __nv_bfloat16 l0 = __float2bfloat16_rn(x[2 * j] - __bfloat162float(h0));
+        const __nv_bfloat16 l1 = __float2bfloat16_rn(x[2 * j + 1] - __bfloat162float(h1));
+        hi[j] = pack_bf16x2(h0, h1);
+        lo[j] = pack_bf16x2(l0, l1);
       }
-#pragma unroll
-      for (int off = 8; off >= 1; off >>= 1)
-        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
-      const float m_new = fmaxf(m[i], tmax);
-      const float ms = m_new * kLog2e;
-      float sum = 0.f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) sum += ptx::ex2(fmaf(z[j], kLog2e, -ms));
-#pragma unroll
-      for (int off = 8; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      s[i] = fmaf(s[i], ptx::ex2((m[i] - m_new) * kLog2e), sum);
-      m[i] = m_new;
-    }
-  }
-
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = row0 + ty * 4 + i;
-    if (r < a.N) {
-      if (tx == 0) a.part[size_t(slab) * size_t(a.N) + size_t(r)] = make_float2(m[i], s[i]);
-      if (got[i]) a.target_logit[r] = zt[i];
+      const uint4 vh = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      const uint4 vl = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      out[g] = vh;
+      out[groups + g] = a.lo_segment == 1 ? vl : vh;
+      out[2 * groups + g] = a.lo_segment == 2 ? vl : vh;
     }
   }
 }
 
-}  // namespace simt
+}  // namespace split
 
 // ----------------------------------------------------------------- merge + mean
 

@@ -59,8 +59,14 @@ def test_workspace_is_O_N_not_O_NV(lib):
     assert lib.flce_workspace_size(4, 0, 8, 0) == 0
     assert lib.flce_workspace_size(4, 10, 0, 0) == 0
     assert lib.flce_workspace_size(4, 10, 8, 7) == 0
-    # independent of dtype and D
-    assert flce.workspace_size(100, 5000, 64) == flce.workspace_size(100, 5000, 4096, 1)
+    # bf16: independent of D
+    assert flce.workspace_size(100, 5000, 64) == flce.workspace_size(100, 5000, 4096)
+    # fp32: plus the bf16 hi/lo split copies of H and W, (rows, 3 * ceil8(D)) each
+    for N, V, D in [(100, 5000, 64), (256, 2048, 256), (7, 9, 5), (1, 1, 1)]:
+        Dp = (D + 7) // 8 * 8
+        r256 = lambda b: (b + 255) // 256 * 256
+        assert flce.workspace_size(N, V, D, 1) == (flce.workspace_size(N, V, D)
+                                                   + r256(6 * Dp * N) + r256(6 * Dp * V))
 
 
 def unit_order(p):
@@ -99,17 +105,16 @@ def test_plan_covers_every_tile_once_and_balances(lib, N, V, D, dtype, sms):
     assert len(order) == p["units"] and len(set(order)) == p["units"]   # each unit exactly once
     assert 1 <= p["group_blocks"] <= p["token_blocks"]
     assert p["workspace_bytes"] == flce.workspace_size(N, V, D, dtype)
-    if dtype == 0:
-        pair = N > 128
-        assert p["ctas_per_unit"] == (2 if pair else 1)
-        assert p["block_rows"] == (256 if pair else 128)
-        workers = sms // 2 if pair else sms
-        assert p["grid"] == min(workers, p["units"]) * p["ctas_per_unit"]
-        assert simulate_makespan(p) == p["makespan_tiles"]
-        total = p["token_blocks"] * p["vocab_tiles"]
-        # within one tile per worker of the perfect split, whenever every worker has work
-        if total >= workers:
-            assert p["makespan_tiles"] <= math.ceil(total / workers) + 1
+    pair = N > 128
+    assert p["ctas_per_unit"] == (2 if pair else 1)
+    assert p["block_rows"] == (256 if pair else 128)
+    workers = sms // 2 if pair else sms
+    assert p["grid"] == min(workers, p["units"]) * p["ctas_per_unit"]
+    assert simulate_makespan(p) == p["makespan_tiles"]
+    total = p["token_blocks"] * p["vocab_tiles"]
+    # within one tile per worker of the perfect split, whenever every worker has work
+    if total >= workers:
+        assert p["makespan_tiles"] <= math.ceil(total / workers) + 1
 
 
 def test_grouped_makespan_matches_simulation_on_random_shapes(lib):

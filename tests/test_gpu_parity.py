@@ -209,3 +209,70 @@ def test_strided_rows_and_int32_targets(dtype, y32):
     # identical to the contiguous call on copies
     ref_gpu = flce.forward(Hs.contiguous(), Ws.contiguous(), yd)
     assert torch.equal(ref_gpu[0], loss)
+
+
+# ---------------------------------------------------------------- fp32 inputs
+# fp32 H and W are split into bf16 hi = bf16(x), lo = bf16(x - hi) and
+# contracted as hi*hi + hi*lo + lo*hi on the tensor cores.  Per product the
+# dropped lo*lo term and the two rounding residues of the lo parts are at most
+# about 3 * 2^-16 |h w|; the fp32 accumulation over K = 3 * ceil8(D) terms
+# adds at most K * 2^-23 of sum |terms| (a loose bound on any summation
+# order).  So |z_gpu - z| <= (3 * 2^-16 + 3 * ceil8(D) * 2^-23) * sum_k |h_k w_k|.
+
+
+def split_error_bound(H, W, y):
+    D = H.shape[1]
+    Dp = (D + 7) // 8 * 8
+    s = np.abs(H.astype(np.float64) * W[y].astype(np.float64)).sum(axis=1)
+    return (3 * 2.0 ** -16 + 3 * Dp * 2.0 ** -23) * s
+
+
+@pytest.mark.parametrize("N,V,D", [(129, 300, 4096), (513, 3000, 9), (300, 2000, 1000), (2, 70000, 24)])
+def test_fp32_more_shapes_every_row(N, V, D):
+    """Ragged D (not a multiple of 8), long D, many vocab slabs, a single CTA tile."""
+    H, W, y = synth.random_inputs(N, V, D, seed=N * 3 + V + D, dtype="fp32")
+    gpu = run(H, W, y)
+    ref = oracle.forward(H, W, y)
+    compare(gpu, ref, mean_ref=oracle.mean(ref["loss"]))
+
+
+def test_fp32_target_logit_within_split_bound():
+    """The target logit is one contraction; its error must respect the derived bound,
+    and stay far below what rounding the fp32 inputs to bf16 would cost."""
+    N, V, D = 512, 4000, 256
+    H, W, y = synth.random_inputs(N, V, D, seed=77, dtype="fp32")
+    gpu = run(H, W, y)
+    ref = oracle.forward(H, W, y)
+    err = np.abs(gpu["target"] - ref["target"])
+    bound = split_error_bound(H, W, y)
+    assert np.all(err <= bound), float((err / bound).max())
+    # rounding H and W to bf16 first would give target-logit errors of about
+    # 2^-9 sqrt(sum (h w)^2) ~ 2e-3 rms here; the split gives about 2^-16 of it
+    assert err.max() < 2e-4
+
+
+def test_fp32_stress_scale_logits():
+    """fp32 rows scaled log-uniformly over [0.1, 10]: logits up to ~+-50."""
+    N, V, D = 384, 9000, 256
+    H, W, y = synth.random_inputs(N, V, D, seed=19, dtype="fp32")
+    sig = np.exp(np.random.default_rng(19).uniform(math.log(0.1), math.log(10.0), V)).astype(np.float32)
+    W = (W * sig[:, None]).astype(np.float32)
+    gpu = run(H, W, y)
+    ref = oracle.forward(H, W, y)
+    compare(gpu, ref, mean_ref=oracle.mean(ref["loss"]))
+
+
+def test_fp32_unaligned_strided_rows():
+    """fp32 row slices at a 4-byte (not 16-byte) offset with an odd row stride:
+    the split kernel's scalar-load path."""
+    import linear_cross_entropy_bf16_b200 as flce
+    N, V, D = 260, 1500, 45
+    H, W, y = synth.random_inputs(N, V, D + 3, seed=23, dtype="fp32")
+    Hd, Wd, yd = to_device(H, W, y)
+    Hs, Ws = Hd[:, 1:1 + D], Wd[:, 3:3 + D]
+    assert Hs.stride(0) == D + 3 and Hs.data_ptr() % 16 != 0
+    loss, lse, tgt, mean = flce.forward_strided(Hs, Ws, yd.to(torch.int32), check=True)
+    ref = oracle.forward(np.ascontiguousarray(H[:, 1:1 + D]), np.ascontiguousarray(W[:, 3:3 + D]), y)
+    gpu = {"loss": loss.cpu().double().numpy(), "lse": lse.cpu().double().numpy(),
+           "target": tgt.cpu().double().numpy(), "mean": float(mean.item())}
+    compare(gpu, ref, mean_ref=oracle.mean(ref["loss"]))
