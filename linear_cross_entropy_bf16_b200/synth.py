@@ -167,3 +167,60 @@ def sample_rows(N: int, k: int, seed: int) -> np.ndarray:
     rng = np.random.default_rng([seed, _S_ROWS])
     inner = rng.choice(np.arange(1, N - 1), size=max(0, k - 2), replace=False)
     return np.sort(np.concatenate([[0, N - 1], inner]).astype(np.int64))
+
+
+# ---------------------------------------------------------------- quantised heads
+
+def pack_codes(q: np.ndarray, bits: int) -> np.ndarray:
+    """Pack unsigned `bits`-bit codes (V, D) into uint32 words (V, D * bits / 32),
+    32 / bits codes per word, element k at bit offset bits * (k mod (32 / bits))."""
+    per = 32 // bits
+    V, D = q.shape
+    q = q.astype(np.uint32).reshape(V, D // per, per)
+    shifts = (np.arange(per, dtype=np.uint32) * bits)[None, None, :]
+    return np.bitwise_or.reduce(q << shifts, axis=2).astype(np.uint32)
+
+
+def quantize_affine(W: np.ndarray, bits: int = 4, group_size: int = 64):
+    """Affine group quantisation of an fp32 (V, D) matrix, MLX-style: per group of
+    `group_size` elements along D, bias = bf16(min), scale = bf16((max - min) / (2^bits - 1))
+    and q = clip(round((w - bias) / scale), 0, 2^bits - 1).
+
+    Returns (wq uint32 (V, D * bits / 32), scales uint16 bf16 bits (V, D / G),
+    biases uint16 bf16 bits (V, D / G)).  This prepares inputs; the loss
+    arithmetic on them lives in the kernels and in the oracle."""
+    V, D = W.shape
+    if D % group_size or bits not in (2, 4, 8):
+        raise ValueError("D must be a multiple of group_size and bits one of 2, 4, 8")
+    ng = D // group_size
+    wq = np.empty((V, D * bits // 32), dtype=np.uint32)
+    sc = np.empty((V, ng), dtype=np.uint16)
+    bi = np.empty((V, ng), dtype=np.uint16)
+    levels = float(2 ** bits - 1)
+    for r0 in range(0, V, CHUNK_ROWS):
+        r1 = min(V, r0 + CHUNK_ROWS)
+        g = W[r0:r1].astype(np.float32).reshape(r1 - r0, ng, group_size)
+        lo = g.min(axis=2)
+        hi = g.max(axis=2)
+        sc[r0:r1] = round_to_bf16_bits(np.maximum((hi - lo) / levels, 1e-12).astype(np.float32))
+        bi[r0:r1] = round_to_bf16_bits(lo)
+        scale = bf16_bits_to_f32(sc[r0:r1])[:, :, None]
+        bias = bf16_bits_to_f32(bi[r0:r1])[:, :, None]
+        q = np.clip(np.rint((g - bias) / scale), 0, levels).astype(np.uint32)
+        wq[r0:r1] = pack_codes(q.reshape(r1 - r0, D), bits)
+    return wq, sc, bi
+
+
+def generate_quantized(w: Workload | str, bits: int = 4, group_size: int = 64,
+                       N: int | None = None, V: int | None = None, D: int | None = None):
+    """(H bf16 bits, (wq, scales, biases), y) for workload `w` with its W (drawn in
+    fp32 by the same recipe) quantised by quantize_affine."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    N = w.N if N is None else N
+    V = w.V if V is None else V
+    D = w.D if D is None else D
+    H = _fill_rows(N, D, w.seed, _S_H, "bf16", None)
+    Wf = _fill_rows(V, D, w.seed, _S_W, "fp32", row_scales(V, D, w.seed, w.w_scale))
+    y = targets(N, V, w.seed, w.targets)
+    return H, quantize_affine(Wf, bits, group_size), y

@@ -73,6 +73,12 @@ def _load():
             lib.oracle_grad_hidden_rows.argtypes = [vp, vp, ctypes.c_int, vp, dp, i64, i64, i64,
                                                     vp, i64, dp, dp, ctypes.c_int]
             lib.oracle_grad_hidden_rows.restype = ctypes.c_int
+            lib.oracle_dequantize.argtypes = [vp, vp, vp, ctypes.c_int, i64, i64, i64, dp]
+            lib.oracle_dequantize.restype = ctypes.c_int
+            lib.oracle_forward_quantized_rows.argtypes = [vp, vp, vp, vp, ctypes.c_int, i64, vp,
+                                                          i64, i64, i64, vp, i64, dp, dp, dp, dp,
+                                                          ctypes.c_int]
+            lib.oracle_forward_quantized_rows.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -209,3 +215,59 @@ def grad_hidden_rows(H: np.ndarray, W: np.ndarray, y: np.ndarray, g, rows, nthre
     if rc != 0:
         raise OracleError(_ERRORS.get(rc, f"oracle error {rc}"))
     return {"dH": dH, "bH": bH}
+
+
+def _quant_arrays(wq, scales, biases, bits, group_size):
+    wq = np.ascontiguousarray(wq)
+    scales = np.ascontiguousarray(scales)
+    biases = np.ascontiguousarray(biases)
+    if wq.dtype != np.uint32 or scales.dtype != np.uint16 or biases.dtype != np.uint16:
+        raise TypeError("wq must be uint32 codes, scales and biases uint16 bf16 bit patterns")
+    V = wq.shape[0]
+    D = wq.shape[1] * (32 // bits)
+    if scales.shape != (V, D // group_size) or biases.shape != scales.shape:
+        raise ValueError("scales and biases must be (V, D / group_size)")
+    return wq, scales, biases, V, D
+
+
+def dequantize(wq: np.ndarray, scales: np.ndarray, biases: np.ndarray, bits: int = 4,
+               group_size: int = 64) -> np.ndarray:
+    """The affine-quantised W (V, D) in float64: W_jk = s_jg q_jk + b_jg (g = k // group_size)."""
+    lib = _load()
+    wq, scales, biases, V, D = _quant_arrays(wq, scales, biases, bits, group_size)
+    W = np.empty((V, D), dtype=np.float64)
+    rc = lib.oracle_dequantize(_ptr(wq), _ptr(scales), _ptr(biases), int(bits), int(group_size),
+                               V, D, _ptr(W))
+    if rc != 0:
+        raise OracleError(_ERRORS.get(rc, f"oracle error {rc}"))
+    return W
+
+
+def forward_quantized(H: np.ndarray, wq: np.ndarray, scales: np.ndarray, biases: np.ndarray,
+                      y: np.ndarray, bits: int = 4, group_size: int = 64, rows=None,
+                      nthreads: int = 0):
+    """forward() with an affine-quantised head; H is (N, D) bf16 bit patterns (uint16)."""
+    lib = _load()
+    H = np.ascontiguousarray(H)
+    if H.dtype != np.uint16 or H.ndim != 2:
+        raise TypeError("H must be (N, D) bf16 bit patterns (uint16)")
+    wq, scales, biases, V, D = _quant_arrays(wq, scales, biases, bits, group_size)
+    N = H.shape[0]
+    if H.shape[1] != D:
+        raise ValueError("H and the quantised W disagree on D")
+    y = np.ascontiguousarray(y, dtype=np.int64)
+    if y.shape != (N,):
+        raise ValueError("y must have length N")
+    if rows is None:
+        rows_arr, n = None, N
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        n = rows_arr.shape[0]
+    out = {k: np.empty(n, dtype=np.float64) for k in ("loss", "lse", "target", "max")}
+    rc = lib.oracle_forward_quantized_rows(_ptr(H), _ptr(wq), _ptr(scales), _ptr(biases), int(bits),
+                                           int(group_size), _ptr(y), N, V, D, _ptr(rows_arr), n,
+                                           _ptr(out["loss"]), _ptr(out["lse"]), _ptr(out["target"]),
+                                           _ptr(out["max"]), int(nthreads))
+    if rc != 0:
+        raise OracleError(_ERRORS.get(rc, f"oracle error {rc}"))
+    return out

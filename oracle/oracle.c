@@ -320,6 +320,130 @@ int oracle_grad_logits_row(const void *H, const void *W, int dtype, const int64_
     return ORACLE_OK;
 }
 
+/*
+ * Quantised output head.
+ *
+ * Source: the same page, section 2: the first (pure MLX) prototype supported
+ * "dense and quantised output heads"; section 9 leaves the quantised variants
+ * out of the measured scope.  The page does not define the format.  Reading:
+ * the affine group quantisation of MLX, the library that prototype is built
+ * on.  Each row j of W is cut into groups of G consecutive elements along D;
+ * group g of row j has a scale s_jg and a bias b_jg (bf16 bit patterns), and
+ * element k holds an unsigned `bits`-bit code q_jk, so that
+ *     W_jk = s_{j, floor(k/G)} * q_jk + b_{j, floor(k/G)}.
+ * The codes of one row are packed 32/bits to a uint32 word, lowest bits
+ * first: element k sits in word floor(k / (32/bits)) of the row at bit offset
+ * bits * (k mod (32/bits)); a row takes D * bits / 32 words.
+ * Supported here: bits in {2, 4, 8}, G in {32, 64, 128}, D a multiple of G.
+ * The loss is the section-1 definition applied to that W, in fp64: every W_jk
+ * is formed exactly (s q is exact in fp64 and so is the sum with b for bf16
+ * operands of any practical range) and each logit is a sequential sum over k.
+ */
+static double bf16_bits_value(uint16_t b) {
+    uint32_t bits = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+static int quant_args_ok(int bits, int64_t G, int64_t D) {
+    if (bits != 2 && bits != 4 && bits != 8) return 0;
+    if (G != 32 && G != 64 && G != 128) return 0;
+    return D >= G && D % G == 0;
+}
+
+/* The code q_jk, unpacked from its word. */
+static uint32_t quant_code(const uint32_t *wq, int bits, int64_t D, int64_t j, int64_t k) {
+    const int64_t per_word = 32 / bits;
+    const uint32_t word = wq[j * (D / per_word) + k / per_word];
+    return (word >> (bits * (int)(k % per_word))) & ((1u << bits) - 1u);
+}
+
+/* W_jk = s_jg q_jk + b_jg with g = floor(k / G). */
+static double dequant_elem(const uint32_t *wq, const uint16_t *scales, const uint16_t *biases,
+                           int bits, int64_t G, int64_t D, int64_t j, int64_t k) {
+    const int64_t g = j * (D / G) + k / G;
+    return bf16_bits_value(scales[g]) * (double)quant_code(wq, bits, D, j, k) +
+           bf16_bits_value(biases[g]);
+}
+
+/* The whole dequantised W (V x D doubles), for small cases. */
+int oracle_dequantize(const uint32_t *wq, const uint16_t *scales, const uint16_t *biases,
+                      int bits, int64_t G, int64_t V, int64_t D, double *W) {
+    if (!wq || !scales || !biases || !W || V < 1 || !quant_args_ok(bits, G, D))
+        return ORACLE_ERR_ARG;
+    for (int64_t j = 0; j < V; ++j)
+        for (int64_t k = 0; k < D; ++k)
+            W[j * D + k] = dequant_elem(wq, scales, biases, bits, G, D, j, k);
+    return ORACLE_OK;
+}
+
+/*
+ * Per-token outputs for a subset of rows with a quantised head: H is (N, D)
+ * bf16 bit patterns; wq, scales and biases hold W as described above.  Same
+ * row selection, outputs and errors as oracle_forward_rows.  Each logit is
+ * z_ij = sum_k H_ik W_jk with W_jk formed on the fly (the full W is never
+ * held), then the same two-pass log-sum-exp.
+ */
+int oracle_forward_quantized_rows(const uint16_t *H, const uint32_t *wq, const uint16_t *scales,
+                                  const uint16_t *biases, int bits, int64_t G,
+                                  const int64_t *y, int64_t N, int64_t V, int64_t D,
+                                  const int64_t *rows, int64_t nrows, double *out_loss,
+                                  double *out_lse, double *out_target, double *out_max,
+                                  int nthreads) {
+    if (!H || !wq || !scales || !biases || !y || N < 0 || V < 1 || nrows < 0 ||
+        !quant_args_ok(bits, G, D))
+        return ORACLE_ERR_ARG;
+    if (!rows && nrows != N) return ORACLE_ERR_ARG;
+    for (int64_t t = 0; t < nrows; ++t) {
+        int64_t i = rows ? rows[t] : t;
+        if (i < 0 || i >= N) return ORACLE_ERR_ARG;
+        if (y[i] < 0 || y[i] >= V) return ORACLE_ERR_TARGET;
+    }
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int status = ORACLE_OK;
+#pragma omp parallel
+    {
+        double *z = (double *)malloc((size_t)V * sizeof(double));
+        double *h = (double *)malloc((size_t)D * sizeof(double));
+        if (!z || !h) {
+#pragma omp atomic write
+            status = ORACLE_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < nrows; ++t) {
+            if (!z || !h) continue;
+            int64_t i = rows ? rows[t] : t;
+            for (int64_t k = 0; k < D; ++k) h[k] = bf16_bits_value(H[i * D + k]);
+            /* Z_i with the dequantised W */
+            for (int64_t j = 0; j < V; ++j) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < D; ++k)
+                    acc += h[k] * dequant_elem(wq, scales, biases, bits, G, D, j, k);
+                z[j] = acc;
+            }
+            double M = z[0];
+            for (int64_t j = 1; j < V; ++j)
+                if (z[j] > M) M = z[j];
+            double S = 0.0;
+            for (int64_t j = 0; j < V; ++j) S += exp(z[j] - M);
+            double lse = M + log(S);
+            double tgt = z[y[i]];
+            if (out_loss) out_loss[t] = lse - tgt;
+            if (out_lse) out_lse[t] = lse;
+            if (out_target) out_target[t] = tgt;
+            if (out_max) out_max[t] = M;
+        }
+        free(z);
+        free(h);
+    }
+    return status;
+}
+
 /* Mean loss: (sum_i loss_i) / n, summed sequentially in fp64.  n == 0 gives NaN. */
 double oracle_mean(const double *loss, int64_t n) {
     if (!loss || n <= 0) return NAN;
