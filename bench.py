@@ -387,6 +387,10 @@ def run_ours(args, w, rank, world, local_rank):
     if args.backward and w.dtype == "bf16":
         line["backward"] = time_backward(flce, H, W, y, lse, N, V, D, tdt, dev, stream, args,
                                          peaks["bf16_tflops"], world)
+    if args.quantized and w.dtype == "bf16":
+        bits, gs = (int(v) for v in args.quantized.split(","))
+        line["quantized"] = time_quantized(flce, H, Wn, y, N, V, D, bits, gs, dev, stream, args,
+                                           peaks["bf16_tflops"], world)
     if world == 1 and not args.no_cpu_baseline:
         rows, secs, cores = oracle_sample(Hn, Wn, yn, args.cpu_seconds, w.seed)
         line["cpu_baseline"] = {"value": rows / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -429,6 +433,51 @@ def time_backward(flce, H, W, y, lse, N, V, D, tdt, dev, stream, args, peak, wor
             "what": "dH and dW of the mean loss from the forward's lse (3 contractions per step)"}
 
 
+def time_quantized(flce, H, Wn, y, N, V, D, bits, gs, dev, stream, args, peak, world):
+    """The forward with the workload's W quantised to `bits`-bit codes in groups of `gs`
+    (affine, MLX layout), on the same H and y, timed like the forward."""
+    import torch
+    wq, sc, bi = synth.quantize_affine(synth.bf16_bits_to_f32(Wn), bits, gs)
+    wqd = torch.from_numpy(wq.view(np.int32)).to(dev)
+    scd = torch.from_numpy(sc).view(torch.bfloat16).to(dev)
+    bid = torch.from_numpy(bi).view(torch.bfloat16).to(dev)
+    ws = torch.empty(flce.quantized_workspace_size(N, V, D, bits, gs), dtype=torch.uint8, device=dev)
+    out = {"loss": torch.empty(N, device=dev), "lse": torch.empty(N, device=dev),
+           "target_logit": torch.empty(N, device=dev), "mean": torch.empty((), device=dev)}
+
+    def step():
+        flce.forward_quantized(H, wqd, scd, bid, y, bits, gs, out=out, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    stream.synchronize()
+    if flce.check(ws, stream) != flce.OK:
+        raise flce.FlceError(flce.check(ws, stream), "forward_quantized")
+    Kq = max(3, args.steps // 2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(Kq):
+            step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks([e0.elapsed_time(e1) / Kq], world, device=dev)[0]
+    flops = 2 * N * V * D
+    Ds = (D + 63) // 64 * 64
+    tensor_flops = 2 * N * V * 2 * Ds      # [H | H] against [hi | lo]
+    head_bytes = wq.nbytes + sc.nbytes + bi.nbytes
+    return {"bits": bits, "group_size": gs, "ms_per_step": ms, "steps": Kq,
+            "tokens_per_s": weak_scaling_tokens_per_s(world, N, ms),
+            "tflops": flops / (ms * 1e-3) / 1e12,
+            "tensor_tflops": tensor_flops / (ms * 1e-3) / 1e12,
+            "tensor_frac_of_bf16_peak": tensor_flops / (ms * 1e-3) / 1e12 / peak,
+            "head_bytes": int(head_bytes), "bf16_head_bytes": int(2 * V * D),
+            "workspace_bytes": int(ws.numel()), "mean_loss": float(out["mean"].item()),
+            "what": "forward with an affine group-quantised head: W expanded per 16384-row chunk "
+                    "to bf16 hi/lo, 2 bf16 products per weight"}
+
+
 def torch_materialised(H, W, y, dev):
     """The materialising forward (cuBLAS logits + logsumexp) timed the same way, for context."""
     import torch
@@ -467,6 +516,8 @@ def main():
     ap.add_argument("--backward", action="store_true",
                     help="also time the backward (dH, dW) and add a 'backward' object to the line")
     ap.add_argument("--backward-steps", type=int, default=10)
+    ap.add_argument("--quantized", default=None, metavar="BITS,GROUP",
+                    help="also time the forward with W quantised (e.g. 4,64) and add a 'quantized' object")
     ap.add_argument("--context", action="store_true", help="also time the materialising torch forward")
     ap.add_argument("--shape", default=None,
                     help="N,V,D: a custom shape with the chosen workload's distributions "

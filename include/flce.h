@@ -324,6 +324,53 @@ FLCE_API flce_status flce_forward_noalloc(const void* H, const void* W, const in
                                           float* out_loss, float* out_lse, float* out_target_logit,
                                           float* out_mean, void* stream);
 
+/*
+ * Quantised output head.
+ *
+ * The page (section 2) says its first, pure-MLX prototype supported dense and
+ * quantised output heads; it does not define the quantised format, and its
+ * measurements leave the quantised variants out (section 9).  Format read
+ * here: MLX's affine group quantisation.  Each row j of W (V, D) is cut into
+ * groups of G consecutive elements along D; group g of row j has a bf16 scale
+ * s_jg and a bf16 bias b_jg, and element k holds an unsigned `bits`-bit code
+ * q_jk, so that
+ *     W_jk = s_{j, k/G} * q_jk + b_{j, k/G}.
+ * The loss is the section-1 operation on that W.
+ *
+ *   H        (N, D) bf16, contiguous, 16-byte aligned
+ *   wq       (V, D * bits / 32) uint32, contiguous, 16-byte aligned: the codes
+ *            of a row packed 32 / bits per word, lowest bits first (element k
+ *            in word k / (32/bits) at bit offset bits * (k mod (32/bits)))
+ *   scales, biases   (V, D / G) bf16 each, contiguous
+ *   bits     2, 4 or 8;  group_size G: 32, 64 or 128;  D a multiple of G
+ *   y, N, V, D, out_*      as flce_forward (int64 targets)
+ *   workspace  >= flce_quantized_workspace_size(N, V, D, bits, group_size)
+ *            bytes, 256-byte aligned; holds the status word flce_check() reads
+ *
+ * How it runs: W is expanded 16384 vocabulary rows at a time into the
+ * workspace as two bf16 K segments per row, hi = bf16(W_jk) and lo =
+ * bf16(W_jk - hi) (W_jk formed in fp32 with one rounding), and the
+ * tensor-core contraction takes [H | H] against [hi | lo]: twice the work of
+ * a bf16 head, with |W - hi - lo| <= 2^-16 |W| per weight.  Each chunk is a
+ * vocabulary shard; their per-token states are merged at the end, in chunk
+ * order.  The workspace is O(N V / 16384 + 16384 D), never O(N V).
+ * Errors: FLCE_ERR_INVALID_ARG for bad sizes, formats, null pointers or a
+ * misaligned workspace / scales / biases; FLCE_ERR_UNSUPPORTED for a
+ * misaligned H or wq, sizes beyond int32 or a device that is not sm_100;
+ * FLCE_ERR_WORKSPACE_TOO_SMALL.  Targets are checked on the device as in
+ * flce_forward.  N == 0 is a no-op that returns FLCE_OK.
+ */
+FLCE_API size_t flce_quantized_workspace_size(int64_t N, int64_t V, int64_t D, int32_t bits,
+                                              int32_t group_size);
+
+FLCE_API flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
+                                            const void* scales, const void* biases,
+                                            int32_t bits, int32_t group_size, const int64_t* y,
+                                            int64_t N, int64_t V, int64_t D, float* out_loss,
+                                            float* out_lse, float* out_target_logit,
+                                            float* out_mean, void* workspace,
+                                            size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,6 +24,7 @@ import torch
 __all__ = [
     "FlceError", "forward", "backward", "partials", "merge", "workspace_size",
     "shard_state", "merge_shards", "forward_vocab_parallel", "forward_strided",
+    "forward_quantized", "quantized_workspace_size",
     "backward_workspace_size", "plan", "check",
     "status_string", "selftest_wait_timeout", "library_path", "load_library",
 ]
@@ -131,6 +132,12 @@ def load_library():
         lib.flce_merge_shards.restype = st
         lib.flce_forward_ex.argtypes = [ctypes.POINTER(ForwardArgs), vp, sz, vp]
         lib.flce_forward_ex.restype = st
+        i32 = ctypes.c_int32
+        lib.flce_quantized_workspace_size.argtypes = [i64, i64, i64, i32, i32]
+        lib.flce_quantized_workspace_size.restype = sz
+        lib.flce_forward_quantized.argtypes = [vp, vp, vp, vp, i32, i32, vp, i64, i64, i64,
+                                               vp, vp, vp, vp, vp, sz, vp]
+        lib.flce_forward_quantized.restype = st
         _lib = lib
         return lib
 
@@ -466,3 +473,51 @@ def forward_noalloc(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, out: dict
             *(t.data_ptr() for t in tensors), _stream_ptr(stream, H.device))
     _raise_on(st, "flce_forward_noalloc")
     return tuple(tensors)
+
+
+def quantized_workspace_size(N: int, V: int, D: int, bits: int = 4, group_size: int = 64) -> int:
+    n = load_library().flce_quantized_workspace_size(int(N), int(V), int(D), int(bits), int(group_size))
+    if n == 0:
+        raise FlceError(ERR_INVALID_ARG, "quantized_workspace_size")
+    return int(n)
+
+
+def forward_quantized(H: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+                      y: torch.Tensor, bits: int = 4, group_size: int = 64, *, out: dict | None = None,
+                      workspace: torch.Tensor | None = None, stream=None, check: bool = False):
+    """flce_forward_quantized: the forward with an affine group-quantised head
+    W = scales * q + biases (MLX layout: wq (V, D * bits / 32) int32/uint32 codes,
+    scales and biases (V, D / group_size) bf16).  Returns (loss, lse, target_logit, mean)."""
+    if H.dtype != torch.bfloat16 or H.dim() != 2 or not H.is_contiguous() or not H.is_cuda:
+        raise ValueError("H must be a contiguous 2-D bf16 CUDA tensor")
+    dev = H.device
+    N, D = H.shape
+    if wq.dtype not in (torch.int32, torch.uint32) or wq.dim() != 2 or not wq.is_contiguous():
+        raise ValueError("wq must be a contiguous 2-D int32/uint32 tensor of packed codes")
+    V = wq.shape[0]
+    if wq.shape[1] * 32 != D * bits:
+        raise ValueError("wq must have D * bits / 32 words per row")
+    for name, t in (("scales", scales), ("biases", biases)):
+        if (t.dtype != torch.bfloat16 or not t.is_contiguous() or t.device != dev
+                or tuple(t.shape) != (V, D // group_size)):
+            raise ValueError(f"{name} must be a contiguous bf16 (V, D / group_size) tensor")
+    if wq.device != dev or y.device != dev or y.dtype != torch.int64 or y.shape != (N,) \
+            or not y.is_contiguous():
+        raise ValueError("wq and y must be on H's device; y contiguous int64 of length N")
+    loss, lse, tgt, mean = _alloc_outputs(N, dev, out)
+    if N == 0:
+        return loss, lse, tgt, mean
+    lib = load_library()
+    need = quantized_workspace_size(N, V, D, bits, group_size)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    nbytes = workspace.numel() * workspace.element_size()
+    sp = _stream_ptr(stream, dev)
+    _raise_on(lib.flce_forward_quantized(H.data_ptr(), wq.data_ptr(), scales.data_ptr(),
+                                         biases.data_ptr(), int(bits), int(group_size), y.data_ptr(),
+                                         N, V, D, loss.data_ptr(), lse.data_ptr(), tgt.data_ptr(),
+                                         mean.data_ptr(), workspace.data_ptr(), nbytes, sp),
+              "flce_forward_quantized")
+    if check:
+        _raise_on(lib.flce_check(workspace.data_ptr(), sp), "flce_forward_quantized (device)")
+    return loss, lse, tgt, mean

@@ -272,6 +272,71 @@ flce_status check_forward_args(const void* H, const void* W, const int64_t* y, i
   return FLCE_OK;
 }
 
+// Device facts and the number of concurrent workers (CTAs or CTA pairs) the
+// contraction kernel gets for N tokens; sets the kernels' shared-memory limit.
+flce_status contraction_workers(int64_t N, DeviceInfo& di, int64_t& workers) {
+  flce_status s = device_info(di);
+  if (s != FLCE_OK) return s;
+  if ((s = set_smem_attr_once()) != FLCE_OK) return s;
+  workers = nominal_workers(di.sms, N);
+  if (use_pair_kernel(N)) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+    workers = resident_pairs(dev, di.sms);
+  }
+  return FLCE_OK;
+}
+
+// The contraction with the online (m, s) epilogue on bf16 operands: opH (N
+// rows, Kh columns, row stride ldh) and opW (V rows, Kw columns, row stride
+// ldw).  The kernel walks Kw in 64-element blocks; H's K coordinate wraps
+// after ceil(Kh / 64) blocks (Kh == Kw except for the quantised head).
+// Writes (m, s) per (slab, token) after the workspace header and the target
+// logits W owns.  reset_header: clear the header (status word) first.
+flce_status launch_contraction(const void* opH, int64_t ldh, int64_t Kh, const void* opW,
+                               int64_t ldw, int64_t Kw, Targets y, int64_t y_offset, int64_t N,
+                               int64_t V, const flce_plan_t& plan, float* out_target, void* ws,
+                               bool reset_header, cudaStream_t st) {
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
+  float2* part = reinterpret_cast<float2*>(wsb + kHeaderBytes);
+  if (reset_header && cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+
+  Schedule sch;
+  sch.token_blocks = int32_t(plan.token_blocks);
+  sch.slabs = plan.slabs;
+  sch.slab_base = plan.slab_base;
+  sch.slab_rem = plan.slab_rem;
+  sch.units = int32_t(plan.units);
+  sch.group_blocks = plan.group_blocks;
+
+  if (!load_encoder()) return FLCE_ERR_CUDA;
+  const bool pair = plan.ctas_per_unit == 2;
+  CUtensorMap tmH, tmW;
+  if (!encode_bf16_rows(&tmH, opH, N, Kh, ldh, tc::BM) ||
+      !encode_bf16_rows(&tmW, opW, V, Kw, ldw, pair ? tc2::HALF_N : tc::BN))
+    return FLCE_ERR_UNSUPPORTED;
+  tc::Args a;
+  a.y = y;
+  a.y_offset = y_offset;
+  a.part = part;
+  a.target_logit = out_target;
+  a.hdr = hdr;
+  a.N = int32_t(N);
+  a.V = int32_t(V);
+  a.D = int32_t(Kw);
+  a.kblocks = int32_t(cdiv(Kw, tc::BK));
+  a.kblocks_h = int32_t(cdiv(Kh, tc::BK));
+  a.sch = sch;
+  a.wait_limit_ns = kDefaultWaitLimitNs;
+  if (pair)
+    tc2::flce_tc2_kernel<<<plan.grid, tc2::NUM_THREADS, tc2::SMEM_BYTES, st>>>(tmH, tmW, a);
+  else
+    tc::flce_tc_kernel<<<plan.grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(tmH, tmW, a);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
 // fp32 inputs: split `src` (rows, D; row stride ld) into its bf16 (rows,
 // 3 Dp) copy at `dst` with hi / lo parts in the segments the operand needs.
 flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, int lo_segment,
@@ -295,26 +360,16 @@ flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, i
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
+// Stage 1 of the forward for bf16 or fp32 H and W (fp32: split first).
 flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t ldw, Targets y,
                             int64_t y_offset, int64_t N, int64_t V, int64_t D, flce_dtype dtype,
                             float* out_target, void* ws, cudaStream_t st) {
   DeviceInfo di;
-  flce_status s = device_info(di);
+  int64_t workers = 0;
+  flce_status s = contraction_workers(N, di, workers);
   if (s != FLCE_OK) return s;
-  if ((s = set_smem_attr_once()) != FLCE_OK) return s;
-  int64_t workers = nominal_workers(di.sms, N);
-  if (use_pair_kernel(N)) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
-    workers = resident_pairs(dev, di.sms);
-  }
   flce_plan_t plan;
   make_plan(N, V, D, dtype, workers, &plan);
-
-  uint8_t* wsb = static_cast<uint8_t*>(ws);
-  WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
-  float2* part = reinterpret_cast<float2*>(wsb + kHeaderBytes);
-  if (cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
 
   // The operands the tensor-core kernels read: H and W themselves (bf16), or
   // their split copies in the workspace (fp32), K = 3 Dp.
@@ -322,6 +377,7 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
   const void* opW = W;
   int64_t K = D;
   if (dtype == FLCE_FP32) {
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
     K = k_extent(D, dtype);
     uint8_t* hs = wsb + state_bytes_for(N, V);
     uint8_t* wsplit = hs + split_bytes_for(N, D);
@@ -332,38 +388,8 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
     ldh = K;
     ldw = K;
   }
-
-  Schedule sch;
-  sch.token_blocks = int32_t(plan.token_blocks);
-  sch.slabs = plan.slabs;
-  sch.slab_base = plan.slab_base;
-  sch.slab_rem = plan.slab_rem;
-  sch.units = int32_t(plan.units);
-  sch.group_blocks = plan.group_blocks;
-
-  if (!load_encoder()) return FLCE_ERR_CUDA;
-  const bool pair = plan.ctas_per_unit == 2;
-  CUtensorMap tmH, tmW;
-  if (!encode_bf16_rows(&tmH, opH, N, K, ldh, tc::BM) ||
-      !encode_bf16_rows(&tmW, opW, V, K, ldw, pair ? tc2::HALF_N : tc::BN))
-    return FLCE_ERR_UNSUPPORTED;
-  tc::Args a;
-  a.y = y;
-  a.y_offset = y_offset;
-  a.part = part;
-  a.target_logit = out_target;
-  a.hdr = hdr;
-  a.N = int32_t(N);
-  a.V = int32_t(V);
-  a.D = int32_t(K);
-  a.kblocks = int32_t(cdiv(K, tc::BK));
-  a.sch = sch;
-  a.wait_limit_ns = kDefaultWaitLimitNs;
-  if (pair)
-    tc2::flce_tc2_kernel<<<plan.grid, tc2::NUM_THREADS, tc2::SMEM_BYTES, st>>>(tmH, tmW, a);
-  else
-    tc::flce_tc_kernel<<<plan.grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(tmH, tmW, a);
-  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+  return launch_contraction(opH, ldh, K, opW, ldw, K, y, y_offset, N, V, plan, out_target, ws,
+                            true, st);
 }
 
 flce_status launch_merge(Targets y, int64_t N, int64_t V, float* out_loss, float* out_lse,
@@ -791,4 +817,133 @@ extern "C" flce_status flce_forward_noalloc(const void* H, const void* W, const 
   // every other scratch byte it reads is written earlier in the same call.
   return flce_forward(H, W, y, N, V, D, dtype, out_loss, out_lse, out_target_logit, out_mean,
                       scratch, size_t(FLCE_NOALLOC_SCRATCH_BYTES), stream);
+}
+
+// ---------------------------------------------------------------- quantised head
+
+namespace {
+
+// Vocabulary rows expanded at a time (a multiple of the 256-column tile).
+constexpr int64_t kQuantChunkRows = 16384;
+
+bool quant_format_ok(int32_t bits, int64_t G, int64_t D) {
+  if (bits != 2 && bits != 4 && bits != 8) return false;
+  if (G != 32 && G != 64 && G != 128) return false;
+  return D >= G && D % G == 0;
+}
+
+// One K segment of the expanded W: D rounded up to the 64-element K block.
+int64_t quant_segment(int64_t D) { return cdiv(D, tc::BK) * tc::BK; }
+
+// Workspace of the quantised forward: the slab state of one chunk (header,
+// partials, the mean's block sums), one float4 per (chunk, token), and the
+// expanded [hi | lo] bf16 rows of one chunk.
+struct QuantLayout {
+  int64_t C = 0, chunks = 0;
+  size_t state = 0, states = 0, expanded = 0, total = 0;
+};
+
+QuantLayout quant_layout(int64_t N, int64_t V, int64_t D) {
+  QuantLayout L;
+  L.C = std::min(V, kQuantChunkRows);
+  L.chunks = cdiv(V, L.C);
+  L.state = state_bytes_for(N, L.C);
+  L.states = align256(size_t(16) * size_t(N) * size_t(L.chunks));
+  L.expanded = align256(size_t(L.C) * size_t(2 * quant_segment(D)) * 2);
+  L.total = L.state + L.states + L.expanded;
+  return L;
+}
+
+flce_status launch_dequant(const uint32_t* wq, const void* scales, const void* biases,
+                           int32_t bits, int32_t G, int64_t row0, int64_t rows, int64_t D,
+                           void* dst, int sms, cudaStream_t st) {
+  quant::Args a;
+  a.wq = wq;
+  a.scales = static_cast<const __nv_bfloat16*>(scales);
+  a.biases = static_cast<const __nv_bfloat16*>(biases);
+  a.row0 = row0;
+  a.rows = rows;
+  a.D = int32_t(D);
+  a.Ds = int32_t(quant_segment(D));
+  a.G = G;
+  a.dst = static_cast<__nv_bfloat16*>(dst);
+  const int64_t warps_per_block = quant::NUM_THREADS / 32;
+  const unsigned blocks = unsigned(std::max<int64_t>(
+      1, std::min<int64_t>(cdiv(rows, warps_per_block), int64_t(sms) * 8)));
+  if (bits == 4)
+    quant::flce_dequant_split_kernel<4><<<blocks, quant::NUM_THREADS, 0, st>>>(a);
+  else if (bits == 8)
+    quant::flce_dequant_split_kernel<8><<<blocks, quant::NUM_THREADS, 0, st>>>(a);
+  else
+    quant::flce_dequant_split_kernel<2><<<blocks, quant::NUM_THREADS, 0, st>>>(a);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" size_t flce_quantized_workspace_size(int64_t N, int64_t V, int64_t D, int32_t bits,
+                                                int32_t group_size) {
+  if (N < 0 || V < 1 || D < 1 || !quant_format_ok(bits, group_size, D)) return 0;
+  return quant_layout(N, V, D).total;
+}
+
+extern "C" flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
+                                              const void* scales, const void* biases,
+                                              int32_t bits, int32_t group_size, const int64_t* y,
+                                              int64_t N, int64_t V, int64_t D, float* out_loss,
+                                              float* out_lse, float* out_target_logit,
+                                              float* out_mean, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  if (N < 0 || V < 1 || D < 1 || !quant_format_ok(bits, group_size, D))
+    return FLCE_ERR_INVALID_ARG;
+  if (N == 0) return FLCE_OK;
+  if (!H || !wq || !scales || !biases || !y || !out_loss || !out_lse || !out_target_logit ||
+      !workspace)
+    return FLCE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      ((reinterpret_cast<uintptr_t>(scales) | reinterpret_cast<uintptr_t>(biases)) & 1u) != 0)
+    return FLCE_ERR_INVALID_ARG;
+  if (!aligned16(H) || !aligned16(wq)) return FLCE_ERR_UNSUPPORTED;
+  if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31) || 2 * quant_segment(D) >= (int64_t(1) << 31))
+    return FLCE_ERR_UNSUPPORTED;
+  const QuantLayout L = quant_layout(N, V, D);
+  if (workspace_bytes < L.total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DeviceInfo di;
+  int64_t workers = 0;
+  flce_status s = contraction_workers(N, di, workers);
+  if (s != FLCE_OK) return s;
+
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
+  float4* states = reinterpret_cast<float4*>(wsb + L.state);
+  void* expanded = wsb + L.state + L.states;
+  const int64_t Ds = quant_segment(D);
+  // One header for the whole call: its status word collects every stage's
+  // findings, and the final merge's block counter starts at zero.
+  if (cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
+  for (int64_t c = 0; c < L.chunks; ++c) {
+    const int64_t c0 = c * L.C;
+    const int64_t rows = std::min(L.C, V - c0);
+    if ((s = launch_dequant(wq, scales, biases, bits, group_size, c0, rows, D, expanded, di.sms,
+                            st)) != FLCE_OK)
+      return s;
+    flce_plan_t plan;
+    make_plan(N, rows, D, FLCE_BF16, workers, &plan);
+    // [H | H] against [hi | lo]: H's K coordinate wraps after Ds.
+    if ((s = launch_contraction(H, D, D, expanded, 2 * Ds, 2 * Ds, Targets{y, 0}, c0, N, rows,
+                                plan, out_target_logit, workspace, false, st)) != FLCE_OK)
+      return s;
+    flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
+        reinterpret_cast<const float2*>(wsb + kHeaderBytes), hdr, y, int32_t(N), c0, rows,
+        int32_t(slab_capacity(rows)), out_target_logit, states + c * N, &hdr->status);
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  }
+  double* block_sums = reinterpret_cast<double*>(
+      wsb + kHeaderBytes + align256(size_t(8) * size_t(N) * size_t(slab_capacity(L.C))));
+  flce_merge_shards_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
+      states, int32_t(L.chunks), y, int32_t(N), V, out_loss, out_lse, out_target_logit, out_mean,
+      block_sums, hdr);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }

@@ -237,7 +237,9 @@ struct Args {
   float* target_logit;     // [N]
   WsHeader* hdr;
   int32_t N, V, D;
-  int32_t kblocks;         // ceil(D / BK)
+  int32_t kblocks;         // K-blocks of W per tile: ceil(K / BK)
+  int32_t kblocks_h;       // K-blocks of H; H's K coordinate wraps modulo this
+                           // (== kblocks, except for the quantised head's [H | H])
   Schedule sch;
   uint64_t wait_limit_ns;
 };
@@ -307,7 +309,7 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
         int slab, tb, t0, nt;
         unit_coords(sch, u, slab, tb, t0, nt);
         for (int t = t0; ok && t < t0 + nt; ++t) {
-          for (int kb = 0; kb < a.kblocks; ++kb) {
+          for (int kb = 0, kh = 0; kb < a.kblocks; ++kb) {
             if (!wait_bounded(ptx::smem_addr(&empty_bar[stage]), phase ^ 1u, abort_flag, status, lim)) {
               ok = false;
               break;
@@ -315,8 +317,9 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
             const uint32_t fb = ptx::smem_addr(&full_bar[stage]);
             const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
             ptx::mbar_arrive_expect_tx(fb, STAGE_BYTES);
-            ptx::tma_load_2d(sa, &tmH, fb, kb * BK, tb * BM);
+            ptx::tma_load_2d(sa, &tmH, fb, kh * BK, tb * BM);
             ptx::tma_load_2d(sa + A_BYTES, &tmW, fb, kb * BK, t * BN);
+            if (++kh == a.kblocks_h) kh = 0;
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) {
@@ -536,7 +539,7 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
         const int hrow = tb * PAIR_M + int(rank) * BM;
         for (int t = t0; ok && t < t0 + nt; ++t) {
           const int wrow = t * BN + int(rank) * HALF_N;
-          for (int kb = 0; kb < a.kblocks; ++kb) {
+          for (int kb = 0, kh = 0; kb < a.kblocks; ++kb) {
             if (!wait_bounded(ptx::smem_addr(&empty_bar[stage]), phase ^ 1u, abort_flag, status,
                               lim)) {
               ok = false;
@@ -546,8 +549,9 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
             const uint32_t fb_even = ptx::map_to_cta(fb_local, 0);
             const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
             if (rank == 0) ptx::mbar_arrive_expect_tx(fb_local, PAIR_TX_BYTES);
-            ptx::tma_load_2d_pair(sa, &tmH, fb_even, kb * BK, hrow);
+            ptx::tma_load_2d_pair(sa, &tmH, fb_even, kh * BK, hrow);
             ptx::tma_load_2d_pair(sa + A_BYTES, &tmW, fb_even, kb * BK, wrow);
+            if (++kh == a.kblocks_h) kh = 0;
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) {
@@ -749,6 +753,99 @@ __global__ void __launch_bounds__(NUM_THREADS) flce_split3_kernel(const Args a) 
 }
 
 }  // namespace split
+
+// ----------------------------------------------------------------- quantised head
+
+// Affine group-quantised W (the MLX format): row j, element k holds an
+// unsigned BITS-bit code q_jk, packed 32 / BITS to a uint32 word with the
+// lowest bits first, and group g = k / G of the row has a bf16 scale s_jg and
+// bias b_jg:  W_jk = s_jg q_jk + b_jg.
+// One chunk of vocabulary rows at a time is expanded into the layout the
+// tensor-core kernels read: per row two K segments of Ds = D rounded up to 64,
+// [hi | lo] with hi = bf16(W_jk) and lo = bf16(W_jk - hi) (zero padded from D
+// to Ds).  H is bf16 already, so H [hi | lo]^T over K = 2 Ds (H's K coordinate
+// wraps after Ds) is H W^T up to |W - hi - lo| <= 2^-16 |W| per weight.
+namespace quant {
+
+constexpr int NUM_THREADS = 256;   // 8 warps, one vocabulary row per warp at a time
+
+struct Args {
+  const uint32_t* wq;             // (V, D * BITS / 32) codes
+  const __nv_bfloat16* scales;    // (V, D / G)
+  const __nv_bfloat16* biases;    // (V, D / G)
+  int64_t row0;                   // first vocabulary row of the chunk
+  int64_t rows;                   // rows in the chunk
+  int32_t D;                      // a multiple of G
+  int32_t Ds;                     // D rounded up to 64
+  int32_t G;                      // 32, 64 or 128
+  __nv_bfloat16* dst;             // (rows, 2 Ds) bf16, contiguous
+};
+
+// The 8 codes of elements k0 .. k0 + 7 (k0 a multiple of 8) of one row.
+template <int BITS>
+__device__ __forceinline__ void load_codes(const uint32_t* row_words, int k0, uint32_t (&q)[8]) {
+  if constexpr (BITS == 4) {
+    const uint32_t w = __ldg(row_words + k0 / 8);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) q[t] = (w >> (4 * t)) & 0xFu;
+  } else if constexpr (BITS == 8) {
+    const uint2 w = __ldg(reinterpret_cast<const uint2*>(row_words + k0 / 4));
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      q[t] = (w.x >> (8 * t)) & 0xFFu;
+      q[t + 4] = (w.y >> (8 * t)) & 0xFFu;
+    }
+  } else {
+    static_assert(BITS == 2, "2, 4 or 8 bits");
+    const uint32_t w = __ldg(row_words + k0 / 16) >> (k0 % 16 == 0 ? 0 : 16);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) q[t] = (w >> (2 * t)) & 0x3u;
+  }
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(NUM_THREADS) flce_dequant_split_kernel(const Args a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = int64_t(gridDim.x) * (NUM_THREADS / 32);
+  const int groups = a.Ds / 8;
+  const int64_t words_per_row = int64_t(a.D) * BITS / 32;
+  const int64_t groups_per_row = a.D / a.G;
+  for (int64_t r = int64_t(blockIdx.x) * (NUM_THREADS / 32) + (threadIdx.x >> 5); r < a.rows;
+       r += warps) {
+    const int64_t j = a.row0 + r;
+    const uint32_t* row_words = a.wq + j * words_per_row;
+    uint4* out = reinterpret_cast<uint4*>(a.dst + r * 2 * int64_t(a.Ds));
+    for (int g = lane; g < groups; g += 32) {
+      const int k0 = g * 8;
+      uint4 vh = make_uint4(0u, 0u, 0u, 0u), vl = vh;
+      if (k0 < a.D) {
+        uint32_t q[8];
+        load_codes<BITS>(row_words, k0, q);
+        const int64_t gi = j * groups_per_row + k0 / a.G;
+        const float sc = __bfloat162float(a.scales[gi]);
+        const float bi = __bfloat162float(a.biases[gi]);
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          // s q + b rounded once to fp32 (s q alone is exact: at most 16 bits)
+          const float w0 = fmaf(sc, float(q[2 * t]), bi);
+          const float w1 = fmaf(sc, float(q[2 * t + 1]), bi);
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(w0);
+          const __nv_bfloat16 h1 = __float2bfloat16_rn(w1);
+          hi[t] = split::pack_bf16x2(h0, h1);
+          lo[t] = split::pack_bf16x2(__float2bfloat16_rn(w0 - __bfloat162float(h0)),
+                                     __float2bfloat16_rn(w1 - __bfloat162float(h1)));
+        }
+        vh = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        vl = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      out[g] = vh;
+      out[groups + g] = vl;
+    }
+  }
+}
+
+}  // namespace quant
 
 // ----------------------------------------------------------------- merge + mean
 

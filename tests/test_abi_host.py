@@ -215,3 +215,34 @@ def test_forward_ex_argument_checks_need_no_gpu(lib):
     assert call(out_lse=None) == flce.ERR_INVALID_ARG
     assert call(N=0) == flce.OK
     assert call(dtype=1, ldh=65, ldw=66, ws_bytes=10) == flce.ERR_WORKSPACE_TOO_SMALL   # fp32: any stride
+
+
+def test_quantized_workspace_and_argument_checks_need_no_gpu(lib):
+    # size: one chunk's slab state + a float4 per (chunk, token) + one chunk of [hi | lo] rows
+    r256 = lambda b: (b + 255) // 256 * 256
+    for N, V, D in [(8192, 151936, 4096), (10, 100, 64), (300, 40000, 192)]:
+        C = min(V, 16384)
+        chunks = math.ceil(V / C)
+        Ds = math.ceil(D / 64) * 64
+        state = flce.workspace_size(N, C, 64)           # bf16 state size depends on (N, V) only
+        want = state + r256(16 * N * chunks) + r256(C * 2 * Ds * 2)
+        assert flce.quantized_workspace_size(N, V, D, 4, 64) == want
+    # far below the 4 N V bytes of logits at the page's shape
+    assert flce.quantized_workspace_size(8192, 151936, 4096, 4, 64) < 4 * 8192 * 151936 / 10
+    for bits, G, D in [(3, 64, 128), (4, 16, 128), (4, 64, 96), (4, 64, 0), (5, 32, 64)]:
+        assert lib.flce_quantized_workspace_size(8, 100, D, bits, G) == 0
+
+    def call(bits=4, G=64, N=16, V=100, D=128, H=FAKE, wq=FAKE, s=FAKE, b=FAKE, y=FAKE,
+             ws=FAKE, ws_bytes=1 << 30):
+        return lib.flce_forward_quantized(H, wq, s, b, bits, G, y, N, V, D, FAKE, FAKE, FAKE, None,
+                                          ws, ws_bytes, None)
+    assert call(bits=3) == flce.ERR_INVALID_ARG
+    assert call(G=16) == flce.ERR_INVALID_ARG
+    assert call(D=96) == flce.ERR_INVALID_ARG            # not a multiple of G
+    assert call(wq=None) == flce.ERR_INVALID_ARG
+    assert call(ws=FAKE + 16) == flce.ERR_INVALID_ARG     # workspace must be 256-byte aligned
+    assert call(s=FAKE + 1) == flce.ERR_INVALID_ARG       # bf16 scales must be 2-byte aligned
+    assert call(H=FAKE + 8) == flce.ERR_UNSUPPORTED       # TMA needs a 16-byte-aligned H
+    assert call(wq=FAKE + 4) == flce.ERR_UNSUPPORTED
+    assert call(ws_bytes=100) == flce.ERR_WORKSPACE_TOO_SMALL
+    assert call(N=0) == flce.OK
