@@ -11,7 +11,9 @@ weak) and the step time is the maximum over ranks.
 
 Also measured: the contraction kernel's own duration (CUDA events around
 flce_partials on the launching stream) for the roofline, an end-to-end leg
-through the public API from pinned host buffers, SM clocks during the timed
+through the C ABI from pinned host buffers (flce_forward_host: H, y and W
+copied in every step, W in chunks that overlap the contraction; results
+copied back), SM clocks during the timed
 region, and the CPU oracle on a bounded sample of the same workload.
 
 ``--impl reference`` times the fp64 CPU oracle instead (the reference arm).
@@ -299,28 +301,46 @@ def run_ours(args, w, rank, world, local_rank):
         raise flce.FlceError(st, "timed region")
     mean_loss = float(mean.item())
 
-    # ---- end to end through the public API from pinned host memory
-    H_d2 = torch.empty_like(H)
-    W_d2 = torch.empty_like(W)
-    y_d2 = torch.empty_like(y)
-    loss_h = torch.empty(N, pin_memory=True)
-    mean_h = torch.empty((), pin_memory=True)
-    out2 = {"loss": torch.empty(N, device=dev), "lse": torch.empty(N, device=dev),
-            "target_logit": torch.empty(N, device=dev), "mean": torch.empty((), device=dev)}
+    # ---- end to end through the public API from pinned host memory:
+    # flce_forward_host copies H and y, streams W in chunks (overlapping the
+    # copies with the contraction) and copies the results back, every step
+    host_ws = None
+    if w.dtype == "bf16":
+        host_ws = torch.empty(flce.host_workspace_size(N, V, D), dtype=torch.uint8, device=dev)
+        copy_stream = torch.cuda.Stream(dev)
+        res_h = {k: torch.empty(N, pin_memory=True) for k in ("loss", "lse", "target_logit")}
+        res_h["mean"] = torch.empty((), pin_memory=True)
+        mean_h = res_h["mean"]
 
-    def e2e_step():
-        H_d2.copy_(H_h, non_blocking=True)
-        W_d2.copy_(W_h, non_blocking=True)
-        y_d2.copy_(y_h, non_blocking=True)
-        flce.forward(H_d2, W_d2, y_d2, out=out2, workspace=ws, stream=stream)
-        loss_h.copy_(out2["loss"], non_blocking=True)
-        mean_h.copy_(out2["mean"], non_blocking=True)
+        def e2e_step():
+            flce.forward_host(H_h, W_h, y_h, device=dev, out=res_h, workspace=host_ws,
+                              stream=stream, copy_stream=copy_stream)
+        d2h = 3 * N * 4 + 4
+    else:
+        H_d2 = torch.empty_like(H)
+        W_d2 = torch.empty_like(W)
+        y_d2 = torch.empty_like(y)
+        loss_h = torch.empty(N, pin_memory=True)
+        mean_h = torch.empty((), pin_memory=True)
+        out2 = {"loss": torch.empty(N, device=dev), "lse": torch.empty(N, device=dev),
+                "target_logit": torch.empty(N, device=dev), "mean": torch.empty((), device=dev)}
+
+        def e2e_step():
+            H_d2.copy_(H_h, non_blocking=True)
+            W_d2.copy_(W_h, non_blocking=True)
+            y_d2.copy_(y_h, non_blocking=True)
+            flce.forward(H_d2, W_d2, y_d2, out=out2, workspace=ws, stream=stream)
+            loss_h.copy_(out2["loss"], non_blocking=True)
+            mean_h.copy_(out2["mean"], non_blocking=True)
+        d2h = N * 4 + 4
 
     Ke = max(3, min(K, args.e2e_steps))
     with torch.cuda.stream(stream):
         for _ in range(3):
             e2e_step()
         stream.synchronize()
+        if host_ws is not None and flce.check(host_ws, stream) != flce.OK:
+            raise flce.FlceError(flce.check(host_ws, stream), "forward_host")
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -330,9 +350,8 @@ def run_ours(args, w, rank, world, local_rank):
         e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / Ke
-    assert abs(float(mean_h.item()) - mean_loss) <= 1e-6 * abs(mean_loss)
+    assert abs(float(mean_h.item()) - mean_loss) <= 1e-5 * abs(mean_loss)
     h2d = H_h.numel() * H_h.element_size() + W_h.numel() * W_h.element_size() + y_h.numel() * 8
-    d2h = N * 4 + 4
 
     # ---- max over ranks
     total_ms, part_avg_ms, e2e_ms = max_over_ranks([total_ms, float(np.mean(part_ms)), e2e_ms],
@@ -380,7 +399,8 @@ def run_ours(args, w, rank, world, local_rank):
                      "flops_per_launch": flops,
                      "traffic": profiled_traffic(w.name, kernel)},
         "e2e": {"value": weak_scaling_tokens_per_s(world, N, e2e_ms), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms,
+                "api": "flce_forward_host" if host_ws is not None else "torch copies + flce_forward"},
         "gpu_launches": 2 * K,
         "clocks": clocks,
     }

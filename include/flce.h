@@ -371,6 +371,51 @@ FLCE_API flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
                                             float* out_mean, void* workspace,
                                             size_t workspace_bytes, void* stream);
 
+/*
+ * The forward on inputs that live in HOST memory, results returned to host
+ * memory: the same operation as flce_forward (section 1 of the page), for
+ * callers whose H, W and y are not on the device (W offloaded to the host,
+ * data loaders that produce pinned host batches).
+ *
+ *   H_host (N, D) bf16, W_host (V, D) bf16, y_host (N) int64: host memory,
+ *            contiguous.  Page-locked (pinned) memory lets the copies run
+ *            asynchronously and overlap the contraction; pageable memory
+ *            works but the copies then block the calling thread.  The host
+ *            buffers must stay valid and unchanged until `stream` has been
+ *            synchronised.
+ *   loss_host (N) fp32 host buffer (required); lse_host, target_logit_host
+ *            (N) and mean_host (1) may be NULL.  They are written by copies
+ *            enqueued on `stream`: read them after synchronising `stream`.
+ *   N, V, D  as flce_forward; bf16 only (fp32 returns FLCE_ERR_UNSUPPORTED),
+ *            D % 8 == 0.
+ *   workspace  device memory, >= flce_forward_host_workspace_size(N, V, D,
+ *            dtype) bytes, 256-byte aligned: device copies of H and y, the
+ *            outputs, two staging buffers of 8192 W rows, and the merge
+ *            state; holds the status word flce_check() reads.
+ *   stream   cudaStream_t for the kernels and the result copies.
+ *   copy_stream  cudaStream_t for the host-to-device copies (a different
+ *            stream overlaps them with the kernels); NULL = use `stream`.
+ *
+ * W crosses PCIe in chunks of 8192 rows into two alternating staging
+ * buffers; each chunk's contraction (a vocabulary shard) starts as soon as
+ * its copy lands and runs while the next chunk is copied, and the chunks'
+ * per-token states are merged in chunk order at the end.  The call first
+ * makes copy_stream wait for the work already queued on `stream`, so calls
+ * on one (stream, workspace) pair may be issued back to back.  The library
+ * creates and destroys a few CUDA events per call and allocates no memory.
+ * Errors as flce_forward; targets are checked on the device.  N == 0 is a
+ * no-op.
+ */
+FLCE_API size_t flce_forward_host_workspace_size(int64_t N, int64_t V, int64_t D,
+                                                 flce_dtype dtype);
+
+FLCE_API flce_status flce_forward_host(const void* H_host, const void* W_host,
+                                       const int64_t* y_host, int64_t N, int64_t V, int64_t D,
+                                       flce_dtype dtype, float* loss_host, float* lse_host,
+                                       float* target_logit_host, float* mean_host,
+                                       void* workspace, size_t workspace_bytes, void* stream,
+                                       void* copy_stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,7 +24,7 @@ import torch
 __all__ = [
     "FlceError", "forward", "backward", "partials", "merge", "workspace_size",
     "shard_state", "merge_shards", "forward_vocab_parallel", "forward_strided",
-    "forward_quantized", "quantized_workspace_size",
+    "forward_quantized", "quantized_workspace_size", "forward_host", "host_workspace_size",
     "backward_workspace_size", "plan", "check",
     "status_string", "selftest_wait_timeout", "library_path", "load_library",
 ]
@@ -138,6 +138,11 @@ def load_library():
         lib.flce_forward_quantized.argtypes = [vp, vp, vp, vp, i32, i32, vp, i64, i64, i64,
                                                vp, vp, vp, vp, vp, sz, vp]
         lib.flce_forward_quantized.restype = st
+        lib.flce_forward_host_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int]
+        lib.flce_forward_host_workspace_size.restype = sz
+        lib.flce_forward_host.argtypes = [vp, vp, vp, i64, i64, i64, ctypes.c_int, vp, vp, vp, vp,
+                                          vp, sz, vp, vp]
+        lib.flce_forward_host.restype = st
         _lib = lib
         return lib
 
@@ -520,4 +525,54 @@ def forward_quantized(H: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, b
               "flce_forward_quantized")
     if check:
         _raise_on(lib.flce_check(workspace.data_ptr(), sp), "flce_forward_quantized (device)")
+    return loss, lse, tgt, mean
+
+
+def host_workspace_size(N: int, V: int, D: int) -> int:
+    n = load_library().flce_forward_host_workspace_size(int(N), int(V), int(D), BF16)
+    if n == 0:
+        raise FlceError(ERR_INVALID_ARG, "host_workspace_size")
+    return int(n)
+
+
+def forward_host(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, *, device=None,
+                 out: dict | None = None, workspace: torch.Tensor | None = None, stream=None,
+                 copy_stream=None, check: bool = False):
+    """flce_forward_host: the forward on CPU tensors H (N, D) bf16, W (V, D) bf16 and
+    y (N) int64 (pin them for overlap), streaming W to `device` chunk by chunk.
+
+    Returns CPU tensors (loss, lse, target_logit, mean); ``out`` may supply them
+    (pinned).  They are valid after `stream` is synchronised (done here when
+    ``check`` is set); until then H, W and y must stay alive and unchanged."""
+    for name, t in (("H", H), ("W", W), ("y", y)):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CPU tensor")
+    if H.dtype != torch.bfloat16 or W.dtype != torch.bfloat16 or H.dim() != 2 or W.dim() != 2 \
+            or H.shape[1] != W.shape[1]:
+        raise ValueError("H (N, D) and W (V, D) must be bf16 with one D")
+    if y.dtype != torch.int64 or y.shape != (H.shape[0],):
+        raise ValueError("y must be int64 of shape (N,)")
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    N, D = H.shape
+    V = W.shape[0]
+    out = out or {}
+    pin = torch.cuda.is_available()
+    def host(key, shape):
+        t = out.get(key)
+        return t if t is not None else torch.empty(shape, dtype=torch.float32, pin_memory=pin)
+    loss, lse, tgt, mean = host("loss", (N,)), host("lse", (N,)), host("target_logit", (N,)), host("mean", ())
+    if N == 0:
+        return loss, lse, tgt, mean
+    lib = load_library()
+    need = host_workspace_size(N, V, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    sp = _stream_ptr(stream, dev)
+    cp = int(copy_stream.cuda_stream) if copy_stream is not None else None
+    _raise_on(lib.flce_forward_host(H.data_ptr(), W.data_ptr(), y.data_ptr(), N, V, D, BF16,
+                                    loss.data_ptr(), lse.data_ptr(), tgt.data_ptr(), mean.data_ptr(),
+                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                    sp, cp), "flce_forward_host")
+    if check:
+        _raise_on(lib.flce_check(workspace.data_ptr(), sp), "flce_forward_host (device)")
     return loss, lse, tgt, mean

@@ -947,3 +947,148 @@ extern "C" flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
       block_sums, hdr);
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------- forward from host memory
+
+namespace {
+
+// Vocabulary rows copied per chunk (a multiple of the 256-column tile).
+constexpr int64_t kHostChunkRows = 8192;
+
+// Workspace of the host-input forward: one chunk's slab state, a float4 per
+// (chunk, token), device copies of H and y, the outputs, and two staging
+// buffers for W chunks.
+struct HostLayout {
+  int64_t C = 0, chunks = 0;
+  size_t state = 0, states = 0, h = 0, y = 0, outs = 0, staging = 0, total = 0;
+};
+
+HostLayout host_layout(int64_t N, int64_t V, int64_t D) {
+  HostLayout L;
+  L.C = std::min(V, kHostChunkRows);
+  L.chunks = cdiv(V, L.C);
+  L.state = state_bytes_for(N, L.C);
+  L.states = align256(size_t(16) * size_t(N) * size_t(L.chunks));
+  L.h = align256(size_t(N) * size_t(D) * 2);
+  L.y = align256(size_t(N) * 8);
+  L.outs = align256(size_t(N) * 12 + 4);
+  L.staging = align256(size_t(L.C) * size_t(D) * 2);
+  L.total = L.state + L.states + L.h + L.y + L.outs + 2 * L.staging;
+  return L;
+}
+
+// Events created for one call; destroyed when the call returns (CUDA keeps a
+// destroyed event's pending work valid).
+struct CallEvents {
+  cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+  bool create() {
+    for (auto& e : ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+    return true;
+  }
+  ~CallEvents() {
+    for (auto& e : ev)
+      if (e) cudaEventDestroy(e);
+  }
+};
+
+}  // namespace
+
+extern "C" size_t flce_forward_host_workspace_size(int64_t N, int64_t V, int64_t D,
+                                                   flce_dtype dtype) {
+  if (!sizes_ok(N, V, D, dtype) || dtype != FLCE_BF16 || D % 8 != 0) return 0;
+  return host_layout(N, V, D).total;
+}
+
+extern "C" flce_status flce_forward_host(const void* H_host, const void* W_host,
+                                         const int64_t* y_host, int64_t N, int64_t V, int64_t D,
+                                         flce_dtype dtype, float* loss_host, float* lse_host,
+                                         float* target_logit_host, float* mean_host,
+                                         void* workspace, size_t workspace_bytes, void* stream,
+                                         void* copy_stream) {
+  if (!sizes_ok(N, V, D, dtype)) return FLCE_ERR_INVALID_ARG;
+  if (N == 0) return FLCE_OK;
+  if (!H_host || !W_host || !y_host || !loss_host || !workspace) return FLCE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FLCE_ERR_INVALID_ARG;
+  if (dtype != FLCE_BF16 || D % 8 != 0) return FLCE_ERR_UNSUPPORTED;
+  if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31) || D >= (int64_t(1) << 31))
+    return FLCE_ERR_UNSUPPORTED;
+  const HostLayout L = host_layout(N, V, D);
+  if (workspace_bytes < L.total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t cs = copy_stream ? static_cast<cudaStream_t>(copy_stream) : st;
+  DeviceInfo di;
+  int64_t workers = 0;
+  flce_status s = contraction_workers(N, di, workers);
+  if (s != FLCE_OK) return s;
+  CallEvents events;
+  if (!events.create()) return FLCE_ERR_CUDA;
+  cudaEvent_t* ready = events.ev;       // [2] staging buffer b holds its chunk
+  cudaEvent_t* freed = events.ev + 2;   // [2] staging buffer b has been read
+  cudaEvent_t start = events.ev[4];     // all work queued on `stream` before this call
+
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
+  size_t off = L.state;
+  float4* states = reinterpret_cast<float4*>(wsb + off);
+  off += L.states;
+  void* Hd = wsb + off;
+  off += L.h;
+  int64_t* yd = reinterpret_cast<int64_t*>(wsb + off);
+  off += L.y;
+  float* loss_d = reinterpret_cast<float*>(wsb + off);
+  float* lse_d = loss_d + N;
+  float* tgt_d = lse_d + N;
+  float* mean_d = tgt_d + N;
+  off += L.outs;
+  uint8_t* staging[2] = {wsb + off, wsb + off + L.staging};
+  const size_t row_bytes = size_t(D) * 2;
+  const uint8_t* Wh = static_cast<const uint8_t*>(W_host);
+
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  // The copies below overwrite H, y and the staging buffers in the workspace:
+  // they wait for earlier work on `stream` (a previous call may still read them).
+  if (cs != st && (!ok(cudaEventRecord(start, st)) || !ok(cudaStreamWaitEvent(cs, start, 0))))
+    return FLCE_ERR_CUDA;
+  if (!ok(cudaMemsetAsync(hdr, 0, kHeaderBytes, st))) return FLCE_ERR_CUDA;
+  // H and y first, on the copy stream, ahead of the W chunks.
+  if (!ok(cudaMemcpyAsync(Hd, H_host, size_t(N) * row_bytes, cudaMemcpyHostToDevice, cs)) ||
+      !ok(cudaMemcpyAsync(yd, y_host, size_t(N) * 8, cudaMemcpyHostToDevice, cs)))
+    return FLCE_ERR_CUDA;
+  for (int64_t c = 0; c < L.chunks; ++c) {
+    const int b = int(c & 1);
+    const int64_t c0 = c * L.C;
+    const int64_t rows = std::min(L.C, V - c0);
+    // Buffer b last held chunk c - 2: wait until its contraction has read it.
+    if (c >= 2 && !ok(cudaStreamWaitEvent(cs, freed[b], 0))) return FLCE_ERR_CUDA;
+    if (!ok(cudaMemcpyAsync(staging[b], Wh + size_t(c0) * row_bytes, size_t(rows) * row_bytes,
+                            cudaMemcpyHostToDevice, cs)) ||
+        !ok(cudaEventRecord(ready[b], cs)) || !ok(cudaStreamWaitEvent(st, ready[b], 0)))
+      return FLCE_ERR_CUDA;
+    flce_plan_t plan;
+    make_plan(N, rows, D, FLCE_BF16, workers, &plan);
+    if ((s = launch_contraction(Hd, D, D, staging[b], D, D, Targets{yd, 0}, c0, N, rows, plan,
+                                tgt_d, workspace, false, st)) != FLCE_OK)
+      return s;
+    flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
+        reinterpret_cast<const float2*>(wsb + kHeaderBytes), hdr, yd, int32_t(N), c0, rows,
+        int32_t(slab_capacity(rows)), tgt_d, states + c * N, &hdr->status);
+    if (!ok(cudaGetLastError()) || !ok(cudaEventRecord(freed[b], st))) return FLCE_ERR_CUDA;
+  }
+  double* block_sums = reinterpret_cast<double*>(
+      wsb + kHeaderBytes + align256(size_t(8) * size_t(N) * size_t(slab_capacity(L.C))));
+  flce_merge_shards_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
+      states, int32_t(L.chunks), yd, int32_t(N), V, loss_d, lse_d, tgt_d, mean_d, block_sums, hdr);
+  if (!ok(cudaGetLastError())) return FLCE_ERR_CUDA;
+  const size_t nb = size_t(N) * 4;
+  if (!ok(cudaMemcpyAsync(loss_host, loss_d, nb, cudaMemcpyDeviceToHost, st)) ||
+      (lse_host && !ok(cudaMemcpyAsync(lse_host, lse_d, nb, cudaMemcpyDeviceToHost, st))) ||
+      (target_logit_host &&
+       !ok(cudaMemcpyAsync(target_logit_host, tgt_d, nb, cudaMemcpyDeviceToHost, st))) ||
+      (mean_host && !ok(cudaMemcpyAsync(mean_host, mean_d, 4, cudaMemcpyDeviceToHost, st))))
+    return FLCE_ERR_CUDA;
+  // The copy stream's last work (the final chunk's copy) is already ordered
+  // before `stream` through ready[]; nothing else is left on it.
+  return FLCE_OK;
+}

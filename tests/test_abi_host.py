@@ -246,3 +246,25 @@ def test_quantized_workspace_and_argument_checks_need_no_gpu(lib):
     assert call(wq=FAKE + 4) == flce.ERR_UNSUPPORTED
     assert call(ws_bytes=100) == flce.ERR_WORKSPACE_TOO_SMALL
     assert call(N=0) == flce.OK
+
+
+def test_forward_host_argument_checks_need_no_gpu(lib):
+    r256 = lambda b: (b + 255) // 256 * 256
+    N, V, D = 300, 20000, 128
+    C = 8192
+    want = (flce.workspace_size(N, C, D) + r256(16 * N * 3) + r256(N * D * 2) + r256(8 * N)
+            + r256(12 * N + 4) + 2 * r256(C * D * 2))
+    assert flce.host_workspace_size(N, V, D) == want
+    assert lib.flce_forward_host_workspace_size(N, V, 12, 0) == 0      # D % 8
+    assert lib.flce_forward_host_workspace_size(N, V, D, 1) == 0       # fp32: not supported
+
+    def call(N=16, V=100, D=64, dtype=0, H=FAKE, W=FAKE, y=FAKE, loss=FAKE, ws=FAKE, ws_bytes=1 << 30):
+        return lib.flce_forward_host(H, W, y, N, V, D, dtype, loss, None, None, None, ws, ws_bytes,
+                                     None, None)
+    assert call(H=None) == flce.ERR_INVALID_ARG
+    assert call(loss=None) == flce.ERR_INVALID_ARG
+    assert call(ws=FAKE + 64) == flce.ERR_INVALID_ARG
+    assert call(dtype=1) == flce.ERR_UNSUPPORTED
+    assert call(D=12) == flce.ERR_UNSUPPORTED
+    assert call(ws_bytes=1000) == flce.ERR_WORKSPACE_TOO_SMALL
+    assert call(N=0) == flce.OK
