@@ -112,9 +112,11 @@ def test_plan_covers_every_tile_once_and_balances(lib, N, V, D, dtype, sms):
     assert p["grid"] == min(workers, p["units"]) * p["ctas_per_unit"]
     assert simulate_makespan(p) == p["makespan_tiles"]
     total = p["token_blocks"] * p["vocab_tiles"]
-    # within one tile per worker of the perfect split, whenever every worker has work
+    # within one tile per worker of the perfect split, whenever every worker has work;
+    # the planner gives up at most 1% of that for slabs of equal length
     if total >= workers:
-        assert p["makespan_tiles"] <= math.ceil(total / workers) + 1
+        bound = math.ceil(total / workers) + 1
+        assert p["makespan_tiles"] <= (bound * 1.01 if p["slab_rem"] == 0 else bound)
 
 
 def test_grouped_makespan_matches_simulation_on_random_shapes(lib):
@@ -138,6 +140,7 @@ def test_headline_plan(lib):
     assert p["token_blocks"] == 32 and p["vocab_tiles"] == 594
     assert p["group_blocks"] == 16             # 16 x 2 MB of H live at a time
     assert p["makespan_tiles"] <= 258          # ceil(32 * 594 / 74) = 257 pair tiles
+    assert p["slab_rem"] == 0                  # equal slabs (99 x 6 tiles) keep the pairs in step
 
 
 def test_plan_rejects_bad_args(lib):
