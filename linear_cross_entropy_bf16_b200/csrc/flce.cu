@@ -613,16 +613,28 @@ inline int64_t round_up(int64_t x, int64_t m) { return cdiv(x, m) * m; }
 
 struct BwdLayout {
   int64_t chunk;
-  size_t off_dz, total;
+  size_t off_dz, off_dzl, off_h3, off_w3, total;
 };
 
-// [256 B header][dZ slice: N x chunk bf16]
-BwdLayout bwd_layout(int64_t N, int64_t V, int64_t D) {
-  (void)D;
+// bf16: [256 B header][dZ slice: N x chunk bf16].
+// fp32 inputs add the lo parts of the dZ slice (N x chunk bf16) and the bf16
+// hi/lo split copies of H (N x 3 Dp, [hi | hi | lo]) and of one chunk of W
+// (chunk x 3 Dp, [hi | lo | hi]).
+BwdLayout bwd_layout(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
   BwdLayout L;
   L.chunk = std::min(round_up(V, kTileCols), kBwdChunkCols);
   L.off_dz = kHeaderBytes;
-  L.total = L.off_dz + align256(size_t(N) * size_t(L.chunk) * 2);
+  size_t end = L.off_dz + align256(size_t(N) * size_t(L.chunk) * 2);
+  L.off_dzl = L.off_h3 = L.off_w3 = 0;
+  if (dtype == FLCE_FP32) {
+    L.off_dzl = end;
+    end += align256(size_t(N) * size_t(L.chunk) * 2);
+    L.off_h3 = end;
+    end += split_bytes_for(N, D);
+    L.off_w3 = end;
+    end += split_bytes_for(L.chunk, D);
+  }
+  L.total = end;
   return L;
 }
 
@@ -677,7 +689,7 @@ flce_status launch_gemm(const CUtensorMap& A, const CUtensorMap& B, const bwd::G
 
 extern "C" size_t flce_backward_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
   if (!sizes_ok(N, V, D, dtype) || N < 1) return 0;
-  return bwd_layout(N, V, D).total;
+  return bwd_layout(N, V, D, dtype).total;
 }
 
 extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t* y,
@@ -689,11 +701,14 @@ extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t
   if (N == 0) return FLCE_OK;
   if (!H || !W || !y || !lse || !dH || !dW || !workspace) return FLCE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FLCE_ERR_INVALID_ARG;
-  if (dtype != FLCE_BF16) return FLCE_ERR_UNSUPPORTED;
   if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31) || D >= (int64_t(1) << 31))
     return FLCE_ERR_UNSUPPORTED;
-  if (D % 8 != 0 || !aligned16(H) || !aligned16(W)) return FLCE_ERR_UNSUPPORTED;
-  const BwdLayout L = bwd_layout(N, V, D);
+  const bool fp32 = dtype == FLCE_FP32;
+  if (!fp32 && (D % 8 != 0 || !aligned16(H) || !aligned16(W))) return FLCE_ERR_UNSUPPORTED;
+  if (fp32 && ((reinterpret_cast<uintptr_t>(H) | reinterpret_cast<uintptr_t>(W)) & 3u))
+    return FLCE_ERR_INVALID_ARG;
+  if (fp32 && k_extent(D, dtype) >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
+  const BwdLayout L = bwd_layout(N, V, D, dtype);
   if (workspace_bytes < L.total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
 
   DeviceInfo di;
@@ -709,20 +724,46 @@ extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
   __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dz);  // (N x chunk)
+  __nv_bfloat16* dzl = fp32 ? reinterpret_cast<__nv_bfloat16*>(ws + L.off_dzl) : nullptr;
   if (cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
 
-  const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(W);
-  CUtensorMap mH_k, mH_mn;
-  if (!encode_bf16_2d(&mH_k, H, N, D, D, bwd::BM) ||     // K1 A: (N, D), K = D
-      !encode_bf16_2d(&mH_mn, H, N, D, D, bwd::BK))      // K3 B: d contiguous, K = N
+  // The bf16 operands.  bf16 inputs: H and W themselves.  fp32 inputs: the
+  // split copies, K1 contracting [hi | hi | lo] against [hi | lo | hi] over
+  // K = 3 Dp; K2 and K3 read the hi and lo segments as strided views.
+  const int64_t Dp = split_segment(D);
+  const int64_t K1 = fp32 ? 3 * Dp : D;   // K of the logits contraction
+  const int64_t ldk = fp32 ? 3 * Dp : D;  // row stride of the H and W operands
+  const __nv_bfloat16* Hb = static_cast<const __nv_bfloat16*>(H);
+  const __nv_bfloat16* W3 = nullptr;
+  if (fp32) {
+    Hb = reinterpret_cast<const __nv_bfloat16*>(ws + L.off_h3);
+    W3 = reinterpret_cast<const __nv_bfloat16*>(ws + L.off_w3);
+    if ((s = launch_split(H, D, N, D, 2, ws + L.off_h3, di.sms, st)) != FLCE_OK) return s;
+  }
+  CUtensorMap mH_k, mH_mn, mH_mn_lo;
+  if (!encode_bf16_2d(&mH_k, Hb, N, K1, ldk, bwd::BM) ||     // K1 A: (N, K1)
+      !encode_bf16_2d(&mH_mn, Hb, N, D, ldk, bwd::BK))       // K3 B (hi): d contiguous, K = N
+    return FLCE_ERR_UNSUPPORTED;
+  if (fp32 && !encode_bf16_2d(&mH_mn_lo, Hb + 2 * Dp, N, D, ldk, bwd::BK))  // K3 B (lo)
     return FLCE_ERR_UNSUPPORTED;
   for (int64_t c0 = 0; c0 < V; c0 += L.chunk) {
     const int64_t clen = std::min(L.chunk, V - c0);
-    CUtensorMap mW_k, mW_mn, mDz_k, mDz_mn;
-    if (!encode_bf16_2d(&mW_k, Wb + c0 * D, clen, D, D, bwd::HALF_N) ||  // K1 B: (clen, D)
-        !encode_bf16_2d(&mW_mn, Wb + c0 * D, clen, D, D, bwd::BK) ||     // K2 B: d contiguous
-        !encode_bf16_2d(&mDz_k, dz, N, clen, L.chunk, bwd::BM) ||        // K2 A: K = vocab
-        !encode_bf16_2d(&mDz_mn, dz, N, clen, L.chunk, bwd::BK))         // K3 A: vocab contiguous
+    const __nv_bfloat16* Wc = static_cast<const __nv_bfloat16*>(W) + c0 * D;
+    if (fp32) {
+      if ((s = launch_split(static_cast<const float*>(W) + c0 * D, D, clen, D, 1,
+                            ws + L.off_w3, di.sms, st)) != FLCE_OK)
+        return s;
+      Wc = W3;
+    }
+    CUtensorMap mW_k, mW_mn, mW_mn_lo, mDz_k, mDz_mn, mDzl_k, mDzl_mn;
+    if (!encode_bf16_2d(&mW_k, Wc, clen, K1, ldk, bwd::HALF_N) ||  // K1 B: (clen, K1)
+        !encode_bf16_2d(&mW_mn, Wc, clen, D, ldk, bwd::BK) ||      // K2 B (hi): d contiguous
+        !encode_bf16_2d(&mDz_k, dz, N, clen, L.chunk, bwd::BM) ||  // K2 A: K = vocab
+        !encode_bf16_2d(&mDz_mn, dz, N, clen, L.chunk, bwd::BK))   // K3 A: vocab contiguous
+      return FLCE_ERR_UNSUPPORTED;
+    if (fp32 && (!encode_bf16_2d(&mW_mn_lo, Wc + Dp, clen, D, ldk, bwd::BK) ||
+                 !encode_bf16_2d(&mDzl_k, dzl, N, clen, L.chunk, bwd::BM) ||
+                 !encode_bf16_2d(&mDzl_mn, dzl, N, clen, L.chunk, bwd::BK)))
       return FLCE_ERR_UNSUPPORTED;
     // K1: dZ for this chunk from the regenerated logits
     bwd::EpiGradLogits e1;
@@ -735,33 +776,40 @@ extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t
     e1.c0 = int32_t(c0);
     e1.clen = int32_t(clen);
     e1.dz = dz;
+    e1.dz_lo = dzl;
     e1.ldz = int32_t(L.chunk);
     e1.status = &hdr->status;
-    s = launch_gemm<bwd::EpiGradLogits, false, false>(mH_k, mW_k, gemm_shape(N, clen, D), e1,
+    s = launch_gemm<bwd::EpiGradLogits, false, false>(mH_k, mW_k, gemm_shape(N, clen, K1), e1,
                                                       &hdr->status, pairs, st);
     if (s != FLCE_OK) return s;
-    // K2: dH (+)= dZ_C W_C
-    bwd::EpiStoreF32 e2;
-    e2.out = dH;
-    e2.ld = int32_t(D);
-    e2.rows = int32_t(N);
-    e2.cols = int32_t(D);
-    e2.row_base = 0;
-    e2.accumulate = c0 > 0 ? 1 : 0;
-    s = launch_gemm<bwd::EpiStoreF32, false, true>(mDz_k, mW_mn, gemm_shape(N, D, clen), e2,
-                                                   &hdr->status, pairs, st);
-    if (s != FLCE_OK) return s;
-    // K3: dW_C = dZ_C^T H
-    bwd::EpiStoreF32 e3;
-    e3.out = dW;
-    e3.ld = int32_t(D);
-    e3.rows = int32_t(clen);
-    e3.cols = int32_t(D);
-    e3.row_base = int32_t(c0);
-    e3.accumulate = 0;
-    s = launch_gemm<bwd::EpiStoreF32, true, true>(mDz_mn, mH_mn, gemm_shape(clen, D, N), e3,
-                                                  &hdr->status, pairs, st);
-    if (s != FLCE_OK) return s;
+    // K2: dH (+)= dZ_C W_C; fp32: dz W_hi + dz W_lo + dz_lo W_hi, in that order
+    const CUtensorMap* k2[3][2] = {{&mDz_k, &mW_mn}, {&mDz_k, &mW_mn_lo}, {&mDzl_k, &mW_mn}};
+    for (int p = 0; p < (fp32 ? 3 : 1); ++p) {
+      bwd::EpiStoreF32 e2;
+      e2.out = dH;
+      e2.ld = int32_t(D);
+      e2.rows = int32_t(N);
+      e2.cols = int32_t(D);
+      e2.row_base = 0;
+      e2.accumulate = (c0 > 0 || p > 0) ? 1 : 0;
+      s = launch_gemm<bwd::EpiStoreF32, false, true>(*k2[p][0], *k2[p][1], gemm_shape(N, D, clen),
+                                                     e2, &hdr->status, pairs, st);
+      if (s != FLCE_OK) return s;
+    }
+    // K3: dW_C = dZ_C^T H; fp32: dz^T H_hi + dz^T H_lo + dz_lo^T H_hi, in that order
+    const CUtensorMap* k3[3][2] = {{&mDz_mn, &mH_mn}, {&mDz_mn, &mH_mn_lo}, {&mDzl_mn, &mH_mn}};
+    for (int p = 0; p < (fp32 ? 3 : 1); ++p) {
+      bwd::EpiStoreF32 e3;
+      e3.out = dW;
+      e3.ld = int32_t(D);
+      e3.rows = int32_t(clen);
+      e3.cols = int32_t(D);
+      e3.row_base = int32_t(c0);
+      e3.accumulate = p > 0 ? 1 : 0;
+      s = launch_gemm<bwd::EpiStoreF32, true, true>(*k3[p][0], *k3[p][1], gemm_shape(clen, D, N),
+                                                    e3, &hdr->status, pairs, st);
+      if (s != FLCE_OK) return s;
+    }
   }
   return FLCE_OK;
 }

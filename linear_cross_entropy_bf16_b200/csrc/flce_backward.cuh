@@ -61,6 +61,26 @@ __device__ __forceinline__ void tile_coords(const GemmShape& s, int t, int& mb, 
 
 // K1: dZ from the regenerated logits.
 struct EpiGradLogits {
+  // 32 values rounded to bf16 at dst (columns col0 .. col0 + 31 of a row,
+  // those below clen), 16-byte stores when all 32 are in the chunk.
+  __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float (&d)[32],
+                                              int col0) const {
+    if (col0 + 32 <= clen) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        __nv_bfloat162 h[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(d[q * 8 + 2 * e], d[q * 8 + 2 * e + 1]);
+        d4[q] = *reinterpret_cast<uint4*>(h);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + j < clen) dst[j] = __float2bfloat16_rn(d[j]);
+    }
+  }
+
   const float* lse;          // (N) from the forward
   const int64_t* y;          // (N)
   const float* grad;         // (N) upstream gradient, or null (then every g_i = 1)
@@ -70,6 +90,8 @@ struct EpiGradLogits {
   int32_t c0;                // first vocabulary row of this chunk
   int32_t clen;              // vocabulary rows in this chunk
   __nv_bfloat16* dz;         // (N x ldz) token-major slice, columns = chunk vocab
+  __nv_bfloat16* dz_lo;      // null, or (N x ldz): bf16(dZ - dz) for fp32 inputs, so that
+                             // dz + dz_lo carries dZ to 2^-16 relative
   int32_t ldz;
   uint32_t* status;
 
@@ -99,20 +121,12 @@ struct EpiGradLogits {
       }
       if (!valid) continue;
       // token-major: 32 consecutive vocab entries of this row
-      __nv_bfloat16* dst = dz + size_t(row) * size_t(ldz) + col0;
-      if (col0 + 32 <= clen) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
+      const size_t at = size_t(row) * size_t(ldz) + col0;
+      store_row32(dz + at, d, col0);
+      if (dz_lo != nullptr) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          __nv_bfloat162 h[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(d[q * 8 + 2 * e], d[q * 8 + 2 * e + 1]);
-          d4[q] = *reinterpret_cast<uint4*>(h);
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (col0 + j < clen) dst[j] = __float2bfloat16_rn(d[j]);
+        for (int j = 0; j < 32; ++j) d[j] -= __bfloat162float(__float2bfloat16_rn(d[j]));
+        store_row32(dz_lo + at, d, col0);
       }
     }
   }

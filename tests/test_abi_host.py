@@ -271,3 +271,13 @@ def test_forward_host_argument_checks_need_no_gpu(lib):
     assert call(D=12) == flce.ERR_UNSUPPORTED
     assert call(ws_bytes=1000) == flce.ERR_WORKSPACE_TOO_SMALL
     assert call(N=0) == flce.OK
+
+
+def test_backward_workspace_fp32_adds_split_copies(lib):
+    r256 = lambda b: (b + 255) // 256 * 256
+    for N, V, D in [(8192, 151936, 4096), (7, 3, 5), (300, 40000, 96)]:
+        chunk = min(math.ceil(V / 256) * 256, 16384)
+        Dp = (D + 7) // 8 * 8
+        bf16 = flce.backward_workspace_size(N, V, D) if D % 8 == 0 else 256 + r256(2 * N * chunk)
+        assert flce.backward_workspace_size(N, V, D, 1) == (
+            bf16 + r256(2 * N * chunk) + r256(6 * Dp * N) + r256(6 * Dp * chunk))

@@ -110,3 +110,57 @@ def test_backward_deterministic_and_flags_bad_targets():
     ws = torch.empty(flce.backward_workspace_size(N, V, D), dtype=torch.uint8, device="cuda")
     flce.backward(Hd, Wd, yb, lse, workspace=ws)
     assert flce.check(ws) == flce.ERR_TARGET_OUT_OF_RANGE
+
+
+# ---------------------------------------------------------------- fp32 inputs
+# fp32 H and W: the logits are regenerated from bf16 hi/lo splits (three bf16
+# products per fp32 product, about 3 * 2^-16 relative each), dZ is kept as a
+# bf16 pair dz + dz_lo (2^-16 relative) and every contraction runs the three
+# products hi*hi, hi*lo, lo*hi.  Every entry must meet the bf16 path's bound
+# above (2^-8 of the magnitude: a guaranteed bound), and the relative
+# Frobenius error must be far below what a bf16 rounding of dZ or of the
+# inputs would leave (about 2e-3): under 1e-4.
+FP32_FROB = 1e-4
+
+
+@pytest.mark.parametrize("N,V,D", [(1, 1, 1), (7, 3, 5), (130, 300, 33), (256, 1000, 128),
+                                   (64, 20000, 64), (300, 2047, 264)])
+def test_backward_fp32_every_element(N, V, D):
+    H, W, y = synth.random_inputs(N, V, D, seed=N + 5 * V + 3 * D, dtype="fp32")
+    g = np.random.default_rng(N + 1).uniform(-1, 1, N)
+    dH, dW = run_backward(H, W, y, g)
+    gf = g.astype(np.float32).astype(np.float64)
+    ref = oracle.backward(H, W, y, gf, bounds=True)
+    for got, r, b, name in ((dH, ref["dH"], ref["bH"], "dH"), (dW, ref["dW"], ref["bW"], "dW")):
+        compare(got, r, b, name)
+        rel = np.linalg.norm(got - r) / max(np.linalg.norm(r), 1e-30)
+        assert rel < FP32_FROB, f"{name}: relative Frobenius error {rel:.2e}"
+
+
+def test_backward_fp32_mean_loss_multi_chunk_vs_bf16_error():
+    """Several vocabulary chunks; and the fp32 path beats the bf16 path on the same values."""
+    import linear_cross_entropy_bf16_b200 as flce
+    N, V, D = 200, 40000, 96
+    H, W, y = synth.random_inputs(N, V, D, seed=51, dtype="fp32")
+    dH, dW = run_backward(H, W, y, None, 1.0 / N)
+    ref = oracle.backward(H, W, y, np.float64(np.float32(1.0 / N)), bounds=True)
+    e32 = [np.linalg.norm(dH - ref["dH"]) / np.linalg.norm(ref["dH"]),
+           np.linalg.norm(dW - ref["dW"]) / np.linalg.norm(ref["dW"])]
+    assert max(e32) < FP32_FROB, e32
+    # the same fp32 values rounded to bf16 and run on the bf16 path, against their own oracle
+    Hb, Wb = synth.round_to_bf16_bits(H), synth.round_to_bf16_bits(W)
+    dHb, dWb = run_backward(Hb, Wb, y, None, 1.0 / N)
+    refb = oracle.backward(Hb, Wb, y, np.float64(np.float32(1.0 / N)))
+    e16 = np.linalg.norm(dHb - refb["dH"]) / np.linalg.norm(refb["dH"])
+    assert e32[0] < e16 / 10, (e32, e16)
+
+
+def test_backward_fp32_deterministic():
+    import linear_cross_entropy_bf16_b200 as flce
+    N, V, D = 300, 17000, 40
+    H, W, y = synth.random_inputs(N, V, D, seed=52, dtype="fp32")
+    Hd, Wd, yd = to_device(H, W, y)
+    _, lse, _, _ = flce.forward(Hd, Wd, yd)
+    a = [t.clone() for t in flce.backward(Hd, Wd, yd, lse)]
+    b = flce.backward(Hd, Wd, yd, lse, check=True)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
