@@ -195,8 +195,9 @@ FLCE_API flce_status flce_merge(const int64_t* y, int64_t N, int64_t V,
  * regenerated tile by tile; vocabulary chunks of up to 16384 rows bound the
  * working slice of dZ to O(N * chunk) (never O(N * V)).
  *
- *   H, W, y, N, V, D, dtype   as for flce_forward (bf16 only for now:
- *                             FLCE_FP32 returns FLCE_ERR_UNSUPPORTED)
+ *   H, W, y, N, V, D, dtype   as for flce_forward (bf16: D % 8 == 0 and
+ *                             16-byte-aligned H, W; fp32: any D, 4-byte
+ *                             alignment)
  *   lse          (N) fp32: out_lse of the forward on the same H, W
  *   grad_loss    (N) fp32 upstream gradient dL/dloss_i, or NULL
  *   dH           (N, D) fp32 row-major, overwritten
@@ -204,10 +205,15 @@ FLCE_API flce_status flce_merge(const int64_t* y, int64_t N, int64_t V,
  *   workspace    >= flce_backward_workspace_size(N, V, D, dtype) bytes,
  *                256-byte aligned (the status word read by flce_check and one
  *                N x chunk slice of dZ in bf16: 256 B + 2 N min(V, 16384) B,
- *                rounded up)
- * dZ is rounded to bf16 before the two gradient contractions (fp32
- * accumulation), so each gradient entry carries an error of at most about
- * 2^-8 times sum_j |dZ_ij| |W_jk| (resp. sum_i |dZ_ij| |H_ik|).
+ *                rounded up; fp32 inputs add a second dZ slice and the bf16
+ *                hi/lo split copies of H and of one W chunk, 6 Dp bytes per
+ *                row, Dp = D rounded up to 8)
+ * bf16 inputs: dZ is rounded to bf16 before the two gradient contractions
+ * (fp32 accumulation), so each gradient entry carries an error of at most
+ * about 2^-8 times sum_j |dZ_ij| |W_jk| (resp. sum_i |dZ_ij| |H_ik|).
+ * fp32 inputs: H, W and dZ are each carried as two bf16 parts (hi + lo, to
+ * 2^-16 relative) and every contraction runs the three products hi*hi +
+ * hi*lo + lo*hi, about 3 * 2^-16 of the same magnitudes.
  * A target outside [0, V) sets FLCE_ERR_TARGET_OUT_OF_RANGE for flce_check.
  * Deterministic run to run.
  */
