@@ -12,7 +12,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libflce.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("flce.cu", "flce_kernels.cuh", "flce_backward.cuh", "ptx_sm100.cuh")] + [
+SOURCES = [os.path.join(CSRC, f) for f in ("flce.cu", "flce_kernels.cuh", "flce_backward.cuh", "flce_schedule.h", "ptx_sm100.cuh")] + [
     os.path.join(ROOT, "include", "flce.h")]
 
 NVCC_FLAGS = [

@@ -26,153 +26,7 @@ using namespace flce;
 
 constexpr uint64_t kDefaultWaitLimitNs = 4000000000ull;  // 4 s in one wait: far beyond any real stage
 
-inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
-
-bool sizes_ok(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
-  if (N < 0 || V < 1 || D < 1) return false;
-  if (dtype != FLCE_BF16 && dtype != FLCE_FP32) return false;
-  return true;
-}
-
-int64_t slab_capacity(int64_t V) { return std::min<int64_t>(cdiv(V, kTileCols), kMaxSlabs); }
-
-// Header, (m, s) partial states and the mean's block sums: what the merge reads.
-size_t state_bytes_for(int64_t N, int64_t V) {
-  const size_t part = align256(size_t(8) * size_t(N) * size_t(slab_capacity(V)));
-  const size_t sums = align256(size_t(8) * size_t(std::max<int64_t>(1, cdiv(N, kMergeThreads))));
-  return kHeaderBytes + part + sums;
-}
-
-// Length of the bf16 K axis the tensor-core kernels contract over: D for bf16
-// inputs; for fp32 inputs three segments (hi / lo parts) of D rounded up to 8.
-int64_t split_segment(int64_t D) { return (D + 7) / 8 * 8; }
-int64_t k_extent(int64_t D, flce_dtype dtype) {
-  return dtype == FLCE_FP32 ? 3 * split_segment(D) : D;
-}
-
-// fp32 inputs: room after the state for the split copies of H and W,
-// (N, 3 Dp) and (V, 3 Dp) bf16, each 256-byte aligned.
-size_t split_bytes_for(int64_t rows, int64_t D) {
-  return align256(size_t(rows) * size_t(3 * split_segment(D)) * 2);
-}
-
-size_t workspace_bytes_for(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
-  size_t b = state_bytes_for(N, V);
-  if (dtype == FLCE_FP32) b += split_bytes_for(N, D) + split_bytes_for(V, D);
-  return b;
-}
-
-// Makespan, in tiles, of the busiest worker when the units of a schedule are
-// handed out round-robin (worker c takes units c, c + g, c + 2g, ...) in the
-// grouped order of unit_coords.  Unit sizes are base + 1 tiles for slabs
-// < rem and base otherwise.  In group k the long units form one contiguous
-// run of rem * gt_k units starting at k * gt * P; a run of L units gives every
-// worker floor(L / g) of them plus one more to L mod g consecutive workers
-// (mod g), which a circular difference array accumulates.
-int64_t grouped_makespan(int64_t tb, int64_t gt, int64_t P, int64_t base, int64_t rem, int64_t g,
-                         std::vector<int64_t>& diff) {
-  const int64_t U = tb * P;
-  diff.assign(size_t(g) + 1, 0);
-  int64_t every = 0;
-  for (int64_t k = 0; k * gt < tb; ++k) {
-    const int64_t gk = std::min(gt, tb - k * gt);
-    const int64_t L = rem * gk;
-    every += L / g;
-    const int64_t r = L % g, a = (k * gt * P) % g;
-    if (r == 0) continue;
-    diff[size_t(a)] += 1;
-    if (a + r <= g) {
-      diff[size_t(a + r)] -= 1;
-    } else {
-      diff[size_t(g)] -= 1;
-      diff[0] += 1;
-      diff[size_t(a + r - g)] -= 1;
-    }
-  }
-  int64_t best = 0, run = 0;
-  for (int64_t c = 0; c < g; ++c) {
-    run += diff[size_t(c)];
-    const int64_t units_c = U / g + (c < U % g ? 1 : 0);
-    best = std::max(best, units_c * base + every + run);
-  }
-  return best;
-}
-
-// Choose P (slabs per token block) for `tb` token blocks in groups of `gt`,
-// `nt` vocab tiles and `g` concurrent workers: the smallest makespan, plus a
-// small per-unit cost (a partial state write and a pipeline restart).
-void choose_slabs(int64_t tb, int64_t gt, int64_t nt, int64_t g, int64_t pcap, int32_t& P_out,
-                  int64_t& makespan_out) {
-  double best = 1e300;
-  int32_t bestP = 1;
-  int64_t best_ms = 0;
-  std::vector<int64_t> diff;
-  for (int64_t P = 1; P <= std::min(nt, pcap); ++P) {
-    const int64_t ms = grouped_makespan(tb, gt, P, nt / P, nt % P, g, diff);
-    // Slabs of unequal length let the workers drift apart over the run, and
-    // the workers that share a W tile then fetch it from HBM at different
-    // times; equal slabs keep them in step.  So a schedule with a remainder
-    // pays 1% of its makespan (at N=8192 V=151936 D=4096 on a B200: 99 equal
-    // slabs of 6 tiles ran 7.70 ms per launch against 7.79 ms for 30 slabs
-    // of 19-20 tiles, sustained under the power cap).
-    const double cost = double(ms) * (nt % P != 0 ? 1.01 : 1.0) + 0.05 * double(cdiv(tb * P, g));
-    if (cost < best - 1e-9) {
-      best = cost;
-      bestP = int32_t(P);
-      best_ms = ms;
-    }
-  }
-  P_out = bestP;
-  makespan_out = best_ms;
-}
-
-// Token blocks per raster group: as many as keep the live part of H within
-// kGroupHBytes, so that it and the W tiles in flight stay in one die's L2
-// partition.
-constexpr int64_t kGroupHBytes = 32ll << 20;
-
-int64_t group_blocks_for(int64_t tb, int64_t block_rows, int64_t D, int64_t elem_bytes) {
-  const int64_t per_block = std::max<int64_t>(1, block_rows * D * elem_bytes);
-  return std::max<int64_t>(1, std::min(tb, kGroupHBytes / per_block));
-}
-
-// The contraction runs on CTA pairs (256-token tiles) unless the batch fits
-// one 128-token tile, where half of every pair tile would be padding.
-bool use_pair_kernel(int64_t N) { return N > tc::BM; }
-
-// `workers`: CTAs (single-CTA kernels) or CTA pairs (pair kernel) that run at once.
-flce_status make_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int64_t workers,
-                      flce_plan_t* p) {
-  std::memset(p, 0, sizeof(*p));
-  p->N = N;
-  p->V = V;
-  p->D = D;
-  p->dtype = int32_t(dtype);
-  p->tile_cols = kTileCols;
-  const bool pair = use_pair_kernel(N);
-  p->ctas_per_unit = pair ? 2 : 1;
-  p->block_rows = pair ? tc2::PAIR_M : tc::BM;
-  p->k_block = tc::BK;
-  p->token_blocks = cdiv(std::max<int64_t>(N, 1), p->block_rows);
-  p->vocab_tiles = cdiv(V, kTileCols);
-  const int64_t g = std::max<int64_t>(1, workers);
-  p->group_blocks = int32_t(group_blocks_for(p->token_blocks, p->block_rows, k_extent(D, dtype), 2));
-  int64_t ms = 0;
-  choose_slabs(p->token_blocks, p->group_blocks, p->vocab_tiles, g, slab_capacity(V), p->slabs,
-               ms);
-  p->slab_base = int32_t(p->vocab_tiles / p->slabs);
-  p->slab_rem = int32_t(p->vocab_tiles % p->slabs);
-  p->units = p->token_blocks * p->slabs;
-  p->grid = int32_t(std::min<int64_t>(g, p->units) * p->ctas_per_unit);
-  p->makespan_tiles = ms;
-  p->workspace_bytes = workspace_bytes_for(N, V, D, dtype);
-  return FLCE_OK;
-}
-
-int64_t nominal_workers(int32_t sms, int64_t N) {
-  return use_pair_kernel(N) ? std::max<int64_t>(1, sms / 2) : int64_t(sms);
-}
+#include "flce_schedule.h"
 
 // ---------------------------------------------------------------- driver entry point
 
