@@ -490,7 +490,34 @@ def time_quantized(flce, H, Wn, y, N, V, D, bits, gs, dev, stream, args, peak, w
     Ds = (D + 63) // 64 * 64
     tensor_flops = 2 * N * V * 2 * Ds      # [H | H] against [hi | lo]
     head_bytes = wq.nbytes + sc.nbytes + bi.nbytes
-    return {"bits": bits, "group_size": gs, "ms_per_step": ms, "steps": Kq,
+    extra = {}
+    if args.backward:
+        # dH of the mean loss for the frozen quantised head
+        bws = torch.empty(flce.backward_quantized_workspace_size(N, V, D, bits, gs),
+                          dtype=torch.uint8, device=dev)
+        dH = torch.empty(N, D, device=dev)
+
+        def bstep():
+            flce.backward_quantized(H, wqd, scd, bid, y, out["lse"], None, 1.0 / N, bits, gs,
+                                    out=dH, workspace=bws, stream=stream)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                bstep()
+        stream.synchronize()
+        if flce.check(bws, stream) != flce.OK:
+            raise flce.FlceError(flce.check(bws, stream), "backward_quantized")
+        Kb = max(3, args.backward_steps)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(Kb):
+                bstep()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        bms = max_over_ranks([e0.elapsed_time(e1) / Kb], world, device=dev)[0]
+        bflops = 2 * N * V * 2 * Ds + 2 * 2 * N * V * D   # logits over [H | H], dZ W_hi + dZ W_lo
+        extra = {"backward_ms_per_step": bms, "backward_tensor_tflops": bflops / (bms * 1e-3) / 1e12,
+                 "backward_what": "dH only (the quantised head is frozen): regenerated logits, 2 GEMMs"}
+    return {**extra, "bits": bits, "group_size": gs, "ms_per_step": ms, "steps": Kq,
             "tokens_per_s": weak_scaling_tokens_per_s(world, N, ms),
             "tflops": flops / (ms * 1e-3) / 1e12,
             "tensor_tflops": tensor_flops / (ms * 1e-3) / 1e12,

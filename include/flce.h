@@ -378,6 +378,36 @@ FLCE_API flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
                                             size_t workspace_bytes, void* stream);
 
 /*
+ * Backward of the forward with a quantised head: dH only.  A quantised head
+ * is frozen while the rest of the model trains (its codes cannot take a
+ * gradient step), so only the hidden-state gradient is formed:
+ *     dZ_ij = g_i (exp(z_ij - lse_i) - [j == y_i]),   dH = dZ W,
+ * with W the dequantised head (same format and arguments as
+ * flce_forward_quantized), g_i and lse as in flce_backward.
+ *   dH         (N, D) fp32 row-major, overwritten
+ *   workspace  >= flce_backward_quantized_workspace_size(N, V, D, bits,
+ *              group_size) bytes, 256-byte aligned: the status word, an
+ *              N x chunk bf16 slice of dZ and one chunk of W expanded to bf16
+ *              [hi | lo] (chunks of 16384 vocabulary rows)
+ * Per chunk: the codes are expanded as in flce_forward_quantized, the logits
+ * regenerated as [H | H] [hi | lo]^T on the tensor cores, dZ rounded to bf16,
+ * and dH accumulates dZ W_hi + dZ W_lo in that order: each entry is within
+ * about 2^-8 sum_j |dZ_ij| |W_jk| of the exact value (as flce_backward on
+ * bf16 inputs).  Errors as flce_forward_quantized; targets are checked on the
+ * device.  Deterministic.  N == 0 is a no-op.
+ */
+FLCE_API size_t flce_backward_quantized_workspace_size(int64_t N, int64_t V, int64_t D,
+                                                       int32_t bits, int32_t group_size);
+
+FLCE_API flce_status flce_backward_quantized(const void* H, const uint32_t* wq,
+                                             const void* scales, const void* biases,
+                                             int32_t bits, int32_t group_size, const int64_t* y,
+                                             const float* lse, const float* grad_loss,
+                                             float grad_scale, int64_t N, int64_t V, int64_t D,
+                                             float* dH, void* workspace, size_t workspace_bytes,
+                                             void* stream);
+
+/*
  * The forward on inputs that live in HOST memory, results returned to host
  * memory: the same operation as flce_forward (section 1 of the page), for
  * callers whose H, W and y are not on the device (W offloaded to the host,

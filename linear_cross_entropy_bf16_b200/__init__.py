@@ -24,7 +24,8 @@ import torch
 __all__ = [
     "FlceError", "forward", "backward", "partials", "merge", "workspace_size",
     "shard_state", "merge_shards", "forward_vocab_parallel", "forward_strided",
-    "forward_quantized", "quantized_workspace_size", "forward_host", "host_workspace_size",
+    "forward_quantized", "quantized_workspace_size", "backward_quantized",
+    "backward_quantized_workspace_size", "forward_host", "host_workspace_size",
     "backward_workspace_size", "plan", "check",
     "status_string", "selftest_wait_timeout", "library_path", "load_library",
 ]
@@ -138,6 +139,11 @@ def load_library():
         lib.flce_forward_quantized.argtypes = [vp, vp, vp, vp, i32, i32, vp, i64, i64, i64,
                                                vp, vp, vp, vp, vp, sz, vp]
         lib.flce_forward_quantized.restype = st
+        lib.flce_backward_quantized_workspace_size.argtypes = [i64, i64, i64, i32, i32]
+        lib.flce_backward_quantized_workspace_size.restype = sz
+        lib.flce_backward_quantized.argtypes = [vp, vp, vp, vp, i32, i32, vp, vp, vp,
+                                                ctypes.c_float, i64, i64, i64, vp, vp, sz, vp]
+        lib.flce_backward_quantized.restype = st
         lib.flce_forward_host_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int]
         lib.flce_forward_host_workspace_size.restype = sz
         lib.flce_forward_host.argtypes = [vp, vp, vp, i64, i64, i64, ctypes.c_int, vp, vp, vp, vp,
@@ -527,6 +533,62 @@ def forward_quantized(H: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, b
         _raise_on(lib.flce_check(workspace.data_ptr(), sp), "flce_forward_quantized (device)")
     return loss, lse, tgt, mean
 
+
+
+def backward_quantized_workspace_size(N: int, V: int, D: int, bits: int = 4, group_size: int = 64) -> int:
+    n = load_library().flce_backward_quantized_workspace_size(int(N), int(V), int(D), int(bits),
+                                                              int(group_size))
+    if n == 0:
+        raise FlceError(ERR_INVALID_ARG, "backward_quantized_workspace_size")
+    return int(n)
+
+
+def backward_quantized(H: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+                       y: torch.Tensor, lse: torch.Tensor, grad: torch.Tensor | None = None,
+                       grad_scale: float = 1.0, bits: int = 4, group_size: int = 64, *,
+                       out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                       stream=None, check: bool = False) -> torch.Tensor:
+    """flce_backward_quantized: dH (N, D) fp32 of sum_i g_i loss_i for a frozen
+    quantised head (arguments as forward_quantized and backward)."""
+    if H.dtype != torch.bfloat16 or H.dim() != 2 or not H.is_contiguous() or not H.is_cuda:
+        raise ValueError("H must be a contiguous 2-D bf16 CUDA tensor")
+    dev = H.device
+    N, D = H.shape
+    V = wq.shape[0]
+    if wq.dtype not in (torch.int32, torch.uint32) or wq.dim() != 2 or not wq.is_contiguous() \
+            or wq.shape[1] * 32 != D * bits:
+        raise ValueError("wq must be contiguous (V, D * bits / 32) int32/uint32 codes")
+    for name, t in (("scales", scales), ("biases", biases)):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or tuple(t.shape) != (V, D // group_size):
+            raise ValueError(f"{name} must be a contiguous bf16 (V, D / group_size) tensor")
+    if lse.dtype != torch.float32 or lse.shape != (N,) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 (N,) tensor")
+    if grad is not None and (grad.dtype != torch.float32 or grad.shape != (N,) or not grad.is_contiguous()):
+        raise ValueError("grad must be a contiguous float32 (N,) tensor")
+    if y.dtype != torch.int64 or y.shape != (N,) or not y.is_contiguous():
+        raise ValueError("y must be contiguous int64 of length N")
+    for t in (wq, scales, biases, y, lse):
+        if t.device != dev:
+            raise ValueError("all tensors must be on H's device")
+    dH = out if out is not None else torch.empty(N, D, dtype=torch.float32, device=dev)
+    if dH.dtype != torch.float32 or tuple(dH.shape) != (N, D) or not dH.is_contiguous() or dH.device != dev:
+        raise ValueError("out must be a contiguous float32 (N, D) tensor on H's device")
+    if N == 0:
+        return dH
+    lib = load_library()
+    need = backward_quantized_workspace_size(N, V, D, bits, group_size)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    sp = _stream_ptr(stream, dev)
+    _raise_on(lib.flce_backward_quantized(H.data_ptr(), wq.data_ptr(), scales.data_ptr(),
+                                          biases.data_ptr(), int(bits), int(group_size), y.data_ptr(),
+                                          lse.data_ptr(), grad.data_ptr() if grad is not None else None,
+                                          float(grad_scale), N, V, D, dH.data_ptr(), workspace.data_ptr(),
+                                          workspace.numel() * workspace.element_size(), sp),
+              "flce_backward_quantized")
+    if check:
+        _raise_on(lib.flce_check(workspace.data_ptr(), sp), "flce_backward_quantized (device)")
+    return dH
 
 def host_workspace_size(N: int, V: int, D: int) -> int:
     n = load_library().flce_forward_host_workspace_size(int(N), int(V), int(D), BF16)

@@ -39,6 +39,8 @@ struct GemmShape {
   int32_t group_m;        // m-blocks per raster group
   int32_t tiles;          // tiles_m * tiles_n
   int32_t kblocks;        // ceil(K / 64)
+  int32_t kblocks_a;      // K-blocks of A; A's K coordinate wraps modulo this (== kblocks,
+                          // except for the quantised head's [H | H])
 };
 
 // Tile t -> (m-block, n-block): groups of group_m m-blocks, n-major inside a
@@ -275,7 +277,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tile_coords(shape, t, mb, nb);
         const int arow = mb * PAIR_M + int(rank) * BM;
         const int brow = nb * BN + int(rank) * HALF_N;
-        for (int kb = 0; kb < shape.kblocks; ++kb) {
+        for (int kb = 0, ka = 0; kb < shape.kblocks; ++kb) {
           if (!wait_bounded(ptx::smem_addr(&empty_bar[stage]), phase ^ 1u, abort_flag, status,
                             lim)) {
             ok = false;
@@ -286,11 +288,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
           if (rank == 0) ptx::mbar_arrive_expect_tx(fb_local, PAIR_TX_BYTES);
           if (kAmn) {  // two 64 (M) x 64 (K) boxes
-            ptx::tma_load_2d_pair(sa, &tmA, fb_even, arow, kb * BK);
-            ptx::tma_load_2d_pair(sa + MN_BOX_BYTES, &tmA, fb_even, arow + MN_CHUNK, kb * BK);
+            ptx::tma_load_2d_pair(sa, &tmA, fb_even, arow, ka * BK);
+            ptx::tma_load_2d_pair(sa + MN_BOX_BYTES, &tmA, fb_even, arow + MN_CHUNK, ka * BK);
           } else {     // one 64 (K) x 128 (M) box
-            ptx::tma_load_2d_pair(sa, &tmA, fb_even, kb * BK, arow);
+            ptx::tma_load_2d_pair(sa, &tmA, fb_even, ka * BK, arow);
           }
+          if (++ka == shape.kblocks_a) ka = 0;
           if (kBmn) {
             ptx::tma_load_2d_pair(sa + A_BYTES, &tmB, fb_even, brow, kb * BK);
             ptx::tma_load_2d_pair(sa + A_BYTES + MN_BOX_BYTES, &tmB, fb_even, brow + MN_CHUNK,

@@ -281,3 +281,22 @@ def test_backward_workspace_fp32_adds_split_copies(lib):
         bf16 = flce.backward_workspace_size(N, V, D) if D % 8 == 0 else 256 + r256(2 * N * chunk)
         assert flce.backward_workspace_size(N, V, D, 1) == (
             bf16 + r256(2 * N * chunk) + r256(6 * Dp * N) + r256(6 * Dp * chunk))
+
+
+def test_quantized_backward_workspace_and_checks_need_no_gpu(lib):
+    r256 = lambda b: (b + 255) // 256 * 256
+    N, V, D = 300, 40000, 96
+    chunk = 16384
+    Ds = 128
+    assert flce.backward_quantized_workspace_size(N, V, D, 4, 32) == 256 + r256(2 * N * chunk) + r256(chunk * 2 * Ds * 2)
+    assert lib.flce_backward_quantized_workspace_size(N, V, D, 4, 64) == 0     # 96 % 64 != 0
+
+    def call(bits=4, G=64, N=16, V=100, D=128, H=FAKE, lse=FAKE, dH=FAKE, ws=FAKE, ws_bytes=1 << 30):
+        return lib.flce_backward_quantized(H, FAKE, FAKE, FAKE, bits, G, FAKE, lse, None, 1.0, N, V, D,
+                                           dH, ws, ws_bytes, None)
+    assert call(bits=3) == flce.ERR_INVALID_ARG
+    assert call(lse=None) == flce.ERR_INVALID_ARG
+    assert call(dH=None) == flce.ERR_INVALID_ARG
+    assert call(H=FAKE + 8) == flce.ERR_UNSUPPORTED
+    assert call(ws_bytes=64) == flce.ERR_WORKSPACE_TOO_SMALL
+    assert call(N=0) == flce.OK

@@ -136,3 +136,51 @@ def test_quantized_page_shape_sampled_rows():
     compare(gpu, ref, rows=rows)
     # logits of a 4-bit head of N(0, 1/D) weights are still about N(0, 1): loss near ln V + 1/2
     assert abs(gpu["mean"] - (math.log(V) + 0.5)) < 0.2
+
+
+# ---------------------------------------------------------------- backward (dH only)
+# dZ is rounded to bf16 before dH = dZ (W_hi + W_lo) is accumulated in fp32,
+# so |d dH_ik| <= 2^-8 sum_j |dZ_ij| |W_jk| (the oracle's bH on the
+# dequantised W; the hi/lo split adds only 2^-16 of it), plus a tiny floor.
+
+
+def run_q_backward(H, wq, s, b, y, bits, G, g=None, scale=1.0):
+    import linear_cross_entropy_bf16_b200 as flce
+    Hd, wqd, sd, bd, yd = to_dev(H, wq, s, b, y)
+    _, lse, _, _ = flce.forward_quantized(Hd, wqd, sd, bd, yd, bits, G, check=True)
+    gd = torch.from_numpy(np.asarray(g, dtype=np.float32)).cuda() if g is not None else None
+    dH = flce.backward_quantized(Hd, wqd, sd, bd, yd, lse, gd, scale, bits, G, check=True)
+    torch.cuda.synchronize()
+    return dH.cpu().double().numpy()
+
+
+@pytest.mark.parametrize("N,V,D,bits,G", [(1, 1, 64, 4, 64), (7, 300, 64, 4, 32),
+                                          (130, 2047, 128, 4, 64), (300, 5000, 96, 2, 32),
+                                          (200, 40000, 64, 8, 64), (257, 16389, 192, 4, 64)])
+def test_quantized_backward_every_element(N, V, D, bits, G):
+    H, wq, s, b, y = inputs(N, V, D, bits, G, seed=3 * N + V + D)
+    g = np.random.default_rng(N).uniform(-1, 1, N)
+    dH = run_q_backward(H, wq, s, b, y, bits, G, g)
+    Wd = oracle.dequantize(wq, s, b, bits, G)
+    Hf = synth.bf16_bits_to_f32(H).astype(np.float64)
+    ref = oracle.backward(Hf, Wd, y, g.astype(np.float32).astype(np.float64), bounds=True)
+    err = np.abs(dH - ref["dH"])
+    lim = 2.0 ** -8 * ref["bH"] + 1e-7
+    worst = np.unravel_index(np.argmax(err - lim), err.shape)
+    assert np.all(err <= lim), (worst, err[worst], lim[worst])
+    assert np.linalg.norm(dH - ref["dH"]) / max(np.linalg.norm(ref["dH"]), 1e-30) < 3e-3
+
+
+def test_quantized_backward_deterministic_and_target_check():
+    import linear_cross_entropy_bf16_b200 as flce
+    N, V, D, bits, G = 300, 20000, 128, 4, 64
+    H, wq, s, b, y = inputs(N, V, D, bits, G, seed=9)
+    Hd, wqd, sd, bd, yd = to_dev(H, wq, s, b, y)
+    _, lse, _, _ = flce.forward_quantized(Hd, wqd, sd, bd, yd, bits, G)
+    a = flce.backward_quantized(Hd, wqd, sd, bd, yd, lse, None, 1.0 / N, bits, G).clone()
+    c = flce.backward_quantized(Hd, wqd, sd, bd, yd, lse, None, 1.0 / N, bits, G, check=True)
+    assert torch.equal(a, c)
+    yb = yd.clone()
+    yb[3] = -1
+    with pytest.raises(flce.FlceError):
+        flce.backward_quantized(Hd, wqd, sd, bd, yb, lse, None, 1.0, bits, G, check=True)
