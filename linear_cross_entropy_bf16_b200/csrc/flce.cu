@@ -78,17 +78,27 @@ flce_status device_info(DeviceInfo& di) {
   return FLCE_OK;
 }
 
-flce_status set_smem_attr_once() {
-  static std::once_flag once;
-  static cudaError_t err = cudaSuccess;
-  std::call_once(once, [] {
-    err = cudaFuncSetAttribute(tc::flce_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               tc::SMEM_BYTES);
-    if (err == cudaSuccess)
-      err = cudaFuncSetAttribute(tc2::flce_tc2_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, tc2::SMEM_BYTES);
-  });
-  return err == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+// A kernel's dynamic shared-memory limit is a per-device setting: raise it
+// once for each (kernel, device) pair, on the current device.
+flce_status ensure_smem_limit(const void* fn, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> done;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& d : done)
+    if (d.first == fn && d.second == dev) return FLCE_OK;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  done.emplace_back(fn, dev);
+  return FLCE_OK;
+}
+
+flce_status set_smem_limits() {
+  flce_status s = ensure_smem_limit(reinterpret_cast<const void*>(tc::flce_tc_kernel),
+                                    tc::SMEM_BYTES);
+  if (s != FLCE_OK) return s;
+  return ensure_smem_limit(reinterpret_cast<const void*>(tc2::flce_tc2_kernel), tc2::SMEM_BYTES);
 }
 
 // CTA pairs of the pair kernel that can be resident at once on the current
@@ -137,7 +147,7 @@ flce_status check_forward_args(const void* H, const void* W, const int64_t* y, i
 flce_status contraction_workers(int64_t N, DeviceInfo& di, int64_t& workers) {
   flce_status s = device_info(di);
   if (s != FLCE_OK) return s;
-  if ((s = set_smem_attr_once()) != FLCE_OK) return s;
+  if ((s = set_smem_limits()) != FLCE_OK) return s;
   workers = nominal_workers(di.sms, N);
   if (use_pair_kernel(N)) {
     int dev = 0;
@@ -527,13 +537,9 @@ bwd::GemmShape gemm_shape(int64_t M, int64_t Nc, int64_t K) {
 template <class Epi, bool kAmn, bool kBmn>
 flce_status launch_gemm(const CUtensorMap& A, const CUtensorMap& B, const bwd::GemmShape& g,
                         const Epi& epi, uint32_t* status, int64_t pairs, cudaStream_t st) {
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(bwd::gemm_pair_kernel<Epi, kAmn, kBmn>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::SMEM_BYTES);
-  });
-  if (attr != cudaSuccess) return FLCE_ERR_CUDA;
+  flce_status s = ensure_smem_limit(
+      reinterpret_cast<const void*>(bwd::gemm_pair_kernel<Epi, kAmn, kBmn>), bwd::SMEM_BYTES);
+  if (s != FLCE_OK) return s;
   const int grid = int(2 * std::min<int64_t>(pairs, g.tiles));
   bwd::gemm_pair_kernel<Epi, kAmn, kBmn><<<grid, bwd::NUM_THREADS, bwd::SMEM_BYTES, st>>>(
       A, B, g, epi, status, kDefaultWaitLimitNs);
@@ -572,7 +578,7 @@ extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t
   if (!load_encoder()) return FLCE_ERR_CUDA;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
-  if ((s = set_smem_attr_once()) != FLCE_OK) return s;
+  if ((s = set_smem_limits()) != FLCE_OK) return s;
   const int64_t pairs = resident_pairs(dev, di.sms);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
@@ -1057,7 +1063,7 @@ extern "C" flce_status flce_backward_quantized(const void* H, const uint32_t* wq
   if (!load_encoder()) return FLCE_ERR_CUDA;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
-  if ((s = set_smem_attr_once()) != FLCE_OK) return s;
+  if ((s = set_smem_limits()) != FLCE_OK) return s;
   const int64_t pairs = resident_pairs(dev, di.sms);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
