@@ -378,6 +378,27 @@ FLCE_API flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
                                             size_t workspace_bytes, void* stream);
 
 /*
+ * Vocabulary-parallel backward: this caller holds W rows [v_offset, v_offset
+ * + V_shard) of a V_total-word vocabulary (as in flce_partials_shard).  With
+ * lse the log-sum-exp over the WHOLE vocabulary (flce_merge_shards), it
+ * writes this shard's rows of dW and this shard's share of dH:
+ *     dH_partial = sum_{j in shard} dZ_ij W_j,     dW_shard = dZ_shard^T H,
+ * so that dH is the sum of dH_partial over the shards (one all-reduce; the
+ * Python binding's backward_vocab_parallel does it over torch.distributed).
+ * A target outside the shard adds no one-hot term here; a target outside
+ * [0, V_total) sets FLCE_ERR_TARGET_OUT_OF_RANGE.  Arguments, workspace
+ * (flce_backward_workspace_size(N, V_shard, D, dtype)), precision and errors
+ * otherwise as flce_backward; FLCE_ERR_INVALID_ARG if the shard does not lie
+ * inside [0, V_total).
+ */
+FLCE_API flce_status flce_backward_shard(const void* H, const void* W_shard, const int64_t* y,
+                                         const float* lse, const float* grad_loss,
+                                         float grad_scale, int64_t N, int64_t V_shard,
+                                         int64_t v_offset, int64_t V_total, int64_t D,
+                                         flce_dtype dtype, float* dH_partial, float* dW_shard,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Backward of the forward with a quantised head: dH only.  A quantised head
  * is frozen while the rest of the model trains (its codes cannot take a
  * gradient step), so only the hidden-state gradient is formed:

@@ -24,6 +24,7 @@ import torch
 __all__ = [
     "FlceError", "forward", "backward", "partials", "merge", "workspace_size",
     "shard_state", "merge_shards", "forward_vocab_parallel", "forward_strided",
+    "backward_shard", "backward_vocab_parallel",
     "forward_quantized", "quantized_workspace_size", "backward_quantized",
     "backward_quantized_workspace_size", "forward_host", "host_workspace_size",
     "backward_workspace_size", "plan", "check",
@@ -139,6 +140,9 @@ def load_library():
         lib.flce_forward_quantized.argtypes = [vp, vp, vp, vp, i32, i32, vp, i64, i64, i64,
                                                vp, vp, vp, vp, vp, sz, vp]
         lib.flce_forward_quantized.restype = st
+        lib.flce_backward_shard.argtypes = [vp, vp, vp, vp, vp, ctypes.c_float, i64, i64, i64, i64,
+                                            i64, ctypes.c_int, vp, vp, vp, sz, vp]
+        lib.flce_backward_shard.restype = st
         lib.flce_backward_quantized_workspace_size.argtypes = [i64, i64, i64, i32, i32]
         lib.flce_backward_quantized_workspace_size.restype = sz
         lib.flce_backward_quantized.argtypes = [vp, vp, vp, vp, i32, i32, vp, vp, vp,
@@ -417,6 +421,61 @@ def forward_vocab_parallel(H: torch.Tensor, W_shard: torch.Tensor, y: torch.Tens
     else:
         gathered = state.unsqueeze(0)
     return merge_shards(gathered, y, V_total, check=check)
+
+
+def backward_shard(H: torch.Tensor, W_shard: torch.Tensor, y: torch.Tensor, lse: torch.Tensor,
+                   v_offset: int, V_total: int, grad: torch.Tensor | None = None,
+                   grad_scale: float = 1.0, *, out: dict | None = None,
+                   workspace: torch.Tensor | None = None, stream=None, check: bool = False):
+    """flce_backward_shard: (dH_partial, dW_shard) for W rows [v_offset, v_offset + V_shard)
+    of a V_total-word vocabulary, with lse over the whole vocabulary."""
+    N, V, D, code = _check_inputs(H, W_shard, y)
+    dev = H.device
+    out = out or {}
+    dH = out.get("dH") if out.get("dH") is not None else torch.empty(N, D, dtype=torch.float32, device=dev)
+    dW = out.get("dW") if out.get("dW") is not None else torch.empty(V, D, dtype=torch.float32, device=dev)
+    for t, shape in ((dH, (N, D)), (dW, (V, D))):
+        if t.dtype != torch.float32 or t.device != dev or not t.is_contiguous() or tuple(t.shape) != shape:
+            raise ValueError("dH and dW must be contiguous float32 (N, D) and (V_shard, D) tensors")
+    if lse.dtype != torch.float32 or lse.shape != (N,) or not lse.is_contiguous() or lse.device != dev:
+        raise ValueError("lse must be a contiguous float32 (N,) tensor on the input device")
+    if grad is not None and (grad.dtype != torch.float32 or grad.shape != (N,) or not grad.is_contiguous()
+                             or grad.device != dev):
+        raise ValueError("grad must be a contiguous float32 (N,) tensor on the input device")
+    if N == 0:
+        dH.zero_()
+        dW.zero_()
+        return dH, dW
+    lib = load_library()
+    need = lib.flce_backward_workspace_size(N, V, D, code)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace.numel() * workspace.element_size() < need:
+        raise FlceError(ERR_WORKSPACE_TOO_SMALL, "backward_shard")
+    sp = _stream_ptr(stream, dev)
+    _raise_on(lib.flce_backward_shard(H.data_ptr(), W_shard.data_ptr(), y.data_ptr(), lse.data_ptr(),
+                                      grad.data_ptr() if grad is not None else None, float(grad_scale),
+                                      N, V, int(v_offset), int(V_total), D, code, dH.data_ptr(),
+                                      dW.data_ptr(), workspace.data_ptr(),
+                                      workspace.numel() * workspace.element_size(), sp),
+              "flce_backward_shard")
+    if check:
+        _raise_on(lib.flce_check(workspace.data_ptr(), sp), "flce_backward_shard (device)")
+    return dH, dW
+
+
+def backward_vocab_parallel(H: torch.Tensor, W_shard: torch.Tensor, y: torch.Tensor, lse: torch.Tensor,
+                            v_offset: int, V_total: int, grad: torch.Tensor | None = None,
+                            grad_scale: float = 1.0, group=None, check: bool = False):
+    """Vocabulary-parallel backward: every rank of `group` passes the same H, y and the
+    whole-vocabulary lse (from forward_vocab_parallel) and its own W shard.  Returns
+    (dH, dW_shard): dH summed over the shards with one all-reduce over
+    torch.distributed (NCCL on GPUs), dW_shard this rank's rows of dW."""
+    import torch.distributed as dist
+    dH, dW = backward_shard(H, W_shard, y, lse, v_offset, V_total, grad, grad_scale, check=check)
+    if dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(dH, op=dist.ReduceOp.SUM, group=group)
+    return dH, dW
 
 
 def partials(H, W, y, target_logit, workspace, stream=None):

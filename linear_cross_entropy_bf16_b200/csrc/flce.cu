@@ -553,11 +553,15 @@ extern "C" size_t flce_backward_workspace_size(int64_t N, int64_t V, int64_t D, 
   return bwd_layout(N, V, D, dtype).total;
 }
 
-extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t* y,
-                                     const float* lse, const float* grad_loss, float grad_scale,
-                                     int64_t N, int64_t V, int64_t D, flce_dtype dtype, float* dH,
-                                     float* dW, void* workspace, size_t workspace_bytes,
-                                     void* stream) {
+namespace {
+
+// The backward over W's rows [0, V) (a whole head, or one vocabulary shard
+// whose first row is vocabulary id y_offset of a V_total-word vocabulary).
+flce_status backward_impl(const void* H, const void* W, const int64_t* y, const float* lse,
+                          const float* grad_loss, float grad_scale, int64_t N, int64_t V,
+                          int64_t y_offset, int64_t V_total, int64_t D, flce_dtype dtype,
+                          float* dH, float* dW, void* workspace, size_t workspace_bytes,
+                          void* stream) {
   if (!sizes_ok(N, V, D, dtype)) return FLCE_ERR_INVALID_ARG;
   if (N == 0) return FLCE_OK;
   if (!H || !W || !y || !lse || !dH || !dW || !workspace) return FLCE_ERR_INVALID_ARG;
@@ -633,7 +637,8 @@ extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t
     e1.grad = grad_loss;
     e1.grad_scale = grad_scale;
     e1.N = int32_t(N);
-    e1.V = int32_t(V);
+    e1.V = int32_t(V_total);
+    e1.y_offset = y_offset;
     e1.c0 = int32_t(c0);
     e1.clen = int32_t(clen);
     e1.dz = dz;
@@ -673,6 +678,30 @@ extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t
     }
   }
   return FLCE_OK;
+}
+
+}  // namespace
+
+extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t* y,
+                                     const float* lse, const float* grad_loss, float grad_scale,
+                                     int64_t N, int64_t V, int64_t D, flce_dtype dtype, float* dH,
+                                     float* dW, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  return backward_impl(H, W, y, lse, grad_loss, grad_scale, N, V, 0, V, D, dtype, dH, dW,
+                       workspace, workspace_bytes, stream);
+}
+
+extern "C" flce_status flce_backward_shard(const void* H, const void* W_shard, const int64_t* y,
+                                           const float* lse, const float* grad_loss,
+                                           float grad_scale, int64_t N, int64_t V_shard,
+                                           int64_t v_offset, int64_t V_total, int64_t D,
+                                           flce_dtype dtype, float* dH_partial, float* dW_shard,
+                                           void* workspace, size_t workspace_bytes,
+                                           void* stream) {
+  if (v_offset < 0 || V_shard < 1 || V_total < v_offset + V_shard || V_total >= (int64_t(1) << 31))
+    return FLCE_ERR_INVALID_ARG;
+  return backward_impl(H, W_shard, y, lse, grad_loss, grad_scale, N, V_shard, v_offset, V_total,
+                       D, dtype, dH_partial, dW_shard, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------- no-allocation entry point
@@ -1097,6 +1126,7 @@ extern "C" flce_status flce_backward_quantized(const void* H, const uint32_t* wq
     e1.grad_scale = grad_scale;
     e1.N = int32_t(N);
     e1.V = int32_t(V);
+    e1.y_offset = 0;
     e1.c0 = int32_t(c0);
     e1.clen = int32_t(clen);
     e1.dz = dz;

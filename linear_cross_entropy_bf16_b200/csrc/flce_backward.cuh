@@ -89,7 +89,8 @@ struct EpiGradLogits {
   float grad_scale;          // multiplies grad
   int32_t N;                 // tokens
   int32_t V;                 // vocabulary size (for the target check)
-  int32_t c0;                // first vocabulary row of this chunk
+  int64_t y_offset;          // vocabulary id of W's first row (a vocabulary shard); else 0
+  int32_t c0;                // first row of this chunk within W
   int32_t clen;              // vocabulary rows in this chunk
   __nv_bfloat16* dz;         // (N x ldz) token-major slice, columns = chunk vocab
   __nv_bfloat16* dz_lo;      // null, or (N x ldz): bf16(dZ - dz) for fp32 inputs, so that
@@ -106,7 +107,7 @@ struct EpiGradLogits {
       gi = grad_scale * (grad ? grad[row] : 1.f);
       const int64_t yi = y[row];
       if (yi < 0 || yi >= V) atomicOr(status, kStatTarget);
-      yrel = yi - c0;
+      yrel = yi - y_offset - c0;
     }
 #pragma unroll 1
     for (int c = 0; c < kTileCols / 32; ++c) {

@@ -65,3 +65,53 @@ def test_target_held_by_no_shard_is_flagged():
     with pytest.raises(flce.FlceError) as e:
         flce.merge_shards(states, yd, 1000, check=True)
     assert e.value.status == flce.ERR_TARGET_OUT_OF_RANGE
+
+
+# ---------------------------------------------------------------- backward
+# Each shard's flce_backward_shard gives its rows of dW and its share of dH;
+# the shares are summed as the ranks' all-reduce would.  dZ is rounded to
+# bf16 (bf16 inputs), so every entry of dH and dW is within 2^-8 of the
+# oracle's magnitude bound (bH, bW), as for the single-GPU backward.
+
+
+@pytest.mark.parametrize("N,V,D,bounds,dtype", [
+    (300, 5000, 128, [0, 2000, 2100, 5000], "bf16"),
+    (129, 40000, 64, [0, 17500, 35000, 40000], "bf16"),   # shards spanning several chunks
+    (200, 3000, 40, [0, 1, 1500, 3000], "fp32"),          # a one-row shard, fp32 inputs
+])
+def test_sharded_backward_matches_oracle(N, V, D, bounds, dtype):
+    import linear_cross_entropy_bf16_b200 as flce
+    H, W, y = synth.random_inputs(N, V, D, seed=V + 7 * len(bounds), dtype=dtype)
+    Hd, Wd, yd = to_device(H, W, y)
+    _, lse, _, _ = flce.forward(Hd, Wd, yd, check=True)
+    g = np.random.default_rng(N).uniform(-1, 1, N)
+    gd = torch.from_numpy(g.astype(np.float32)).cuda()
+    dH = torch.zeros(N, D, dtype=torch.float64, device="cuda")
+    dW = []
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        part, dWs = flce.backward_shard(Hd, Wd[a:b].contiguous(), yd, lse, a, V, gd, check=True)
+        dH += part.double()
+        dW.append(dWs)
+    dW = torch.cat(dW).cpu().double().numpy()
+    dH = dH.cpu().numpy()
+    ref = oracle.backward(H, W, y, g.astype(np.float32).astype(np.float64), bounds=True)
+    for got, r, bnd, name in ((dH, ref["dH"], ref["bH"], "dH"), (dW, ref["dW"], ref["bW"], "dW")):
+        err = np.abs(got - r)
+        lim = 2.0 ** -8 * bnd + 1e-7
+        assert np.all(err <= lim), (name, float((err - lim).max()))
+    # dW rows do not depend on how the vocabulary is cut: equal to the unsharded backward's
+    _, dW_full = flce.backward(Hd, Wd, yd, lse, gd, check=True)
+    assert np.array_equal(dW, dW_full.cpu().double().numpy())
+
+
+def test_sharded_backward_flags_targets_outside_the_vocabulary():
+    import linear_cross_entropy_bf16_b200 as flce
+    N, V, D = 64, 1000, 64
+    H, W, y = synth.random_inputs(N, V, D, seed=53)
+    Hd, Wd, yd = to_device(H, W, y)
+    _, lse, _, _ = flce.forward(Hd, Wd, yd, check=True)
+    yb = yd.clone()
+    yb[3] = V + 5
+    with pytest.raises(flce.FlceError) as e:
+        flce.backward_shard(Hd, Wd[600:].contiguous(), yb, lse, 600, V, check=True)
+    assert e.value.status == flce.ERR_TARGET_OUT_OF_RANGE

@@ -140,3 +140,55 @@ def test_vocab_parallel_exchange_on_two_gloo_ranks():
         assert p.exitcode == 0
     for rank, dloss, dmean in out:
         assert dloss < 1e-12 and abs(dmean) < 1e-12
+
+
+def _vpb_worker(rank, world, port, q):
+    """backward_vocab_parallel's all-reduce on two gloo ranks; the kernel step is
+    replaced by an fp64 restatement of one shard's dH share and dW rows."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import linear_cross_entropy_bf16_b200 as flce
+        rng = np.random.default_rng(8)
+        N, V, D = 6, 10, 4
+        H = torch.from_numpy(rng.standard_normal((N, D)))
+        W = torch.from_numpy(rng.standard_normal((V, D)))
+        y = torch.from_numpy(rng.integers(0, V, N))
+        lse = torch.logsumexp(H @ W.T, dim=1)
+        cut = [0, 3, 10]
+        a, b = cut[rank], cut[rank + 1]
+
+        def fake_shard(H_, W_shard, y_, lse_, v_offset, V_total, grad=None, grad_scale=1.0, **kw):
+            z = H_ @ W_shard.T
+            p = torch.exp(z - lse_[:, None])
+            rel = y_ - v_offset
+            own = (rel >= 0) & (rel < W_shard.shape[0])
+            onehot = torch.zeros_like(p)
+            onehot[own, rel[own]] = 1.0
+            dz = grad_scale * (p - onehot)
+            return dz @ W_shard, dz.T @ H_
+
+        flce.backward_shard = fake_shard
+        dH, dW = flce.backward_vocab_parallel(H, W[a:b].contiguous(), y, lse, a, V, grad_scale=1.0 / N)
+        Hr = H.clone().requires_grad_(True)
+        Wr = W.clone().requires_grad_(True)
+        torch.nn.functional.cross_entropy(Hr @ Wr.T, y).backward()
+        q.put((rank, float((dH - Hr.grad).abs().max()), float((dW - Wr.grad[a:b]).abs().max())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_vocab_parallel_backward_allreduce_on_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_vpb_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=240) for _ in procs]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    for rank, ddH, ddW in out:
+        assert ddH < 1e-12 and ddW < 1e-12
