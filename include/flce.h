@@ -390,13 +390,18 @@ FLCE_API flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
  * (flce_backward_workspace_size(N, V_shard, D, dtype)), precision and errors
  * otherwise as flce_backward; FLCE_ERR_INVALID_ARG if the shard does not lie
  * inside [0, V_total).
+ *   dh_ready_event  a cudaEvent_t or NULL: recorded on `stream` as soon as
+ *            dH_partial is final, before the last chunk's dW GEMMs, so that a
+ *            collective on dH (on another stream waiting for the event) can
+ *            overlap them.
  */
 FLCE_API flce_status flce_backward_shard(const void* H, const void* W_shard, const int64_t* y,
                                          const float* lse, const float* grad_loss,
                                          float grad_scale, int64_t N, int64_t V_shard,
                                          int64_t v_offset, int64_t V_total, int64_t D,
                                          flce_dtype dtype, float* dH_partial, float* dW_shard,
-                                         void* workspace, size_t workspace_bytes, void* stream);
+                                         void* workspace, size_t workspace_bytes, void* stream,
+                                         void* dh_ready_event);
 
 /*
  * Backward of the forward with a quantised head: dH only.  A quantised head

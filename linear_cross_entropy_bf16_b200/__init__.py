@@ -141,7 +141,7 @@ def load_library():
                                                vp, vp, vp, vp, vp, sz, vp]
         lib.flce_forward_quantized.restype = st
         lib.flce_backward_shard.argtypes = [vp, vp, vp, vp, vp, ctypes.c_float, i64, i64, i64, i64,
-                                            i64, ctypes.c_int, vp, vp, vp, sz, vp]
+                                            i64, ctypes.c_int, vp, vp, vp, sz, vp, vp]
         lib.flce_backward_shard.restype = st
         lib.flce_backward_quantized_workspace_size.argtypes = [i64, i64, i64, i32, i32]
         lib.flce_backward_quantized_workspace_size.restype = sz
@@ -192,6 +192,21 @@ def plan(N: int, V: int, D: int, dtype=torch.bfloat16, sm_count: int = 148) -> d
     _raise_on(load_library().flce_plan(int(N), int(V), int(D), code, int(sm_count), ctypes.byref(p)),
               "plan")
     return p.as_dict()
+
+
+_side_streams: dict = {}
+
+
+def _side_stream(device) -> "torch.cuda.Stream":
+    """One extra stream per device for collectives that overlap the kernels."""
+    key = torch.device(device).index
+    if key not in _side_streams:
+        _side_streams[key] = torch.cuda.Stream(device)
+    return _side_streams[key]
+
+
+def _event_ptr(event) -> int | None:
+    return int(event.cuda_event) if event is not None else None
 
 
 def _stream_ptr(stream, device) -> int:
@@ -426,9 +441,11 @@ def forward_vocab_parallel(H: torch.Tensor, W_shard: torch.Tensor, y: torch.Tens
 def backward_shard(H: torch.Tensor, W_shard: torch.Tensor, y: torch.Tensor, lse: torch.Tensor,
                    v_offset: int, V_total: int, grad: torch.Tensor | None = None,
                    grad_scale: float = 1.0, *, out: dict | None = None,
-                   workspace: torch.Tensor | None = None, stream=None, check: bool = False):
+                   workspace: torch.Tensor | None = None, stream=None, dh_ready=None,
+                   check: bool = False):
     """flce_backward_shard: (dH_partial, dW_shard) for W rows [v_offset, v_offset + V_shard)
-    of a V_total-word vocabulary, with lse over the whole vocabulary."""
+    of a V_total-word vocabulary, with lse over the whole vocabulary.  ``dh_ready``
+    (a torch.cuda.Event) is recorded once dH_partial is final, before the last dW GEMMs."""
     N, V, D, code = _check_inputs(H, W_shard, y)
     dev = H.device
     out = out or {}
@@ -457,7 +474,8 @@ def backward_shard(H: torch.Tensor, W_shard: torch.Tensor, y: torch.Tensor, lse:
                                       grad.data_ptr() if grad is not None else None, float(grad_scale),
                                       N, V, int(v_offset), int(V_total), D, code, dH.data_ptr(),
                                       dW.data_ptr(), workspace.data_ptr(),
-                                      workspace.numel() * workspace.element_size(), sp),
+                                      workspace.numel() * workspace.element_size(), sp,
+                                      _event_ptr(dh_ready)),
               "flce_backward_shard")
     if check:
         _raise_on(lib.flce_check(workspace.data_ptr(), sp), "flce_backward_shard (device)")
@@ -472,9 +490,29 @@ def backward_vocab_parallel(H: torch.Tensor, W_shard: torch.Tensor, y: torch.Ten
     (dH, dW_shard): dH summed over the shards with one all-reduce over
     torch.distributed (NCCL on GPUs), dW_shard this rank's rows of dW."""
     import torch.distributed as dist
-    dH, dW = backward_shard(H, W_shard, y, lse, v_offset, V_total, grad, grad_scale, check=check)
-    if dist.is_initialized() and dist.get_world_size(group) > 1:
+    multi = dist.is_initialized() and dist.get_world_size(group) > 1
+    if not (multi and H.is_cuda):
+        dH, dW = backward_shard(H, W_shard, y, lse, v_offset, V_total, grad, grad_scale, check=check)
+        if multi:
+            dist.all_reduce(dH, op=dist.ReduceOp.SUM, group=group)
+        return dH, dW
+    # The all-reduce of dH runs on a side stream as soon as dH is final, while
+    # the last dW GEMMs finish on the compute stream.
+    main = torch.cuda.current_stream(H.device)
+    side = _side_stream(H.device)
+    ready = torch.cuda.Event()
+    ws = torch.empty(backward_workspace_size(H.shape[0], W_shard.shape[0], H.shape[1], H.dtype),
+                     dtype=torch.uint8, device=H.device)
+    dH, dW = backward_shard(H, W_shard, y, lse, v_offset, V_total, grad, grad_scale, workspace=ws,
+                            stream=main, dh_ready=ready)
+    side.wait_event(ready)
+    with torch.cuda.stream(side):
         dist.all_reduce(dH, op=dist.ReduceOp.SUM, group=group)
+    dH.record_stream(side)
+    main.wait_stream(side)
+    if check:
+        _raise_on(load_library().flce_check(ws.data_ptr(), _stream_ptr(main, H.device)),
+                  "backward_vocab_parallel (device)")
     return dH, dW
 
 

@@ -561,7 +561,7 @@ flce_status backward_impl(const void* H, const void* W, const int64_t* y, const 
                           const float* grad_loss, float grad_scale, int64_t N, int64_t V,
                           int64_t y_offset, int64_t V_total, int64_t D, flce_dtype dtype,
                           float* dH, float* dW, void* workspace, size_t workspace_bytes,
-                          void* stream) {
+                          void* stream, cudaEvent_t dh_ready) {
   if (!sizes_ok(N, V, D, dtype)) return FLCE_ERR_INVALID_ARG;
   if (N == 0) return FLCE_OK;
   if (!H || !W || !y || !lse || !dH || !dW || !workspace) return FLCE_ERR_INVALID_ARG;
@@ -662,6 +662,10 @@ flce_status backward_impl(const void* H, const void* W, const int64_t* y, const 
                                                      e2, &hdr->status, pairs, st);
       if (s != FLCE_OK) return s;
     }
+    // dH is final once the last chunk's dH GEMMs are queued: a collective on
+    // it can start while the dW GEMMs below finish.
+    if (dh_ready && c0 + L.chunk >= V && cudaEventRecord(dh_ready, st) != cudaSuccess)
+      return FLCE_ERR_CUDA;
     // K3: dW_C = dZ_C^T H; fp32: dz^T H_hi + dz^T H_lo + dz_lo^T H_hi, in that order
     const CUtensorMap* k3[3][2] = {{&mDz_mn, &mH_mn}, {&mDz_mn, &mH_mn_lo}, {&mDzl_mn, &mH_mn}};
     for (int p = 0; p < (fp32 ? 3 : 1); ++p) {
@@ -688,7 +692,7 @@ extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t
                                      float* dW, void* workspace, size_t workspace_bytes,
                                      void* stream) {
   return backward_impl(H, W, y, lse, grad_loss, grad_scale, N, V, 0, V, D, dtype, dH, dW,
-                       workspace, workspace_bytes, stream);
+                       workspace, workspace_bytes, stream, nullptr);
 }
 
 extern "C" flce_status flce_backward_shard(const void* H, const void* W_shard, const int64_t* y,
@@ -697,11 +701,12 @@ extern "C" flce_status flce_backward_shard(const void* H, const void* W_shard, c
                                            int64_t v_offset, int64_t V_total, int64_t D,
                                            flce_dtype dtype, float* dH_partial, float* dW_shard,
                                            void* workspace, size_t workspace_bytes,
-                                           void* stream) {
+                                           void* stream, void* dh_ready_event) {
   if (v_offset < 0 || V_shard < 1 || V_total < v_offset + V_shard || V_total >= (int64_t(1) << 31))
     return FLCE_ERR_INVALID_ARG;
   return backward_impl(H, W_shard, y, lse, grad_loss, grad_scale, N, V_shard, v_offset, V_total,
-                       D, dtype, dH_partial, dW_shard, workspace, workspace_bytes, stream);
+                       D, dtype, dH_partial, dW_shard, workspace, workspace_bytes, stream,
+                       static_cast<cudaEvent_t>(dh_ready_event));
 }
 
 // ---------------------------------------------------------------- no-allocation entry point

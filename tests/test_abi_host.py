@@ -305,7 +305,7 @@ def test_quantized_backward_workspace_and_checks_need_no_gpu(lib):
 def test_backward_shard_checks_need_no_gpu(lib):
     def call(V_shard=100, v_offset=0, V_total=1000, N=16):
         return lib.flce_backward_shard(FAKE, FAKE, FAKE, FAKE, None, 1.0, N, V_shard, v_offset, V_total,
-                                       64, 0, FAKE, FAKE, FAKE, 1 << 30, None)
+                                       64, 0, FAKE, FAKE, FAKE, 1 << 30, None, None)
     assert call(v_offset=-1) == flce.ERR_INVALID_ARG
     assert call(v_offset=950) == flce.ERR_INVALID_ARG        # shard runs past V_total
     assert call(V_shard=0) == flce.ERR_INVALID_ARG

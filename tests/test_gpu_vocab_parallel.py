@@ -115,3 +115,52 @@ def test_sharded_backward_flags_targets_outside_the_vocabulary():
     with pytest.raises(flce.FlceError) as e:
         flce.backward_shard(Hd, Wd[600:].contiguous(), yb, lse, 600, V, check=True)
     assert e.value.status == flce.ERR_TARGET_OUT_OF_RANGE
+
+
+def _vp_backward_rank(rank, world, port, q):
+    """One rank of backward_vocab_parallel on CUDA tensors (gloo carries the all-reduce,
+    so both ranks can share the one GPU; no kernel of one rank waits on the other)."""
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import linear_cross_entropy_bf16_b200 as flce
+        from linear_cross_entropy_bf16_b200 import synth as sy
+        from tests.flce_testing import to_device as td
+        N, V, D = 256, 20000, 128
+        H, W, y = sy.random_inputs(N, V, D, seed=60)
+        Hd, Wd, yd = td(H, W, y)
+        _, lse, _, _ = flce.forward(Hd, Wd, yd, check=True)
+        cut = [0, 12000, V]
+        a, b = cut[rank], cut[rank + 1]
+        dH, dW = flce.backward_vocab_parallel(Hd, Wd[a:b].contiguous(), yd, lse, a, V,
+                                              grad_scale=1.0 / N, check=True)
+        torch.cuda.synchronize()
+        dH_full, dW_full = flce.backward(Hd, Wd, yd, lse, None, 1.0 / N, check=True)
+        rel = float((dH - dH_full).norm() / dH_full.norm())
+        q.put((rank, rel, bool(torch.equal(dW, dW_full[a:b]))))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_backward_vocab_parallel_overlapped_allreduce_two_ranks_one_gpu():
+    import socket
+    import torch.multiprocessing as mp
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_vp_backward_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=300) for _ in procs]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    for rank, rel, same_dw in out:
+        assert rel < 1e-5, (rank, rel)        # the shares' sum vs the unsharded dH (fp32 sums)
+        assert same_dw
