@@ -37,7 +37,13 @@ class OracleError(RuntimeError):
 
 
 def build(force: bool = False) -> str:
-    """Compile ``oracle.c`` into ``liboracle.so`` (no fast-math: fp64 sums stay in order)."""
+    """Compile ``oracle.c`` into ``liboracle.so`` (no fast-math: fp64 sums stay in order).
+
+    With ORACLE_LIB_PATH set (only the mutation tests do this: they build a
+    copy of oracle.c with one planted mistake), that shared object is used
+    instead and nothing is compiled here."""
+    if os.environ.get("ORACLE_LIB_PATH"):
+        return os.environ["ORACLE_LIB_PATH"]
     stale = (not os.path.exists(_LIB_PATH)) or (
         os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
     if force or stale:
@@ -52,8 +58,7 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            build()
-            lib = ctypes.CDLL(_LIB_PATH)
+            lib = ctypes.CDLL(build())
             vp, i64, dp = ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p
             lib.oracle_forward_rows.argtypes = [vp, vp, ctypes.c_int, vp, i64, i64, i64,
                                                 vp, i64, dp, dp, dp, dp, ctypes.c_int]

@@ -1,0 +1,87 @@
+"""The oracle's pins catch planted mistakes (CPU only).
+
+Each mutant is a copy of oracle/oracle.c with one plausible mistake planted
+(a dropped term, a wrong sign, a wrong index, a swapped operand order, a
+wrong base or shift), compiled with gcc into a temporary shared object.  The
+CPU pin suites then run against it in a subprocess (ORACLE_LIB_PATH points
+the oracle module at the mutant) and must fail.  The unmutated source,
+compiled the same way, must pass: the harness itself is sound.
+"""
+import os
+import subprocess
+import sys
+from concurrent.futures import ThreadPoolExecutor
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "oracle.c")
+
+FWD = ["tests/test_oracle_pins.py", "tests/test_golden_pages.py"]
+BWD = ["tests/test_oracle_backward_pins.py"]
+QNT = ["tests/test_oracle_quant_pins.py"]
+
+# (name, text in oracle.c, replacement, which occurrence of the text, pin files
+# that cover the mutated function)
+MUTANTS = [
+    ("lse drops the max shift", "double lse = M + log(S);", "double lse = log(S);", 0, FWD),
+    ("loss sign flipped", "out_loss[t] = lse - tgt;", "out_loss[t] = tgt - lse;", 0, FWD),
+    ("target logit off by one column", "double tgt = z[y[i]];",
+     "double tgt = z[y[i] > 0 ? y[i] - 1 : 0];", 0, FWD),
+    ("logit pairs H_ik with W_j,D-1-k", "load_elem(W, dtype, j * D + k)",
+     "load_elem(W, dtype, j * D + (D - 1 - k))", 0, FWD),
+    ("sum of exponentials drops column 0", "for (int64_t j = 0; j < V; ++j) S += exp(z[j] - M);",
+     "for (int64_t j = 1; j < V; ++j) S += exp(z[j] - M);", 0, FWD),
+    ("exp taken base 2", "S += exp(z[j] - M);", "S += exp2(z[j] - M);", 0, FWD),
+    ("bf16 widened by 15 bits", "((const uint16_t *)base)[idx]) << 16;",
+     "((const uint16_t *)base)[idx]) << 15;", 0, FWD),
+    ("mean divides by n - 1", "return acc / (double)n;", "return acc / (double)(n - 1);", 0, FWD),
+    ("backward one-hot sign flipped", "(exp(z[j] - lse[i]) - (j == y[i] ? 1.0 : 0.0))",
+     "(exp(z[j] - lse[i]) + (j == y[i] ? 1.0 : 0.0))", 0, BWD),
+    ("backward dH drops the W factor", "acc += z[j] * w;", "acc += z[j];", 0, BWD),
+    ("backward dW drops the H factor", "acc += dz[i] * h;", "acc += dz[i];", 0, BWD),
+    ("quantised codes read highest first", "(word >> (bits * (int)(k % per_word)))",
+     "(word >> (bits * (int)(per_word - 1 - k % per_word)))", 0, QNT),
+    ("quantised groups in reverse order", "const int64_t g = j * (D / G) + k / G;",
+     "const int64_t g = j * (D / G) + (D / G - 1 - k / G);", 0, QNT),
+    ("quantised bias dropped", "bf16_bits_value(biases[g]);", "0.0 * bf16_bits_value(biases[g]);",
+     0, QNT),
+]
+
+
+def build_variant(tmp_path, name, text):
+    src = tmp_path / f"{name}.c"
+    src.write_text(text)
+    lib = tmp_path / f"{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", str(lib),
+                           str(src), "-lm"])
+    return str(lib)
+
+
+def run_pins(lib, pins, stop_first=True):
+    env = dict(os.environ, ORACLE_LIB_PATH=lib, OMP_NUM_THREADS="2")
+    cmd = [sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider", "-m", "not gpu"] + pins
+    if stop_first:
+        cmd.insert(3, "-x")
+    return subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+
+
+def test_unmutated_oracle_passes_the_pins(tmp_path):
+    r = run_pins(build_variant(tmp_path, "original", open(SRC).read()), FWD + BWD + QNT,
+                 stop_first=False)
+    assert r.returncode == 0, r.stdout[-2000:]
+
+
+def test_pins_catch_every_planted_mistake(tmp_path):
+    text = open(SRC).read()
+    jobs = []
+    for n, (name, old, new, occurrence, pins) in enumerate(MUTANTS):
+        parts = text.split(old)
+        assert len(parts) > occurrence + 1, f"mutation target not found: {old!r}"
+        mutated = old.join(parts[:occurrence + 1]) + new + old.join(parts[occurrence + 1:])
+        assert mutated != text
+        jobs.append((name, build_variant(tmp_path, f"mutant{n}", mutated), pins))
+    workers = max(1, min(8, (os.cpu_count() or 2) // 2))
+    with ThreadPoolExecutor(workers) as ex:
+        results = list(ex.map(lambda j: (j[0], run_pins(j[1], j[2])), jobs))
+    survivors = [name for name, r in results
+                 if r.returncode == 0 or not ("failed" in r.stdout or "error" in r.stdout.lower())]
+    assert not survivors, f"no pin caught: {survivors}"
