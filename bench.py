@@ -78,6 +78,30 @@ def profiled_traffic(workload: str, kernel: str):
     return float(m_tr.group(1))
 
 
+def run_environment(dev) -> dict:
+    """What ran: source identity, GPU, driver and library versions."""
+    import torch
+    env = {"kernel_sources_sha256": kernel_sources_sha256(), "gpu": torch.cuda.get_device_name(dev),
+           "torch": torch.__version__, "cuda_runtime": torch.version.cuda}
+    try:
+        h = hashlib.sha256()
+        with open(os.path.abspath(__file__), "rb") as f:
+            h.update(f.read())
+        env["bench_sha256"] = h.hexdigest()
+        out = subprocess.run(["nvidia-smi", "--query-gpu=driver_version", "--format=csv,noheader",
+                              f"--id={torch.cuda.current_device()}"],
+                             capture_output=True, text=True, timeout=20)
+        if out.returncode == 0:
+            env["driver"] = out.stdout.strip()
+        g = subprocess.run(["git", "rev-parse", "HEAD"], cwd=ROOT, capture_output=True, text=True,
+                           timeout=20)
+        if g.returncode == 0:
+            env["git"] = g.stdout.strip()
+    except (OSError, subprocess.SubprocessError):
+        pass
+    return env
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -405,6 +429,9 @@ def run_ours(args, w, rank, world, local_rank):
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms,
                 "api": "flce_forward_host" if host_ws is not None else "torch copies + flce_forward"},
         "gpu_launches": 2 * K,
+        "kernel_ms_stats": {"median": float(np.median(part_ms)), "min": float(np.min(part_ms)),
+                            "max": float(np.max(part_ms))},
+        "env": run_environment(dev),
         "clocks": clocks,
     }
     if args.backward and w.dtype == "bf16":
