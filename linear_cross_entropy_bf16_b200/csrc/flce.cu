@@ -8,6 +8,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -23,6 +24,17 @@
 namespace {
 
 using namespace flce;
+
+// A named NVTX range around each public entry point that enqueues GPU work,
+// so profiler timelines show which library call issued which kernels.  NVTX
+// is header-only and does nothing unless a profiling tool is attached.
+struct TraceRange {
+  explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+  ~TraceRange() { nvtxRangePop(); }
+  TraceRange(const TraceRange&) = delete;
+  TraceRange& operator=(const TraceRange&) = delete;
+};
+#define FLCE_TRACE() TraceRange flce_trace_range_(__func__)
 
 constexpr uint64_t kDefaultWaitLimitNs = 4000000000ull;  // 4 s in one wait: far beyond any real stage
 
@@ -303,6 +315,7 @@ flce_status flce_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int32_t
 flce_status flce_partials(const void* H, const void* W, const int64_t* y, int64_t N, int64_t V,
                           int64_t D, flce_dtype dtype, float* out_target_logit, void* workspace,
                           size_t workspace_bytes, void* stream) {
+  FLCE_TRACE();
   flce_status s = check_forward_args(H, W, y, N, V, D, dtype, workspace, workspace_bytes);
   if (s != FLCE_OK || N == 0) return s;
   if (!out_target_logit) return FLCE_ERR_INVALID_ARG;
@@ -313,6 +326,7 @@ flce_status flce_partials(const void* H, const void* W, const int64_t* y, int64_
 flce_status flce_merge(const int64_t* y, int64_t N, int64_t V, float* out_loss, float* out_lse,
                        float* out_target_logit, float* out_mean, const void* workspace,
                        size_t workspace_bytes, void* stream) {
+  FLCE_TRACE();
   if (N < 0 || V < 1) return FLCE_ERR_INVALID_ARG;
   if (N == 0) return FLCE_OK;
   if (!y || !out_loss || !out_lse || !out_target_logit || !workspace) return FLCE_ERR_INVALID_ARG;
@@ -327,6 +341,7 @@ flce_status flce_forward(const void* H, const void* W, const int64_t* y, int64_t
                          int64_t D, flce_dtype dtype, float* out_loss, float* out_lse,
                          float* out_target_logit, float* out_mean, void* workspace,
                          size_t workspace_bytes, void* stream) {
+  FLCE_TRACE();
   flce_status s = check_forward_args(H, W, y, N, V, D, dtype, workspace, workspace_bytes);
   if (s != FLCE_OK || N == 0) return s;
   if (!out_loss || !out_lse || !out_target_logit) return FLCE_ERR_INVALID_ARG;
@@ -340,6 +355,7 @@ flce_status flce_forward(const void* H, const void* W, const int64_t* y, int64_t
 
 flce_status flce_forward_ex(const flce_forward_args* a, void* workspace, size_t workspace_bytes,
                             void* stream) {
+  FLCE_TRACE();
   if (!a) return FLCE_ERR_INVALID_ARG;
   const flce_dtype dtype = flce_dtype(a->dtype);
   if (!sizes_ok(a->N, a->V, a->D, dtype)) return FLCE_ERR_INVALID_ARG;
@@ -366,6 +382,7 @@ flce_status flce_partials_shard(const void* H, const void* W_shard, const int64_
                                 int64_t V_shard, int64_t v_offset, int64_t D, flce_dtype dtype,
                                 float* out_target_logit, void* workspace, size_t workspace_bytes,
                                 void* stream) {
+  FLCE_TRACE();
   if (v_offset < 0) return FLCE_ERR_INVALID_ARG;
   flce_status s =
       check_forward_args(H, W_shard, y, N, V_shard, D, dtype, workspace, workspace_bytes);
@@ -379,6 +396,7 @@ flce_status flce_partials_shard(const void* H, const void* W_shard, const int64_
 flce_status flce_shard_state(const int64_t* y, int64_t N, int64_t V_shard, int64_t v_offset,
                              const float* target_logit, const void* workspace,
                              size_t workspace_bytes, float* out_state, void* stream) {
+  FLCE_TRACE();
   if (N < 0 || V_shard < 1 || v_offset < 0) return FLCE_ERR_INVALID_ARG;
   if (N == 0) return FLCE_OK;
   if (!y || !target_logit || !workspace || !out_state) return FLCE_ERR_INVALID_ARG;
@@ -406,6 +424,7 @@ flce_status flce_merge_shards(const float* states, int32_t G, const int64_t* y, 
                               int64_t V_total, float* out_loss, float* out_lse,
                               float* out_target_logit, float* out_mean, void* scratch,
                               size_t scratch_bytes, void* stream) {
+  FLCE_TRACE();
   if (G < 1 || N < 0 || V_total < 1) return FLCE_ERR_INVALID_ARG;
   if (N == 0) return FLCE_OK;
   if (!states || !y || !out_loss || !out_lse || !out_target_logit || !scratch)
@@ -691,6 +710,7 @@ extern "C" flce_status flce_backward(const void* H, const void* W, const int64_t
                                      int64_t N, int64_t V, int64_t D, flce_dtype dtype, float* dH,
                                      float* dW, void* workspace, size_t workspace_bytes,
                                      void* stream) {
+  FLCE_TRACE();
   return backward_impl(H, W, y, lse, grad_loss, grad_scale, N, V, 0, V, D, dtype, dH, dW,
                        workspace, workspace_bytes, stream, nullptr);
 }
@@ -702,6 +722,7 @@ extern "C" flce_status flce_backward_shard(const void* H, const void* W_shard, c
                                            flce_dtype dtype, float* dH_partial, float* dW_shard,
                                            void* workspace, size_t workspace_bytes,
                                            void* stream, void* dh_ready_event) {
+  FLCE_TRACE();
   if (v_offset < 0 || V_shard < 1 || V_total < v_offset + V_shard || V_total >= (int64_t(1) << 31))
     return FLCE_ERR_INVALID_ARG;
   return backward_impl(H, W_shard, y, lse, grad_loss, grad_scale, N, V_shard, v_offset, V_total,
@@ -843,6 +864,7 @@ extern "C" flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
                                               float* out_lse, float* out_target_logit,
                                               float* out_mean, void* workspace,
                                               size_t workspace_bytes, void* stream) {
+  FLCE_TRACE();
   if (N < 0 || V < 1 || D < 1 || !quant_format_ok(bits, group_size, D))
     return FLCE_ERR_INVALID_ARG;
   if (N == 0) return FLCE_OK;
@@ -955,6 +977,7 @@ extern "C" flce_status flce_forward_host(const void* H_host, const void* W_host,
                                          float* target_logit_host, float* mean_host,
                                          void* workspace, size_t workspace_bytes, void* stream,
                                          void* copy_stream) {
+  FLCE_TRACE();
   if (!sizes_ok(N, V, D, dtype)) return FLCE_ERR_INVALID_ARG;
   if (N == 0) return FLCE_OK;
   if (!H_host || !W_host || !y_host || !loss_host || !workspace) return FLCE_ERR_INVALID_ARG;
@@ -1076,6 +1099,7 @@ extern "C" flce_status flce_backward_quantized(const void* H, const uint32_t* wq
                                                float grad_scale, int64_t N, int64_t V, int64_t D,
                                                float* dH, void* workspace, size_t workspace_bytes,
                                                void* stream) {
+  FLCE_TRACE();
   if (N < 0 || V < 1 || D < 1 || !quant_format_ok(bits, group_size, D))
     return FLCE_ERR_INVALID_ARG;
   if (N == 0) return FLCE_OK;
