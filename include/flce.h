@@ -90,7 +90,7 @@ typedef struct {
 /* Bytes of device workspace that flce_forward / flce_partials need for this
  * problem: a 256-byte header, the per-(slab, token) partial states (8 bytes
  * each, at most 512 slabs per token, so O(N), never O(N*V)), and one fp64
- * per 256 tokens for the mean.  fp32 inputs add the bf16 split copies of H
+ * per 32 tokens for the mean.  fp32 inputs add the bf16 split copies of H
  * and W, 6 * Dp bytes per row of each (Dp = D rounded up to 8): O((N + V) D),
  * still never O(N*V).  Depends only on its arguments (not on the device).
  * Returns 0 for invalid arguments (N < 0, V < 1, D < 1, unknown dtype).  Host
@@ -310,7 +310,7 @@ FLCE_API flce_status flce_selftest_wait_timeout(void* workspace, size_t workspac
  *   - A problem whose flce_workspace_size(N, V, D, dtype) exceeds
  *     FLCE_NOALLOC_SCRATCH_BYTES is rejected with FLCE_ERR_WORKSPACE_TOO_SMALL
  *     and nothing is enqueued.  With V >= 131072 (512 slab states per token)
- *     that means N <= 16383.
+ *     that means N <= 16382.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current.  Make that first call
  *     before any stream capture on that device.

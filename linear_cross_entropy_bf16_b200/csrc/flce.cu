@@ -292,8 +292,8 @@ flce_status launch_merge(Targets y, int64_t N, int64_t V, float* out_loss, float
   m.V = int32_t(V);
   m.max_slabs = int32_t(slab_capacity(V));
   (void)ws_bytes;
-  const int blocks = int(cdiv(N, kMergeThreads));
-  flce_merge_kernel<<<blocks, kMergeThreads, 0, st>>>(m);
+  const int blocks = int(cdiv(N, kMergeTokensPerBlock));
+  flce_merge_kernel<<<blocks, kMergeBlockThreads, 0, st>>>(m);
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 

@@ -858,38 +858,60 @@ struct MergeArgs {
   float* loss;
   float* lse;
   float* mean;          // may be null
-  double* block_sums;   // [gridDim.x]
+  double* block_sums;   // [gridDim.x]: one per kMergeTokensPerBlock tokens
   WsHeader* hdr;
   int32_t N, V;
   int32_t max_slabs;    // capacity of the partial array in this workspace
 };
 
-// One thread per token: m = max_p m_p, s = sum_p s_p exp(m_p - m) over the P
-// slab states in slab order (fp64), lse = m + log s, loss = lse - z_target.
-// The mean is a fixed-order fp64 reduction: a shuffle tree per block, then the
-// last block to finish sums the block results in block order.
-__global__ void __launch_bounds__(kMergeThreads) flce_merge_kernel(const MergeArgs a) {
-  __shared__ double warp_sums[kMergeThreads / 32];
+// The merge spreads each token's P slab states over kMergeLanes lanes of one
+// warp (lane l takes slabs l, l + 16, ...), so no thread walks a long chain of
+// dependent loads: m = max_p m_p (a shuffle max), s = sum_p s_p exp(m_p - m)
+// in fp64 (each lane sums its slabs in slab order, then a fixed xor-shuffle
+// tree adds the lanes), lse = m + log s, loss = lse - z_target.  The mean is
+// a fixed-order fp64 reduction: per block, then the last block to finish
+// reduces the block results with a fixed strided-then-tree order.  Results are
+// bitwise identical run to run.
+constexpr int kMergeLanes = 16;                 // lanes per token
+constexpr int kMergeTokensPerBlock = 32;
+constexpr int kMergeBlockThreads = kMergeLanes * kMergeTokensPerBlock;   // 512
+
+__global__ void __launch_bounds__(kMergeBlockThreads) flce_merge_kernel(const MergeArgs a) {
+  __shared__ double tok_loss[kMergeTokensPerBlock];
+  __shared__ double red[kMergeBlockThreads / 32];
   __shared__ bool is_last;
-  const int i = blockIdx.x * kMergeThreads + threadIdx.x;
+  const int lane = threadIdx.x % kMergeLanes;
+  const int tok = threadIdx.x / kMergeLanes;
+  const int i = blockIdx.x * kMergeTokensPerBlock + tok;
   const WsHeader h = *a.hdr;
   const bool ws_ok = h.magic == kWsMagic && h.N == a.N && h.V == a.V && h.slabs >= 1 &&
                      h.slabs <= a.max_slabs;
+  const bool live = i < a.N;
+  const int P = ws_ok ? h.slabs : 0;
+  // every lane of a 16-lane group takes part in the shuffles (same token,
+  // same trip counts), so the masks are full
+  float M = -INFINITY;
+  if (live)
+    for (int p = lane; p < P; p += kMergeLanes) M = fmaxf(M, a.part[size_t(p) * a.N + i].x);
+#pragma unroll
+  for (int off = kMergeLanes / 2; off >= 1; off >>= 1)
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off, kMergeLanes));
+  double S = 0.0;
+  if (live)
+    for (int p = lane; p < P; p += kMergeLanes) {
+      const float2 st = a.part[size_t(p) * a.N + i];
+      S += double(st.y) * exp(double(st.x) - double(M));
+    }
+#pragma unroll
+  for (int off = kMergeLanes / 2; off >= 1; off >>= 1)
+    S += __shfl_xor_sync(0xffffffffu, S, off, kMergeLanes);
   double l = 0.0;
-  if (i < a.N) {
+  if (live && lane == 0) {
     float loss_f, lse_f;
     if (!ws_ok) {
       loss_f = lse_f = __int_as_float(0x7fc00000);
       if (i == 0) atomicOr(&a.hdr->status, kStatBadWs);
     } else {
-      const int P = h.slabs;
-      float M = -INFINITY;
-      for (int p = 0; p < P; ++p) M = fmaxf(M, a.part[size_t(p) * a.N + i].x);
-      double S = 0.0;
-      for (int p = 0; p < P; ++p) {
-        const float2 st = a.part[size_t(p) * a.N + i];
-        S += double(st.y) * exp(double(st.x) - double(M));
-      }
       const double lse = double(M) + log(S);
       const int64_t yi = a.y[i];
       lse_f = float(lse);
@@ -906,25 +928,32 @@ __global__ void __launch_bounds__(kMergeThreads) flce_merge_kernel(const MergeAr
     l = double(loss_f);
   }
   if (a.mean == nullptr) return;
-  // fixed-order block reduction
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) l += __shfl_down_sync(0xffffffffu, l, off);
-  if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = l;
+  // fixed-order block sum over the block's tokens
+  if (lane == 0) tok_loss[tok] = l;
   __syncthreads();
   if (threadIdx.x == 0) {
     double b = 0.0;
-    for (int w = 0; w < kMergeThreads / 32; ++w) b += warp_sums[w];
+    for (int t = 0; t < kMergeTokensPerBlock; ++t) b += tok_loss[t];
     a.block_sums[blockIdx.x] = b;
     __threadfence();
     const uint32_t ticket = atomicAdd(&a.hdr->counter, 1u);
     is_last = ticket == gridDim.x - 1;
   }
   __syncthreads();
-  if (is_last && threadIdx.x == 0) {
-    __threadfence();
-    const volatile double* bs = a.block_sums;
+  if (!is_last) return;
+  // the last block: thread t sums block results t, t + 512, ... in order,
+  // then warps and the block reduce in a fixed tree
+  __threadfence();
+  const volatile double* bs = a.block_sums;
+  double v = 0.0;
+  for (int b = threadIdx.x; b < int(gridDim.x); b += kMergeBlockThreads) v += bs[b];
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
     double total = 0.0;
-    for (int b = 0; b < int(gridDim.x); ++b) total += bs[b];
+    for (int w = 0; w < kMergeBlockThreads / 32; ++w) total += red[w];
     *a.mean = float(total / double(a.N));
     a.hdr->counter = 0;
   }

@@ -22,7 +22,10 @@ int64_t slab_capacity(int64_t V) { return std::min<int64_t>(cdiv(V, kTileCols), 
 // Header, (m, s) partial states and the mean's block sums: what the merge reads.
 size_t state_bytes_for(int64_t N, int64_t V) {
   const size_t part = align256(size_t(8) * size_t(N) * size_t(slab_capacity(V)));
-  const size_t sums = align256(size_t(8) * size_t(std::max<int64_t>(1, cdiv(N, kMergeThreads))));
+  // block results of the mean: one per kMergeTokensPerBlock tokens (the merge
+  // kernel), which also covers one per kMergeThreads tokens (the shard merge)
+  const size_t sums =
+      align256(size_t(8) * size_t(std::max<int64_t>(1, cdiv(N, kMergeTokensPerBlock))));
   return kHeaderBytes + part + sums;
 }
 

@@ -52,7 +52,7 @@ def test_workspace_is_O_N_not_O_NV(lib):
         ws = flce.workspace_size(N, V, D)
         slabs = min(math.ceil(V / 256), 512)
         assert ws >= 256 + 8 * N * slabs
-        assert ws <= 256 + 8 * N * 512 + 256 + 8 * (N // 256 + 1) + 512
+        assert ws <= 256 + 8 * N * 512 + 256 + 8 * (N // 32 + 1) + 512
         if V >= 100000:
             assert ws < 4 * N * V / 50        # the logits it replaces are 4 N V bytes
     assert lib.flce_workspace_size(-1, 10, 8, 0) == 0

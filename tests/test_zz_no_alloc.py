@@ -76,7 +76,10 @@ def test_noalloc_rejects_problems_beyond_its_scratch(lib):
         flce.forward_noalloc(H, W, y, out)
     assert e.value.status == flce.ERR_WORKSPACE_TOO_SMALL
     # the largest problem that fits runs, through the Python binding too
-    n_max = 16383
+    n_max = 16300
+    while flce.workspace_size(n_max + 1, 131072, 64) <= flce.NOALLOC_SCRATCH_BYTES:
+        n_max += 1
+    assert 16000 < n_max < 16384
     H2, W2, y2 = synth.random_inputs(n_max, 131072, 64, seed=23)
     Hd, Wd, yd = to_device(H2, W2, y2)
     out = {k: torch.empty(n_max, device="cuda") for k in ("loss", "lse", "target_logit")}
