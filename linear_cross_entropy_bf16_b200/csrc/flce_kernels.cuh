@@ -186,11 +186,14 @@ __device__ __forceinline__ void fold_tile(uint32_t taddr, int ncols, int64_t rel
 #pragma unroll
       for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
     const float m_new = fmaxf(m, mx[0]);
-    const float ms = m_new * kLog2e;
-    // sum_j exp(z_j - m') as 2^(z_j log2 e - m' log2 e)
+    const float ms = __fmul_rn(m_new, kLog2e);
+    // sum_j exp(z_j - m') as 2^(z_j log2 e - m' log2 e).  The product and the
+    // difference are rounded separately (no fused multiply-add), so the
+    // column holding the maximum contributes exactly 2^0 = 1: s >= 1, hence
+    // lse >= max_j z_j >= z_target and every loss is >= 0 (exactly 0 for V = 1).
     float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int j = 0; j < 32; ++j) e[j & 3] += ptx::ex2(fmaf(z[j], kLog2e, -ms));
+    for (int j = 0; j < 32; ++j) e[j & 3] += ptx::ex2(__fsub_rn(__fmul_rn(z[j], kLog2e), ms));
     // s' = s exp(m - m') + sum; m = -inf on the first chunk gives exp(-inf) = 0
     s = fmaf(s, ptx::ex2((m - m_new) * kLog2e), (e[0] + e[1]) + (e[2] + e[3]));
     m = m_new;

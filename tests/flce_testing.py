@@ -51,7 +51,8 @@ def check_properties(gpu, V):
     """Properties that hold at any size: finite, loss >= 0, lse >= target, mean = average."""
     import math
     assert np.all(np.isfinite(gpu["loss"])) and np.all(np.isfinite(gpu["lse"]))
-    assert np.all(gpu["loss"] >= -LOSS_TOL)
+    # the maximum's own term is exactly 1, so lse >= max z >= target logit: never negative
+    assert np.all(gpu["loss"] >= 0.0)
     assert np.all(gpu["lse"] + LSE_TOL >= gpu["target"])
     # loss = lse - target logit, up to fp32 rounding of the stored lse
     assert np.all(np.abs(gpu["loss"] - (gpu["lse"] - gpu["target"])) <= 4e-7 * (1 + np.abs(gpu["lse"])) + 1e-6)

@@ -1,0 +1,78 @@
+"""Edge cases through every Python entry point on the GPU: empty batches, a
+one-word vocabulary, and logits in the thousands (the online max must keep
+every exponent finite)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_cross_entropy_bf16_b200 import synth
+from tests.flce_testing import compare, run, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from linear_cross_entropy_bf16_b200 import build
+    build.build()
+    oracle.build()
+
+
+def test_empty_batch_everywhere():
+    """N = 0: every entry point returns empty results and launches nothing."""
+    import linear_cross_entropy_bf16_b200 as flce
+    V, D = 1000, 64
+    H = torch.empty(0, D, dtype=torch.bfloat16, device="cuda")
+    W = torch.randn(V, D, device="cuda").bfloat16()
+    y = torch.empty(0, dtype=torch.int64, device="cuda")
+    lse0 = torch.empty(0, device="cuda")
+    loss, lse, tgt, mean = flce.forward(H, W, y, check=False)
+    assert loss.numel() == lse.numel() == tgt.numel() == 0 and math.isnan(mean.item())
+    assert flce.forward_strided(H, W, y.to(torch.int32))[0].numel() == 0
+    assert flce.forward(H.float(), W.float(), y)[0].numel() == 0
+    dH, dW = flce.backward(H, W, y, lse0)
+    assert dH.shape == (0, D) and dW.shape == (V, D) and not dW.abs().any()
+    dHs, dWs = flce.backward_shard(H, W[:300].contiguous(), y, lse0, 0, V)
+    assert dHs.shape == (0, D) and not dWs.abs().any()
+    Wq = torch.zeros(V, D * 4 // 32, dtype=torch.int32, device="cuda")
+    sc = torch.ones(V, D // 64, dtype=torch.bfloat16, device="cuda")
+    assert flce.forward_quantized(H, Wq, sc, sc, y, 4, 64)[0].numel() == 0
+    assert flce.backward_quantized(H, Wq, sc, sc, y, lse0, None, 1.0, 4, 64).shape == (0, D)
+    res = flce.forward_host(H.cpu(), W.cpu(), y.cpu())
+    assert res[0].numel() == 0
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_one_word_vocabulary_gives_zero_loss(dtype):
+    """V = 1: lse equals the only logit, so every loss is exactly 0."""
+    H, W, _ = synth.random_inputs(300, 1, 128, seed=81, dtype=dtype)
+    y = np.zeros(300, dtype=np.int64)
+    gpu = run(H, W, y)
+    assert np.all(gpu["loss"] == 0.0)
+    np.testing.assert_array_equal(gpu["lse"], gpu["target"])
+    ref = oracle.forward(H, W, y)
+    compare(gpu, ref, mean_ref=None)
+
+
+@pytest.mark.parametrize("scale", [30.0, 300.0])
+def test_logits_in_the_thousands(scale):
+    """Rows scaled so logits reach about +-scale * 10 (several thousand at the top
+    scale): exp(z - m) stays in range only through the running max."""
+    N, V, D = 260, 3000, 128
+    H, W, y = synth.random_inputs(N, V, D, seed=82)
+    Hs = synth.round_to_bf16_bits(synth.bf16_bits_to_f32(H) * np.float32(scale))
+    gpu = run(Hs, W, y)
+    ref = oracle.forward(Hs, W, y)
+    assert np.abs(ref["max"]).max() > 3 * scale
+    assert np.all(np.isfinite(gpu["loss"]))
+    # lse and the target logit carry fp32 rounding of values of this size: the
+    # 1e-3 bar scales with the logit magnitude here (relative 2^-20 of |max z|)
+    tol = np.maximum(1e-3, 2.0 ** -20 * np.abs(ref["max"]))
+    for key in ("loss", "lse", "target"):
+        assert np.all(np.abs(gpu[key] - ref[key]) <= 2 * tol), key
