@@ -25,6 +25,7 @@ __all__ = [
     "FlceError", "forward", "backward", "partials", "merge", "workspace_size",
     "shard_state", "merge_shards", "forward_vocab_parallel", "forward_strided",
     "backward_shard", "backward_vocab_parallel",
+    "linear_cross_entropy", "linear_cross_entropy_quantized",
     "forward_quantized", "quantized_workspace_size", "backward_quantized",
     "backward_quantized_workspace_size", "forward_host", "host_workspace_size",
     "backward_workspace_size", "plan", "check",
@@ -735,3 +736,93 @@ def forward_host(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, *, device=No
     if check:
         _raise_on(lib.flce_check(workspace.data_ptr(), sp), "flce_forward_host (device)")
     return loss, lse, tgt, mean
+
+
+# ---------------------------------------------------------------- autograd
+
+
+class _LinearCrossEntropy(torch.autograd.Function):
+    """loss = cross_entropy(H W^T, y) with the fused kernels in both directions."""
+
+    @staticmethod
+    def forward(ctx, H, W, y, reduction):
+        loss, lse, _, mean = forward(H, W, y)
+        ctx.save_for_backward(H, W, y, lse)
+        ctx.reduction = reduction
+        if reduction == "mean":
+            return mean
+        if reduction == "sum":
+            return mean * H.shape[0] if H.shape[0] else mean.new_zeros(())
+        return loss
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        H, W, y, lse = ctx.saved_tensors
+        N = H.shape[0]
+        need_h, need_w = ctx.needs_input_grad[0], ctx.needs_input_grad[1]
+        if not (need_h or need_w):
+            return None, None, None, None
+        grad_out = grad_out.float()
+        if ctx.reduction == "none":
+            g, scale = grad_out.contiguous(), 1.0
+        else:
+            # the upstream scalar times 1/N (mean) or 1 (sum), applied on the device
+            g = grad_out.reshape(1).expand(N).contiguous()
+            scale = 1.0 / N if (ctx.reduction == "mean" and N) else 1.0
+        dH, dW = backward(H, W, y, lse, g, scale)
+        return (dH.to(H.dtype) if need_h else None, dW.to(W.dtype) if need_w else None, None, None)
+
+
+def linear_cross_entropy(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor,
+                         reduction: str = "mean") -> torch.Tensor:
+    """Differentiable fused linear cross-entropy: cross_entropy(H @ W.T, y) without the
+    (N, V) logits, in the forward (flce_forward) and the backward (flce_backward).
+
+    H (N, D) and W (V, D) bf16 or fp32 on one CUDA device, y (N) int64.  reduction:
+    "mean" (default), "sum" or "none" (per-token losses).  Gradients come back in the
+    inputs' dtypes (computed in fp32)."""
+    if reduction not in ("mean", "sum", "none"):
+        raise ValueError("reduction must be 'mean', 'sum' or 'none'")
+    return _LinearCrossEntropy.apply(H, W, y, reduction)
+
+
+class _LinearCrossEntropyQuantized(torch.autograd.Function):
+    """The same with a frozen affine-quantised head: gradients for H only."""
+
+    @staticmethod
+    def forward(ctx, H, wq, scales, biases, y, bits, group_size, reduction):
+        loss, lse, _, mean = forward_quantized(H, wq, scales, biases, y, bits, group_size)
+        ctx.save_for_backward(H, wq, scales, biases, y, lse)
+        ctx.args = (bits, group_size, reduction)
+        if reduction == "mean":
+            return mean
+        if reduction == "sum":
+            return mean * H.shape[0] if H.shape[0] else mean.new_zeros(())
+        return loss
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        H, wq, scales, biases, y, lse = ctx.saved_tensors
+        bits, group_size, reduction = ctx.args
+        none = (None,) * 7
+        if not ctx.needs_input_grad[0]:
+            return (None,) + none
+        N = H.shape[0]
+        grad_out = grad_out.float()
+        if reduction == "none":
+            g, scale = grad_out.contiguous(), 1.0
+        else:
+            g = grad_out.reshape(1).expand(N).contiguous()
+            scale = 1.0 / N if (reduction == "mean" and N) else 1.0
+        dH = backward_quantized(H, wq, scales, biases, y, lse, g, scale, bits, group_size)
+        return (dH.to(H.dtype),) + none
+
+
+def linear_cross_entropy_quantized(H: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor,
+                                   biases: torch.Tensor, y: torch.Tensor, bits: int = 4,
+                                   group_size: int = 64, reduction: str = "mean") -> torch.Tensor:
+    """Differentiable loss with a frozen quantised head (MLX affine layout, as
+    forward_quantized); only H receives a gradient."""
+    if reduction not in ("mean", "sum", "none"):
+        raise ValueError("reduction must be 'mean', 'sum' or 'none'")
+    return _LinearCrossEntropyQuantized.apply(H, wq, scales, biases, y, bits, group_size, reduction)
