@@ -783,7 +783,11 @@ def linear_cross_entropy(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor,
     inputs' dtypes (computed in fp32)."""
     if reduction not in ("mean", "sum", "none"):
         raise ValueError("reduction must be 'mean', 'sum' or 'none'")
-    return _LinearCrossEntropy.apply(H, W, y, reduction)
+    if y.dtype == torch.int32:
+        y = y.long()
+    # the kernels take contiguous rows; a strided view is copied first (the copy
+    # is an ordinary differentiable op, so gradients still reach the original)
+    return _LinearCrossEntropy.apply(H.contiguous(), W.contiguous(), y.contiguous(), reduction)
 
 
 class _LinearCrossEntropyQuantized(torch.autograd.Function):
@@ -825,4 +829,7 @@ def linear_cross_entropy_quantized(H: torch.Tensor, wq: torch.Tensor, scales: to
     forward_quantized); only H receives a gradient."""
     if reduction not in ("mean", "sum", "none"):
         raise ValueError("reduction must be 'mean', 'sum' or 'none'")
-    return _LinearCrossEntropyQuantized.apply(H, wq, scales, biases, y, bits, group_size, reduction)
+    if y.dtype == torch.int32:
+        y = y.long()
+    return _LinearCrossEntropyQuantized.apply(H.contiguous(), wq, scales, biases, y.contiguous(), bits,
+                                              group_size, reduction)

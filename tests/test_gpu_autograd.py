@@ -99,3 +99,21 @@ def test_quantized_head_gradient_for_H():
     ref.backward()
     assert abs(loss.item() - ref.item()) <= 1e-5 * abs(ref.item())
     assert rel(Hd.grad, Hr.grad) < 1e-2
+
+
+def test_int32_targets_and_strided_inputs():
+    """int32 targets and a row-strided H (a slice of a wider activation) go through."""
+    import linear_cross_entropy_bf16_b200 as flce
+    N, V, D = 200, 3000, 64
+    H, W, y = synth.random_inputs(N, V, D + 32, seed=95)
+    Hwide = torch.from_numpy(H).view(torch.bfloat16).cuda().requires_grad_(True)
+    Wd = torch.from_numpy(W).view(torch.bfloat16).cuda()[:, :D].contiguous().requires_grad_(True)
+    y32 = torch.from_numpy(y).cuda().to(torch.int32)
+    Hs = Hwide[:, 16:16 + D]                      # strided rows
+    loss = flce.linear_cross_entropy(Hs, Wd, y32)
+    loss.backward()
+    ref_loss, ref_dH, ref_dW = reference(Hs, Wd, y32.long(), "mean", torch.tensor(1.0, device="cuda"),
+                                         torch.float32)
+    assert abs(loss.item() - ref_loss.item()) <= 1e-3
+    assert Hwide.grad is not None and not Hwide.grad[:, :16].float().abs().any()
+    assert rel(Hwide.grad[:, 16:16 + D], ref_dH) < 1e-2 and rel(Wd.grad, ref_dW) < 1e-2
