@@ -380,7 +380,39 @@ def run_ours(args, w, rank, world, local_rank):
     assert abs(float(mean_h.item()) - mean_loss) <= 1e-5 * abs(mean_loss)
     h2d = H_h.numel() * H_h.element_size() + W_h.numel() * W_h.element_size() + y_h.numel() * 8
 
+    # ---- the same with the head resident on the device (a training or
+    # inference step, where W is a parameter): H and y copied in from pinned
+    # host memory, the results copied out, every step
+    H_r = torch.empty_like(H)
+    y_r = torch.empty_like(y)
+    res_r = {k: torch.empty(N, pin_memory=True) for k in ("loss", "lse", "target_logit")}
+    res_r["mean"] = torch.empty((), pin_memory=True)
+    out_r = {"loss": torch.empty(N, device=dev), "lse": torch.empty(N, device=dev),
+             "target_logit": torch.empty(N, device=dev), "mean": torch.empty((), device=dev)}
+
+    def resident_step():
+        H_r.copy_(H_h, non_blocking=True)
+        y_r.copy_(y_h, non_blocking=True)
+        flce.forward(H_r, W, y_r, out=out_r, workspace=ws, stream=stream)
+        for k in res_r:
+            res_r[k].copy_(out_r[k], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            resident_step()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(Ke):
+            resident_step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    resident_ms = e0.elapsed_time(e1) / Ke
+    assert abs(float(res_r["mean"].item()) - mean_loss) <= 1e-6 * abs(mean_loss)
+
     # ---- max over ranks
+    resident_ms = max_over_ranks([resident_ms], world, device=dev)[0]
     total_ms, part_avg_ms, e2e_ms = max_over_ranks([total_ms, float(np.mean(part_ms)), e2e_ms],
                                                    world, device=dev)
 
@@ -428,6 +460,11 @@ def run_ours(args, w, rank, world, local_rank):
         "e2e": {"value": weak_scaling_tokens_per_s(world, N, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms,
                 "api": "flce_forward_host" if host_ws is not None else "torch copies + flce_forward"},
+        "e2e_resident_head": {"value": weak_scaling_tokens_per_s(world, N, resident_ms), "unit": "tokens/s",
+                              "h2d_bytes_per_step": int(H_h.numel() * H_h.element_size() + y_h.numel() * 8),
+                              "d2h_bytes_per_step": int(3 * N * 4 + 4), "ms_per_step": resident_ms,
+                              "what": "W resident on the device (a parameter); H and y copied in and the "
+                                      "results out every step, around flce_forward"},
         "gpu_launches": 2 * K,
         "kernel_ms_stats": {"median": float(np.median(part_ms)), "min": float(np.min(part_ms)),
                             "max": float(np.max(part_ms))},
