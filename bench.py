@@ -416,13 +416,23 @@ def run_ours(args, w, rank, world, local_rank):
     total_ms, part_avg_ms, e2e_ms = max_over_ranks([total_ms, float(np.mean(part_ms)), e2e_ms],
                                                    world, device=dev)
 
+    # the optional legs take their own max over ranks: every rank runs them
+    peaks, peak_kind = measured_peaks()
+    extra = {}
+    if args.backward and w.dtype == "bf16":
+        extra["backward"] = time_backward(flce, H, W, y, lse, N, V, D, tdt, dev, stream, args,
+                                          peaks["bf16_tflops"], world)
+    if args.quantized and w.dtype == "bf16":
+        bits, gs = (int(v) for v in args.quantized.split(","))
+        extra["quantized"] = time_quantized(flce, H, Wn, y, N, V, D, bits, gs, dev, stream, args,
+                                            peaks["bf16_tflops"], world)
+
     if rank != 0:
         return 0
 
     ms_step = total_ms / K
     tokens_per_s = weak_scaling_tokens_per_s(world, N, ms_step)
     flops = w.flops
-    peaks, peak_kind = measured_peaks()
     achieved = flops / (part_avg_ms * 1e-3) / 1e12
     p = flce.plan(N, V, D, tdt)
     # fp32 inputs run on the same kernels after the bf16 hi/lo split (three
@@ -471,13 +481,7 @@ def run_ours(args, w, rank, world, local_rank):
         "env": run_environment(dev),
         "clocks": clocks,
     }
-    if args.backward and w.dtype == "bf16":
-        line["backward"] = time_backward(flce, H, W, y, lse, N, V, D, tdt, dev, stream, args,
-                                         peaks["bf16_tflops"], world)
-    if args.quantized and w.dtype == "bf16":
-        bits, gs = (int(v) for v in args.quantized.split(","))
-        line["quantized"] = time_quantized(flce, H, Wn, y, N, V, D, bits, gs, dev, stream, args,
-                                           peaks["bf16_tflops"], world)
+    line.update(extra)
     if world == 1 and not args.no_cpu_baseline:
         rows, secs, cores = oracle_sample(Hn, Wn, yn, args.cpu_seconds, w.seed)
         line["cpu_baseline"] = {"value": rows / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
