@@ -83,3 +83,33 @@ def test_random_quantised_heads_every_row(N, V, D, bits, G):
     gpu = {"loss": loss.cpu().double().numpy(), "lse": lse.cpu().double().numpy(),
            "target": tgt.cpu().double().numpy(), "mean": float(mean.item())}
     compare(gpu, ref, mean_ref=oracle.mean(ref["loss"]))
+
+
+def draw_backward(n=10, seed=2028, budget=1.2e9):
+    rng = np.random.default_rng(seed)
+    out = []
+    while len(out) < n:
+        dtype = "fp32" if rng.random() < 0.4 else "bf16"
+        N = int(rng.choice([1, 7, 128, 129, 256, 300, 513]))
+        V = int(np.exp(rng.uniform(0.0, np.log(40000.0))))
+        D = int(rng.integers(1, 49)) * 8 if dtype == "bf16" else int(rng.integers(1, 200))
+        if N * V * D <= budget:
+            out.append((dtype, N, V, D))
+    return out
+
+
+@pytest.mark.parametrize("dtype,N,V,D", draw_backward())
+def test_random_shapes_backward_every_element(dtype, N, V, D):
+    """dH and dW of sum_i g_i loss_i on every element, within 2^-8 of the oracle's
+    magnitude bound (the bf16 rounding of dZ; fp32 inputs do far better)."""
+    import linear_cross_entropy_bf16_b200 as flce
+    H, W, y = synth.random_inputs(N, V, D, seed=3 * N + V + D, dtype=dtype)
+    Hd, Wd, yd = to_device(H, W, y)
+    _, lse, _, _ = flce.forward(Hd, Wd, yd, check=True)
+    g = np.random.default_rng(N + V).uniform(-1, 1, N)
+    gd = torch.from_numpy(g.astype(np.float32)).cuda()
+    dH, dW = flce.backward(Hd, Wd, yd, lse, gd, 1.0, check=True)
+    ref = oracle.backward(H, W, y, g.astype(np.float32).astype(np.float64), bounds=True)
+    for got, r, b in ((dH, ref["dH"], ref["bH"]), (dW, ref["dW"], ref["bW"])):
+        err = np.abs(got.cpu().double().numpy() - r)
+        assert np.all(err <= 2.0 ** -8 * b + 1e-7), float((err - 2.0 ** -8 * b).max())
