@@ -40,7 +40,7 @@ constexpr uint64_t kDefaultWaitLimitNs = 4000000000ull;  // 4 s in one wait: far
 
 #include "flce_schedule.h"
 
-// ---------------------------------------------------------------- driver entry point
+// ---------------------------------------------------------------- tensor maps, device facts, launches
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -919,6 +919,126 @@ extern "C" flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- quantised head: backward
+
+namespace {
+
+// [256 B header][dZ slice: N x chunk bf16][one chunk of W expanded: chunk x 2 Ds bf16]
+struct QuantBwdLayout {
+  int64_t chunk = 0;
+  size_t off_dz = 0, off_exp = 0, total = 0;
+};
+
+QuantBwdLayout quant_bwd_layout(int64_t N, int64_t V, int64_t D) {
+  QuantBwdLayout L;
+  L.chunk = std::min(round_up(V, kTileCols), kBwdChunkCols);
+  L.off_dz = kHeaderBytes;
+  L.off_exp = L.off_dz + align256(size_t(N) * size_t(L.chunk) * 2);
+  L.total = L.off_exp + align256(size_t(L.chunk) * size_t(2 * quant_segment(D)) * 2);
+  return L;
+}
+
+}  // namespace
+
+extern "C" size_t flce_backward_quantized_workspace_size(int64_t N, int64_t V, int64_t D,
+                                                         int32_t bits, int32_t group_size) {
+  if (N < 1 || V < 1 || D < 1 || !quant_format_ok(bits, group_size, D)) return 0;
+  return quant_bwd_layout(N, V, D).total;
+}
+
+extern "C" flce_status flce_backward_quantized(const void* H, const uint32_t* wq,
+                                               const void* scales, const void* biases,
+                                               int32_t bits, int32_t group_size, const int64_t* y,
+                                               const float* lse, const float* grad_loss,
+                                               float grad_scale, int64_t N, int64_t V, int64_t D,
+                                               float* dH, void* workspace, size_t workspace_bytes,
+                                               void* stream) {
+  FLCE_TRACE();
+  if (N < 0 || V < 1 || D < 1 || !quant_format_ok(bits, group_size, D))
+    return FLCE_ERR_INVALID_ARG;
+  if (N == 0) return FLCE_OK;
+  if (!H || !wq || !scales || !biases || !y || !lse || !dH || !workspace)
+    return FLCE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      ((reinterpret_cast<uintptr_t>(scales) | reinterpret_cast<uintptr_t>(biases)) & 1u) != 0)
+    return FLCE_ERR_INVALID_ARG;
+  if (!aligned16(H) || !aligned16(wq)) return FLCE_ERR_UNSUPPORTED;
+  if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31) ||
+      2 * quant_segment(D) >= (int64_t(1) << 31))
+    return FLCE_ERR_UNSUPPORTED;
+  const QuantBwdLayout L = quant_bwd_layout(N, V, D);
+  if (workspace_bytes < L.total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+
+  DeviceInfo di;
+  flce_status s = device_info(di);
+  if (s != FLCE_OK) return s;
+  if (!load_encoder()) return FLCE_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if ((s = set_smem_limits()) != FLCE_OK) return s;
+  const int64_t pairs = resident_pairs(dev, di.sms);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+  __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dz);
+  const __nv_bfloat16* ex = reinterpret_cast<const __nv_bfloat16*>(ws + L.off_exp);
+  const int64_t Ds = quant_segment(D);
+  if (cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
+
+  CUtensorMap mH_k;
+  if (!encode_bf16_2d(&mH_k, H, N, D, D, bwd::BM)) return FLCE_ERR_UNSUPPORTED;  // K1 A
+  for (int64_t c0 = 0; c0 < V; c0 += L.chunk) {
+    const int64_t clen = std::min(L.chunk, V - c0);
+    // W rows [c0, c0 + clen) as bf16 [hi | lo] (row stride 2 Ds)
+    if ((s = launch_dequant(wq, scales, biases, bits, group_size, c0, clen, D, ws + L.off_exp,
+                            di.sms, st)) != FLCE_OK)
+      return s;
+    CUtensorMap mW_k, mW_hi, mW_lo, mDz_k;
+    if (!encode_bf16_2d(&mW_k, ex, clen, 2 * Ds, 2 * Ds, bwd::HALF_N) ||  // K1 B: [hi | lo]
+        !encode_bf16_2d(&mW_hi, ex, clen, D, 2 * Ds, bwd::BK) ||          // K2 B: hi, MN-major
+        !encode_bf16_2d(&mW_lo, ex + Ds, clen, D, 2 * Ds, bwd::BK) ||     // K2 B: lo, MN-major
+        !encode_bf16_2d(&mDz_k, dz, N, clen, L.chunk, bwd::BM))           // K2 A
+      return FLCE_ERR_UNSUPPORTED;
+    // K1: logits [H | H] [hi | lo]^T over K = 2 Ds (H's K coordinate wraps
+    // after Ds), then dZ for the chunk
+    bwd::EpiGradLogits e1;
+    e1.lse = lse;
+    e1.y = y;
+    e1.grad = grad_loss;
+    e1.grad_scale = grad_scale;
+    e1.N = int32_t(N);
+    e1.V = int32_t(V);
+    e1.y_offset = 0;
+    e1.c0 = int32_t(c0);
+    e1.clen = int32_t(clen);
+    e1.dz = dz;
+    e1.dz_lo = nullptr;
+    e1.ldz = int32_t(L.chunk);
+    e1.status = &hdr->status;
+    bwd::GemmShape g1 = gemm_shape(N, clen, 2 * Ds);
+    g1.kblocks_a = int32_t(Ds / bwd::BK);
+    s = launch_gemm<bwd::EpiGradLogits, false, false>(mH_k, mW_k, g1, e1, &hdr->status, pairs,
+                                                      st);
+    if (s != FLCE_OK) return s;
+    // K2: dH (+)= dZ_C W_hi + dZ_C W_lo, in that order
+    const CUtensorMap* bs[2] = {&mW_hi, &mW_lo};
+    for (int p = 0; p < 2; ++p) {
+      bwd::EpiStoreF32 e2;
+      e2.out = dH;
+      e2.ld = int32_t(D);
+      e2.rows = int32_t(N);
+      e2.cols = int32_t(D);
+      e2.row_base = 0;
+      e2.accumulate = (c0 > 0 || p > 0) ? 1 : 0;
+      s = launch_gemm<bwd::EpiStoreF32, false, true>(mDz_k, *bs[p], gemm_shape(N, D, clen), e2,
+                                                     &hdr->status, pairs, st);
+      if (s != FLCE_OK) return s;
+    }
+  }
+  return FLCE_OK;
+}
+
 // ---------------------------------------------------------------- forward from host memory
 
 namespace {
@@ -1062,125 +1182,5 @@ extern "C" flce_status flce_forward_host(const void* H_host, const void* W_host,
     return FLCE_ERR_CUDA;
   // The copy stream's last work (the final chunk's copy) is already ordered
   // before `stream` through ready[]; nothing else is left on it.
-  return FLCE_OK;
-}
-
-// ---------------------------------------------------------------- quantised head: backward
-
-namespace {
-
-// [256 B header][dZ slice: N x chunk bf16][one chunk of W expanded: chunk x 2 Ds bf16]
-struct QuantBwdLayout {
-  int64_t chunk = 0;
-  size_t off_dz = 0, off_exp = 0, total = 0;
-};
-
-QuantBwdLayout quant_bwd_layout(int64_t N, int64_t V, int64_t D) {
-  QuantBwdLayout L;
-  L.chunk = std::min(round_up(V, kTileCols), kBwdChunkCols);
-  L.off_dz = kHeaderBytes;
-  L.off_exp = L.off_dz + align256(size_t(N) * size_t(L.chunk) * 2);
-  L.total = L.off_exp + align256(size_t(L.chunk) * size_t(2 * quant_segment(D)) * 2);
-  return L;
-}
-
-}  // namespace
-
-extern "C" size_t flce_backward_quantized_workspace_size(int64_t N, int64_t V, int64_t D,
-                                                         int32_t bits, int32_t group_size) {
-  if (N < 1 || V < 1 || D < 1 || !quant_format_ok(bits, group_size, D)) return 0;
-  return quant_bwd_layout(N, V, D).total;
-}
-
-extern "C" flce_status flce_backward_quantized(const void* H, const uint32_t* wq,
-                                               const void* scales, const void* biases,
-                                               int32_t bits, int32_t group_size, const int64_t* y,
-                                               const float* lse, const float* grad_loss,
-                                               float grad_scale, int64_t N, int64_t V, int64_t D,
-                                               float* dH, void* workspace, size_t workspace_bytes,
-                                               void* stream) {
-  FLCE_TRACE();
-  if (N < 0 || V < 1 || D < 1 || !quant_format_ok(bits, group_size, D))
-    return FLCE_ERR_INVALID_ARG;
-  if (N == 0) return FLCE_OK;
-  if (!H || !wq || !scales || !biases || !y || !lse || !dH || !workspace)
-    return FLCE_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
-      ((reinterpret_cast<uintptr_t>(scales) | reinterpret_cast<uintptr_t>(biases)) & 1u) != 0)
-    return FLCE_ERR_INVALID_ARG;
-  if (!aligned16(H) || !aligned16(wq)) return FLCE_ERR_UNSUPPORTED;
-  if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31) ||
-      2 * quant_segment(D) >= (int64_t(1) << 31))
-    return FLCE_ERR_UNSUPPORTED;
-  const QuantBwdLayout L = quant_bwd_layout(N, V, D);
-  if (workspace_bytes < L.total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
-
-  DeviceInfo di;
-  flce_status s = device_info(di);
-  if (s != FLCE_OK) return s;
-  if (!load_encoder()) return FLCE_ERR_CUDA;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
-  if ((s = set_smem_limits()) != FLCE_OK) return s;
-  const int64_t pairs = resident_pairs(dev, di.sms);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
-  __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dz);
-  const __nv_bfloat16* ex = reinterpret_cast<const __nv_bfloat16*>(ws + L.off_exp);
-  const int64_t Ds = quant_segment(D);
-  if (cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
-
-  CUtensorMap mH_k;
-  if (!encode_bf16_2d(&mH_k, H, N, D, D, bwd::BM)) return FLCE_ERR_UNSUPPORTED;  // K1 A
-  for (int64_t c0 = 0; c0 < V; c0 += L.chunk) {
-    const int64_t clen = std::min(L.chunk, V - c0);
-    // W rows [c0, c0 + clen) as bf16 [hi | lo] (row stride 2 Ds)
-    if ((s = launch_dequant(wq, scales, biases, bits, group_size, c0, clen, D, ws + L.off_exp,
-                            di.sms, st)) != FLCE_OK)
-      return s;
-    CUtensorMap mW_k, mW_hi, mW_lo, mDz_k;
-    if (!encode_bf16_2d(&mW_k, ex, clen, 2 * Ds, 2 * Ds, bwd::HALF_N) ||  // K1 B: [hi | lo]
-        !encode_bf16_2d(&mW_hi, ex, clen, D, 2 * Ds, bwd::BK) ||          // K2 B: hi, MN-major
-        !encode_bf16_2d(&mW_lo, ex + Ds, clen, D, 2 * Ds, bwd::BK) ||     // K2 B: lo, MN-major
-        !encode_bf16_2d(&mDz_k, dz, N, clen, L.chunk, bwd::BM))           // K2 A
-      return FLCE_ERR_UNSUPPORTED;
-    // K1: logits [H | H] [hi | lo]^T over K = 2 Ds (H's K coordinate wraps
-    // after Ds), then dZ for the chunk
-    bwd::EpiGradLogits e1;
-    e1.lse = lse;
-    e1.y = y;
-    e1.grad = grad_loss;
-    e1.grad_scale = grad_scale;
-    e1.N = int32_t(N);
-    e1.V = int32_t(V);
-    e1.y_offset = 0;
-    e1.c0 = int32_t(c0);
-    e1.clen = int32_t(clen);
-    e1.dz = dz;
-    e1.dz_lo = nullptr;
-    e1.ldz = int32_t(L.chunk);
-    e1.status = &hdr->status;
-    bwd::GemmShape g1 = gemm_shape(N, clen, 2 * Ds);
-    g1.kblocks_a = int32_t(Ds / bwd::BK);
-    s = launch_gemm<bwd::EpiGradLogits, false, false>(mH_k, mW_k, g1, e1, &hdr->status, pairs,
-                                                      st);
-    if (s != FLCE_OK) return s;
-    // K2: dH (+)= dZ_C W_hi + dZ_C W_lo, in that order
-    const CUtensorMap* bs[2] = {&mW_hi, &mW_lo};
-    for (int p = 0; p < 2; ++p) {
-      bwd::EpiStoreF32 e2;
-      e2.out = dH;
-      e2.ld = int32_t(D);
-      e2.rows = int32_t(N);
-      e2.cols = int32_t(D);
-      e2.row_base = 0;
-      e2.accumulate = (c0 > 0 || p > 0) ? 1 : 0;
-      s = launch_gemm<bwd::EpiStoreF32, false, true>(mDz_k, *bs[p], gemm_shape(N, D, clen), e2,
-                                                     &hdr->status, pairs, st);
-      if (s != FLCE_OK) return s;
-    }
-  }
   return FLCE_OK;
 }
