@@ -1,10 +1,19 @@
-"""Fused linear cross-entropy forward for NVIDIA B200 (sm_100a).
+"""Fused linear cross-entropy for NVIDIA B200 (sm_100a).
 
 For hidden states H (N, D), an output projection W (V, D) and targets y (N),
 computes loss_i = logsumexp(H_i W^T) - H_i . W_{y_i}, the log-sum-exp, the
 target logit and the mean loss without ever forming the (N, V) logits
 (D. Ineshin, "Een gefuseerde forward-kernel voor lineaire cross-entropy op
-Apple-GPU's", 2026, section 1).
+Apple-GPU's", 2026, section 1), and the gradients dH, dW from the saved
+log-sum-exp.
+
+Entry points: ``forward`` / ``backward`` (bf16 or fp32), ``forward_strided``
+(strided rows, int32 targets), ``forward_quantized`` / ``backward_quantized``
+(an affine group-quantised head), ``forward_host`` (inputs and results in
+host memory), the vocabulary-parallel ``forward_vocab_parallel`` /
+``backward_vocab_parallel`` and their per-shard pieces, ``forward_noalloc``,
+and the differentiable loss layers ``linear_cross_entropy`` /
+``linear_cross_entropy_quantized``.
 
 This module is a thin ctypes binding over ``libflce.so`` (C ABI in
 ``include/flce.h``): it checks and marshals torch tensors, allocates outputs
