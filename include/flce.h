@@ -1,6 +1,7 @@
 /*
- * flce.h — C ABI of libflce.so: the fused linear cross-entropy forward on
- * NVIDIA B200 (sm_100a).
+ * flce.h — C ABI of libflce.so: the fused linear cross-entropy forward and
+ * backward on NVIDIA B200 (sm_100a), with fp32, quantised-head,
+ * host-input, vocabulary-parallel and no-allocation variants.
  *
  * The operation (D. Ineshin, "Een gefuseerde forward-kernel voor lineaire
  * cross-entropy op Apple-GPU's", 2026, section 1): for hidden states H (N, D),

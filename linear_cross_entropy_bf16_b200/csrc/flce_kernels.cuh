@@ -15,13 +15,19 @@
 //     double-buffered fp32 TMEM accumulator, and warps 2-5 (one TMEM lane,
 //     i.e. one token, per thread) fold each finished tile into (m, s) and
 //     capture the target logit.  Logits never leave TMEM/registers.
+//   * flce_tc2_kernel: the same on CTA pairs (cta_group::2, 256x256 tiles,
+//     6-stage ring): each CTA stages its own 128 token rows and half of the
+//     W tile, the even CTA issues the pair MMAs.  Used for N > 128.
 //   * flce_split3_kernel: for fp32 inputs, splits H and W into bf16 hi/lo
 //     parts laid out along a tripled K axis, so that the same tensor-core
 //     kernels compute the three-product fp32 emulation Hhi Whi + Hhi Wlo +
 //     Hlo Whi.
+//   * flce_dequant_split_kernel: expands one chunk of an affine
+//     group-quantised head into bf16 [hi | lo] rows for the same kernels.
 //   * flce_merge_kernel: combines the P slab states of each token in a fixed
 //     order (the recurrence of section 1 applied to whole slabs), writes
-//     lse/loss, and reduces the mean deterministically in fp64.
+//     lse/loss, and reduces the mean deterministically in fp64; the shard
+//     kernels do the same across vocabulary shards or chunks.
 #pragma once
 
 #include <cstdint>
