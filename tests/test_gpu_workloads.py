@@ -20,7 +20,7 @@ from tests.flce_testing import check_properties, compare, run, to_device
 
 pytestmark = pytest.mark.gpu
 
-SAMPLE_ROWS = int(os.environ.get("FLCE_ORACLE_ROWS", "128"))
+SAMPLE_ROWS = int(os.environ.get("FLCE_ORACLE_ROWS", "256"))
 
 
 @pytest.fixture(scope="module", autouse=True)
