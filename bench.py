@@ -29,6 +29,7 @@ import re
 import shutil
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -120,8 +121,10 @@ class ClockSampler:
 
     def __init__(self, gpu_index: int):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv") \
-            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/flce_clocks_{os.getpid()}.csv"
+        # the raw samples go to FLCE_BENCH_CLOCKS_DIR when set (to keep them), else a temp file
+        out_dir = os.environ.get("FLCE_BENCH_CLOCKS_DIR")
+        self.path = os.path.join(out_dir, f"clocks_rank{gpu_index}.csv") if out_dir \
+            else os.path.join(tempfile.gettempdir(), f"flce_clocks_{os.getpid()}_{gpu_index}.csv")
         self.gpu_index = gpu_index
 
     def start(self):
