@@ -76,3 +76,20 @@ def test_logits_in_the_thousands(scale):
     tol = np.maximum(1e-3, 2.0 ** -20 * np.abs(ref["max"]))
     for key in ("loss", "lse", "target"):
         assert np.all(np.abs(gpu[key] - ref[key]) <= 2 * tol), key
+
+
+@pytest.mark.parametrize("N,V,D", [(256, 1 << 20, 128), (65536, 4096, 64), (256, 2048, 16384)])
+def test_extreme_extents(N, V, D):
+    """A million-word vocabulary (4096 tiles, the 512-slab cap), 65536 tokens, and
+    D = 16384: sampled rows against the oracle, properties on every row."""
+    import linear_cross_entropy_bf16_b200 as flce
+    from tests.flce_testing import check_properties
+    H, W, y = synth.random_inputs(N, V, D, seed=N + V + D)
+    Hd, Wd, yd = to_device(H, W, y)
+    loss, lse, tgt, mean = flce.forward(Hd, Wd, yd, check=True)
+    gpu = {"loss": loss.cpu().double().numpy(), "lse": lse.cpu().double().numpy(),
+           "target": tgt.cpu().double().numpy(), "mean": float(mean.item())}
+    check_properties(gpu, V)
+    rows = synth.sample_rows(N, 48, seed=7)
+    ref = oracle.forward(H, W, y, rows=rows)
+    compare(gpu, ref, rows=rows)
