@@ -92,8 +92,8 @@ typedef struct {
  * problem: a 256-byte header, the per-(slab, token) partial states (8 bytes
  * each, at most 512 slabs per token, so O(N), never O(N*V)), and one fp64
  * per 32 tokens for the mean.  fp32 inputs add the bf16 split copies of H
- * and W, 6 * Dp bytes per row of each (Dp = D rounded up to 8): O((N + V) D),
- * still never O(N*V).  Depends only on its arguments (not on the device).
+ * ([hi | hi | lo], 6 Dp bytes per row) and W ([hi | lo], 4 Dp bytes per row),
+ * Dp = D rounded up to 64: O((N + V) D), still never O(N*V).  Depends only on its arguments (not on the device).
  * Returns 0 for invalid arguments (N < 0, V < 1, D < 1, unknown dtype).  Host
  * only; never touches the GPU. */
 FLCE_API size_t flce_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype dtype);

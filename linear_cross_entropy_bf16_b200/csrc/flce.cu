@@ -171,14 +171,16 @@ flce_status contraction_workers(int64_t N, DeviceInfo& di, int64_t& workers) {
 
 // The contraction with the online (m, s) epilogue on bf16 operands: opH (N
 // rows, Kh columns, row stride ldh) and opW (V rows, Kw columns, row stride
-// ldw).  The kernel walks Kw in 64-element blocks; H's K coordinate wraps
-// after ceil(Kh / 64) blocks (Kh == Kw except for the quantised head).
-// Writes (m, s) per (slab, token) after the workspace header and the target
-// logits W owns.  reset_header: clear the header (status word) first.
+// ldw).  The kernel walks K in 64-element blocks; H's K coordinate wraps
+// after ceil(Kh / 64) blocks and W's after ceil(Kw / 64) (Kh == Kw == K
+// except for the quantised head, whose [H | H] wraps H, and for fp32
+// inputs, whose [hi | lo] W wraps W).  Writes (m, s) per (slab, token) after
+// the workspace header and the target logits W owns.  reset_header: clear
+// the header (status word) first.
 flce_status launch_contraction(const void* opH, int64_t ldh, int64_t Kh, const void* opW,
-                               int64_t ldw, int64_t Kw, Targets y, int64_t y_offset, int64_t N,
-                               int64_t V, const flce_plan_t& plan, float* out_target, void* ws,
-                               bool reset_header, cudaStream_t st) {
+                               int64_t ldw, int64_t Kw, int64_t K, Targets y, int64_t y_offset,
+                               int64_t N, int64_t V, const flce_plan_t& plan, float* out_target,
+                               void* ws, bool reset_header, cudaStream_t st) {
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
   float2* part = reinterpret_cast<float2*>(wsb + kHeaderBytes);
@@ -207,9 +209,10 @@ flce_status launch_contraction(const void* opH, int64_t ldh, int64_t Kh, const v
   a.hdr = hdr;
   a.N = int32_t(N);
   a.V = int32_t(V);
-  a.D = int32_t(Kw);
-  a.kblocks = int32_t(cdiv(Kw, tc::BK));
+  a.D = int32_t(K);
+  a.kblocks = int32_t(cdiv(K, tc::BK));
   a.kblocks_h = int32_t(cdiv(Kh, tc::BK));
+  a.kblocks_w = int32_t(cdiv(Kw, tc::BK));
   a.sch = sch;
   a.wait_limit_ns = kDefaultWaitLimitNs;
   if (pair)
@@ -220,15 +223,16 @@ flce_status launch_contraction(const void* opH, int64_t ldh, int64_t Kh, const v
 }
 
 // fp32 inputs: split `src` (rows, D; row stride ld) into its bf16 (rows,
-// 3 Dp) copy at `dst` with hi / lo parts in the segments the operand needs.
-flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, int lo_segment,
-                         void* dst, int sms, cudaStream_t st) {
+// nseg Dp) copy at `dst`: lo in segment lo_segment, hi in the others.
+flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, int64_t Dp,
+                         int nseg, int lo_segment, void* dst, int sms, cudaStream_t st) {
   split::Args a;
   a.src = static_cast<const float*>(src);
   a.ld = ld;
   a.rows = rows;
   a.D = int32_t(D);
-  a.Dp = int32_t(split_segment(D));
+  a.Dp = int32_t(Dp);
+  a.nseg = nseg;
   a.lo_segment = lo_segment;
   a.dst = static_cast<__nv_bfloat16*>(dst);
   const int64_t warps_per_block = split::NUM_THREADS / 32;
@@ -254,23 +258,26 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
   make_plan(N, V, D, dtype, workers, &plan);
 
   // The operands the tensor-core kernels read: H and W themselves (bf16), or
-  // their split copies in the workspace (fp32), K = 3 Dp.
+  // their split copies in the workspace (fp32): H as [hi | hi | lo] and W as
+  // [hi | lo], K = 3 Dp with W's K coordinate wrapping after 2 Dp.
   const void* opH = H;
   const void* opW = W;
-  int64_t K = D;
+  int64_t K = D, Kw = D;
   if (dtype == FLCE_FP32) {
     uint8_t* wsb = static_cast<uint8_t*>(ws);
-    K = k_extent(D, dtype);
+    const int64_t Dp = fwd_split_segment(D);
+    K = 3 * Dp;
+    Kw = 2 * Dp;
     uint8_t* hs = wsb + state_bytes_for(N, V);
-    uint8_t* wsplit = hs + split_bytes_for(N, D);
-    if ((s = launch_split(H, ldh, N, D, 2, hs, di.sms, st)) != FLCE_OK) return s;
-    if ((s = launch_split(W, ldw, V, D, 1, wsplit, di.sms, st)) != FLCE_OK) return s;
+    uint8_t* wsplit = hs + fwd_split_h_bytes(N, D);
+    if ((s = launch_split(H, ldh, N, D, Dp, 3, 2, hs, di.sms, st)) != FLCE_OK) return s;
+    if ((s = launch_split(W, ldw, V, D, Dp, 2, 1, wsplit, di.sms, st)) != FLCE_OK) return s;
     opH = hs;
     opW = wsplit;
     ldh = K;
-    ldw = K;
+    ldw = Kw;
   }
-  return launch_contraction(opH, ldh, K, opW, ldw, K, y, y_offset, N, V, plan, out_target, ws,
+  return launch_contraction(opH, ldh, K, opW, ldw, Kw, K, y, y_offset, N, V, plan, out_target, ws,
                             true, st);
 }
 
@@ -513,9 +520,9 @@ BwdLayout bwd_layout(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
     L.off_dzl = end;
     end += align256(size_t(N) * size_t(L.chunk) * 2);
     L.off_h3 = end;
-    end += split_bytes_for(N, D);
+    end += bwd_split_bytes_for(N, D);
     L.off_w3 = end;
-    end += split_bytes_for(L.chunk, D);
+    end += bwd_split_bytes_for(L.chunk, D);
   }
   L.total = end;
   return L;
@@ -614,7 +621,7 @@ flce_status backward_impl(const void* H, const void* W, const int64_t* y, const 
   // The bf16 operands.  bf16 inputs: H and W themselves.  fp32 inputs: the
   // split copies, K1 contracting [hi | hi | lo] against [hi | lo | hi] over
   // K = 3 Dp; K2 and K3 read the hi and lo segments as strided views.
-  const int64_t Dp = split_segment(D);
+  const int64_t Dp = bwd_split_segment(D);
   const int64_t K1 = fp32 ? 3 * Dp : D;   // K of the logits contraction
   const int64_t ldk = fp32 ? 3 * Dp : D;  // row stride of the H and W operands
   const __nv_bfloat16* Hb = static_cast<const __nv_bfloat16*>(H);
@@ -622,7 +629,7 @@ flce_status backward_impl(const void* H, const void* W, const int64_t* y, const 
   if (fp32) {
     Hb = reinterpret_cast<const __nv_bfloat16*>(ws + L.off_h3);
     W3 = reinterpret_cast<const __nv_bfloat16*>(ws + L.off_w3);
-    if ((s = launch_split(H, D, N, D, 2, ws + L.off_h3, di.sms, st)) != FLCE_OK) return s;
+    if ((s = launch_split(H, D, N, D, Dp, 3, 2, ws + L.off_h3, di.sms, st)) != FLCE_OK) return s;
   }
   CUtensorMap mH_k, mH_mn, mH_mn_lo;
   if (!encode_bf16_2d(&mH_k, Hb, N, K1, ldk, bwd::BM) ||     // K1 A: (N, K1)
@@ -634,7 +641,7 @@ flce_status backward_impl(const void* H, const void* W, const int64_t* y, const 
     const int64_t clen = std::min(L.chunk, V - c0);
     const __nv_bfloat16* Wc = static_cast<const __nv_bfloat16*>(W) + c0 * D;
     if (fp32) {
-      if ((s = launch_split(static_cast<const float*>(W) + c0 * D, D, clen, D, 1,
+      if ((s = launch_split(static_cast<const float*>(W) + c0 * D, D, clen, D, Dp, 3, 1,
                             ws + L.off_w3, di.sms, st)) != FLCE_OK)
         return s;
       Wc = W3;
@@ -903,8 +910,8 @@ extern "C" flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
     flce_plan_t plan;
     make_plan(N, rows, D, FLCE_BF16, workers, &plan);
     // [H | H] against [hi | lo]: H's K coordinate wraps after Ds.
-    if ((s = launch_contraction(H, D, D, expanded, 2 * Ds, 2 * Ds, Targets{y, 0}, c0, N, rows,
-                                plan, out_target_logit, workspace, false, st)) != FLCE_OK)
+    if ((s = launch_contraction(H, D, D, expanded, 2 * Ds, 2 * Ds, 2 * Ds, Targets{y, 0}, c0, N,
+                                rows, plan, out_target_logit, workspace, false, st)) != FLCE_OK)
       return s;
     flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
         reinterpret_cast<const float2*>(wsb + kHeaderBytes), hdr, y, int32_t(N), c0, rows,
@@ -1160,7 +1167,7 @@ extern "C" flce_status flce_forward_host(const void* H_host, const void* W_host,
       return FLCE_ERR_CUDA;
     flce_plan_t plan;
     make_plan(N, rows, D, FLCE_BF16, workers, &plan);
-    if ((s = launch_contraction(Hd, D, D, staging[b], D, D, Targets{yd, 0}, c0, N, rows, plan,
+    if ((s = launch_contraction(Hd, D, D, staging[b], D, D, D, Targets{yd, 0}, c0, N, rows, plan,
                                 tgt_d, workspace, false, st)) != FLCE_OK)
       return s;
     flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(

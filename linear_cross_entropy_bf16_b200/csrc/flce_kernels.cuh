@@ -246,9 +246,11 @@ struct Args {
   float* target_logit;     // [N]
   WsHeader* hdr;
   int32_t N, V, D;
-  int32_t kblocks;         // K-blocks of W per tile: ceil(K / BK)
+  int32_t kblocks;         // K-blocks per tile: ceil(K / BK)
   int32_t kblocks_h;       // K-blocks of H; H's K coordinate wraps modulo this
                            // (== kblocks, except for the quantised head's [H | H])
+  int32_t kblocks_w;       // K-blocks of W; W's K coordinate wraps modulo this
+                           // (== kblocks, except for fp32 inputs' [hi | lo] W)
   Schedule sch;
   uint64_t wait_limit_ns;
 };
@@ -318,7 +320,7 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
         int slab, tb, t0, nt;
         unit_coords(sch, u, slab, tb, t0, nt);
         for (int t = t0; ok && t < t0 + nt; ++t) {
-          for (int kb = 0, kh = 0; kb < a.kblocks; ++kb) {
+          for (int kb = 0, kh = 0, kw = 0; kb < a.kblocks; ++kb) {
             if (!wait_bounded(ptx::smem_addr(&empty_bar[stage]), phase ^ 1u, abort_flag, status, lim)) {
               ok = false;
               break;
@@ -327,8 +329,9 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
             const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
             ptx::mbar_arrive_expect_tx(fb, STAGE_BYTES);
             ptx::tma_load_2d(sa, &tmH, fb, kh * BK, tb * BM);
-            ptx::tma_load_2d(sa + A_BYTES, &tmW, fb, kb * BK, t * BN);
+            ptx::tma_load_2d(sa + A_BYTES, &tmW, fb, kw * BK, t * BN);
             if (++kh == a.kblocks_h) kh = 0;
+            if (++kw == a.kblocks_w) kw = 0;
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) {
@@ -548,7 +551,7 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
         const int hrow = tb * PAIR_M + int(rank) * BM;
         for (int t = t0; ok && t < t0 + nt; ++t) {
           const int wrow = t * BN + int(rank) * HALF_N;
-          for (int kb = 0, kh = 0; kb < a.kblocks; ++kb) {
+          for (int kb = 0, kh = 0, kw = 0; kb < a.kblocks; ++kb) {
             if (!wait_bounded(ptx::smem_addr(&empty_bar[stage]), phase ^ 1u, abort_flag, status,
                               lim)) {
               ok = false;
@@ -559,8 +562,9 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
             const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
             if (rank == 0) ptx::mbar_arrive_expect_tx(fb_local, PAIR_TX_BYTES);
             ptx::tma_load_2d_pair(sa, &tmH, fb_even, kh * BK, hrow);
-            ptx::tma_load_2d_pair(sa + A_BYTES, &tmW, fb_even, kb * BK, wrow);
+            ptx::tma_load_2d_pair(sa + A_BYTES, &tmW, fb_even, kw * BK, wrow);
             if (++kh == a.kblocks_h) kh = 0;
+            if (++kw == a.kblocks_w) kw = 0;
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) {
@@ -692,11 +696,13 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
 // the bfloat16 artificial intelligence datatype for higher-precision
 // computations", ARITH 2019):  hi = bf16(x),  lo = bf16(x - hi),  so that
 // |x - hi - lo| <= 2^-16 |x|.  Laying H out as [hi | hi | lo] and W as
-// [hi | lo | hi] along K (three segments of Dp = D rounded up to 8, zero
-// padded) turns one bf16 contraction over 3 Dp into
+// [hi | lo] along K (segments of Dp = D rounded up to 64, zero padded), with
+// W's K coordinate wrapping after its two segments, turns one bf16
+// contraction over 3 Dp into
 //   Z = Hhi Whi^T + Hhi Wlo^T + Hlo Whi^T
 // with fp32 accumulation in TMEM: each product h w is off by at most about
 // 3 * 2^-16 |h w| (the dropped lo*lo term and the two rounding residues).
+// (The backward lays W out as [hi | lo | hi] instead: its GEMM wraps only A.)
 namespace split {
 
 constexpr int NUM_THREADS = 256;   // 8 warps, one row per warp at a time
@@ -706,9 +712,10 @@ struct Args {
   int64_t ld;
   int64_t rows;
   int32_t D;
-  int32_t Dp;             // D rounded up to a multiple of 8
-  int32_t lo_segment;     // 1 (W: [hi | lo | hi]) or 2 (H: [hi | hi | lo])
-  __nv_bfloat16* dst;     // (rows, 3 Dp) bf16, contiguous
+  int32_t Dp;             // one segment: D rounded up (to 64 for the forward, 8 for the backward)
+  int32_t nseg;           // segments per row: 3, or 2 for [hi | lo]
+  int32_t lo_segment;     // the segment that holds lo; every other one holds hi
+  __nv_bfloat16* dst;     // (rows, nseg Dp) bf16, contiguous
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 a, __nv_bfloat16 b) {
@@ -727,11 +734,15 @@ __global__ void __launch_bounds__(NUM_THREADS) flce_split3_kernel(const Args a) 
   for (int64_t r = int64_t(blockIdx.x) * (NUM_THREADS / 32) + (threadIdx.x >> 5); r < a.rows;
        r += warps) {
     const float* row = a.src + r * a.ld;
-    uint4* out = reinterpret_cast<uint4*>(a.dst + r * 3 * int64_t(a.Dp));
+    uint4* out = reinterpret_cast<uint4*>(a.dst + r * a.nseg * int64_t(a.Dp));
     for (int g = lane; g < groups; g += 32) {
       const int k0 = g * 8;
       float x[8];
-      if (kVec) {
+      if (k0 >= a.D) {
+        // zero padding from D to the segment length: nothing of the row is read
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x[j] = 0.f;
+      } else if (kVec) {        // D % 8 == 0: all 8 elements lie inside the row
         const float4 u = __ldg(reinterpret_cast<const float4*>(row + k0));
         const float4 v = __ldg(reinterpret_cast<const float4*>(row + k0 + 4));
         x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
@@ -754,9 +765,7 @@ __global__ void __launch_bounds__(NUM_THREADS) flce_split3_kernel(const Args a) 
       }
       const uint4 vh = make_uint4(hi[0], hi[1], hi[2], hi[3]);
       const uint4 vl = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      out[g] = vh;
-      out[groups + g] = a.lo_segment == 1 ? vl : vh;
-      out[2 * groups + g] = a.lo_segment == 2 ? vl : vh;
+      for (int seg = 0; seg < a.nseg; ++seg) out[seg * groups + g] = seg == a.lo_segment ? vl : vh;
     }
   }
 }
