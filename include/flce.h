@@ -193,8 +193,8 @@ FLCE_API flce_status flce_merge(const int64_t* y, int64_t N, int64_t V,
  * loss).  Differentiating section 1 of the page:
  *     dZ_ij = g_i (exp(z_ij - lse_i) - [j == y_i]),   dH = dZ W,   dW = dZ^T H.
  * As on the page, the forward's log-sum-exp is kept and the logits are
- * regenerated tile by tile; vocabulary chunks of up to 16384 rows bound the
- * working slice of dZ to O(N * chunk) (never O(N * V)).
+ * regenerated tile by tile; vocabulary chunks (32768 rows for bf16, 16384 for
+ * fp32) bound the working slice of dZ to O(N * chunk) (never O(N * V)).
  *
  *   H, W, y, N, V, D, dtype   as for flce_forward (bf16: D % 8 == 0 and
  *                             16-byte-aligned H, W; fp32: any D, 4-byte
@@ -205,8 +205,10 @@ FLCE_API flce_status flce_merge(const int64_t* y, int64_t N, int64_t V,
  *   dW           (V, D) fp32 row-major, overwritten
  *   workspace    >= flce_backward_workspace_size(N, V, D, dtype) bytes,
  *                256-byte aligned (the status word read by flce_check and one
- *                N x chunk slice of dZ in bf16: 256 B + 2 N min(V, 16384) B,
- *                rounded up; fp32 inputs add a second dZ slice and the bf16
+ *                N x chunk slice of dZ in bf16: 256 B + 2 N chunk B, chunk =
+ *                min(V rounded up to 256, 32768 (bf16) or 16384 (fp32)),
+ *                each part rounded up to
+ *                256 B; fp32 inputs add a second dZ slice and the bf16
  *                hi/lo split copies of H and of one W chunk, 6 Dp bytes per
  *                row, Dp = D rounded up to 8)
  * bf16 inputs: dZ is rounded to bf16 before the two gradient contractions

@@ -276,11 +276,13 @@ def test_forward_host_argument_checks_need_no_gpu(lib):
 def test_backward_workspace_fp32_adds_split_copies(lib):
     r256 = lambda b: (b + 255) // 256 * 256
     for N, V, D in [(8192, 151936, 4096), (7, 3, 5), (300, 40000, 96)]:
-        chunk = min(math.ceil(V / 256) * 256, 16384)
+        chunk = min(math.ceil(V / 256) * 256, 32768)       # bf16
+        chunk32 = min(math.ceil(V / 256) * 256, 16384)     # fp32
         Dp = (D + 7) // 8 * 8
-        bf16 = flce.backward_workspace_size(N, V, D) if D % 8 == 0 else 256 + r256(2 * N * chunk)
+        if D % 8 == 0:
+            assert flce.backward_workspace_size(N, V, D) == 256 + r256(2 * N * chunk)
         assert flce.backward_workspace_size(N, V, D, 1) == (
-            bf16 + r256(2 * N * chunk) + r256(6 * Dp * N) + r256(6 * Dp * chunk))
+            256 + 2 * r256(2 * N * chunk32) + r256(6 * Dp * N) + r256(6 * Dp * chunk32))
 
 
 def test_quantized_backward_workspace_and_checks_need_no_gpu(lib):

@@ -140,8 +140,7 @@ def _vp_backward_rank(rank, world, port, q):
                                               grad_scale=1.0 / N, check=True)
         torch.cuda.synchronize()
         dH_full, dW_full = flce.backward(Hd, Wd, yd, lse, None, 1.0 / N, check=True)
-        rel = float((dH - dH_full).norm() / dH_full.norm())
-        q.put((rank, rel, bool(torch.equal(dW, dW_full[a:b]))))
+        q.put((rank, dH.cpu().numpy(), dH_full.cpu().numpy(), bool(torch.equal(dW, dW_full[a:b]))))
     finally:
         dist.destroy_process_group()
 
@@ -161,6 +160,17 @@ def test_backward_vocab_parallel_overlapped_allreduce_two_ranks_one_gpu():
     for p in procs:
         p.join(60)
         assert p.exitcode == 0
-    for rank, rel, same_dw in out:
-        assert rel < 1e-5, (rank, rel)        # the shares' sum vs the unsharded dH (fp32 sums)
+    # Both sides contract the same bf16 dZ with the same W; only the grouping of
+    # the fp32 sums over the vocabulary differs (one sum over all V rows against
+    # two shard sums and their all-reduce), so each entry of the two dH differs
+    # by at most 2 (V + 1) 2^-24 sum_j |dZ_ij| |W_jk| (the oracle's bH, scaled
+    # by 1 + 2^-8 for dZ's rounding to bf16).
+    N, V, D = 256, 20000, 128
+    H, W, y = synth.random_inputs(N, V, D, seed=60)
+    ref = oracle.backward(H, W, y, np.float64(np.float32(1.0 / N)), bounds=True)
+    lim = 2 * (V + 1) * 2.0 ** -24 * (1 + 2.0 ** -8) * ref["bH"] + 1e-12
+    for rank, dH, dH_full, same_dw in out:
+        err = np.abs(dH.astype(np.float64) - dH_full)
+        assert np.all(err <= lim), (rank, float((err / lim).max()))
+        assert np.linalg.norm(dH - dH_full) / np.linalg.norm(dH_full) < 1e-4
         assert same_dw
