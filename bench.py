@@ -16,6 +16,11 @@ copied in every step, W in chunks that overlap the contraction; results
 copied back), SM clocks during the timed
 region, and the CPU oracle on a bounded sample of the same workload.
 
+Optional legs, each added to the same line as its own object: ``--backward``
+(dH and dW), ``--quantized BITS,GROUP`` (a quantised head, with its dH when
+``--backward`` is given too) and ``--fp32`` (the same workload's fp32 samples,
+not rounded to bf16: forward, and backward with ``--backward``).
+
 ``--impl reference`` times the fp64 CPU oracle instead (the reference arm).
 """
 from __future__ import annotations
@@ -429,6 +434,8 @@ def run_ours(args, w, rank, world, local_rank):
         bits, gs = (int(v) for v in args.quantized.split(","))
         extra["quantized"] = time_quantized(flce, H, Wn, y, N, V, D, bits, gs, dev, stream, args,
                                             peaks["bf16_tflops"], world)
+    if args.fp32 and w.dtype == "bf16":
+        extra["fp32"] = time_fp32(flce, w, rank, y, dev, stream, args, peaks["bf16_tflops"], world)
 
     if rank != 0:
         return 0
@@ -559,7 +566,7 @@ def time_quantized(flce, H, Wn, y, N, V, D, bits, gs, dev, stream, args, peak, w
     ms = max_over_ranks([e0.elapsed_time(e1) / Kq], world, device=dev)[0]
     flops = 2 * N * V * D
     Ds = (D + 63) // 64 * 64
-    tensor_flops = 2 * N * V * 2 * Ds      # [H | H] against [hi | lo]
+    tensor_flops = 2 * N * V * 2 * Ds      # H hi^T + H lo^T
     head_bytes = wq.nbytes + sc.nbytes + bi.nbytes
     extra = {}
     if args.backward:
@@ -585,7 +592,7 @@ def time_quantized(flce, H, Wn, y, N, V, D, bits, gs, dev, stream, args, peak, w
         e1.record(stream)
         torch.cuda.synchronize(dev)
         bms = max_over_ranks([e0.elapsed_time(e1) / Kb], world, device=dev)[0]
-        bflops = 2 * N * V * 2 * Ds + 2 * 2 * N * V * D   # logits over [H | H], dZ W_hi + dZ W_lo
+        bflops = 2 * N * V * 2 * Ds + 2 * 2 * N * V * D   # logits H hi^T + H lo^T, dZ W_hi + dZ W_lo
         extra = {"backward_ms_per_step": bms, "backward_tensor_tflops": bflops / (bms * 1e-3) / 1e12,
                  "backward_what": "dH only (the quantised head is frozen): regenerated logits, 2 GEMMs"}
     return {**extra, "bits": bits, "group_size": gs, "ms_per_step": ms, "steps": Kq,
@@ -597,6 +604,71 @@ def time_quantized(flce, H, Wn, y, N, V, D, bits, gs, dev, stream, args, peak, w
             "workspace_bytes": int(ws.numel()), "mean_loss": float(out["mean"].item()),
             "what": "forward with an affine group-quantised head: W expanded per 16384-row chunk "
                     "to bf16 hi/lo, 2 bf16 products per weight"}
+
+
+def time_fp32(flce, w, rank, y, dev, stream, args, peak, world):
+    """The forward (and with --backward the backward) on the same workload drawn in fp32:
+    the samples the bf16 inputs are rounded from, kept as they are.  Each call splits H
+    and W into bf16 hi/lo parts and runs three bf16 products per fp32 product."""
+    import dataclasses
+
+    import torch
+    N, V, D = w.N, w.V, w.D
+    Hn, Wn, _ = synth.generate(dataclasses.replace(w, dtype="fp32"), token_stream=rank)
+    H = torch.from_numpy(Hn).to(dev)
+    W = torch.from_numpy(Wn).to(dev)
+    del Hn, Wn
+    ws = torch.empty(flce.workspace_size(N, V, D, torch.float32), dtype=torch.uint8, device=dev)
+    out = {"loss": torch.empty(N, device=dev), "lse": torch.empty(N, device=dev),
+           "target_logit": torch.empty(N, device=dev), "mean": torch.empty((), device=dev)}
+
+    def timed(fn, steps, what, ws_check):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+        stream.synchronize()
+        if flce.check(ws_check, stream) != flce.OK:
+            raise flce.FlceError(flce.check(ws_check, stream), what)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(steps):
+                fn()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if flce.check(ws_check, stream) != flce.OK:
+            raise flce.FlceError(flce.check(ws_check, stream), what)
+        return max_over_ranks([e0.elapsed_time(e1) / steps], world, device=dev)[0]
+
+    Kf = max(3, args.steps // 5)
+    ms = timed(lambda: flce.forward(H, W, y, out=out, workspace=ws, stream=stream), Kf,
+               "forward (fp32)", ws)
+    Dp = (D + 63) // 64 * 64
+    tensor_flops = 2 * N * V * 3 * Dp          # hi hi + hi lo + lo hi per K block
+    res = {"ms_per_step": ms, "steps": Kf, "tokens_per_s": weak_scaling_tokens_per_s(world, N, ms),
+           "tflops": 2 * N * V * D / (ms * 1e-3) / 1e12,
+           "tensor_tflops": tensor_flops / (ms * 1e-3) / 1e12,
+           "tensor_frac_of_bf16_peak": tensor_flops / (ms * 1e-3) / 1e12 / peak,
+           "workspace_bytes": int(ws.numel()), "mean_loss": float(out["mean"].item()),
+           "what": "fp32 H and W (the workload's samples before bf16 rounding): each call splits "
+                   "them into bf16 hi/lo and runs 3 bf16 products per fp32 product; tflops counts "
+                   "2 N V D, tensor_tflops the bf16 products"}
+    if args.backward:
+        bws = torch.empty(flce.backward_workspace_size(N, V, D, torch.float32), dtype=torch.uint8,
+                          device=dev)
+        grads = {"dH": torch.empty(N, D, device=dev), "dW": torch.empty(V, D, device=dev)}
+        Kb = max(3, args.backward_steps // 2)
+        bms = timed(lambda: flce.backward(H, W, y, out["lse"], None, 1.0 / N, out=grads,
+                                          workspace=bws, stream=stream), Kb, "backward (fp32)", bws)
+        Db = (D + 7) // 8 * 8
+        btensor = 2 * N * V * 3 * Db + 2 * 3 * 2 * N * V * D    # logits over 3 segments; 3 + 3 products
+        res.update({"backward_ms_per_step": bms, "backward_steps": Kb,
+                    "backward_tflops": 3 * 2 * N * V * D / (bms * 1e-3) / 1e12,
+                    "backward_tensor_tflops": btensor / (bms * 1e-3) / 1e12,
+                    "backward_workspace_bytes": int(bws.numel())})
+        del bws, grads
+    del H, W, ws
+    return res
 
 
 def torch_materialised(H, W, y, dev):
@@ -640,6 +712,9 @@ def main():
     ap.add_argument("--quantized", default=None, metavar="BITS,GROUP",
                     help="also time the forward with W quantised (e.g. 4,64) and add a 'quantized' object")
     ap.add_argument("--context", action="store_true", help="also time the materialising torch forward")
+    ap.add_argument("--fp32", action="store_true",
+                    help="also time the forward (and with --backward the backward) on the workload's "
+                         "fp32 samples and add an 'fp32' object")
     ap.add_argument("--shape", default=None,
                     help="N,V,D: a custom shape with the chosen workload's distributions "
                          "(used for small profiling captures; not a reported workload)")

@@ -92,8 +92,9 @@ typedef struct {
  * problem: a 256-byte header, the per-(slab, token) partial states (8 bytes
  * each, at most 512 slabs per token, so O(N), never O(N*V)), and one fp64
  * per 32 tokens for the mean.  fp32 inputs add the bf16 split copies of H
- * ([hi | hi | lo], 6 Dp bytes per row) and W ([hi | lo], 4 Dp bytes per row),
- * Dp = D rounded up to 64: O((N + V) D), still never O(N*V).  Depends only on its arguments (not on the device).
+ * and W ([hi | lo], 4 Dp bytes per row each), Dp = D rounded up to 64:
+ * O((N + V) D), still never O(N*V).  Depends only on its arguments (not on
+ * the device).
  * Returns 0 for invalid arguments (N < 0, V < 1, D < 1, unknown dtype).  Host
  * only; never touches the GPU. */
 FLCE_API size_t flce_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype dtype);
@@ -359,8 +360,9 @@ FLCE_API flce_status flce_forward_noalloc(const void* H, const void* W, const in
  * How it runs: W is expanded 16384 vocabulary rows at a time into the
  * workspace as two bf16 K segments per row, hi = bf16(W_jk) and lo =
  * bf16(W_jk - hi) (W_jk formed in fp32 with one rounding), and the
- * tensor-core contraction takes [H | H] against [hi | lo]: twice the work of
- * a bf16 head, with |W - hi - lo| <= 2^-16 |W| per weight.  Each chunk is a
+ * tensor-core contraction stages each K block of H once with both parts of
+ * W and forms H hi^T + H lo^T: twice the tensor work of a bf16 head, with
+ * |W - hi - lo| <= 2^-16 |W| per weight.  Each chunk is a
  * vocabulary shard; their per-token states are merged at the end, in chunk
  * order.  The workspace is O(N V / 16384 + 16384 D), never O(N V).
  * Errors: FLCE_ERR_INVALID_ARG for bad sizes, formats, null pointers or a

@@ -106,11 +106,20 @@ flce_status ensure_smem_limit(const void* fn, int bytes) {
   return FLCE_OK;
 }
 
-flce_status set_smem_limits() {
-  flce_status s = ensure_smem_limit(reinterpret_cast<const void*>(tc::flce_tc_kernel),
-                                    tc::SMEM_BYTES);
+template <int L>
+flce_status set_smem_limits_for() {
+  flce_status s = ensure_smem_limit(reinterpret_cast<const void*>(tc::flce_tc_kernel<L>),
+                                    tc::Cfg<L>::SMEM_BYTES);
   if (s != FLCE_OK) return s;
-  return ensure_smem_limit(reinterpret_cast<const void*>(tc2::flce_tc2_kernel), tc2::SMEM_BYTES);
+  return ensure_smem_limit(reinterpret_cast<const void*>(tc2::flce_tc2_kernel<L>),
+                           tc2::Cfg<L>::SMEM_BYTES);
+}
+
+flce_status set_smem_limits() {
+  flce_status s = set_smem_limits_for<tc::kPlain>();
+  if (s == FLCE_OK) s = set_smem_limits_for<tc::kSplitW>();
+  if (s == FLCE_OK) s = set_smem_limits_for<tc::kSplitHW>();
+  return s;
 }
 
 // CTA pairs of the pair kernel that can be resident at once on the current
@@ -124,8 +133,10 @@ int64_t resident_pairs(int dev, int sms) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(sms & ~1), 1, 1);
   cfg.blockDim = dim3(tc2::NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = tc2::SMEM_BYTES;
-  if (cudaOccupancyMaxActiveClusters(&n, tc2::flce_tc2_kernel, &cfg) != cudaSuccess || n < 1) {
+  // every layout of the pair kernel takes the same 192 KiB ring (one CTA per SM)
+  cfg.dynamicSmemBytes = tc2::Cfg<tc::kPlain>::SMEM_BYTES;
+  if (cudaOccupancyMaxActiveClusters(&n, tc2::flce_tc2_kernel<tc::kPlain>, &cfg) != cudaSuccess ||
+      n < 1) {
     (void)cudaGetLastError();
     n = sms / 2;
   }
@@ -169,18 +180,36 @@ flce_status contraction_workers(int64_t N, DeviceInfo& di, int64_t& workers) {
   return FLCE_OK;
 }
 
-// The contraction with the online (m, s) epilogue on bf16 operands: opH (N
-// rows, Kh columns, row stride ldh) and opW (V rows, Kw columns, row stride
-// ldw).  The kernel walks K in 64-element blocks; H's K coordinate wraps
-// after ceil(Kh / 64) blocks and W's after ceil(Kw / 64) (Kh == Kw == K
-// except for the quantised head, whose [H | H] wraps H, and for fp32
-// inputs, whose [hi | lo] W wraps W).  Writes (m, s) per (slab, token) after
-// the workspace header and the target logits W owns.  reset_header: clear
-// the header (status word) first.
-flce_status launch_contraction(const void* opH, int64_t ldh, int64_t Kh, const void* opW,
-                               int64_t ldw, int64_t Kw, int64_t K, Targets y, int64_t y_offset,
-                               int64_t N, int64_t V, const flce_plan_t& plan, float* out_target,
-                               void* ws, bool reset_header, cudaStream_t st) {
+// The bf16 operands of one contraction: rows of H (N rows) and of W (V rows),
+// `cols_*` columns stored with row stride `ld_*` elements.  The kernel walks
+// `kblocks` 64-element K blocks.  In the split layouts (tc::StageLayout) the
+// lo part of K block kb sits `seg_*` columns after its hi part in the same
+// row: fp32 inputs split into [hi | lo] H and W rows (kSplitHW), a quantised
+// head expanded into [hi | lo] W rows against H itself (kSplitW).
+struct Operands {
+  const void* H;
+  int64_t ldh, cols_h, seg_h;
+  const void* W;
+  int64_t ldw, cols_w, seg_w;
+  int64_t kblocks;
+  int layout;  // tc::StageLayout
+};
+
+template <int L>
+void launch_contraction_kernel(bool pair, unsigned grid, const CUtensorMap& tmH,
+                               const CUtensorMap& tmW, const tc::Args& a, cudaStream_t st) {
+  if (pair)
+    tc2::flce_tc2_kernel<L><<<grid, tc2::NUM_THREADS, tc2::Cfg<L>::SMEM_BYTES, st>>>(tmH, tmW, a);
+  else
+    tc::flce_tc_kernel<L><<<grid, tc::NUM_THREADS, tc::Cfg<L>::SMEM_BYTES, st>>>(tmH, tmW, a);
+}
+
+// The contraction with the online (m, s) epilogue.  Writes (m, s) per (slab,
+// token) after the workspace header and the target logits W owns.
+// reset_header: clear the header (status word) first.
+flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, int64_t N,
+                               int64_t V, const flce_plan_t& plan, float* out_target, void* ws,
+                               bool reset_header, cudaStream_t st) {
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
   float2* part = reinterpret_cast<float2*>(wsb + kHeaderBytes);
@@ -198,8 +227,8 @@ flce_status launch_contraction(const void* opH, int64_t ldh, int64_t Kh, const v
   if (!load_encoder()) return FLCE_ERR_CUDA;
   const bool pair = plan.ctas_per_unit == 2;
   CUtensorMap tmH, tmW;
-  if (!encode_bf16_rows(&tmH, opH, N, Kh, ldh, tc::BM) ||
-      !encode_bf16_rows(&tmW, opW, V, Kw, ldw, pair ? tc2::HALF_N : tc::BN))
+  if (!encode_bf16_rows(&tmH, op.H, N, op.cols_h, op.ldh, tc::BM) ||
+      !encode_bf16_rows(&tmW, op.W, V, op.cols_w, op.ldw, pair ? tc2::HALF_N : tc::BN))
     return FLCE_ERR_UNSUPPORTED;
   tc::Args a;
   a.y = y;
@@ -209,16 +238,19 @@ flce_status launch_contraction(const void* opH, int64_t ldh, int64_t Kh, const v
   a.hdr = hdr;
   a.N = int32_t(N);
   a.V = int32_t(V);
-  a.D = int32_t(K);
-  a.kblocks = int32_t(cdiv(K, tc::BK));
-  a.kblocks_h = int32_t(cdiv(Kh, tc::BK));
-  a.kblocks_w = int32_t(cdiv(Kw, tc::BK));
+  a.D = int32_t(op.kblocks * tc::BK);
+  a.kblocks = int32_t(op.kblocks);
+  a.seg_h = int32_t(op.seg_h);
+  a.seg_w = int32_t(op.seg_w);
   a.sch = sch;
   a.wait_limit_ns = kDefaultWaitLimitNs;
-  if (pair)
-    tc2::flce_tc2_kernel<<<plan.grid, tc2::NUM_THREADS, tc2::SMEM_BYTES, st>>>(tmH, tmW, a);
-  else
-    tc::flce_tc_kernel<<<plan.grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(tmH, tmW, a);
+  const unsigned grid = unsigned(plan.grid);
+  switch (op.layout) {
+    case tc::kPlain: launch_contraction_kernel<tc::kPlain>(pair, grid, tmH, tmW, a, st); break;
+    case tc::kSplitW: launch_contraction_kernel<tc::kSplitW>(pair, grid, tmH, tmW, a, st); break;
+    case tc::kSplitHW: launch_contraction_kernel<tc::kSplitHW>(pair, grid, tmH, tmW, a, st); break;
+    default: return FLCE_ERR_INVALID_ARG;
+  }
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
@@ -258,27 +290,19 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
   make_plan(N, V, D, dtype, workers, &plan);
 
   // The operands the tensor-core kernels read: H and W themselves (bf16), or
-  // their split copies in the workspace (fp32): H as [hi | hi | lo] and W as
-  // [hi | lo], K = 3 Dp with W's K coordinate wrapping after 2 Dp.
-  const void* opH = H;
-  const void* opW = W;
-  int64_t K = D, Kw = D;
+  // their [hi | lo] split copies in the workspace (fp32), each K block's four
+  // parts staged together for the three products hi hi + hi lo + lo hi.
+  Operands op{H, ldh, D, 0, W, ldw, D, 0, cdiv(D, tc::BK), tc::kPlain};
   if (dtype == FLCE_FP32) {
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     const int64_t Dp = fwd_split_segment(D);
-    K = 3 * Dp;
-    Kw = 2 * Dp;
     uint8_t* hs = wsb + state_bytes_for(N, V);
     uint8_t* wsplit = hs + fwd_split_h_bytes(N, D);
-    if ((s = launch_split(H, ldh, N, D, Dp, 3, 2, hs, di.sms, st)) != FLCE_OK) return s;
+    if ((s = launch_split(H, ldh, N, D, Dp, 2, 1, hs, di.sms, st)) != FLCE_OK) return s;
     if ((s = launch_split(W, ldw, V, D, Dp, 2, 1, wsplit, di.sms, st)) != FLCE_OK) return s;
-    opH = hs;
-    opW = wsplit;
-    ldh = K;
-    ldw = Kw;
+    op = Operands{hs, 2 * Dp, 2 * Dp, Dp, wsplit, 2 * Dp, 2 * Dp, Dp, Dp / tc::BK, tc::kSplitHW};
   }
-  return launch_contraction(opH, ldh, K, opW, ldw, Kw, K, y, y_offset, N, V, plan, out_target, ws,
-                            true, st);
+  return launch_contraction(op, y, y_offset, N, V, plan, out_target, ws, true, st);
 }
 
 flce_status launch_merge(Targets y, int64_t N, int64_t V, float* out_loss, float* out_lse,
@@ -916,9 +940,10 @@ extern "C" flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
       return s;
     flce_plan_t plan;
     make_plan(N, rows, D, FLCE_BF16, workers, &plan);
-    // [H | H] against [hi | lo]: H's K coordinate wraps after Ds.
-    if ((s = launch_contraction(H, D, D, expanded, 2 * Ds, 2 * Ds, 2 * Ds, Targets{y, 0}, c0, N,
-                                rows, plan, out_target_logit, workspace, false, st)) != FLCE_OK)
+    // H against the chunk's [hi | lo] rows: H W_hi^T + H W_lo^T per K block
+    const Operands op{H, D, D, 0, expanded, 2 * Ds, 2 * Ds, Ds, Ds / tc::BK, tc::kSplitW};
+    if ((s = launch_contraction(op, Targets{y, 0}, c0, N, rows, plan, out_target_logit, workspace,
+                                false, st)) != FLCE_OK)
       return s;
     flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
         reinterpret_cast<const float2*>(wsb + kHeaderBytes), hdr, y, int32_t(N), c0, rows,
@@ -1174,8 +1199,9 @@ extern "C" flce_status flce_forward_host(const void* H_host, const void* W_host,
       return FLCE_ERR_CUDA;
     flce_plan_t plan;
     make_plan(N, rows, D, FLCE_BF16, workers, &plan);
-    if ((s = launch_contraction(Hd, D, D, staging[b], D, D, D, Targets{yd, 0}, c0, N, rows, plan,
-                                tgt_d, workspace, false, st)) != FLCE_OK)
+    const Operands op{Hd, D, D, 0, staging[b], D, D, 0, cdiv(D, tc::BK), tc::kPlain};
+    if ((s = launch_contraction(op, Targets{yd, 0}, c0, N, rows, plan, tgt_d, workspace, false,
+                                st)) != FLCE_OK)
       return s;
     flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
         reinterpret_cast<const float2*>(wsb + kHeaderBytes), hdr, yd, int32_t(N), c0, rows,

@@ -18,10 +18,12 @@
 //   * flce_tc2_kernel: the same on CTA pairs (cta_group::2, 256x256 tiles,
 //     6-stage ring): each CTA stages its own 128 token rows and half of the
 //     W tile, the even CTA issues the pair MMAs.  Used for N > 128.
-//   * flce_split3_kernel: for fp32 inputs, splits H and W into bf16 hi/lo
-//     parts laid out along a tripled K axis, so that the same tensor-core
-//     kernels compute the three-product fp32 emulation Hhi Whi + Hhi Wlo +
-//     Hlo Whi.
+//   * Both are templates on the stage layout (tc::StageLayout): one H and one
+//     W block per K block for bf16 inputs; H with W's hi and lo blocks for a
+//     quantised head (two products); H's and W's hi and lo blocks for fp32
+//     inputs (three products, Hhi Whi + Hhi Wlo + Hlo Whi).
+//   * flce_split3_kernel: for fp32 inputs, splits H and W into bf16 [hi | lo]
+//     rows for the split layout (three segments for the backward's GEMMs).
 //   * flce_dequant_split_kernel: expands one chunk of an affine
 //     group-quantised head into bf16 [hi | lo] rows for the same kernels.
 //   * flce_merge_kernel: combines the P slab states of each token in a fixed
@@ -210,18 +212,50 @@ __device__ __forceinline__ void fold_tile(uint32_t taddr, int ncols, int64_t rel
 
 namespace tc {
 
+// What one pipeline stage holds for one 64-wide K block, and the products the
+// MMA issuer forms from it into the tile's accumulator:
+//   kPlain    H and W blocks: H W^T (bf16 inputs).
+//   kSplitW   H, W_hi, W_lo: H W_hi^T + H W_lo^T (a quantised head expanded to
+//             bf16 hi + lo; H is staged once for both products).
+//   kSplitHW  H_hi, H_lo, W_hi, W_lo: hi hi + hi lo + lo hi (fp32 inputs split
+//             into bf16 hi + lo, the bf16x3 scheme; four blocks feed three
+//             products, and every block is used while it is in shared memory).
+// The lo blocks come from the same tensor maps as the hi blocks, `seg_h` /
+// `seg_w` elements further along the row.
+enum StageLayout : int { kPlain = 0, kSplitW = 1, kSplitHW = 2 };
+
+template <int L>
+struct Layout {
+  static constexpr int NA = L == kSplitHW ? 2 : 1;                    // H blocks per stage
+  static constexpr int NB = L == kPlain ? 1 : 2;                      // W blocks per stage
+  static constexpr int NP = L == kPlain ? 1 : (L == kSplitW ? 2 : 3); // products per stage
+  // product p reads H block pa(p) and W block pb(p)
+  static __device__ __forceinline__ int pa(int p) { return (L == kSplitHW && p == 2) ? 1 : 0; }
+  static __device__ __forceinline__ int pb(int p) { return p == 1 ? 1 : 0; }
+};
+
+// Pipeline depth for a stage of `stage_bytes`: as many as fit in 192 KiB.
+constexpr int stages_for(int stage_bytes) { return (192 * 1024) / stage_bytes; }
+
 constexpr int BM = 128;                      // tokens per tile (UMMA M, TMEM lanes)
 constexpr int BN = kTileCols;                // vocab columns per tile (UMMA N)
 constexpr int BK = 64;                       // bf16 per K block = 128 B = one swizzle row
 constexpr int UMMA_K = 16;                   // K per tcgen05.mma (32 bytes)
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;         // 16 KiB
-constexpr int B_BYTES = BN * BK * 2;         // 32 KiB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int A_BYTES = BM * BK * 2;         // 16 KiB per H block
+constexpr int B_BYTES = BN * BK * 2;         // 32 KiB per W block
 constexpr int NUM_THREADS = 192;             // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int EPI_WARPS = 4;
 constexpr uint32_t TMEM_COLS = 512;          // two BN-column fp32 accumulators
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+// Stage geometry per layout: 4 stages of 48 KiB (kPlain), 2 of 80 KiB
+// (kSplitW), 2 of 96 KiB (kSplitHW).
+template <int L>
+struct Cfg {
+  static constexpr int STAGE_BYTES = Layout<L>::NA * A_BYTES + Layout<L>::NB * B_BYTES;
+  static constexpr int STAGES = stages_for(STAGE_BYTES);
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(STAGES >= 2 && 2 * STAGES + 6 <= 32, "stage ring and barriers");
+};
 
 // Instruction descriptor of tcgen05.mma kind::f16: D fp32 (bits 4-5 = 1),
 // A and B bf16 (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0),
@@ -246,18 +280,20 @@ struct Args {
   float* target_logit;     // [N]
   WsHeader* hdr;
   int32_t N, V, D;
-  int32_t kblocks;         // K-blocks per tile: ceil(K / BK)
-  int32_t kblocks_h;       // K-blocks of H; H's K coordinate wraps modulo this
-                           // (== kblocks, except for the quantised head's [H | H])
-  int32_t kblocks_w;       // K-blocks of W; W's K coordinate wraps modulo this
-                           // (== kblocks, except for fp32 inputs' [hi | lo] W)
+  int32_t kblocks;         // K-blocks per tile: ceil(K / BK) over one (hi) segment
+  int32_t seg_h;           // split layouts: column of H's lo block 0 (elements); else 0
+  int32_t seg_w;           // split layouts: column of W's lo block 0 (elements); else 0
   Schedule sch;
   uint64_t wait_limit_ns;
 };
 
+template <int L>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW,
                const Args a) {
+  using LY = Layout<L>;
+  constexpr int STAGES = Cfg<L>::STAGES;
+  constexpr int STAGE_BYTES = Cfg<L>::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the swizzle atoms
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -320,7 +356,7 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
         int slab, tb, t0, nt;
         unit_coords(sch, u, slab, tb, t0, nt);
         for (int t = t0; ok && t < t0 + nt; ++t) {
-          for (int kb = 0, kh = 0, kw = 0; kb < a.kblocks; ++kb) {
+          for (int kb = 0; kb < a.kblocks; ++kb) {
             if (!wait_bounded(ptx::smem_addr(&empty_bar[stage]), phase ^ 1u, abort_flag, status, lim)) {
               ok = false;
               break;
@@ -328,10 +364,13 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
             const uint32_t fb = ptx::smem_addr(&full_bar[stage]);
             const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
             ptx::mbar_arrive_expect_tx(fb, STAGE_BYTES);
-            ptx::tma_load_2d(sa, &tmH, fb, kh * BK, tb * BM);
-            ptx::tma_load_2d(sa + A_BYTES, &tmW, fb, kw * BK, t * BN);
-            if (++kh == a.kblocks_h) kh = 0;
-            if (++kw == a.kblocks_w) kw = 0;
+#pragma unroll
+            for (int i = 0; i < LY::NA; ++i)
+              ptx::tma_load_2d(sa + i * A_BYTES, &tmH, fb, kb * BK + i * a.seg_h, tb * BM);
+#pragma unroll
+            for (int i = 0; i < LY::NB; ++i)
+              ptx::tma_load_2d(sa + LY::NA * A_BYTES + i * B_BYTES, &tmW, fb, kb * BK + i * a.seg_w,
+                               t * BN);
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) {
@@ -373,10 +412,15 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
             ptx::tc_fence_after_sync();
             const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
 #pragma unroll
-            for (int k = 0; k < BK / UMMA_K; ++k) {
-              const uint64_t ad = sw128_desc(sa + k * UMMA_K * 2);
-              const uint64_t bd = sw128_desc(sa + A_BYTES + k * UMMA_K * 2);
-              ptx::mma_bf16(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+            for (int p = 0; p < LY::NP; ++p) {
+              const uint32_t sa_a = sa + LY::pa(p) * A_BYTES;
+              const uint32_t sa_b = sa + LY::NA * A_BYTES + LY::pb(p) * B_BYTES;
+#pragma unroll
+              for (int k = 0; k < BK / UMMA_K; ++k) {
+                const uint64_t ad = sw128_desc(sa_a + k * UMMA_K * 2);
+                const uint64_t bd = sw128_desc(sa_b + k * UMMA_K * 2);
+                ptx::mma_bf16(d_tmem, ad, bd, kIdesc, (kb | p | k) != 0 ? 1u : 0u);
+              }
             }
             ptx::mma_commit(ptx::smem_addr(&empty_bar[stage]));  // slot free once read
             if (++stage == STAGES) {
@@ -467,24 +511,36 @@ constexpr int BN = kTileCols;                // vocab columns per tile (UMMA N)
 constexpr int HALF_N = BN / 2;               // W rows staged by each CTA
 constexpr int BK = 64;
 constexpr int UMMA_K = 16;
-constexpr int STAGES = 6;
-constexpr int A_BYTES = BM * BK * 2;         // 16 KiB
-constexpr int B_BYTES = HALF_N * BK * 2;     // 16 KiB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr uint32_t PAIR_TX_BYTES = 2 * STAGE_BYTES;  // both CTAs' copies complete on the even CTA
+constexpr int A_BYTES = BM * BK * 2;         // 16 KiB per H block
+constexpr int B_BYTES = HALF_N * BK * 2;     // 16 KiB per W block (this CTA's half of the tile)
 constexpr int NUM_THREADS = 192;             // warp 0 TMA, warp 1 MMA (even CTA), warps 2..5 epilogue
 constexpr int EPI_WARPS = 4;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr uint16_t kPairMask = 0x3;
+
+// Stage geometry per layout: 6 stages of 32 KiB (kPlain), 4 of 48 KiB
+// (kSplitW), 3 of 64 KiB (kSplitHW); both CTAs' copies of a stage complete
+// on the even CTA's barrier.
+template <int L>
+struct Cfg {
+  static constexpr int STAGE_BYTES = tc::Layout<L>::NA * A_BYTES + tc::Layout<L>::NB * B_BYTES;
+  static constexpr int STAGES = tc::stages_for(STAGE_BYTES);
+  static constexpr uint32_t PAIR_TX_BYTES = 2 * STAGE_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+  static_assert(STAGES >= 2 && 2 * STAGES + 6 <= 32, "stage ring and barriers");
+};
 
 // kind::f16 descriptor as in the single-CTA kernel, with M = 256 (bits 24-28).
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
                             (uint32_t(PAIR_M >> 4) << 24);
 
+template <int L>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW,
                 const tc::Args a) {
+  using LY = tc::Layout<L>;
+  constexpr int STAGES = Cfg<L>::STAGES;
+  constexpr int STAGE_BYTES = Cfg<L>::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -551,7 +607,7 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
         const int hrow = tb * PAIR_M + int(rank) * BM;
         for (int t = t0; ok && t < t0 + nt; ++t) {
           const int wrow = t * BN + int(rank) * HALF_N;
-          for (int kb = 0, kh = 0, kw = 0; kb < a.kblocks; ++kb) {
+          for (int kb = 0; kb < a.kblocks; ++kb) {
             if (!wait_bounded(ptx::smem_addr(&empty_bar[stage]), phase ^ 1u, abort_flag, status,
                               lim)) {
               ok = false;
@@ -560,11 +616,14 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
             const uint32_t fb_local = ptx::smem_addr(&full_bar[stage]);
             const uint32_t fb_even = ptx::map_to_cta(fb_local, 0);
             const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
-            if (rank == 0) ptx::mbar_arrive_expect_tx(fb_local, PAIR_TX_BYTES);
-            ptx::tma_load_2d_pair(sa, &tmH, fb_even, kh * BK, hrow);
-            ptx::tma_load_2d_pair(sa + A_BYTES, &tmW, fb_even, kw * BK, wrow);
-            if (++kh == a.kblocks_h) kh = 0;
-            if (++kw == a.kblocks_w) kw = 0;
+            if (rank == 0) ptx::mbar_arrive_expect_tx(fb_local, Cfg<L>::PAIR_TX_BYTES);
+#pragma unroll
+            for (int i = 0; i < LY::NA; ++i)
+              ptx::tma_load_2d_pair(sa + i * A_BYTES, &tmH, fb_even, kb * BK + i * a.seg_h, hrow);
+#pragma unroll
+            for (int i = 0; i < LY::NB; ++i)
+              ptx::tma_load_2d_pair(sa + LY::NA * A_BYTES + i * B_BYTES, &tmW, fb_even,
+                                    kb * BK + i * a.seg_w, wrow);
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) {
@@ -609,10 +668,15 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
             ptx::tc_fence_after_sync();
             const uint32_t sa = ptx::smem_addr(smem + stage * STAGE_BYTES);
 #pragma unroll
-            for (int k = 0; k < BK / UMMA_K; ++k) {
-              const uint64_t ad = tc::sw128_desc(sa + k * UMMA_K * 2);
-              const uint64_t bd = tc::sw128_desc(sa + A_BYTES + k * UMMA_K * 2);
-              ptx::mma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+            for (int p = 0; p < LY::NP; ++p) {
+              const uint32_t sa_a = sa + LY::pa(p) * A_BYTES;
+              const uint32_t sa_b = sa + LY::NA * A_BYTES + LY::pb(p) * B_BYTES;
+#pragma unroll
+              for (int k = 0; k < BK / UMMA_K; ++k) {
+                const uint64_t ad = tc::sw128_desc(sa_a + k * UMMA_K * 2);
+                const uint64_t bd = tc::sw128_desc(sa_b + k * UMMA_K * 2);
+                ptx::mma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb | p | k) != 0 ? 1u : 0u);
+              }
             }
             ptx::mma_commit_pair_mc(ptx::smem_addr(&empty_bar[stage]), kPairMask);
             if (++stage == STAGES) {
@@ -695,14 +759,14 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
 // every value into two bf16 values (Henry, Tang and Heinecke, "Leveraging
 // the bfloat16 artificial intelligence datatype for higher-precision
 // computations", ARITH 2019):  hi = bf16(x),  lo = bf16(x - hi),  so that
-// |x - hi - lo| <= 2^-16 |x|.  Laying H out as [hi | hi | lo] and W as
-// [hi | lo] along K (segments of Dp = D rounded up to 64, zero padded), with
-// W's K coordinate wrapping after its two segments, turns one bf16
-// contraction over 3 Dp into
+// |x - hi - lo| <= 2^-16 |x|.  The forward lays H and W out as [hi | lo]
+// rows (segments of Dp = D rounded up to 64, zero padded); the contraction
+// kernels stage the four parts of each K block together (tc::kSplitHW) and
+// accumulate
 //   Z = Hhi Whi^T + Hhi Wlo^T + Hlo Whi^T
-// with fp32 accumulation in TMEM: each product h w is off by at most about
-// 3 * 2^-16 |h w| (the dropped lo*lo term and the two rounding residues).
-// (The backward lays W out as [hi | lo | hi] instead: its GEMM wraps only A.)
+// in fp32 in TMEM: each product h w is off by at most about 3 * 2^-16 |h w|
+// (the dropped lo*lo term and the two rounding residues).  (The backward lays
+// H out as [hi | hi | lo] and W as [hi | lo | hi] and walks K = 3 segments.)
 namespace split {
 
 constexpr int NUM_THREADS = 256;   // 8 warps, one row per warp at a time
@@ -781,8 +845,9 @@ __global__ void __launch_bounds__(NUM_THREADS) flce_split3_kernel(const Args a) 
 // One chunk of vocabulary rows at a time is expanded into the layout the
 // tensor-core kernels read: per row two K segments of Ds = D rounded up to 64,
 // [hi | lo] with hi = bf16(W_jk) and lo = bf16(W_jk - hi) (zero padded from D
-// to Ds).  H is bf16 already, so H [hi | lo]^T over K = 2 Ds (H's K coordinate
-// wraps after Ds) is H W^T up to |W - hi - lo| <= 2^-16 |W| per weight.
+// to Ds).  H is bf16 already: the contraction kernels stage each K block of H
+// once beside both parts of W (tc::kSplitW) and accumulate H hi^T + H lo^T,
+// which is H W^T up to |W - hi - lo| <= 2^-16 |W| per weight.
 namespace quant {
 
 constexpr int NUM_THREADS = 256;   // 8 warps, one vocabulary row per warp at a time

@@ -29,23 +29,23 @@ size_t state_bytes_for(int64_t N, int64_t V) {
   return kHeaderBytes + part + sums;
 }
 
-// fp32 inputs run on bf16 hi / lo parts.  The forward lays H out as
-// [hi | hi | lo] and W as [hi | lo] (the kernel wraps W's K coordinate after
-// two segments), so a segment must end on a 64-element K block: D rounded up
-// to 64.  The backward lays both out in three segments of D rounded up to 8.
+// fp32 inputs run on bf16 hi / lo parts.  The forward lays H and W out as
+// [hi | lo] rows (the kernel stages a K block of each part side by side), so a
+// segment must end on a 64-element K block: D rounded up to 64.  The backward
+// lays both out in three segments of D rounded up to 8.
 int64_t fwd_split_segment(int64_t D) { return (D + 63) / 64 * 64; }
 int64_t bwd_split_segment(int64_t D) { return (D + 7) / 8 * 8; }
 
-// Length of the bf16 K axis the forward's tensor-core kernels walk: D for
-// bf16 inputs, three hi / lo segments for fp32 inputs.
+// bf16 elements per row of the operands the forward's tensor-core kernels
+// stage: D for bf16 inputs, the hi and lo segments for fp32 inputs.
 int64_t k_extent(int64_t D, flce_dtype dtype) {
-  return dtype == FLCE_FP32 ? 3 * fwd_split_segment(D) : D;
+  return dtype == FLCE_FP32 ? 2 * fwd_split_segment(D) : D;
 }
 
-// Workspace for the forward's split copies of fp32 inputs: H (N, 3 Dp) and
+// Workspace for the forward's split copies of fp32 inputs: H (N, 2 Dp) and
 // W (V, 2 Dp) bf16, each 256-byte aligned.
 size_t fwd_split_h_bytes(int64_t N, int64_t D) {
-  return align256(size_t(N) * size_t(3 * fwd_split_segment(D)) * 2);
+  return align256(size_t(N) * size_t(2 * fwd_split_segment(D)) * 2);
 }
 size_t fwd_split_w_bytes(int64_t V, int64_t D) {
   return align256(size_t(V) * size_t(2 * fwd_split_segment(D)) * 2);

@@ -61,12 +61,12 @@ def test_workspace_is_O_N_not_O_NV(lib):
     assert lib.flce_workspace_size(4, 10, 8, 7) == 0
     # bf16: independent of D
     assert flce.workspace_size(100, 5000, 64) == flce.workspace_size(100, 5000, 4096)
-    # fp32: plus the bf16 hi/lo split copies, H (N, 3 Dp) and W (V, 2 Dp), Dp = ceil64(D)
+    # fp32: plus the bf16 hi/lo split copies, H (N, 2 Dp) and W (V, 2 Dp), Dp = ceil64(D)
     for N, V, D in [(100, 5000, 64), (256, 2048, 256), (7, 9, 5), (1, 1, 1), (3, 4, 65)]:
         Dp = (D + 63) // 64 * 64
         r256 = lambda b: (b + 255) // 256 * 256
         assert flce.workspace_size(N, V, D, 1) == (flce.workspace_size(N, V, D)
-                                                   + r256(6 * Dp * N) + r256(4 * Dp * V))
+                                                   + r256(4 * Dp * N) + r256(4 * Dp * V))
 
 
 def unit_order(p):

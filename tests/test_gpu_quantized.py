@@ -3,7 +3,7 @@
 The head is MLX's affine group format, W = s * q + b per group of G along D
 (the page's section 2 mentions quantised heads without a format; this is the
 reading the library and the oracle both take).  The GPU expands W to bf16
-[hi | lo] and contracts [H | H] against it: per weight |W - hi - lo| <=
+[hi | lo] and forms H hi^T + H lo^T per K block: per weight |W - hi - lo| <=
 2^-16 |W|, so the bar is the forward's: |d loss|, |d lse| <= 1e-3 per token,
 |d mean| / |mean| <= 1e-5.
 """
