@@ -156,7 +156,12 @@ flce_status make_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int64_t
   p->token_blocks = cdiv(std::max<int64_t>(N, 1), p->block_rows);
   p->vocab_tiles = cdiv(V, kTileCols);
   const int64_t g = std::max<int64_t>(1, workers);
-  p->group_blocks = int32_t(group_blocks_for(p->token_blocks, p->block_rows, k_extent(D, dtype), 2));
+  // Sized by the bf16 rows of H (for fp32 inputs: their hi parts).  fp32's
+  // [hi | lo] rows hold twice the bytes per block, yet at N=8192 V=151936
+  // D=4096 a group of 16 blocks (64 MB of H) measured faster than one sized by
+  // the full rows (7 blocks: 23.1-23.5 against 24.6-25.2 ms; DRAM reads 30.1
+  // against 35.4 GB per launch): fewer slabs in flight share each W tile.
+  p->group_blocks = int32_t(group_blocks_for(p->token_blocks, p->block_rows, D, 2));
   int64_t ms = 0;
   choose_slabs(p->token_blocks, p->group_blocks, p->vocab_tiles, g, slab_capacity(V), p->slabs,
                ms);
