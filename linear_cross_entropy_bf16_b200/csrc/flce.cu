@@ -119,6 +119,7 @@ flce_status set_smem_limits() {
   flce_status s = set_smem_limits_for<tc::kPlain>();
   if (s == FLCE_OK) s = set_smem_limits_for<tc::kSplitW>();
   if (s == FLCE_OK) s = set_smem_limits_for<tc::kSplitHW>();
+  if (s == FLCE_OK) s = set_smem_limits_for<tc::kPlain1>();
   return s;
 }
 
@@ -181,11 +182,12 @@ flce_status contraction_workers(int64_t N, DeviceInfo& di, int64_t& workers) {
 }
 
 // The bf16 operands of one contraction: rows of H (N rows) and of W (V rows),
-// `cols_*` columns stored with row stride `ld_*` elements.  The kernel walks
-// `kblocks` 64-element K blocks.  In the split layouts (tc::StageLayout) the
-// lo part of K block kb sits `seg_*` columns after its hi part in the same
-// row: fp32 inputs split into [hi | lo] H and W rows (kSplitHW), a quantised
-// head expanded into [hi | lo] W rows against H itself (kSplitW).
+// `cols_*` columns stored with row stride `ld_*` elements.  The kernel runs
+// `kblocks` pipeline stages per tile (tc::StageLayout): kPlain stages K
+// blocks 2j and 2j + 1 (seg_* = 64, the next block); in the split layouts the
+// lo part of K block kb sits seg_* columns after its hi part in the same row:
+// fp32 inputs split into [hi | lo] H and W rows (kSplitHW), a quantised head
+// expanded into [hi | lo] W rows against H itself (kSplitW).
 struct Operands {
   const void* H;
   int64_t ldh, cols_h, seg_h;
@@ -194,6 +196,20 @@ struct Operands {
   int64_t kblocks;
   int layout;  // tc::StageLayout
 };
+
+// Batches of at most this many tokens stream W from HBM faster than the
+// tensor cores consume it, so they run the one-K-block ring (tc::kPlain1);
+// larger ones stage two K blocks per stage (tc::kPlain).  At V=151936
+// D=4096 on B200 the one-block ring streamed W 2-6% faster at N = 1..256, and
+// the two-block ring ran the N=8192 forward 6.5% faster.
+constexpr int64_t kStreamBoundTokens = 256;
+
+Operands bf16_operands(const void* H, int64_t ldh, const void* W, int64_t ldw, int64_t N,
+                       int64_t D) {
+  if (N <= kStreamBoundTokens)
+    return Operands{H, ldh, D, 0, W, ldw, D, 0, cdiv(D, tc::BK), tc::kPlain1};
+  return Operands{H, ldh, D, tc::BK, W, ldw, D, tc::BK, cdiv(D, 2 * tc::BK), tc::kPlain};
+}
 
 template <int L>
 void launch_contraction_kernel(bool pair, unsigned grid, const CUtensorMap& tmH,
@@ -249,6 +265,7 @@ flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, 
     case tc::kPlain: launch_contraction_kernel<tc::kPlain>(pair, grid, tmH, tmW, a, st); break;
     case tc::kSplitW: launch_contraction_kernel<tc::kSplitW>(pair, grid, tmH, tmW, a, st); break;
     case tc::kSplitHW: launch_contraction_kernel<tc::kSplitHW>(pair, grid, tmH, tmW, a, st); break;
+    case tc::kPlain1: launch_contraction_kernel<tc::kPlain1>(pair, grid, tmH, tmW, a, st); break;
     default: return FLCE_ERR_INVALID_ARG;
   }
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
@@ -292,7 +309,7 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
   // The operands the tensor-core kernels read: H and W themselves (bf16), or
   // their [hi | lo] split copies in the workspace (fp32), each K block's four
   // parts staged together for the three products hi hi + hi lo + lo hi.
-  Operands op{H, ldh, D, 0, W, ldw, D, 0, cdiv(D, tc::BK), tc::kPlain};
+  Operands op = bf16_operands(H, ldh, W, ldw, N, D);
   if (dtype == FLCE_FP32) {
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     const int64_t Dp = fwd_split_segment(D);
@@ -1199,7 +1216,7 @@ extern "C" flce_status flce_forward_host(const void* H_host, const void* W_host,
       return FLCE_ERR_CUDA;
     flce_plan_t plan;
     make_plan(N, rows, D, FLCE_BF16, workers, &plan);
-    const Operands op{Hd, D, D, 0, staging[b], D, D, 0, cdiv(D, tc::BK), tc::kPlain};
+    const Operands op = bf16_operands(Hd, D, staging[b], D, N, D);
     if ((s = launch_contraction(op, Targets{yd, 0}, c0, N, rows, plan, tgt_d, workspace, false,
                                 st)) != FLCE_OK)
       return s;

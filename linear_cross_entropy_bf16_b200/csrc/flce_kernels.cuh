@@ -10,18 +10,19 @@
 // B200 design (not the page's one-dispatch-per-tile chain):
 //   * flce_tc_kernel: a persistent, warp-specialised tcgen05 GEMM.  One CTA
 //     per SM walks work units (128 tokens x one vocab slab of 256-column
-//     tiles).  Warp 0 streams H and W K-blocks with TMA into a 4-stage
-//     shared-memory ring, warp 1 issues 128x256x16 bf16 MMAs into a
+//     tiles).  Warp 0 streams H and W K-blocks with TMA into a shared-memory
+//     ring (192 KiB), warp 1 issues 128x256x16 bf16 MMAs into a
 //     double-buffered fp32 TMEM accumulator, and warps 2-5 (one TMEM lane,
 //     i.e. one token, per thread) fold each finished tile into (m, s) and
 //     capture the target logit.  Logits never leave TMEM/registers.
-//   * flce_tc2_kernel: the same on CTA pairs (cta_group::2, 256x256 tiles,
-//     6-stage ring): each CTA stages its own 128 token rows and half of the
+//   * flce_tc2_kernel: the same on CTA pairs (cta_group::2, 256x256 tiles):
+//     each CTA stages its own 128 token rows and half of the
 //     W tile, the even CTA issues the pair MMAs.  Used for N > 128.
-//   * Both are templates on the stage layout (tc::StageLayout): one H and one
-//     W block per K block for bf16 inputs; H with W's hi and lo blocks for a
-//     quantised head (two products); H's and W's hi and lo blocks for fp32
-//     inputs (three products, Hhi Whi + Hhi Wlo + Hlo Whi).
+//   * Both are templates on the stage layout (tc::StageLayout): H and W
+//     blocks of two consecutive K blocks per stage for bf16 inputs; H with
+//     W's hi and lo blocks for a quantised head (two products); H's and W's
+//     hi and lo blocks for fp32 inputs (three products, Hhi Whi + Hhi Wlo +
+//     Hlo Whi).
 //   * flce_split3_kernel: for fp32 inputs, splits H and W into bf16 [hi | lo]
 //     rows for the split layout (three segments for the backward's GEMMs).
 //   * flce_dequant_split_kernel: expands one chunk of an affine
@@ -212,26 +213,38 @@ __device__ __forceinline__ void fold_tile(uint32_t taddr, int ncols, int64_t rel
 
 namespace tc {
 
-// What one pipeline stage holds for one 64-wide K block, and the products the
-// MMA issuer forms from it into the tile's accumulator:
-//   kPlain    H and W blocks: H W^T (bf16 inputs).
-//   kSplitW   H, W_hi, W_lo: H W_hi^T + H W_lo^T (a quantised head expanded to
-//             bf16 hi + lo; H is staged once for both products).
-//   kSplitHW  H_hi, H_lo, W_hi, W_lo: hi hi + hi lo + lo hi (fp32 inputs split
-//             into bf16 hi + lo, the bf16x3 scheme; four blocks feed three
-//             products, and every block is used while it is in shared memory).
-// The lo blocks come from the same tensor maps as the hi blocks, `seg_h` /
-// `seg_w` elements further along the row.
-enum StageLayout : int { kPlain = 0, kSplitW = 1, kSplitHW = 2 };
+// What one pipeline stage holds (64-column K blocks of H and W, 128 B swizzle
+// rows) and the products the MMA issuer forms from it into the tile's
+// accumulator, each product being four 16-deep MMAs:
+//   kPlain    H and W blocks of two consecutive K blocks: H W^T over 128 K
+//             columns per stage (bf16 inputs).  Two products per barrier
+//             round trip: with one K block per stage the tensor pipe idled
+//             about 9% of its active cycles between stages, and the headline
+//             forward ran 6.5% slower.
+//   kSplitW   H, W_hi, W_lo of one K block: H W_hi^T + H W_lo^T (a quantised
+//             head expanded to bf16 hi + lo; H is staged once for both).
+//   kSplitHW  H_hi, H_lo, W_hi, W_lo of one K block: hi hi + hi lo + lo hi
+//             (fp32 inputs split into bf16 hi + lo, the bf16x3 scheme; four
+//             blocks feed three products while they are in shared memory).
+//   kPlain1   H and W blocks of one K block (bf16 inputs, batches small
+//             enough that streaming W from HBM bounds the contraction: the
+//             deeper ring of smaller stages keeps more bytes in flight).
+// The second block of a pair comes from the same tensor map, `seg_h` /
+// `seg_w` elements further along the row: the next K block (kPlain, 64) or
+// the lo part of the same K block (the split layouts, one segment).
+enum StageLayout : int { kPlain = 0, kSplitW = 1, kSplitHW = 2, kPlain1 = 3 };
 
 template <int L>
 struct Layout {
-  static constexpr int NA = L == kSplitHW ? 2 : 1;                    // H blocks per stage
-  static constexpr int NB = L == kPlain ? 1 : 2;                      // W blocks per stage
-  static constexpr int NP = L == kPlain ? 1 : (L == kSplitW ? 2 : 3); // products per stage
+  static constexpr int NA = (L == kSplitW || L == kPlain1) ? 1 : 2;    // H blocks per stage
+  static constexpr int NB = L == kPlain1 ? 1 : 2;                      // W blocks per stage
+  static constexpr int NP = L == kSplitHW ? 3 : (L == kPlain1 ? 1 : 2); // products per stage
+  static constexpr int KSTEP = L == kPlain ? 128 : 64;                 // K columns per stage
   // product p reads H block pa(p) and W block pb(p)
-  static __device__ __forceinline__ int pa(int p) { return (L == kSplitHW && p == 2) ? 1 : 0; }
-  static __device__ __forceinline__ int pb(int p) { return p == 1 ? 1 : 0; }
+  static __device__ __forceinline__ int pa(int p) {
+    return L == kPlain ? p : ((L == kSplitHW && p == 2) ? 1 : 0);
+  }
+  static __device__ __forceinline__ int pb(int p) { return L == kPlain ? p : (p == 1 ? 1 : 0); }
 };
 
 // Pipeline depth for a stage of `stage_bytes`: as many as fit in 192 KiB.
@@ -247,8 +260,8 @@ constexpr int NUM_THREADS = 192;             // warp 0 TMA, warp 1 MMA, warps 2.
 constexpr int EPI_WARPS = 4;
 constexpr uint32_t TMEM_COLS = 512;          // two BN-column fp32 accumulators
 
-// Stage geometry per layout: 4 stages of 48 KiB (kPlain), 2 of 80 KiB
-// (kSplitW), 2 of 96 KiB (kSplitHW).
+// Stage geometry per layout: 2 stages of 96 KiB (kPlain, kSplitHW), 2 of
+// 80 KiB (kSplitW), 4 of 48 KiB (kPlain1).
 template <int L>
 struct Cfg {
   static constexpr int STAGE_BYTES = Layout<L>::NA * A_BYTES + Layout<L>::NB * B_BYTES;
@@ -280,7 +293,7 @@ struct Args {
   float* target_logit;     // [N]
   WsHeader* hdr;
   int32_t N, V, D;
-  int32_t kblocks;         // K-blocks per tile: ceil(K / BK) over one (hi) segment
+  int32_t kblocks;         // stages per tile: K steps of Layout<L>::KSTEP columns
   int32_t seg_h;           // split layouts: column of H's lo block 0 (elements); else 0
   int32_t seg_w;           // split layouts: column of W's lo block 0 (elements); else 0
   Schedule sch;
@@ -366,11 +379,11 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
             ptx::mbar_arrive_expect_tx(fb, STAGE_BYTES);
 #pragma unroll
             for (int i = 0; i < LY::NA; ++i)
-              ptx::tma_load_2d(sa + i * A_BYTES, &tmH, fb, kb * BK + i * a.seg_h, tb * BM);
+              ptx::tma_load_2d(sa + i * A_BYTES, &tmH, fb, kb * LY::KSTEP + i * a.seg_h, tb * BM);
 #pragma unroll
             for (int i = 0; i < LY::NB; ++i)
-              ptx::tma_load_2d(sa + LY::NA * A_BYTES + i * B_BYTES, &tmW, fb, kb * BK + i * a.seg_w,
-                               t * BN);
+              ptx::tma_load_2d(sa + LY::NA * A_BYTES + i * B_BYTES, &tmW, fb,
+                               kb * LY::KSTEP + i * a.seg_w, t * BN);
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) {
@@ -518,9 +531,9 @@ constexpr int EPI_WARPS = 4;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint16_t kPairMask = 0x3;
 
-// Stage geometry per layout: 6 stages of 32 KiB (kPlain), 4 of 48 KiB
-// (kSplitW), 3 of 64 KiB (kSplitHW); both CTAs' copies of a stage complete
-// on the even CTA's barrier.
+// Stage geometry per layout: 3 stages of 64 KiB (kPlain, kSplitHW), 4 of
+// 48 KiB (kSplitW), 6 of 32 KiB (kPlain1); both CTAs' copies of a stage
+// complete on the even CTA's barrier.
 template <int L>
 struct Cfg {
   static constexpr int STAGE_BYTES = tc::Layout<L>::NA * A_BYTES + tc::Layout<L>::NB * B_BYTES;
@@ -619,11 +632,12 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
             if (rank == 0) ptx::mbar_arrive_expect_tx(fb_local, Cfg<L>::PAIR_TX_BYTES);
 #pragma unroll
             for (int i = 0; i < LY::NA; ++i)
-              ptx::tma_load_2d_pair(sa + i * A_BYTES, &tmH, fb_even, kb * BK + i * a.seg_h, hrow);
+              ptx::tma_load_2d_pair(sa + i * A_BYTES, &tmH, fb_even, kb * LY::KSTEP + i * a.seg_h,
+                                    hrow);
 #pragma unroll
             for (int i = 0; i < LY::NB; ++i)
               ptx::tma_load_2d_pair(sa + LY::NA * A_BYTES + i * B_BYTES, &tmW, fb_even,
-                                    kb * BK + i * a.seg_w, wrow);
+                                    kb * LY::KSTEP + i * a.seg_w, wrow);
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) {
