@@ -184,7 +184,8 @@ flce_status contraction_workers(int64_t N, DeviceInfo& di, int64_t& workers) {
 // The bf16 operands of one contraction: rows of H (N rows) and of W (V rows),
 // `cols_*` columns stored with row stride `ld_*` elements.  The kernel runs
 // `kblocks` pipeline stages per tile (tc::StageLayout): kPlain stages K
-// blocks 2j and 2j + 1 (seg_* = 64, the next block); in the split layouts the
+// blocks 2j and 2j + 1 (seg_* = 64, the next block), kPlain1 one K block
+// (seg_* unused); in the split layouts the
 // lo part of K block kb sits seg_* columns after its hi part in the same row:
 // fp32 inputs split into [hi | lo] H and W rows (kSplitHW), a quantised head
 // expanded into [hi | lo] W rows against H itself (kSplitW).
