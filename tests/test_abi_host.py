@@ -141,6 +141,10 @@ def test_headline_plan(lib):
     assert p["group_blocks"] == 16             # 16 x 2 MB of H live at a time
     assert p["makespan_tiles"] <= 258          # ceil(32 * 594 / 74) = 257 pair tiles
     assert p["slab_rem"] == 0                  # equal slabs (99 x 6 tiles) keep the pairs in step
+    # fp32 inputs: the same schedule; the raster group counts only H's hi part
+    # (16 blocks, not the 7 that the [hi | lo] rows' bytes would allow)
+    q = flce.plan(8192, 151936, 4096, 1, sm_count=148)
+    assert q["group_blocks"] == 16 and q["slabs"] == p["slabs"] and q["units"] == p["units"]
 
 
 def test_plan_rejects_bad_args(lib):
