@@ -135,8 +135,8 @@ FLCE_API flce_status flce_forward(const void* H, const void* W, const int64_t* y
 /* Element type of the targets y in flce_forward_ex. */
 typedef enum { FLCE_INDEX_INT64 = 0, FLCE_INDEX_INT32 = 1 } flce_index_dtype;
 
-/* Arguments of flce_forward_ex: those of flce_forward plus row strides and
- * the target type. */
+/* Arguments of flce_forward_ex: those of flce_forward plus row strides, the
+ * target type and an optional sum of the losses. */
 typedef struct {
   const void* H;            /* (N, D) rows, row stride ldh elements */
   int64_t ldh;              /* >= D; 0 means D.  bf16: a multiple of 8 */
@@ -150,6 +150,8 @@ typedef struct {
   float* out_lse;           /* (N) */
   float* out_target_logit;  /* (N) */
   float* out_mean;          /* (1) or NULL */
+  float* out_sum;           /* (1) or NULL: sum_i out_loss[i], the fp64 total that the
+                               mean divides by N, rounded once to fp32 */
 } flce_forward_args;
 
 /*
@@ -267,14 +269,15 @@ FLCE_API size_t flce_merge_shards_scratch_size(int64_t N);
 
 /* Merges G shard states, laid out [G][N] float4 in shard order (any order
  * gives the same lse up to rounding; a fixed order makes it deterministic),
- * into per-token loss, lse and target logit and the mean (out_mean may be
- * NULL).  A token whose target is outside [0, V_total) or is held by no
+ * into per-token loss, lse and target logit, the mean (out_mean may be
+ * NULL) and the sum of the losses (out_sum may be NULL; the fp64 total that
+ * the mean divides by N, rounded once).  A token whose target is outside [0, V_total) or is held by no
  * shard or by more than one gets NaN and sets FLCE_ERR_TARGET_OUT_OF_RANGE
  * in the scratch status word (read with flce_check(scratch, stream)). */
 FLCE_API flce_status flce_merge_shards(const float* states, int32_t G, const int64_t* y, int64_t N,
                                        int64_t V_total, float* out_loss, float* out_lse,
-                                       float* out_target_logit, float* out_mean, void* scratch,
-                                       size_t scratch_bytes, void* stream);
+                                       float* out_target_logit, float* out_mean, float* out_sum,
+                                       void* scratch, size_t scratch_bytes, void* stream);
 
 /* Waits for `stream`, then reads the workspace status word left by the last
  * flce_forward / flce_partials + flce_merge that used this workspace.
@@ -317,7 +320,11 @@ FLCE_API flce_status flce_selftest_wait_timeout(void* workspace, size_t workspac
  *     that means N <= 16382.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current.  Make that first call
- *     before any stream capture on that device.
+ *     before any stream capture on that device.  The address is cached with
+ *     the id of the CUDA context it belongs to; a call in another context
+ *     (a non-primary context, or the primary context re-created after
+ *     cudaDeviceReset) looks it up again, so it too should come before any
+ *     capture in that context.
  *   - All calls on one device share the array, and it keeps the contents of
  *     the last call.  Each call resets the header words it needs before its
  *     kernels run.  Calls whose work overlaps on the GPU (different streams,
@@ -353,7 +360,9 @@ FLCE_API flce_status flce_forward_noalloc(const void* H, const void* W, const in
  *            in word k / (32/bits) at bit offset bits * (k mod (32/bits)))
  *   scales, biases   (V, D / G) bf16 each, contiguous
  *   bits     2, 4 or 8;  group_size G: 32, 64 or 128;  D a multiple of G
- *   y, N, V, D, out_*      as flce_forward (int64 targets)
+ *   y, N, V, D, out_*      as flce_forward (int64 targets); out_sum (1) fp32 or
+ *            NULL receives the sum of the losses (the fp64 total that the
+ *            mean divides by N, rounded once)
  *   workspace  >= flce_quantized_workspace_size(N, V, D, bits, group_size)
  *            bytes, 256-byte aligned; holds the status word flce_check() reads
  *
@@ -379,7 +388,7 @@ FLCE_API flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
                                             int32_t bits, int32_t group_size, const int64_t* y,
                                             int64_t N, int64_t V, int64_t D, float* out_loss,
                                             float* out_lse, float* out_target_logit,
-                                            float* out_mean, void* workspace,
+                                            float* out_mean, float* out_sum, void* workspace,
                                             size_t workspace_bytes, void* stream);
 
 /*

@@ -77,6 +77,7 @@ class ForwardArgs(ctypes.Structure):
         ("dtype", ctypes.c_int32), ("N", ctypes.c_int64), ("V", ctypes.c_int64),
         ("D", ctypes.c_int64), ("out_loss", ctypes.c_void_p), ("out_lse", ctypes.c_void_p),
         ("out_target_logit", ctypes.c_void_p), ("out_mean", ctypes.c_void_p),
+        ("out_sum", ctypes.c_void_p),
     ]
 
 
@@ -140,7 +141,8 @@ def load_library():
         lib.flce_shard_state.restype = st
         lib.flce_merge_shards_scratch_size.argtypes = [i64]
         lib.flce_merge_shards_scratch_size.restype = sz
-        lib.flce_merge_shards.argtypes = [vp, ctypes.c_int32, vp, i64, i64, vp, vp, vp, vp, vp, sz, vp]
+        lib.flce_merge_shards.argtypes = [vp, ctypes.c_int32, vp, i64, i64, vp, vp, vp, vp, vp, vp, sz,
+                                          vp]
         lib.flce_merge_shards.restype = st
         lib.flce_forward_ex.argtypes = [ctypes.POINTER(ForwardArgs), vp, sz, vp]
         lib.flce_forward_ex.restype = st
@@ -148,7 +150,7 @@ def load_library():
         lib.flce_quantized_workspace_size.argtypes = [i64, i64, i64, i32, i32]
         lib.flce_quantized_workspace_size.restype = sz
         lib.flce_forward_quantized.argtypes = [vp, vp, vp, vp, i32, i32, vp, i64, i64, i64,
-                                               vp, vp, vp, vp, vp, sz, vp]
+                                               vp, vp, vp, vp, vp, vp, sz, vp]
         lib.flce_forward_quantized.restype = st
         lib.flce_backward_shard.argtypes = [vp, vp, vp, vp, vp, ctypes.c_float, i64, i64, i64, i64,
                                             i64, ctypes.c_int, vp, vp, vp, sz, vp, vp]
@@ -257,6 +259,19 @@ def _alloc_outputs(N, device, out):
     return loss, lse, tgt, mean
 
 
+def _sum_output(N, device, out):
+    """Device pointer of out["sum"] (a 0-d fp32 tensor that receives the sum of the
+    losses), or None; with N == 0 the sum is written here as 0."""
+    t = (out or {}).get("sum")
+    if t is None:
+        return None
+    if t.dtype != torch.float32 or t.device != device or t.numel() != 1:
+        raise ValueError("out['sum'] must be a one-element float32 tensor on the input device")
+    if N == 0:
+        t.zero_()
+    return t.data_ptr()
+
+
 def _workspace(N, V, D, code, device, workspace):
     need = load_library().flce_workspace_size(int(N), int(V), int(D), code)
     if workspace is None:
@@ -348,7 +363,9 @@ def backward(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, lse: torch.Tenso
 def forward_strided(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, *, out: dict | None = None,
                     workspace: torch.Tensor | None = None, stream=None, check: bool = False):
     """flce_forward_ex: like forward(), for H and W whose rows are strided (each row
-    contiguous, row stride >= D) and int32 or int64 targets."""
+    contiguous, row stride >= D) and int32 or int64 targets.  ``out["sum"]`` (a 0-d
+    fp32 tensor) also receives the sum of the losses, from the same fp64 total as the
+    mean."""
     for name, t in (("H", H), ("W", W)):
         if not t.is_cuda or t.dim() != 2 or t.stride(1) != 1 or t.stride(0) < t.shape[1]:
             raise ValueError(f"{name} must be a 2-D CUDA tensor with contiguous rows")
@@ -361,12 +378,13 @@ def forward_strided(H: torch.Tensor, W: torch.Tensor, y: torch.Tensor, *, out: d
     code = _dtype_code(H)
     dev = H.device
     loss, lse, tgt, mean = _alloc_outputs(N, dev, out)
+    sum_ptr = _sum_output(N, dev, out)
     if N == 0:
         return loss, lse, tgt, mean
     ws = _workspace(N, V, D, code, dev, workspace)
     a = ForwardArgs(H.data_ptr(), H.stride(0), W.data_ptr(), W.stride(0), y.data_ptr(),
                     INDEX_INT32 if y.dtype == torch.int32 else INDEX_INT64, code, N, V, D,
-                    loss.data_ptr(), lse.data_ptr(), tgt.data_ptr(), mean.data_ptr())
+                    loss.data_ptr(), lse.data_ptr(), tgt.data_ptr(), mean.data_ptr(), sum_ptr)
     sp = _stream_ptr(stream, dev)
     lib = load_library()
     _raise_on(lib.flce_forward_ex(ctypes.byref(a), ws.data_ptr(), ws.numel() * ws.element_size(), sp),
@@ -403,8 +421,9 @@ def shard_state(H: torch.Tensor, W_shard: torch.Tensor, y: torch.Tensor, v_offse
 
 
 def merge_shards(states: torch.Tensor, y: torch.Tensor, V_total: int, *, stream=None,
-                 check: bool = False):
-    """Merge (G, N, 4) shard states (in shard order) into (loss, lse, target_logit, mean)."""
+                 check: bool = False, out_sum: torch.Tensor | None = None):
+    """Merge (G, N, 4) shard states (in shard order) into (loss, lse, target_logit, mean);
+    ``out_sum`` (a 0-d fp32 tensor) also receives the sum of the losses."""
     if states.dim() != 3 or states.shape[2] != 4 or states.dtype != torch.float32 or not states.is_contiguous():
         raise ValueError("states must be a contiguous float32 (G, N, 4) tensor")
     G, N = states.shape[0], states.shape[1]
@@ -412,6 +431,7 @@ def merge_shards(states: torch.Tensor, y: torch.Tensor, V_total: int, *, stream=
     f32 = dict(dtype=torch.float32, device=dev)
     loss, lse, tgt = (torch.empty(N, **f32) for _ in range(3))
     mean = torch.full((), float("nan"), **f32)
+    sum_ptr = _sum_output(N, dev, {"sum": out_sum})
     if N == 0:
         return loss, lse, tgt, mean
     lib = load_library()
@@ -419,7 +439,8 @@ def merge_shards(states: torch.Tensor, y: torch.Tensor, V_total: int, *, stream=
     sp = _stream_ptr(stream, dev)
     _raise_on(lib.flce_merge_shards(states.data_ptr(), G, y.data_ptr(), N, int(V_total),
                                     loss.data_ptr(), lse.data_ptr(), tgt.data_ptr(), mean.data_ptr(),
-                                    scratch.data_ptr(), scratch.numel(), sp), "flce_merge_shards")
+                                    sum_ptr, scratch.data_ptr(), scratch.numel(), sp),
+              "flce_merge_shards")
     if check:
         _raise_on(lib.flce_check(scratch.data_ptr(), sp), "flce_merge_shards (device)")
     return loss, lse, tgt, mean
@@ -605,7 +626,8 @@ def forward_quantized(H: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, b
                       workspace: torch.Tensor | None = None, stream=None, check: bool = False):
     """flce_forward_quantized: the forward with an affine group-quantised head
     W = scales * q + biases (MLX layout: wq (V, D * bits / 32) int32/uint32 codes,
-    scales and biases (V, D / group_size) bf16).  Returns (loss, lse, target_logit, mean)."""
+    scales and biases (V, D / group_size) bf16).  Returns (loss, lse, target_logit, mean);
+    ``out["sum"]`` (a 0-d fp32 tensor) also receives the sum of the losses."""
     if H.dtype != torch.bfloat16 or H.dim() != 2 or not H.is_contiguous() or not H.is_cuda:
         raise ValueError("H must be a contiguous 2-D bf16 CUDA tensor")
     dev = H.device
@@ -623,6 +645,7 @@ def forward_quantized(H: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, b
             or not y.is_contiguous():
         raise ValueError("wq and y must be on H's device; y contiguous int64 of length N")
     loss, lse, tgt, mean = _alloc_outputs(N, dev, out)
+    sum_ptr = _sum_output(N, dev, out)
     if N == 0:
         return loss, lse, tgt, mean
     lib = load_library()
@@ -634,7 +657,7 @@ def forward_quantized(H: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, b
     _raise_on(lib.flce_forward_quantized(H.data_ptr(), wq.data_ptr(), scales.data_ptr(),
                                          biases.data_ptr(), int(bits), int(group_size), y.data_ptr(),
                                          N, V, D, loss.data_ptr(), lse.data_ptr(), tgt.data_ptr(),
-                                         mean.data_ptr(), workspace.data_ptr(), nbytes, sp),
+                                         mean.data_ptr(), sum_ptr, workspace.data_ptr(), nbytes, sp),
               "flce_forward_quantized")
     if check:
         _raise_on(lib.flce_check(workspace.data_ptr(), sp), "flce_forward_quantized (device)")
@@ -755,13 +778,14 @@ class _LinearCrossEntropy(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, H, W, y, reduction):
-        loss, lse, _, mean = forward(H, W, y)
+        total = torch.empty((), dtype=torch.float32, device=H.device)
+        loss, lse, _, mean = forward_strided(H, W, y, out={"sum": total})
         ctx.save_for_backward(H, W, y, lse)
         ctx.reduction = reduction
         if reduction == "mean":
             return mean
         if reduction == "sum":
-            return mean * H.shape[0] if H.shape[0] else mean.new_zeros(())
+            return total
         return loss
 
     @staticmethod
@@ -804,13 +828,15 @@ class _LinearCrossEntropyQuantized(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, H, wq, scales, biases, y, bits, group_size, reduction):
-        loss, lse, _, mean = forward_quantized(H, wq, scales, biases, y, bits, group_size)
+        total = torch.empty((), dtype=torch.float32, device=H.device)
+        loss, lse, _, mean = forward_quantized(H, wq, scales, biases, y, bits, group_size,
+                                               out={"sum": total})
         ctx.save_for_backward(H, wq, scales, biases, y, lse)
         ctx.args = (bits, group_size, reduction)
         if reduction == "mean":
             return mean
         if reduction == "sum":
-            return mean * H.shape[0] if H.shape[0] else mean.new_zeros(())
+            return total
         return loss
 
     @staticmethod

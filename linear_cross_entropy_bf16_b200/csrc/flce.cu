@@ -324,7 +324,8 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
 }
 
 flce_status launch_merge(Targets y, int64_t N, int64_t V, float* out_loss, float* out_lse,
-                         float* out_target, float* out_mean, const void* ws, size_t ws_bytes,
+                         float* out_target, float* out_mean, float* out_sum, const void* ws,
+                         size_t ws_bytes,
                          cudaStream_t st) {
   uint8_t* wsb = static_cast<uint8_t*>(const_cast<void*>(ws));
   MergeArgs m;
@@ -337,6 +338,7 @@ flce_status launch_merge(Targets y, int64_t N, int64_t V, float* out_loss, float
   m.loss = out_loss;
   m.lse = out_lse;
   m.mean = out_mean;
+  m.sum = out_sum;
   m.N = int32_t(N);
   m.V = int32_t(V);
   m.max_slabs = int32_t(slab_capacity(V));
@@ -382,7 +384,8 @@ flce_status flce_merge(const int64_t* y, int64_t N, int64_t V, float* out_loss, 
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FLCE_ERR_INVALID_ARG;
   if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
   if (workspace_bytes < state_bytes_for(N, V)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
-  return launch_merge(Targets{y, 0}, N, V, out_loss, out_lse, out_target_logit, out_mean, workspace,
+  return launch_merge(Targets{y, 0}, N, V, out_loss, out_lse, out_target_logit, out_mean, nullptr,
+                      workspace,
                       workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -398,7 +401,8 @@ flce_status flce_forward(const void* H, const void* W, const int64_t* y, int64_t
   s = launch_partials(H, D, W, D, Targets{y, 0}, 0, N, V, D, dtype, out_target_logit, workspace,
                       st);
   if (s != FLCE_OK) return s;
-  return launch_merge(Targets{y, 0}, N, V, out_loss, out_lse, out_target_logit, out_mean, workspace,
+  return launch_merge(Targets{y, 0}, N, V, out_loss, out_lse, out_target_logit, out_mean, nullptr,
+                      workspace,
                       workspace_bytes, st);
 }
 
@@ -424,6 +428,7 @@ flce_status flce_forward_ex(const flce_forward_args* a, void* workspace, size_t 
                       workspace, st);
   if (s != FLCE_OK) return s;
   return launch_merge(y, a->N, a->V, a->out_loss, a->out_lse, a->out_target_logit, a->out_mean,
+                      a->out_sum,
                       workspace, workspace_bytes, st);
 }
 
@@ -471,7 +476,8 @@ size_t flce_merge_shards_scratch_size(int64_t N) {
 
 flce_status flce_merge_shards(const float* states, int32_t G, const int64_t* y, int64_t N,
                               int64_t V_total, float* out_loss, float* out_lse,
-                              float* out_target_logit, float* out_mean, void* scratch,
+                              float* out_target_logit, float* out_mean, float* out_sum,
+                              void* scratch,
                               size_t scratch_bytes, void* stream) {
   FLCE_TRACE();
   if (G < 1 || N < 0 || V_total < 1) return FLCE_ERR_INVALID_ARG;
@@ -488,7 +494,7 @@ flce_status flce_merge_shards(const float* states, int32_t G, const int64_t* y, 
   if (cudaMemsetAsync(sb, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
   flce_merge_shards_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
       reinterpret_cast<const float4*>(states), G, y, int32_t(N), V_total, out_loss, out_lse,
-      out_target_logit, out_mean, reinterpret_cast<double*>(sb + kHeaderBytes),
+      out_target_logit, out_mean, out_sum, reinterpret_cast<double*>(sb + kHeaderBytes),
       reinterpret_cast<WsHeader*>(sb));
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
@@ -799,27 +805,76 @@ namespace {
 
 // Every GPU on which this library's module is loaded holds this array until
 // the process exits.  In host code the name is only a stand-in: the device
-// address comes from cudaGetSymbolAddress, once per device.
+// address comes from cudaGetSymbolAddress, with the device current.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FLCE_NOALLOC_SCRATCH_BYTES];
 
+// The looked-up address is cached per device together with the id of the
+// CUDA context it was found in (cuCtxGetId: unique for the life of the
+// process, never reused).  A call made in another context (a non-primary
+// context, or a primary context re-created after cudaDeviceReset, which
+// reloads the module elsewhere) looks the address up again.
 constexpr int kMaxDevices = 64;
+struct NoallocSlot {
+  unsigned long long ctx_id = 0;
+  void* ptr = nullptr;
+};
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+NoallocSlot g_noalloc_slot[kMaxDevices];
 
-// Device address of the scratch array on the current device (looked up on the
-// first call for that device, with that device current).
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+PfnCtxGetCurrent g_ctx_get_current = nullptr;
+PfnCtxGetId g_ctx_get_id = nullptr;
+std::once_flag g_ctx_fns_once;
+
+bool load_ctx_fns() {
+  std::call_once(g_ctx_fns_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_current = reinterpret_cast<PfnCtxGetCurrent>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_id = reinterpret_cast<PfnCtxGetId>(fn);
+  });
+  return g_ctx_get_current != nullptr && g_ctx_get_id != nullptr;
+}
+
+// Id of the context current on this thread; binds the current device's primary
+// context first if none is current (the runtime does so on its first call).
+flce_status current_ctx_id(unsigned long long* id) {
+  if (!load_ctx_fns()) return FLCE_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return FLCE_ERR_CUDA;
+  if (ctx == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return FLCE_ERR_CUDA;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return FLCE_ERR_CUDA;
+  }
+  return g_ctx_get_id(ctx, id) == CUDA_SUCCESS ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+// Device address of the scratch array in the current context (looked up on
+// the first call in that context, with its device current).
 flce_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return FLCE_ERR_UNSUPPORTED;
+  unsigned long long id = 0;
+  flce_status s = current_ctx_id(&id);
+  if (s != FLCE_OK) return s;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  NoallocSlot& slot = g_noalloc_slot[dev];
+  if (slot.ptr == nullptr || slot.ctx_id != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return FLCE_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
+    slot.ptr = p;
+    slot.ctx_id = id;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return FLCE_OK;
 }
 
@@ -830,6 +885,7 @@ extern "C" flce_status flce_forward_noalloc(const void* H, const void* W, const 
                                             float* out_loss, float* out_lse,
                                             float* out_target_logit, float* out_mean,
                                             void* stream) {
+  FLCE_TRACE();
   if (!sizes_ok(N, V, D, dtype)) return FLCE_ERR_INVALID_ARG;
   if (N == 0) return FLCE_OK;
   // The problem must fit the built-in scratch; nothing larger is ever allocated.
@@ -918,7 +974,7 @@ extern "C" flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
                                               int32_t bits, int32_t group_size, const int64_t* y,
                                               int64_t N, int64_t V, int64_t D, float* out_loss,
                                               float* out_lse, float* out_target_logit,
-                                              float* out_mean, void* workspace,
+                                              float* out_mean, float* out_sum, void* workspace,
                                               size_t workspace_bytes, void* stream) {
   FLCE_TRACE();
   if (N < 0 || V < 1 || D < 1 || !quant_format_ok(bits, group_size, D))
@@ -972,6 +1028,7 @@ extern "C" flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
       wsb + kHeaderBytes + align256(size_t(8) * size_t(N) * size_t(slab_capacity(L.C))));
   flce_merge_shards_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
       states, int32_t(L.chunks), y, int32_t(N), V, out_loss, out_lse, out_target_logit, out_mean,
+      out_sum,
       block_sums, hdr);
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
@@ -1229,7 +1286,8 @@ extern "C" flce_status flce_forward_host(const void* H_host, const void* W_host,
   double* block_sums = reinterpret_cast<double*>(
       wsb + kHeaderBytes + align256(size_t(8) * size_t(N) * size_t(slab_capacity(L.C))));
   flce_merge_shards_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
-      states, int32_t(L.chunks), yd, int32_t(N), V, loss_d, lse_d, tgt_d, mean_d, block_sums, hdr);
+      states, int32_t(L.chunks), yd, int32_t(N), V, loss_d, lse_d, tgt_d, mean_d, nullptr,
+      block_sums, hdr);
   if (!ok(cudaGetLastError())) return FLCE_ERR_CUDA;
   const size_t nb = size_t(N) * 4;
   if (!ok(cudaMemcpyAsync(loss_host, loss_d, nb, cudaMemcpyDeviceToHost, st)) ||

@@ -955,6 +955,7 @@ struct MergeArgs {
   float* loss;
   float* lse;
   float* mean;          // may be null
+  float* sum;           // may be null: sum_i loss_i from the same fp64 total as the mean
   double* block_sums;   // [gridDim.x]: one per kMergeTokensPerBlock tokens
   WsHeader* hdr;
   int32_t N, V;
@@ -967,8 +968,9 @@ struct MergeArgs {
 // in fp64 (each lane sums its slabs in slab order, then a fixed xor-shuffle
 // tree adds the lanes), lse = m + log s, loss = lse - z_target.  The mean is
 // a fixed-order fp64 reduction: per block, then the last block to finish
-// reduces the block results with a fixed strided-then-tree order.  Results are
-// bitwise identical run to run.
+// reduces the block results with a fixed strided-then-tree order; the same
+// fp64 total, rounded once, is the sum of the losses.  Results are bitwise
+// identical run to run.
 constexpr int kMergeLanes = 16;                 // lanes per token
 constexpr int kMergeTokensPerBlock = 32;
 constexpr int kMergeBlockThreads = kMergeLanes * kMergeTokensPerBlock;   // 512
@@ -1024,7 +1026,7 @@ __global__ void __launch_bounds__(kMergeBlockThreads) flce_merge_kernel(const Me
     a.lse[i] = lse_f;
     l = double(loss_f);
   }
-  if (a.mean == nullptr) return;
+  if (a.mean == nullptr && a.sum == nullptr) return;
   // fixed-order block sum over the block's tokens
   if (lane == 0) tok_loss[tok] = l;
   __syncthreads();
@@ -1051,7 +1053,8 @@ __global__ void __launch_bounds__(kMergeBlockThreads) flce_merge_kernel(const Me
   if (threadIdx.x == 0) {
     double total = 0.0;
     for (int w = 0; w < kMergeBlockThreads / 32; ++w) total += red[w];
-    *a.mean = float(total / double(a.N));
+    if (a.mean != nullptr) *a.mean = float(total / double(a.N));
+    if (a.sum != nullptr) *a.sum = float(total);
     a.hdr->counter = 0;
   }
 }
@@ -1091,10 +1094,10 @@ __global__ void __launch_bounds__(kMergeThreads) flce_shard_state_kernel(
 // Combines the per-token states of G shards (in shard order): m = max_r m_r,
 // s = sum_r s_r exp(m_r - m), lse = m + log s; the target logit comes from
 // the shard that holds it (exactly one for a valid target); loss = lse -
-// target; mean as in flce_merge_kernel.
+// target; mean and sum as in flce_merge_kernel.
 __global__ void __launch_bounds__(kMergeThreads) flce_merge_shards_kernel(
     const float4* states, int32_t G, const int64_t* y, int32_t N, int64_t V_total, float* loss,
-    float* lse, float* target_logit, float* mean, double* block_sums, WsHeader* hdr) {
+    float* lse, float* target_logit, float* mean, float* sum, double* block_sums, WsHeader* hdr) {
   __shared__ double warp_sums[kMergeThreads / 32];
   __shared__ bool is_last;
   const int i = blockIdx.x * kMergeThreads + threadIdx.x;
@@ -1127,7 +1130,7 @@ __global__ void __launch_bounds__(kMergeThreads) flce_merge_shards_kernel(
     target_logit[i] = t;
     l = double(loss_f);
   }
-  if (mean == nullptr) return;
+  if (mean == nullptr && sum == nullptr) return;
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) l += __shfl_down_sync(0xffffffffu, l, off);
   if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = l;
@@ -1146,7 +1149,8 @@ __global__ void __launch_bounds__(kMergeThreads) flce_merge_shards_kernel(
     const volatile double* bs = block_sums;
     double total = 0.0;
     for (int b = 0; b < int(gridDim.x); ++b) total += bs[b];
-    *mean = float(total / double(N));
+    if (mean != nullptr) *mean = float(total / double(N));
+    if (sum != nullptr) *sum = float(total);
     hdr->counter = 0;
   }
 }

@@ -78,6 +78,9 @@ def _load():
             lib.oracle_grad_hidden_rows.argtypes = [vp, vp, ctypes.c_int, vp, dp, i64, i64, i64,
                                                     vp, i64, dp, dp, ctypes.c_int]
             lib.oracle_grad_hidden_rows.restype = ctypes.c_int
+            lib.oracle_grad_weight_rows.argtypes = [vp, vp, ctypes.c_int, vp, dp, i64, i64, i64,
+                                                    vp, i64, dp, dp, dp, ctypes.c_int]
+            lib.oracle_grad_weight_rows.restype = ctypes.c_int
             lib.oracle_dequantize.argtypes = [vp, vp, vp, ctypes.c_int, i64, i64, i64, dp]
             lib.oracle_dequantize.restype = ctypes.c_int
             lib.oracle_forward_quantized_rows.argtypes = [vp, vp, vp, vp, ctypes.c_int, i64, vp,
@@ -220,6 +223,31 @@ def grad_hidden_rows(H: np.ndarray, W: np.ndarray, y: np.ndarray, g, rows, nthre
     if rc != 0:
         raise OracleError(_ERRORS.get(rc, f"oracle error {rc}"))
     return {"dH": dH, "bH": bH}
+
+
+def grad_weight_rows(H: np.ndarray, W: np.ndarray, y: np.ndarray, g, vocab_rows,
+                     nthreads: int = 0):
+    """dW (and its magnitude bound bW) for the selected vocabulary rows only, plus every
+    token's lse.  Costs one full logits row per token (for lse) and one logits column
+    per selected vocabulary row."""
+    lib = _load()
+    H, dt = _as_storage(H)
+    W, dt_w = _as_storage(W)
+    if dt != dt_w:
+        raise TypeError("H and W must share one storage type")
+    N, D = H.shape
+    V = W.shape[0]
+    y = np.ascontiguousarray(y, dtype=np.int64)
+    gv = np.ascontiguousarray(np.broadcast_to(np.asarray(g, dtype=np.float64), (N,)))
+    vrows = np.ascontiguousarray(vocab_rows, dtype=np.int64)
+    dW = np.empty((vrows.shape[0], D))
+    bW = np.empty((vrows.shape[0], D))
+    lse = np.empty(N)
+    rc = lib.oracle_grad_weight_rows(_ptr(H), _ptr(W), dt, _ptr(y), _ptr(gv), N, V, D, _ptr(vrows),
+                                     vrows.shape[0], _ptr(dW), _ptr(bW), _ptr(lse), int(nthreads))
+    if rc != 0:
+        raise OracleError(_ERRORS.get(rc, f"oracle error {rc}"))
+    return {"dW": dW, "bW": bW, "lse": lse}
 
 
 def _quant_arrays(wq, scales, biases, bits, group_size):

@@ -302,6 +302,90 @@ int oracle_grad_hidden_rows(const void *H, const void *W, int dtype, const int64
     return status;
 }
 
+/* dW rows only (vocabulary rows vrows[t], t < nvrows), with their magnitudes
+ * bW, and optionally every token's lse.  Row j of dW is
+ *     dW_j = sum_i dZ_ij H_i,   dZ_ij = g_i (exp(z_ij - lse_i) - [j == y_i]),
+ * which needs the log-sum-exp of EVERY token (the whole logits of each row),
+ * but only column j of the logits.  So: pass 1 computes lse_i for all N rows
+ * (two passes over a materialised row, as oracle_forward_rows), pass 2 forms
+ * each selected dW row from its recomputed logits column (as pass 2 of
+ * oracle_backward).  g is indexed by token; lse_out may be NULL. */
+int oracle_grad_weight_rows(const void *H, const void *W, int dtype, const int64_t *y,
+                            const double *g, int64_t N, int64_t V, int64_t D,
+                            const int64_t *vrows, int64_t nvrows, double *dW, double *bW,
+                            double *lse_out, int nthreads) {
+    if (!H || !W || !y || !g || !vrows || !dW || N < 1 || V < 1 || D < 1 || nvrows < 0)
+        return ORACLE_ERR_ARG;
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP32 && dtype != ORACLE_FP64) return ORACLE_ERR_ARG;
+    for (int64_t t = 0; t < nvrows; ++t)
+        if (vrows[t] < 0 || vrows[t] >= V) return ORACLE_ERR_ARG;
+    for (int64_t i = 0; i < N; ++i)
+        if (y[i] < 0 || y[i] >= V) return ORACLE_ERR_TARGET;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    double *lse = (double *)malloc((size_t)N * sizeof(double));
+    if (!lse) return ORACLE_ERR_NOMEM;
+    int status = ORACLE_OK;
+    /* pass 1: every token's log-sum-exp */
+#pragma omp parallel
+    {
+        double *z = (double *)malloc((size_t)V * sizeof(double));
+        if (!z) {
+#pragma omp atomic write
+            status = ORACLE_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < N; ++i) {
+            if (!z) continue;
+            for (int64_t j = 0; j < V; ++j) z[j] = logit(H, W, dtype, i, j, D);
+            double M = z[0];
+            for (int64_t j = 1; j < V; ++j)
+                if (z[j] > M) M = z[j];
+            double S = 0.0;
+            for (int64_t j = 0; j < V; ++j) S += exp(z[j] - M);
+            lse[i] = M + log(S);
+        }
+        free(z);
+    }
+    /* pass 2: the selected dW rows */
+    if (status == ORACLE_OK) {
+#pragma omp parallel
+        {
+            double *dz = (double *)malloc((size_t)N * sizeof(double));
+            if (!dz) {
+#pragma omp atomic write
+                status = ORACLE_ERR_NOMEM;
+            }
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t t = 0; t < nvrows; ++t) {
+                if (!dz) continue;
+                const int64_t j = vrows[t];
+                for (int64_t i = 0; i < N; ++i)
+                    dz[i] = g[i] * (exp(logit(H, W, dtype, i, j, D) - lse[i]) -
+                                    (j == y[i] ? 1.0 : 0.0));
+                for (int64_t k = 0; k < D; ++k) {
+                    double acc = 0.0, mag = 0.0;
+                    for (int64_t i = 0; i < N; ++i) {
+                        double h = load_elem(H, dtype, i * D + k);
+                        acc += dz[i] * h;
+                        mag += fabs(dz[i]) * fabs(h);
+                    }
+                    dW[t * D + k] = acc;
+                    if (bW) bW[t * D + k] = mag;
+                }
+            }
+            free(dz);
+        }
+    }
+    if (status == ORACLE_OK && lse_out)
+        for (int64_t i = 0; i < N; ++i) lse_out[i] = lse[i];
+    free(lse);
+    return status;
+}
+
 /* dL/dZ for one row i (V values), given upstream gradient g_i: the vector the
  * backward contracts with W and H.  For tests of the gradient definition. */
 int oracle_grad_logits_row(const void *H, const void *W, int dtype, const int64_t *y, double g_i,

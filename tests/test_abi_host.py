@@ -242,7 +242,7 @@ def test_quantized_workspace_and_argument_checks_need_no_gpu(lib):
     def call(bits=4, G=64, N=16, V=100, D=128, H=FAKE, wq=FAKE, s=FAKE, b=FAKE, y=FAKE,
              ws=FAKE, ws_bytes=1 << 30):
         return lib.flce_forward_quantized(H, wq, s, b, bits, G, y, N, V, D, FAKE, FAKE, FAKE, None,
-                                          ws, ws_bytes, None)
+                                          None, ws, ws_bytes, None)
     assert call(bits=3) == flce.ERR_INVALID_ARG
     assert call(G=16) == flce.ERR_INVALID_ARG
     assert call(D=96) == flce.ERR_INVALID_ARG            # not a multiple of G

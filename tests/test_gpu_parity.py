@@ -276,3 +276,51 @@ def test_fp32_unaligned_strided_rows():
     gpu = {"loss": loss.cpu().double().numpy(), "lse": lse.cpu().double().numpy(),
            "target": tgt.cpu().double().numpy(), "mean": float(mean.item())}
     compare(gpu, ref, mean_ref=oracle.mean(ref["loss"]))
+
+
+# ---------------------------------------------------------------- sum of the losses
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_loss_sum_output(dtype):
+    """out_sum of flce_forward_ex, flce_forward_quantized and flce_merge_shards: the
+    merge's fp64 total of the per-token losses, rounded once, against the oracle's
+    exactly rounded sum (math.fsum of its fp64 losses), within the mean's relative bar."""
+    import linear_cross_entropy_bf16_b200 as flce
+    from tests.flce_testing import MEAN_RTOL
+    N, V, D = 700, 3000, 128
+    H, W, y = synth.random_inputs(N, V, D, seed=77, dtype=dtype)
+    ref = oracle.forward(H, W, y)
+    want = math.fsum(ref["loss"].tolist())
+    Hd, Wd, yd = to_device(H, W, y)
+    total = torch.full((), float("nan"), device="cuda:0")
+    loss, _, _, mean = flce.forward_strided(Hd, Wd, yd, out={"sum": total}, check=True)
+    got = float(total.item())
+    assert abs(got - want) <= MEAN_RTOL * abs(want), (got, want)
+    # the same fp64 total as the mean, rounded once each
+    assert abs(got - float(mean.item()) * N) <= 1e-6 * abs(got)
+    # vocabulary shards merged: the same sum
+    states = torch.stack([flce.shard_state(Hd, Wd[a:b].contiguous(), yd, a)
+                          for a, b in ((0, 1000), (1000, V))]).contiguous()
+    total2 = torch.full((), float("nan"), device="cuda:0")
+    flce.merge_shards(states, yd, V, check=True, out_sum=total2)
+    assert abs(float(total2.item()) - want) <= MEAN_RTOL * abs(want)
+
+
+def test_loss_sum_output_quantized():
+    import linear_cross_entropy_bf16_b200 as flce
+    from tests.flce_testing import MEAN_RTOL
+    N, V, D, bits, G = 300, 2000, 128, 4, 64
+    H, Wf, y = synth.random_inputs(N, V, D, seed=78, dtype="fp32")
+    H = synth.round_to_bf16_bits(H)
+    wq, sc, bi = synth.quantize_affine(Wf, bits, G)
+    ref = oracle.forward_quantized(H, wq, sc, bi, y, bits, G)
+    want = math.fsum(ref["loss"].tolist())
+    dev = torch.device("cuda:0")
+    Hd = torch.from_numpy(H).view(torch.bfloat16).to(dev)
+    total = torch.full((), float("nan"), device=dev)
+    flce.forward_quantized(Hd, torch.from_numpy(wq.view(np.int32)).to(dev),
+                           torch.from_numpy(sc).view(torch.bfloat16).to(dev),
+                           torch.from_numpy(bi).view(torch.bfloat16).to(dev),
+                           torch.from_numpy(y).to(dev), bits, G, out={"sum": total}, check=True)
+    assert abs(float(total.item()) - want) <= MEAN_RTOL * abs(want)

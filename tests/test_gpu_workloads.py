@@ -89,6 +89,41 @@ def test_backward_workload_n1024_every_element():
     _within(dW.cpu().double().numpy(), ref["dW"], ref["bW"])
 
 
+def _dw_fixture(name, H, W, y):
+    """The oracle's sampled dW rows for workload `name` (tests/golden/make_dw_rows.py),
+    after checking that they were computed from these very inputs."""
+    import hashlib
+    path = os.path.join(os.path.dirname(__file__), "golden", f"dw_rows_{name}.npz")
+    f = np.load(path)
+    h = hashlib.sha256()
+    for a in (H, W, y):
+        h.update(np.ascontiguousarray(a).tobytes())
+    assert str(f["input_sha256"]) == h.hexdigest(), "inputs differ from those the fixture was made from"
+    return f
+
+
+@pytest.mark.parametrize("name", [synth.HEADLINE, "n4096_v128256_d4096_zipf"])
+def test_backward_full_size_dW_rows_every_element(name):
+    """At full size the backward runs in several 32768-row vocabulary chunks; the
+    sampled dW rows (chunk edges, the first and last rows, targets, seeded rows) are
+    compared element by element with the oracle's (every token's lse recomputed in
+    fp64), within the derived bound 2^-8 sum_i |dZ_ij| |H_ik|."""
+    H, W, y, dH, dW = _backward(name)
+    f = _dw_fixture(name, H, W, y)
+    assert float(f["g"]) == float(np.float32(1.0 / H.shape[0]))
+    rows = torch.from_numpy(f["vocab_rows"]).cuda()
+    got = dW[rows].cpu().double().numpy()
+    ref, bound = f["dW"].astype(np.float64), f["bW"].astype(np.float64)
+    # dW entries here are ~1e-7 (g = 1/N), so no absolute slack: the bound alone
+    err = np.abs(got - ref)
+    assert np.all(err <= 2.0 ** -8 * bound + 1e-15), float((err / np.maximum(bound, 1e-300)).max())
+    # and the comparison is not vacuous: the bound is small against the values
+    assert np.median(2.0 ** -8 * bound / np.maximum(np.abs(ref), 1e-300)) < 1.0
+    # the rows straddle the chunk edges of the backward
+    edges = {int(r) % 32768 for r in f["vocab_rows"]}
+    assert 0 in edges and 32767 in edges
+
+
 def test_backward_headline_sampled_rows_and_properties():
     """The page's shape: sampled dH rows against the oracle; dW by its exact zero-sum."""
     H, W, y, dH, dW = _backward(synth.HEADLINE)

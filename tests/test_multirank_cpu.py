@@ -192,3 +192,136 @@ def test_vocab_parallel_backward_allreduce_on_two_gloo_ranks():
         assert p.exitcode == 0
     for rank, ddH, ddW in out:
         assert ddH < 1e-12 and ddW < 1e-12
+
+
+def _bench_vp_worker(rank, world, port, q):
+    """bench.vocab_parallel_legs (the `--parallel vocab` step) on two gloo ranks: the
+    kernel steps are replaced by fp64 restatements, the exchange and the per-stage
+    timing are the benchmark's own."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        import linear_cross_entropy_bf16_b200 as flce
+        rng = np.random.default_rng(11)
+        N, V, D = 7, 13, 5
+        H = torch.from_numpy(rng.standard_normal((N, D)))
+        W = torch.from_numpy(rng.standard_normal((V, D)))
+        y = torch.from_numpy(rng.integers(0, V, N))
+        a, b = bench.vocab_shard_bounds(V, world, rank)
+
+        def fake_state(H_, W_shard, y_, v_offset, **kw):
+            z = H_ @ W_shard.T
+            m = z.max(dim=1).values
+            s = torch.exp(z - m[:, None]).sum(dim=1)
+            rel = y_ - v_offset
+            own = (rel >= 0) & (rel < W_shard.shape[0])
+            t = torch.where(own, z[torch.arange(z.shape[0]), rel.clamp(0, W_shard.shape[0] - 1)], 0.0)
+            return torch.stack([m, s, t, own.double()], dim=1)
+
+        def fake_merge(states, y_, V_total, **kw):
+            m = states[..., 0].max(dim=0).values
+            s = (states[..., 1] * torch.exp(states[..., 0] - m)).sum(dim=0)
+            lse = m + torch.log(s)
+            t = (states[..., 2] * states[..., 3]).sum(dim=0)
+            return lse - t, lse, t, (lse - t).mean()
+
+        def fake_shard(H_, W_shard, y_, lse_, v_offset, V_total, grad=None, grad_scale=1.0, **kw):
+            p = torch.exp(H_ @ W_shard.T - lse_[:, None])
+            rel = y_ - v_offset
+            own = (rel >= 0) & (rel < W_shard.shape[0])
+            onehot = torch.zeros_like(p)
+            onehot[own, rel[own]] = 1.0
+            dz = grad_scale * (p - onehot)
+            return dz @ W_shard, dz.T @ H_
+
+        flce.shard_state, flce.merge_shards, flce.backward_shard = fake_state, fake_merge, fake_shard
+        res = bench.vocab_parallel_legs(flce, H, W[a:b].contiguous(), y, a, V, world, steps=3, warmup=1)
+        Hr, Wr = H.clone().requires_grad_(True), W.clone().requires_grad_(True)
+        ref = torch.nn.functional.cross_entropy(Hr @ Wr.T, y, reduction="none")
+        ref.mean().backward()
+        q.put((rank, float((res["loss"] - ref.detach()).abs().max()),
+               float((res["dH"] - Hr.grad).abs().max()), float((res["dW_shard"] - Wr.grad[a:b]).abs().max()),
+               res["forward"], res["backward"]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_vocab_parallel_legs_on_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_bench_vp_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=240) for _ in procs]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    for rank, dloss, ddH, ddW, fw, bw in out:
+        assert dloss < 1e-12 and ddH < 1e-12 and ddW < 1e-12
+        for key in ("compute_ms", "exchange_ms", "merge_ms", "ms_per_step"):
+            assert fw[key] >= 0.0
+        assert fw["exchange_bytes_per_rank"] == 16 * 7
+        assert bw["ms_per_step"] > 0.0 and bw["exchange_alone_ms"] >= 0.0
+        assert bw["exchange_bytes_per_rank"] == 4 * 7 * 5 * 2 * 1 // 2
+
+
+def test_vocab_shard_bounds_cover_the_vocabulary():
+    import bench
+    for V, G in [(151936, 8), (13, 2), (5, 4), (1, 1)]:
+        bounds = [bench.vocab_shard_bounds(V, G, r) for r in range(G)]
+        assert bounds[0][0] == 0 and bounds[-1][1] == V
+        assert all(bounds[r][1] == bounds[r + 1][0] for r in range(G - 1))
+
+
+def test_both_arms_print_the_same_config():
+    import bench
+    from linear_cross_entropy_bf16_b200 import synth
+    w = synth.WORKLOADS[synth.HEADLINE]
+    for world in (1, 8):
+        for par in ("token", "vocab"):
+            assert bench.workload_config(w, world, par) == bench.workload_config(w, world, par)
+    c = bench.workload_config(w, 1)
+    assert c["workload"] == synth.HEADLINE and c["global_batch"] == 8192 and "no flush" in c["l2"]
+    assert "flushed" in bench.workload_config(synth.WORKLOADS["n1024_v32000_d1024"], 1)["l2"]
+
+
+def test_sustained_summary_bins_chunks_by_clock(tmp_path):
+    """The sustained window's clock matching: samples inside each chunk's host time
+    span set its clock bin; kernel medians and rates per bin."""
+    import bench
+    s = bench.ClockSampler(0)
+    s.path = str(tmp_path / "c.csv")
+    t = 1_700_000_000.0
+    with open(s.path, "w") as f:
+        for i in range(40):
+            ts = datetime_str(t + 0.05 * i)
+            mhz = 1900 if i < 20 else 1300
+            f.write(f"{ts}, 0, {mhz}, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, "
+                    f"{'Active' if i >= 20 else 'Not Active'}\n")
+    s.proc, s.f = _Done(), open(os.devnull, "w")
+    s.stop()
+    assert len(s.rows) == 40
+    chunks = [(t, t + 0.9, [1.0, 1.0, 1.2], [1.1, 1.1, 1.3]), (t + 1.0, t + 1.95, [1.5, 1.5, 1.6], [1.6] * 3)]
+    peaks = {"bf16_tflops": 1000.0, "bf16_tflops_sustained": 800.0}
+    res = bench.sustained_summary(chunks, 1e12, 100, peaks, s)
+    assert res["steps"] == 6 and res["kernel_ms_median"] == pytest.approx(1.35)
+    assert [b["sm_mhz_bin"] for b in res["by_clock"]] == [1300, 1900]
+    assert res["by_clock"][1]["kernel_ms_median"] == pytest.approx(1.0)
+    assert res["clocks"]["reasons"] == ["sw_power_cap"]
+    assert res["tflops"] == pytest.approx(1e12 / 1.35e-3 / 1e12)
+
+
+class _Done:
+    def terminate(self):
+        pass
+
+    def wait(self, *_):
+        return 0
+
+
+def datetime_str(epoch):
+    import datetime
+    return datetime.datetime.fromtimestamp(epoch).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]

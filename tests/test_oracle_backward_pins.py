@@ -157,3 +157,80 @@ def test_hidden_rows_match_full_backward(oracle_mod):
     sub = oracle_mod.grad_hidden_rows(H, W, y, g, rows)
     np.testing.assert_array_equal(sub["dH"], full["dH"][rows])
     np.testing.assert_array_equal(sub["bH"], full["bH"][rows])
+
+
+# ---------------------------------------------------------------- dW row sampler
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_weight_rows_match_torch_autograd(oracle_mod, dtype):
+    """The sampled dW rows against torch autograd on fp64 logits (an independent
+    differentiation of the same definition), every element."""
+    rng = np.random.default_rng(40)
+    N, V, D = 37, 500, 24
+    Hs = rng.standard_normal((N, D)).astype(np.float32)
+    Ws = (rng.standard_normal((V, D)) / 5).astype(np.float32)
+    H, W = (synth.round_to_bf16_bits(Hs), synth.round_to_bf16_bits(Ws)) if dtype == "bf16" else (Hs, Ws)
+    y = rng.integers(0, V, N)
+    y[:5] = 499                                   # one row that is many tokens' target
+    g = rng.uniform(-1, 1, N)
+    rows = np.array([499, 0, 250, int(y[7]), 1, 499])
+    out = oracle_mod.grad_weight_rows(H, W, y, g, rows)
+    Ht = torch.tensor(f64(H))
+    Wt = torch.tensor(f64(W), requires_grad=True)
+    loss = torch.nn.functional.cross_entropy(Ht @ Wt.T, torch.from_numpy(y), reduction="none")
+    (loss * torch.from_numpy(g)).sum().backward()
+    np.testing.assert_allclose(out["dW"], Wt.grad.numpy()[rows], rtol=1e-10, atol=1e-13)
+    # every token's lse, against the same logits
+    lse = torch.logsumexp(Ht @ Wt.detach().T, dim=1).numpy()
+    np.testing.assert_allclose(out["lse"], lse, rtol=1e-13, atol=1e-13)
+
+
+def test_weight_rows_finite_differences(oracle_mod):
+    """Central differences of the oracle's own forward on fp64 inputs."""
+    rng = np.random.default_rng(41)
+    N, V, D = 6, 9, 5
+    H = rng.standard_normal((N, D))
+    W = rng.standard_normal((V, D)) / 2
+    y = rng.integers(0, V, N)
+    g = rng.uniform(0.2, 1.5, N)
+    rows = np.array([int(y[0]), 8, 3])
+    out = oracle_mod.grad_weight_rows(H, W, y, g, rows)
+    eps = 1e-6
+    for t, j in enumerate(rows):
+        for k in range(D):
+            Wp, Wm = W.copy(), W.copy()
+            Wp[j, k] += eps
+            Wm[j, k] -= eps
+            fd = (weighted_loss(oracle_mod, H, Wp, y, g) - weighted_loss(oracle_mod, H, Wm, y, g)) / (2 * eps)
+            assert out["dW"][t, k] == pytest.approx(fd, rel=1e-6, abs=1e-8)
+
+
+def test_weight_rows_magnitudes_and_zero_sum(oracle_mod):
+    """bW is sum_i |dZ_ij| |H_ik| (exact brute force on a tiny case), and the rows of
+    the whole vocabulary sum to zero (sum_j dZ_ij = 0)."""
+    rng = np.random.default_rng(42)
+    N, V, D = 3, 4, 3
+    H = synth.round_to_bf16_bits(rng.standard_normal((N, D)).astype(np.float32))
+    W = synth.round_to_bf16_bits(rng.standard_normal((V, D)).astype(np.float32))
+    y = np.array([2, 0, 2])
+    g = np.array([0.75, -1.5, 1.0])
+    out = oracle_mod.grad_weight_rows(H, W, y, g, np.arange(V))
+    Hq = [[Fraction(float(v)) for v in r] for r in f64(H)]
+    Wq = [[Fraction(float(v)) for v in r] for r in f64(W)]
+    mpmath.mp.dps = 50
+    dz = []
+    for i in range(N):
+        z = [mpmath.mpf(float(sum(Hq[i][k] * Wq[j][k] for k in range(D)))) for j in range(V)]
+        lse = mpmath.log(mpmath.fsum(mpmath.e ** v for v in z))
+        dz.append([g[i] * (mpmath.e ** (z[j] - lse) - (1 if j == y[i] else 0)) for j in range(V)])
+    for j in range(V):
+        for k in range(D):
+            ref = mpmath.fsum(dz[i][j] * float(Hq[i][k]) for i in range(N))
+            mag = mpmath.fsum(abs(dz[i][j]) * abs(float(Hq[i][k])) for i in range(N))
+            assert out["dW"][j, k] == pytest.approx(float(ref), rel=1e-12, abs=1e-14)
+            assert out["bW"][j, k] == pytest.approx(float(mag), rel=1e-12, abs=1e-14)
+    H2, W2, y2 = synth.random_inputs(50, 300, 16, seed=43)
+    full = oracle_mod.grad_weight_rows(H2, W2, y2, 1.0 / 50, np.arange(300))
+    scale = np.abs(full["dW"]).sum(axis=0).max()
+    assert np.abs(full["dW"].sum(axis=0)).max() <= 1e-12 * max(1.0, scale)

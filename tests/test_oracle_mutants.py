@@ -22,6 +22,7 @@ QNT = ["tests/test_oracle_quant_pins.py"]
 FR = "int oracle_forward_rows("
 QR = "int oracle_forward_quantized_rows("
 BW = "int oracle_backward("
+WR = "int oracle_grad_weight_rows("
 
 # (name, text in oracle.c, replacement, which occurrence of the text, pin files
 # that cover the mutated function, the function the mutation must land in)
@@ -43,6 +44,13 @@ MUTANTS = [
      "(exp(z[j] - lse[i]) + (j == y[i] ? 1.0 : 0.0))", 0, BWD, BW),
     ("backward dH drops the W factor", "acc += z[j] * w;", "acc += z[j];", 0, BWD, BW),
     ("backward dW drops the H factor", "acc += dz[i] * h;", "acc += dz[i];", 0, BWD, BW),
+    ("dW row sampler flips the one-hot sign", "(exp(logit(H, W, dtype, i, j, D) - lse[i]) -\n"
+     "                                    (j == y[i] ? 1.0 : 0.0));",
+     "(exp(logit(H, W, dtype, i, j, D) - lse[i]) +\n"
+     "                                    (j == y[i] ? 1.0 : 0.0));", 1, BWD, WR),
+    ("dW row sampler's lse drops the max shift", "lse[i] = M + log(S);", "lse[i] = log(S);", 1, BWD, WR),
+    ("dW row sampler pairs dZ with the wrong token", "acc += dz[i] * h;",
+     "acc += dz[N - 1 - i] * h;", 1, BWD, WR),
     ("quantised codes read highest first", "(word >> (bits * (int)(k % per_word)))",
      "(word >> (bits * (int)(per_word - 1 - k % per_word)))", 0, QNT, "static uint32_t quant_code("),
     ("quantised groups in reverse order", "const int64_t g = j * (D / G) + k / G;",

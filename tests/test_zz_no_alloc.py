@@ -4,9 +4,9 @@ Such callers (code running inside an allocator or memory-pool callback, or a
 runtime that owns the whole device memory budget) cannot hand over a
 workspace, so this entry point uses a fixed scratch array built into the
 library.  The test calls it through the C ABI (ctypes) twice in a row, with
-different inputs, and checks each result against flce_forward with a
-caller-supplied workspace, within the tolerances of the other GPU tests.
-The file is named to be collected last.
+different inputs, and checks each result against the fp64 oracle on every row
+and against flce_forward with a caller-supplied workspace, within the
+tolerances of the other GPU tests.  The file is named to be collected last.
 """
 import ctypes
 
@@ -14,8 +14,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from linear_cross_entropy_bf16_b200 import synth
-from tests.flce_testing import LOSS_TOL, LSE_TOL, MEAN_RTOL, TARGET_TOL, to_device
+from tests.flce_testing import LOSS_TOL, LSE_TOL, MEAN_RTOL, TARGET_TOL, compare, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -27,6 +28,7 @@ def lib():
     import linear_cross_entropy_bf16_b200 as flce
     from linear_cross_entropy_bf16_b200 import build
     build.build()
+    oracle.build()
     L = flce.load_library()
     fn = L.flce_forward_noalloc
     fn.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 3 + [ctypes.c_int] + [ctypes.c_void_p] * 5
@@ -55,6 +57,12 @@ def test_noalloc_matches_forward_twice_in_a_row(lib, dtype, shape):
         H, W, y = synth.random_inputs(N, V, D, seed=seed, dtype=dtype)
         Hd, Wd, yd = to_device(H, W, y)
         got = call_noalloc(lib, Hd, Wd, yd, code)
+        # against the oracle on every row
+        want = oracle.forward(H, W, y)
+        compare({"loss": got[0].cpu().double().numpy(), "lse": got[1].cpu().double().numpy(),
+                 "target": got[2].cpu().double().numpy(), "mean": float(got[3].item())},
+                want, mean_ref=oracle.mean(want["loss"]))
+        # and against the forward with a caller-supplied workspace
         ref = flce.forward(Hd, Wd, yd, check=True)
         torch.cuda.synchronize()
         for g, r, tol in zip(got[:3], ref[:3], (LOSS_TOL, LSE_TOL, TARGET_TOL)):
