@@ -14,8 +14,9 @@ over ranks; `--parallel vocab` splits W's rows over the ranks instead (one
 all-gather of 16 bytes per token per step; scaling is strong).
 
 Also measured in the default run, each in its own object of the same line:
-  * roofline: the contraction kernel's median duration (CUDA events on its
-    stream) over a sustained window of at least --sustain-seconds, against the
+  * roofline: the forward is one kernel launch (the contraction with the
+    merge in its epilogue); its median duration (CUDA events on its stream)
+    over a sustained window of at least --sustain-seconds, against the
     measured bf16 peaks, with the SM clock sampled during that window (median,
     and the kernel's rate binned by clock); the burst figures of the K steps
     beside it;
@@ -148,7 +149,8 @@ def workload_config(w, world: int, parallel: str = "token") -> dict:
             "parallelism": ("single GPU" if world == 1 else
                             f"dp{world}" if parallel == "token" else f"vocab-parallel over {world} GPUs"),
             "l2": (f"inputs larger than L2 (W is {w.V * w.D * elem / 1e9:.2f} GB), no flush" if big else
-                   f"L2 flushed between steps (a {FLUSH_BYTES >> 20} MiB write)")}
+                   f"L2 flushed between steps (a {FLUSH_BYTES >> 20} MiB write, then a "
+                   f"{FLUSH_BYTES >> 20} MiB read so that no dirty line is written back during the step)")}
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -252,9 +254,9 @@ def oracle_rows_timed(H, W, y, rows):
 
 
 def cpu_baseline_for(w, H, W, y, rows_cap: int):
-    """cpu_baseline object: the oracle on every row (small workloads) or on the
-    seeded row sample the tests use (large ones)."""
-    rows = synth.sample_rows(w.N, rows_cap, w.seed)
+    """cpu_baseline object: the oracle on every row (workloads of at most 1024
+    tokens) or on the seeded row sample the tests use (larger ones)."""
+    rows = synth.sample_rows(w.N, w.N if w.N <= 1024 else rows_cap, w.seed)
     _, secs, cores = oracle_rows_timed(H, W, y, rows)
     return {"value": len(rows) / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "seconds": secs, "rows": int(len(rows)), "s_per_token": secs / len(rows),
@@ -336,43 +338,37 @@ def sync(device):
 
 
 class ForwardTimer:
-    """One forward step as the two stages of flce_forward with CUDA events on the
-    launching stream: the contraction kernel (flce_partials) and the merge."""
+    """One forward step: flce_forward, one kernel launch (the contraction with the
+    merge in its epilogue) after a small header reset, between two CUDA events on
+    the launching stream."""
 
     def __init__(self, flce, H, W, y, dev, stream):
         import torch
         N, V, D = H.shape[0], W.shape[0], H.shape[1]
         self.flce, self.H, self.W, self.y, self.stream, self.dev = flce, H, W, y, stream, dev
-        self.V = V
         self.ws = torch.empty(flce.workspace_size(N, V, D, H.dtype), dtype=torch.uint8, device=dev)
-        self.loss, self.lse, self.tgt = (torch.empty(N, device=dev) for _ in range(3))
-        self.mean = torch.empty((), device=dev)
-
-    def launch(self):
-        self.flce.partials(self.H, self.W, self.y, self.tgt, self.ws, stream=self.stream)
-
-    def merge(self):
-        self.flce.merge(self.y, self.V, self.loss, self.lse, self.tgt, self.mean, self.ws,
-                        stream=self.stream)
+        self.out = {"loss": torch.empty(N, device=dev), "lse": torch.empty(N, device=dev),
+                    "target_logit": torch.empty(N, device=dev), "mean": torch.empty((), device=dev)}
+        self.lse, self.mean = self.out["lse"], self.out["mean"]
 
     def run(self, steps: int, flush=None):
-        """Times `steps` steps; returns per-step (kernel ms, step ms) and the total ms
-        from the first step's start to the last step's end."""
+        """Times `steps` steps; returns the per-step times (ms) and the total ms from the
+        first step's start to the last step's end.  `flush`: a (write, read) pair of
+        buffers larger than L2, written and then read between steps."""
         import torch
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
         with torch.cuda.stream(self.stream):
             for k in range(steps):
                 if flush is not None:
-                    flush.zero_()
+                    flush[0].zero_()
+                    flush[1].sum(dtype=torch.float32)
                 ev[k][0].record(self.stream)
-                self.launch()
+                self.flce.forward(self.H, self.W, self.y, out=self.out, workspace=self.ws,
+                                  stream=self.stream)
                 ev[k][1].record(self.stream)
-                self.merge()
-                ev[k][2].record(self.stream)
         torch.cuda.synchronize(self.dev)
-        kern = [ev[k][0].elapsed_time(ev[k][1]) for k in range(steps)]
-        step = [ev[k][0].elapsed_time(ev[k][2]) for k in range(steps)]
-        return kern, step, ev[0][0].elapsed_time(ev[steps - 1][2])
+        step = [ev[k][0].elapsed_time(ev[k][1]) for k in range(steps)]
+        return step, ev[0][0].elapsed_time(ev[steps - 1][1])
 
     def check(self, what):
         st = self.flce.check(self.ws, self.stream)
@@ -388,24 +384,25 @@ def roofline_numbers(flops: float, kernel_ms: float, peaks: dict) -> dict:
 
 def sustained_window(timer: ForwardTimer, seconds: float, chunk_steps: int = 20):
     """Back-to-back steps for at least `seconds`, in chunks of `chunk_steps` whose host
-    time spans are matched to the clock samples.  Returns the chunks (t0, t1, kernel
-    ms list, step ms list)."""
+    time spans are matched to the clock samples.  Returns the chunks (t0, t1, step ms
+    list)."""
     chunks = []
     t_end = time.time() + seconds
     while time.time() < t_end or len(chunks) < 3:
         sync(timer.dev)
         t0 = time.time()
-        kern, step, _ = timer.run(chunk_steps)
-        chunks.append((t0, time.time(), kern, step))
+        step, _ = timer.run(chunk_steps)
+        chunks.append((t0, time.time(), step))
     return chunks
 
 
 def sustained_summary(chunks, flops: float, N: int, peaks: dict, sampler: ClockSampler) -> dict:
+    """Medians of the sustained window's steps (the forward is one kernel launch, so
+    the step time is the kernel's), their rate against the peaks, and by clock."""
     kern = [v for c in chunks for v in c[2]]
-    step = [v for c in chunks for v in c[3]]
     km = median(kern)
     res = {"seconds": chunks[-1][1] - chunks[0][0], "steps": len(kern),
-           "ms_per_step_median": median(step), "tokens_per_s_median_step": N / (median(step) * 1e-3),
+           "ms_per_step_median": km, "tokens_per_s_median_step": N / (km * 1e-3),
            "kernel_ms_median": km, "kernel_ms_mean": float(np.mean(kern)),
            "kernel_ms_p10": float(np.percentile(kern, 10)), "kernel_ms_p90": float(np.percentile(kern, 90)),
            **roofline_numbers(flops, km, peaks)}
@@ -417,7 +414,7 @@ def sustained_summary(chunks, flops: float, N: int, peaks: dict, sampler: ClockS
         res["frac_of_per_cycle_peak_at_median_clock"] = res["tflops"] / per_cycle
         # per chunk: the clock samples that fall inside its host time span
         bins = {}
-        for t0, t1, kc, _ in chunks:
+        for t0, t1, kc in chunks:
             mhz = [r[1] for r in sampler.rows if t0 <= r[0] <= t1 and r[3] > 300]
             if not mhz:
                 continue
@@ -485,7 +482,7 @@ def run_ours(args, w, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize(dev)
     t_timed = time.time()
-    part_ms, step_ms, total_ms = fwd.run(K)
+    part_ms, total_ms = fwd.run(K)
     t_timed_end = time.time()
     if world > 1:
         dist.barrier()
@@ -523,7 +520,8 @@ def run_ours(args, w, rank, world, local_rank):
     host_inputs = {w.name: (Hn, Wn, yn)}
     if "workloads" in legs and world == 1:
         workloads = {}
-        flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        flush = (torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev),
+                 torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev))
         for name, wl in synth.WORKLOADS.items():
             if name == w.name:
                 continue
@@ -570,7 +568,7 @@ def run_ours(args, w, rank, world, local_rank):
         "sustained": sustained,
         "e2e": e2e["e2e"],
         "e2e_resident_head": e2e["resident"],
-        "gpu_launches": 2 * K,
+        "gpu_launches": K,
         "kernel_ms_stats": {"median": median(part_ms), "min": float(np.min(part_ms)),
                             "max": float(np.max(part_ms)), "mean": float(np.mean(part_ms))},
         "env": run_environment(dev),
@@ -619,9 +617,9 @@ def time_workload(flce, w, dev, stream, args, peaks, flush):
     for _ in range(3):
         t.run(1, flush if needs_flush else None)
     steps = max(20, args.steps)
-    kern, step, _ = t.run(steps, flush if needs_flush else None)
+    kern, _ = t.run(steps, flush if needs_flush else None)
     t.check(w.name)
-    km, sm = median(kern), median(step)
+    km = sm = median(kern)
     p = flce.plan(w.N, w.V, w.D, H.dtype)
     res = {"N": w.N, "V": w.V, "D": w.D, "input_dtype": w.dtype, "targets": w.targets,
            "steps": steps, "ms_per_step": sm, "tokens_per_s": w.N / (sm * 1e-3),

@@ -89,9 +89,9 @@ typedef struct {
 } flce_plan_t;
 
 /* Bytes of device workspace that flce_forward / flce_partials need for this
- * problem: a 256-byte header, the per-(slab, token) partial states (8 bytes
- * each, at most 512 slabs per token, so O(N), never O(N*V)), and one fp64
- * per 32 tokens for the mean.  fp32 inputs add the bf16 split copies of H
+ * problem: a 256-byte header, one 4-byte arrival counter per 128 tokens, the
+ * per-(slab, token) partial states (8 bytes each, at most 512 slabs per
+ * token, so O(N), never O(N*V)), and one fp64 per 128 tokens for the mean.  fp32 inputs add the bf16 split copies of H
  * and W ([hi | lo], 4 Dp bytes per row each), Dp = D rounded up to 64:
  * O((N + V) D), still never O(N*V).  Depends only on its arguments (not on
  * the device).
@@ -121,6 +121,11 @@ FLCE_API flce_status flce_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype
  *                contents on entry are ignored; it holds the status word that
  *                flce_check() reads until the next call that uses it
  *   stream       cudaStream_t
+ * One kernel launch (after a reset of the workspace header, and for fp32
+ * inputs the split of H and W): the CTA that writes the last vocab slab's
+ * state of a 128-token row block merges that block in the same kernel, and
+ * the one that merges the last row block forms the mean.  The results equal
+ * those of flce_partials followed by flce_merge bit for bit.
  * A row whose target is out of range gets NaN loss and NaN target logit and
  * sets FLCE_ERR_TARGET_OUT_OF_RANGE for flce_check().  N == 0 is a no-op that
  * returns FLCE_OK and writes nothing (out_mean untouched).
@@ -317,7 +322,7 @@ FLCE_API flce_status flce_selftest_wait_timeout(void* workspace, size_t workspac
  *   - A problem whose flce_workspace_size(N, V, D, dtype) exceeds
  *     FLCE_NOALLOC_SCRATCH_BYTES is rejected with FLCE_ERR_WORKSPACE_TOO_SMALL
  *     and nothing is enqueued.  With V >= 131072 (512 slab states per token)
- *     that means N <= 16382.
+ *     that means N <= 16383.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current.  Make that first call
  *     before any stream capture on that device.  The address is cached with

@@ -221,17 +221,30 @@ void launch_contraction_kernel(bool pair, unsigned grid, const CUtensorMap& tmH,
     tc::flce_tc_kernel<L><<<grid, tc::NUM_THREADS, tc::Cfg<L>::SMEM_BYTES, st>>>(tmH, tmW, a);
 }
 
+// Outputs of the merge when it runs inside the contraction kernel (the whole
+// forward in one launch); see tc::fused_merge.
+struct MergeOutputs {
+  float* loss;
+  float* lse;
+  float* mean;  // may be null
+  float* sum;   // may be null
+};
+
 // The contraction with the online (m, s) epilogue.  Writes (m, s) per (slab,
-// token) after the workspace header and the target logits W owns.
-// reset_header: clear the header (status word) first.
+// token) into the workspace's state and the target logits W owns; with
+// `merged` also the merged loss, lse, mean and sum (then y_offset must be 0
+// and V the whole vocabulary).  reset_header: clear the header (status word)
+// and the row-block counters first.
 flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, int64_t N,
                                int64_t V, const flce_plan_t& plan, float* out_target, void* ws,
-                               bool reset_header, cudaStream_t st) {
+                               bool reset_header, cudaStream_t st,
+                               const MergeOutputs* merged = nullptr) {
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
-  float2* part = reinterpret_cast<float2*>(wsb + kHeaderBytes);
-  if (reset_header && cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess)
-    return FLCE_ERR_CUDA;
+  const StateLayout L = state_layout(N, V);
+  float2* part = reinterpret_cast<float2*>(wsb + L.part);
+  if (merged != nullptr && (!reset_header || y_offset != 0)) return FLCE_ERR_INVALID_ARG;
+  if (reset_header && cudaMemsetAsync(hdr, 0, L.part, st) != cudaSuccess) return FLCE_ERR_CUDA;
 
   Schedule sch;
   sch.token_blocks = int32_t(plan.token_blocks);
@@ -261,6 +274,16 @@ flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, 
   a.seg_w = int32_t(op.seg_w);
   a.sch = sch;
   a.wait_limit_ns = kDefaultWaitLimitNs;
+  a.fm = tc::FusedMerge{};
+  if (merged != nullptr) {
+    a.fm.arrivals = reinterpret_cast<uint32_t*>(wsb + L.counters);
+    a.fm.loss = merged->loss;
+    a.fm.lse = merged->lse;
+    a.fm.mean = merged->mean;
+    a.fm.sum = merged->sum;
+    a.fm.block_sums = reinterpret_cast<double*>(wsb + L.sums);
+    a.fm.row_blocks = int32_t(plan.token_blocks * plan.ctas_per_unit);
+  }
   const unsigned grid = unsigned(plan.grid);
   switch (op.layout) {
     case tc::kPlain: launch_contraction_kernel<tc::kPlain>(pair, grid, tmH, tmW, a, st); break;
@@ -296,10 +319,12 @@ flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, i
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
-// Stage 1 of the forward for bf16 or fp32 H and W (fp32: split first).
+// Stage 1 of the forward for bf16 or fp32 H and W (fp32: split first); with
+// `merged`, the whole forward (the merge runs inside the contraction kernel).
 flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t ldw, Targets y,
                             int64_t y_offset, int64_t N, int64_t V, int64_t D, flce_dtype dtype,
-                            float* out_target, void* ws, cudaStream_t st) {
+                            float* out_target, void* ws, cudaStream_t st,
+                            const MergeOutputs* merged = nullptr) {
   DeviceInfo di;
   int64_t workers = 0;
   flce_status s = contraction_workers(N, di, workers);
@@ -320,7 +345,7 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
     if ((s = launch_split(W, ldw, V, D, Dp, 2, 1, wsplit, di.sms, st)) != FLCE_OK) return s;
     op = Operands{hs, 2 * Dp, 2 * Dp, Dp, wsplit, 2 * Dp, 2 * Dp, Dp, Dp / tc::BK, tc::kSplitHW};
   }
-  return launch_contraction(op, y, y_offset, N, V, plan, out_target, ws, true, st);
+  return launch_contraction(op, y, y_offset, N, V, plan, out_target, ws, true, st, merged);
 }
 
 flce_status launch_merge(Targets y, int64_t N, int64_t V, float* out_loss, float* out_lse,
@@ -328,11 +353,11 @@ flce_status launch_merge(Targets y, int64_t N, int64_t V, float* out_loss, float
                          size_t ws_bytes,
                          cudaStream_t st) {
   uint8_t* wsb = static_cast<uint8_t*>(const_cast<void*>(ws));
+  const StateLayout L = state_layout(N, V);
   MergeArgs m;
   m.hdr = reinterpret_cast<WsHeader*>(wsb);
-  m.part = reinterpret_cast<const float2*>(wsb + kHeaderBytes);
-  m.block_sums = reinterpret_cast<double*>(
-      wsb + kHeaderBytes + align256(size_t(8) * size_t(N) * size_t(slab_capacity(V))));
+  m.part = reinterpret_cast<const float2*>(wsb + L.part);
+  m.block_sums = reinterpret_cast<double*>(wsb + L.sums);
   m.y = y;
   m.target_logit = out_target;
   m.loss = out_loss;
@@ -397,13 +422,10 @@ flce_status flce_forward(const void* H, const void* W, const int64_t* y, int64_t
   flce_status s = check_forward_args(H, W, y, N, V, D, dtype, workspace, workspace_bytes);
   if (s != FLCE_OK || N == 0) return s;
   if (!out_loss || !out_lse || !out_target_logit) return FLCE_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = launch_partials(H, D, W, D, Targets{y, 0}, 0, N, V, D, dtype, out_target_logit, workspace,
-                      st);
-  if (s != FLCE_OK) return s;
-  return launch_merge(Targets{y, 0}, N, V, out_loss, out_lse, out_target_logit, out_mean, nullptr,
-                      workspace,
-                      workspace_bytes, st);
+  // one launch: the merge runs in the contraction kernel's epilogue
+  const MergeOutputs merged{out_loss, out_lse, out_mean, nullptr};
+  return launch_partials(H, D, W, D, Targets{y, 0}, 0, N, V, D, dtype, out_target_logit, workspace,
+                         static_cast<cudaStream_t>(stream), &merged);
 }
 
 flce_status flce_forward_ex(const flce_forward_args* a, void* workspace, size_t workspace_bytes,
@@ -424,12 +446,9 @@ flce_status flce_forward_ex(const flce_forward_args* a, void* workspace, size_t 
   if (ldh >= (int64_t(1) << 31) || ldw >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Targets y{a->y, a->y_dtype == FLCE_INDEX_INT32 ? 1 : 0};
-  s = launch_partials(a->H, ldh, a->W, ldw, y, 0, a->N, a->V, a->D, dtype, a->out_target_logit,
-                      workspace, st);
-  if (s != FLCE_OK) return s;
-  return launch_merge(y, a->N, a->V, a->out_loss, a->out_lse, a->out_target_logit, a->out_mean,
-                      a->out_sum,
-                      workspace, workspace_bytes, st);
+  const MergeOutputs merged{a->out_loss, a->out_lse, a->out_mean, a->out_sum};
+  return launch_partials(a->H, ldh, a->W, ldw, y, 0, a->N, a->V, a->D, dtype, a->out_target_logit,
+                         workspace, st, &merged);
 }
 
 flce_status flce_partials_shard(const void* H, const void* W_shard, const int64_t* y, int64_t N,
@@ -463,7 +482,8 @@ flce_status flce_shard_state(const int64_t* y, int64_t N, int64_t V_shard, int64
   const WsHeader* hdr = reinterpret_cast<const WsHeader*>(wsb);
   flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0,
                             static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const float2*>(wsb + kHeaderBytes), hdr, y, int32_t(N), v_offset, V_shard,
+      reinterpret_cast<const float2*>(wsb + state_layout(N, V_shard).part), hdr, y, int32_t(N),
+      v_offset, V_shard,
       int32_t(slab_capacity(V_shard)), target_logit, reinterpret_cast<float4*>(out_state),
       const_cast<uint32_t*>(&hdr->status));
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
@@ -1020,12 +1040,12 @@ extern "C" flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
                                 false, st)) != FLCE_OK)
       return s;
     flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
-        reinterpret_cast<const float2*>(wsb + kHeaderBytes), hdr, y, int32_t(N), c0, rows,
+        reinterpret_cast<const float2*>(wsb + state_layout(N, rows).part), hdr, y, int32_t(N), c0,
+        rows,
         int32_t(slab_capacity(rows)), out_target_logit, states + c * N, &hdr->status);
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   }
-  double* block_sums = reinterpret_cast<double*>(
-      wsb + kHeaderBytes + align256(size_t(8) * size_t(N) * size_t(slab_capacity(L.C))));
+  double* block_sums = reinterpret_cast<double*>(wsb + state_layout(N, L.C).sums);
   flce_merge_shards_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
       states, int32_t(L.chunks), y, int32_t(N), V, out_loss, out_lse, out_target_logit, out_mean,
       out_sum,
@@ -1279,12 +1299,12 @@ extern "C" flce_status flce_forward_host(const void* H_host, const void* W_host,
                                 st)) != FLCE_OK)
       return s;
     flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
-        reinterpret_cast<const float2*>(wsb + kHeaderBytes), hdr, yd, int32_t(N), c0, rows,
+        reinterpret_cast<const float2*>(wsb + state_layout(N, rows).part), hdr, yd, int32_t(N), c0,
+        rows,
         int32_t(slab_capacity(rows)), tgt_d, states + c * N, &hdr->status);
     if (!ok(cudaGetLastError()) || !ok(cudaEventRecord(freed[b], st))) return FLCE_ERR_CUDA;
   }
-  double* block_sums = reinterpret_cast<double*>(
-      wsb + kHeaderBytes + align256(size_t(8) * size_t(N) * size_t(slab_capacity(L.C))));
+  double* block_sums = reinterpret_cast<double*>(wsb + state_layout(N, L.C).sums);
   flce_merge_shards_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
       states, int32_t(L.chunks), yd, int32_t(N), V, loss_d, lse_d, tgt_d, mean_d, nullptr,
       block_sums, hdr);

@@ -18,6 +18,10 @@
 //   * flce_tc2_kernel: the same on CTA pairs (cta_group::2, 256x256 tiles):
 //     each CTA stages its own 128 token rows and half of the
 //     W tile, the even CTA issues the pair MMAs.  Used for N > 128.
+//   * In the forward both also merge (tc::fused_merge): the CTA that writes
+//     the last slab state of a 128-token row block merges that block in its
+//     epilogue, and the one that merges the last row block forms the mean,
+//     so the whole forward is one launch.
 //   * Both are templates on the stage layout (tc::StageLayout): H and W
 //     blocks of two consecutive K blocks per stage for bf16 inputs; H with
 //     W's hi and lo blocks for a quantised head (two products); H's and W's
@@ -27,10 +31,11 @@
 //     rows for the split layout (three segments for the backward's GEMMs).
 //   * flce_dequant_split_kernel: expands one chunk of an affine
 //     group-quantised head into bf16 [hi | lo] rows for the same kernels.
-//   * flce_merge_kernel: combines the P slab states of each token in a fixed
-//     order (the recurrence of section 1 applied to whole slabs), writes
-//     lse/loss, and reduces the mean deterministically in fp64; the shard
-//     kernels do the same across vocabulary shards or chunks.
+//   * flce_merge_kernel: the same merge as a kernel of its own, after the
+//     contraction alone (flce_partials): combines the P slab states of each
+//     token in a fixed order (the recurrence of section 1 applied to whole
+//     slabs), writes lse/loss, and reduces the mean deterministically in
+//     fp64; the shard kernels do the same across vocabulary shards or chunks.
 #pragma once
 
 #include <cstdint>
@@ -46,7 +51,8 @@ namespace flce {
 constexpr int kTileCols = 256;   // vocab columns per tile (UMMA N, TMEM columns)
 constexpr int kMaxSlabs = 512;   // partial states per token, at most
 
-// workspace layout: [header 256 B][partials float2[P][N]][block sums double[ceil(N/256)]]
+// workspace layout: [header 256 B][row-block arrival counters][partials float2[P][N]]
+// [block sums double]; the host's state_layout() gives the offsets
 constexpr size_t kHeaderBytes = 256;
 constexpr uint32_t kWsMagic = 0x464C4345u;  // "FLCE"
 
@@ -209,6 +215,81 @@ __device__ __forceinline__ void fold_tile(uint32_t taddr, int ncols, int64_t rel
   }
 }
 
+// ----------------------------------------------------------------- merge helpers
+
+// The merge of one token's P slab states part[p * N] (p = 0 .. P-1), the
+// recurrence of section 1 applied to whole slabs in slab order:
+// m = max_p m_p, s = sum_p s_p exp(m_p - m), accumulated in fp64, with a
+// running maximum over batches of 16 slabs (sixteen independent loads in
+// flight, one pass); returns lse = m + log s (log in fp64).  Each factor
+// exp(m_p - m) is evaluated as 2^((m_p - m) log2 e) on the SFU, as the
+// contraction's own exponentials are: relative error about 2^-22 per term,
+// and the slab holding the maximum contributes exactly s_p.  Every slab holds
+// at least one real column, so m is finite.
+__device__ __forceinline__ double merge_slab_states(const float2* part, int P, int N) {
+  constexpr int kBatch = 16;
+  float M = -INFINITY;
+  double S = 0.0;
+  for (int p0 = 0; p0 < P; p0 += kBatch) {
+    float2 st[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j)
+      st[j] = p0 + j < P ? __ldcg(part + size_t(p0 + j) * size_t(N)) : make_float2(-INFINITY, 0.f);
+    float mb = st[0].x;
+#pragma unroll
+    for (int j = 1; j < kBatch; ++j) mb = fmaxf(mb, st[j].x);
+    if (mb > M) {  // rescale the running sum (on the first batch S = 0 and 2^-inf = 0)
+      S *= double(ptx::ex2(__fmul_rn(M - mb, kLog2e)));
+      M = mb;
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j)
+      S += double(st[j].y * ptx::ex2(__fmul_rn(st[j].x - M, kLog2e)));
+  }
+  return double(M) + log(S);
+}
+
+// Fixed-order sum of one value per thread over 128 threads (four warps): a
+// warp shuffle tree, then the four warps in order.  `sync` is a barrier over
+// the 128 threads; the result is valid in thread 0.
+template <class Sync>
+__device__ __forceinline__ double sum128(double v, int t, volatile double* red, Sync sync) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
+  if ((t & 31) == 0) red[t >> 5] = v;
+  sync();
+  return ((red[0] + red[1]) + red[2]) + red[3];
+}
+
+// Row block `rb` (128 tokens, thread t holding token loss `l`) records its
+// loss sum; the row block that finishes last of `nblocks` adds the block sums
+// (thread t: blocks t, t + 128, ... in order, then sum128) into the mean and
+// the sum, and resets the counter.  The same order for any set of finishing
+// times, so results are bitwise deterministic.
+template <class Sync>
+__device__ __forceinline__ void rowblock_finish(double l, int t, int rb, int nblocks,
+                                                double* block_sums, uint32_t* counter, float* mean,
+                                                float* sum, int N, volatile double* red,
+                                                volatile int* flag, Sync sync) {
+  const double b = sum128(l, t, red, sync);
+  if (t == 0) {
+    block_sums[rb] = b;
+    __threadfence();
+    *flag = atomicAdd(counter, 1u) == uint32_t(nblocks - 1);
+  }
+  sync();
+  if (!*flag || (mean == nullptr && sum == nullptr)) return;
+  __threadfence();  // every block sum, seen through the counter
+  double v = 0.0;
+  for (int r = t; r < nblocks; r += 128) v += __ldcg(block_sums + r);
+  const double total = sum128(v, t, red, sync);
+  if (t == 0) {
+    if (mean != nullptr) *mean = float(total / double(N));
+    if (sum != nullptr) *sum = float(total);
+    *counter = 0;
+  }
+}
+
 // ----------------------------------------------------------------- tcgen05 kernel
 
 namespace tc {
@@ -267,7 +348,7 @@ struct Cfg {
   static constexpr int STAGE_BYTES = Layout<L>::NA * A_BYTES + Layout<L>::NB * B_BYTES;
   static constexpr int STAGES = stages_for(STAGE_BYTES);
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-  static_assert(STAGES >= 2 && 2 * STAGES + 6 <= 32, "stage ring and barriers");
+  static_assert(STAGES >= 2 && 2 * STAGES + 11 <= 32, "stage ring, barriers and merge scratch");
 };
 
 // Instruction descriptor of tcgen05.mma kind::f16: D fp32 (bits 4-5 = 1),
@@ -286,6 +367,19 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
          (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
+// The merge fused into the contraction (the whole forward in one kernel):
+// where to count slab arrivals per 128-token row block and where the merged
+// results go.  arrivals == nullptr: the kernel only writes the slab states.
+struct FusedMerge {
+  uint32_t* arrivals;   // [row blocks] slab states written so far (zeroed before the launch)
+  float* loss;          // [N]
+  float* lse;           // [N]
+  float* mean;          // may be null
+  float* sum;           // may be null
+  double* block_sums;   // [row blocks] fixed-order loss sum of each row block
+  int32_t row_blocks;   // token blocks x CTAs per unit: 128 tokens each
+};
+
 struct Args {
   Targets y;
   int64_t y_offset;        // first vocabulary id of W's rows (a vocabulary shard); 0 otherwise
@@ -298,7 +392,51 @@ struct Args {
   int32_t seg_w;           // split layouts: column of W's lo block 0 (elements); else 0
   Schedule sch;
   uint64_t wait_limit_ns;
+  FusedMerge fm;
 };
+
+// Barrier over the 128 epilogue threads (warps 2-5) of a contraction CTA:
+// named barrier 1 (warps 0 and 1 keep streaming and issuing meanwhile).
+struct EpiSync {
+  __device__ __forceinline__ void operator()() const { ptx::named_bar_sync(1, 128); }
+};
+
+// Called by all 128 epilogue threads after the CTA wrote its (m, s) states
+// of one vocab slab for the 128 tokens of row block `rb` (thread t owns token
+// `row`; `yi` is its target).  Counts the slab in; the CTA that brings in a
+// row block's last slab merges that block (merge_slab_states per token, lse,
+// loss = lse - z_target, NaN and the status bit for a target outside [0, V)),
+// and the CTA that merges the last row block forms the mean and the sum
+// (rowblock_finish).  `flag` and `red` are this CTA's shared memory.  The
+// arithmetic is flce_merge_kernel's, so the one-launch forward and the
+// two-stage one agree bit for bit; which CTA merges a block changes nothing.
+__device__ __forceinline__ void fused_merge(const Args& a, int rb, int row, bool valid, int64_t yi,
+                                            int t, volatile int* flag, volatile double* red) {
+  const EpiSync epi_sync;
+  __threadfence();  // this thread's state and target logit, visible device-wide
+  epi_sync();
+  if (t == 0) *flag = atomicAdd(&a.fm.arrivals[rb], 1u) == uint32_t(a.sch.slabs - 1);
+  epi_sync();
+  if (!*flag) return;
+  __threadfence();  // the other CTAs' states of this block, seen through the counter
+  double l = 0.0;
+  if (valid) {
+    const double lse = merge_slab_states(a.part + row, a.sch.slabs, a.N);
+    float loss_f;
+    if (yi < 0 || yi >= a.V) {  // no slab holds the target: invalid input
+      loss_f = __int_as_float(0x7fc00000);
+      a.target_logit[row] = loss_f;
+      atomicOr(&a.hdr->status, kStatTarget);
+    } else {
+      loss_f = float(lse - double(__ldcg(a.target_logit + row)));
+    }
+    a.fm.loss[row] = loss_f;
+    a.fm.lse[row] = float(lse);
+    l = double(loss_f);
+  }
+  rowblock_finish(l, t, rb, a.fm.row_blocks, a.fm.block_sums, &a.hdr->counter, a.fm.mean,
+                  a.fm.sum, a.N, red, flag, epi_sync);
+}
 
 template <int L>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -319,6 +457,8 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
   uint64_t* done_bar = bars + 2 * STAGES + 4;    // all MMAs retired
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* merge_flag = abort_flag + 1;                                   // fused merge: decision
+  double* merge_red = reinterpret_cast<double*>(bars + 2 * STAGES + 7);  // fused merge: [4] warp sums
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -492,6 +632,8 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
         a.part[size_t(slab) * size_t(a.N) + size_t(row)] = make_float2(m, s);
         if (got) a.target_logit[row] = zt;
       }
+      if (a.fm.arrivals != nullptr)
+        fused_merge(a, tb, row, valid, yi, threadIdx.x - 64, merge_flag, merge_red);
     }
   }
 
@@ -540,7 +682,7 @@ struct Cfg {
   static constexpr int STAGES = tc::stages_for(STAGE_BYTES);
   static constexpr uint32_t PAIR_TX_BYTES = 2 * STAGE_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
-  static_assert(STAGES >= 2 && 2 * STAGES + 6 <= 32, "stage ring and barriers");
+  static_assert(STAGES >= 2 && 2 * STAGES + 11 <= 32, "stage ring, barriers and merge scratch");
 };
 
 // kind::f16 descriptor as in the single-CTA kernel, with M = 256 (bits 24-28).
@@ -565,6 +707,8 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
   uint64_t* done_bar = bars + 2 * STAGES + 4;    // (even CTA) all MMAs retired
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* merge_flag = abort_flag + 1;                                   // fused merge: decision
+  double* merge_red = reinterpret_cast<double*>(bars + 2 * STAGES + 7);  // fused merge: [4] warp sums
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -749,6 +893,9 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
         a.part[size_t(slab) * size_t(a.N) + size_t(row)] = make_float2(m, s);
         if (got) a.target_logit[row] = zt;
       }
+      if (a.fm.arrivals != nullptr)
+        tc::fused_merge(a, 2 * tb + int(rank), row, valid, yi, threadIdx.x - 64, merge_flag,
+                        merge_red);
     }
   }
 
@@ -962,56 +1109,33 @@ struct MergeArgs {
   int32_t max_slabs;    // capacity of the partial array in this workspace
 };
 
-// The merge spreads each token's P slab states over kMergeLanes lanes of one
-// warp (lane l takes slabs l, l + 16, ...), so no thread walks a long chain of
-// dependent loads: m = max_p m_p (a shuffle max), s = sum_p s_p exp(m_p - m)
-// in fp64 (each lane sums its slabs in slab order, then a fixed xor-shuffle
-// tree adds the lanes), lse = m + log s, loss = lse - z_target.  The mean is
-// a fixed-order fp64 reduction: per block, then the last block to finish
-// reduces the block results with a fixed strided-then-tree order; the same
-// fp64 total, rounded once, is the sum of the losses.  Results are bitwise
-// identical run to run.
-constexpr int kMergeLanes = 16;                 // lanes per token
-constexpr int kMergeTokensPerBlock = 32;
-constexpr int kMergeBlockThreads = kMergeLanes * kMergeTokensPerBlock;   // 512
+// The two-stage forward's merge (after flce_partials): one thread per token,
+// one 128-token row block per CTA, with exactly the fused merge's arithmetic
+// (merge_slab_states, then rowblock_finish for the mean and the sum), so the
+// two-stage forward and the one-launch forward agree bit for bit.
+constexpr int kMergeTokensPerBlock = 128;
+constexpr int kMergeBlockThreads = kMergeTokensPerBlock;
+
+struct BlockSync {
+  __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
 
 __global__ void __launch_bounds__(kMergeBlockThreads) flce_merge_kernel(const MergeArgs a) {
-  __shared__ double tok_loss[kMergeTokensPerBlock];
-  __shared__ double red[kMergeBlockThreads / 32];
-  __shared__ bool is_last;
-  const int lane = threadIdx.x % kMergeLanes;
-  const int tok = threadIdx.x / kMergeLanes;
-  const int i = blockIdx.x * kMergeTokensPerBlock + tok;
+  __shared__ double red[4];
+  __shared__ int flag;
+  const int t = threadIdx.x;
+  const int i = blockIdx.x * kMergeTokensPerBlock + t;
   const WsHeader h = *a.hdr;
   const bool ws_ok = h.magic == kWsMagic && h.N == a.N && h.V == a.V && h.slabs >= 1 &&
                      h.slabs <= a.max_slabs;
-  const bool live = i < a.N;
-  const int P = ws_ok ? h.slabs : 0;
-  // every lane of a 16-lane group takes part in the shuffles (same token,
-  // same trip counts), so the masks are full
-  float M = -INFINITY;
-  if (live)
-    for (int p = lane; p < P; p += kMergeLanes) M = fmaxf(M, a.part[size_t(p) * a.N + i].x);
-#pragma unroll
-  for (int off = kMergeLanes / 2; off >= 1; off >>= 1)
-    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off, kMergeLanes));
-  double S = 0.0;
-  if (live)
-    for (int p = lane; p < P; p += kMergeLanes) {
-      const float2 st = a.part[size_t(p) * a.N + i];
-      S += double(st.y) * exp(double(st.x) - double(M));
-    }
-#pragma unroll
-  for (int off = kMergeLanes / 2; off >= 1; off >>= 1)
-    S += __shfl_xor_sync(0xffffffffu, S, off, kMergeLanes);
   double l = 0.0;
-  if (live && lane == 0) {
+  if (i < a.N) {
     float loss_f, lse_f;
     if (!ws_ok) {
       loss_f = lse_f = __int_as_float(0x7fc00000);
       if (i == 0) atomicOr(&a.hdr->status, kStatBadWs);
     } else {
-      const double lse = double(M) + log(S);
+      const double lse = merge_slab_states(a.part + i, h.slabs, a.N);
       const int64_t yi = a.y[i];
       lse_f = float(lse);
       if (yi < 0 || yi >= a.V) {
@@ -1026,37 +1150,8 @@ __global__ void __launch_bounds__(kMergeBlockThreads) flce_merge_kernel(const Me
     a.lse[i] = lse_f;
     l = double(loss_f);
   }
-  if (a.mean == nullptr && a.sum == nullptr) return;
-  // fixed-order block sum over the block's tokens
-  if (lane == 0) tok_loss[tok] = l;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double b = 0.0;
-    for (int t = 0; t < kMergeTokensPerBlock; ++t) b += tok_loss[t];
-    a.block_sums[blockIdx.x] = b;
-    __threadfence();
-    const uint32_t ticket = atomicAdd(&a.hdr->counter, 1u);
-    is_last = ticket == gridDim.x - 1;
-  }
-  __syncthreads();
-  if (!is_last) return;
-  // the last block: thread t sums block results t, t + 512, ... in order,
-  // then warps and the block reduce in a fixed tree
-  __threadfence();
-  const volatile double* bs = a.block_sums;
-  double v = 0.0;
-  for (int b = threadIdx.x; b < int(gridDim.x); b += kMergeBlockThreads) v += bs[b];
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double total = 0.0;
-    for (int w = 0; w < kMergeBlockThreads / 32; ++w) total += red[w];
-    if (a.mean != nullptr) *a.mean = float(total / double(a.N));
-    if (a.sum != nullptr) *a.sum = float(total);
-    a.hdr->counter = 0;
-  }
+  rowblock_finish(l, t, int(blockIdx.x), int(gridDim.x), a.block_sums, &a.hdr->counter, a.mean,
+                  a.sum, a.N, red, &flag, BlockSync{});
 }
 
 // ----------------------------------------------------------------- vocabulary shards

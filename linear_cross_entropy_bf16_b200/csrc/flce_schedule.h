@@ -19,15 +19,33 @@ bool sizes_ok(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
 
 int64_t slab_capacity(int64_t V) { return std::min<int64_t>(cdiv(V, kTileCols), kMaxSlabs); }
 
-// Header, (m, s) partial states and the mean's block sums: what the merge reads.
-size_t state_bytes_for(int64_t N, int64_t V) {
-  const size_t part = align256(size_t(8) * size_t(N) * size_t(slab_capacity(V)));
+// 128-token row blocks the fused merge counts: two per 256-token block, which
+// covers one per 128-token block of the single-CTA kernel.
+int64_t row_block_capacity(int64_t N) { return 2 * cdiv(std::max<int64_t>(N, 1), 256); }
+
+// Byte offsets in the workspace of the forward's state: the header, one
+// arrival counter per row block (zeroed with the header before every call),
+// the (m, s) partial states [slab][token], and the block sums of the mean.
+struct StateLayout {
+  size_t counters = 0, part = 0, sums = 0, total = 0;
+};
+
+StateLayout state_layout(int64_t N, int64_t V) {
+  StateLayout L;
+  L.counters = kHeaderBytes;
+  L.part = L.counters + align256(size_t(4) * size_t(row_block_capacity(N)));
+  L.sums = L.part + align256(size_t(8) * size_t(N) * size_t(slab_capacity(V)));
   // block results of the mean: one per kMergeTokensPerBlock tokens (the merge
   // kernel), which also covers one per kMergeThreads tokens (the shard merge)
-  const size_t sums =
-      align256(size_t(8) * size_t(std::max<int64_t>(1, cdiv(N, kMergeTokensPerBlock))));
-  return kHeaderBytes + part + sums;
+  // and one per row block (the fused merge)
+  const int64_t nsums =
+      std::max<int64_t>({1, cdiv(N, kMergeTokensPerBlock), row_block_capacity(N)});
+  L.total = L.sums + align256(size_t(8) * size_t(nsums));
+  return L;
 }
+
+// Header, counters, (m, s) partial states and the mean's block sums.
+size_t state_bytes_for(int64_t N, int64_t V) { return state_layout(N, V).total; }
 
 // fp32 inputs run on bf16 hi / lo parts.  The forward lays H and W out as
 // [hi | lo] rows (the kernel stages a K block of each part side by side), so a

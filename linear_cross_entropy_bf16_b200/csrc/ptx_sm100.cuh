@@ -136,6 +136,11 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&u)[32]
       : "memory");
 }
 
+// Barrier `id` (1-15) among `nthreads` threads (whole warps) of the CTA.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // 2^x on the special-function unit (approximate, flush-to-zero).
 __device__ __forceinline__ float ex2(float x) {
   float y;

@@ -304,7 +304,7 @@ def test_sustained_summary_bins_chunks_by_clock(tmp_path):
     s.proc, s.f = _Done(), open(os.devnull, "w")
     s.stop()
     assert len(s.rows) == 40
-    chunks = [(t, t + 0.9, [1.0, 1.0, 1.2], [1.1, 1.1, 1.3]), (t + 1.0, t + 1.95, [1.5, 1.5, 1.6], [1.6] * 3)]
+    chunks = [(t, t + 0.9, [1.0, 1.0, 1.2]), (t + 1.0, t + 1.95, [1.5, 1.5, 1.6])]
     peaks = {"bf16_tflops": 1000.0, "bf16_tflops_sustained": 800.0}
     res = bench.sustained_summary(chunks, 1e12, 100, peaks, s)
     assert res["steps"] == 6 and res["kernel_ms_median"] == pytest.approx(1.35)
