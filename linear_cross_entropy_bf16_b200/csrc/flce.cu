@@ -244,6 +244,7 @@ flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, 
   const StateLayout L = state_layout(N, V);
   float2* part = reinterpret_cast<float2*>(wsb + L.part);
   if (merged != nullptr && (!reset_header || y_offset != 0)) return FLCE_ERR_INVALID_ARG;
+  // the header and the row-block counters
   if (reset_header && cudaMemsetAsync(hdr, 0, L.part, st) != cudaSuccess) return FLCE_ERR_CUDA;
 
   Schedule sch;
@@ -296,9 +297,13 @@ flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, 
 }
 
 // fp32 inputs: split `src` (rows, D; row stride ld) into its bf16 (rows,
-// nseg Dp) copy at `dst`: lo in segment lo_segment, hi in the others.
+// nseg Dp) copy at `dst`: lo in segment lo_segment, hi in the others.  With
+// src2 (rows2 rows, row stride ld2, copy at dst2) a second matrix of the same
+// D is split in the same launch.
 flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, int64_t Dp,
-                         int nseg, int lo_segment, void* dst, int sms, cudaStream_t st) {
+                         int nseg, int lo_segment, void* dst, int sms, cudaStream_t st,
+                         const void* src2 = nullptr, int64_t ld2 = 0, int64_t rows2 = 0,
+                         void* dst2 = nullptr) {
   split::Args a;
   a.src = static_cast<const float*>(src);
   a.ld = ld;
@@ -308,14 +313,20 @@ flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, i
   a.nseg = nseg;
   a.lo_segment = lo_segment;
   a.dst = static_cast<__nv_bfloat16*>(dst);
+  split::Args b = a;
+  b.src = static_cast<const float*>(src2);
+  b.ld = ld2;
+  b.rows = src2 != nullptr ? rows2 : 0;
+  b.dst = static_cast<__nv_bfloat16*>(dst2);
   const int64_t warps_per_block = split::NUM_THREADS / 32;
   const int64_t blocks = std::max<int64_t>(
-      1, std::min<int64_t>(cdiv(rows, warps_per_block), int64_t(sms) * 8));
-  const bool vec = D % 8 == 0 && ld % 4 == 0 && aligned16(src);
+      1, std::min<int64_t>(cdiv(rows + b.rows, warps_per_block), int64_t(sms) * 8));
+  const bool vec = D % 8 == 0 && ld % 4 == 0 && aligned16(src) &&
+                   (b.rows == 0 || (ld2 % 4 == 0 && aligned16(src2)));
   if (vec)
-    split::flce_split3_kernel<true><<<unsigned(blocks), split::NUM_THREADS, 0, st>>>(a);
+    split::flce_split3_kernel<true><<<unsigned(blocks), split::NUM_THREADS, 0, st>>>(a, b);
   else
-    split::flce_split3_kernel<false><<<unsigned(blocks), split::NUM_THREADS, 0, st>>>(a);
+    split::flce_split3_kernel<false><<<unsigned(blocks), split::NUM_THREADS, 0, st>>>(a, b);
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
@@ -341,8 +352,9 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
     const int64_t Dp = fwd_split_segment(D);
     uint8_t* hs = wsb + state_bytes_for(N, V);
     uint8_t* wsplit = hs + fwd_split_h_bytes(N, D);
-    if ((s = launch_split(H, ldh, N, D, Dp, 2, 1, hs, di.sms, st)) != FLCE_OK) return s;
-    if ((s = launch_split(W, ldw, V, D, Dp, 2, 1, wsplit, di.sms, st)) != FLCE_OK) return s;
+    // H and W in one launch
+    if ((s = launch_split(H, ldh, N, D, Dp, 2, 1, hs, di.sms, st, W, ldw, V, wsplit)) != FLCE_OK)
+      return s;
     op = Operands{hs, 2 * Dp, 2 * Dp, Dp, wsplit, 2 * Dp, 2 * Dp, Dp, Dp / tc::BK, tc::kSplitHW};
   }
   return launch_contraction(op, y, y_offset, N, V, plan, out_target, ws, true, st, merged);

@@ -274,12 +274,13 @@ __device__ __forceinline__ void rowblock_finish(double l, int t, int rb, int nbl
   const double b = sum128(l, t, red, sync);
   if (t == 0) {
     block_sums[rb] = b;
-    __threadfence();
-    *flag = atomicAdd(counter, 1u) == uint32_t(nblocks - 1);
+    __threadfence();  // release: this block sum before the count
+    const bool last = atomicAdd(counter, 1u) == uint32_t(nblocks - 1);
+    if (last) __threadfence();  // acquire: every block sum, seen through the count
+    *flag = last;
   }
-  sync();
+  sync();  // the other threads read block sums after thread 0's acquire, through L2 only
   if (!*flag || (mean == nullptr && sum == nullptr)) return;
-  __threadfence();  // every block sum, seen through the counter
   double v = 0.0;
   for (int r = t; r < nblocks; r += 128) v += __ldcg(block_sums + r);
   const double total = sum128(v, t, red, sync);
@@ -413,12 +414,19 @@ struct EpiSync {
 __device__ __forceinline__ void fused_merge(const Args& a, int rb, int row, bool valid, int64_t yi,
                                             int t, volatile int* flag, volatile double* red) {
   const EpiSync epi_sync;
-  __threadfence();  // this thread's state and target logit, visible device-wide
+  // Every epilogue thread has written its state and target logit; the barrier
+  // orders those writes before thread 0's release fence and count, and the
+  // CTA that counts last acquires them (and all other CTAs' states of this
+  // block) before its barrier.  The merge reads them through L2 (ld.cg).
   epi_sync();
-  if (t == 0) *flag = atomicAdd(&a.fm.arrivals[rb], 1u) == uint32_t(a.sch.slabs - 1);
+  if (t == 0) {
+    __threadfence();
+    const bool last = atomicAdd(&a.fm.arrivals[rb], 1u) == uint32_t(a.sch.slabs - 1);
+    if (last) __threadfence();
+    *flag = last;
+  }
   epi_sync();
   if (!*flag) return;
-  __threadfence();  // the other CTAs' states of this block, seen through the counter
   double l = 0.0;
   if (valid) {
     const double lse = merge_slab_states(a.part + row, a.sch.slabs, a.N);
@@ -478,12 +486,6 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
     ptx::fence_proxy_async_smem();
     ptx::prefetch_tensormap(&tmH);
     ptx::prefetch_tensormap(&tmW);
-    if (blockIdx.x == 0) {
-      a.hdr->slabs = a.sch.slabs;
-      a.hdr->N = a.N;
-      a.hdr->V = a.V;
-      a.hdr->magic = kWsMagic;
-    }
   }
   if (warp == 1) {
     ptx::tmem_alloc(ptx::smem_addr(tmem_slot), TMEM_COLS);
@@ -493,6 +495,12 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
   __syncthreads();
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  if (threadIdx.x == 0 && blockIdx.x == 0) {
+    a.hdr->slabs = a.sch.slabs;
+    a.hdr->N = a.N;
+    a.hdr->V = a.V;
+    a.hdr->magic = kWsMagic;
+  }
 
   uint32_t* status = &a.hdr->status;
   const uint64_t lim = a.wait_limit_ns;
@@ -731,12 +739,6 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
     ptx::fence_proxy_async_smem();
     ptx::prefetch_tensormap(&tmH);
     ptx::prefetch_tensormap(&tmW);
-    if (blockIdx.x == 0) {
-      a.hdr->slabs = a.sch.slabs;
-      a.hdr->N = a.N;
-      a.hdr->V = a.V;
-      a.hdr->magic = kWsMagic;
-    }
   }
   if (warp == 1) {
     ptx::tmem_alloc_pair(ptx::smem_addr(tmem_slot), TMEM_COLS);
@@ -746,6 +748,12 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
   ptx::cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  if (threadIdx.x == 0 && blockIdx.x == 0) {
+    a.hdr->slabs = a.sch.slabs;
+    a.hdr->N = a.N;
+    a.hdr->V = a.V;
+    a.hdr->magic = kWsMagic;
+  }
 
   uint32_t* status = &a.hdr->status;
   const uint64_t lim = a.wait_limit_ns;
@@ -949,15 +957,23 @@ __device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 a, __nv_bfloat16 b
 
 // Each lane converts groups of 8 consecutive elements of its warp's row: it
 // loads 32 bytes of fp32 (two float4 when `kVec`, i.e. D % 8 == 0, ld % 4 ==
-// 0 and a 16-byte-aligned base) and stores 16 bytes to each of the three
-// segments.  Purely bandwidth-bound: 4 bytes in, 6 bytes out per element.
+// 0 and a 16-byte-aligned base) and stores 16 bytes to each of the
+// segments.  Purely bandwidth-bound: 4 bytes in, 4 or 6 bytes out per
+// element.  One launch splits two matrices (the forward's H and W): the rows
+// of `first`, then those of `second` (second.rows may be 0); both share D, Dp
+// and the segment layout.
 template <bool kVec>
-__global__ void __launch_bounds__(NUM_THREADS) flce_split3_kernel(const Args a) {
+__global__ void __launch_bounds__(NUM_THREADS) flce_split3_kernel(const Args first,
+                                                                  const Args second) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = int64_t(gridDim.x) * (NUM_THREADS / 32);
-  const int groups = a.Dp / 8;
-  for (int64_t r = int64_t(blockIdx.x) * (NUM_THREADS / 32) + (threadIdx.x >> 5); r < a.rows;
-       r += warps) {
+  const int groups = first.Dp / 8;
+  const int64_t total = first.rows + second.rows;
+  for (int64_t rr = int64_t(blockIdx.x) * (NUM_THREADS / 32) + (threadIdx.x >> 5); rr < total;
+       rr += warps) {
+    const bool in_first = rr < first.rows;
+    const Args& a = in_first ? first : second;
+    const int64_t r = in_first ? rr : rr - first.rows;
     const float* row = a.src + r * a.ld;
     uint4* out = reinterpret_cast<uint4*>(a.dst + r * a.nseg * int64_t(a.Dp));
     for (int g = lane; g < groups; g += 32) {
