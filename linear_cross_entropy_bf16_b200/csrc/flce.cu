@@ -195,7 +195,8 @@ struct Operands {
   const void* W;
   int64_t ldw, cols_w, seg_w;
   int64_t kblocks;
-  int layout;  // tc::StageLayout
+  int layout;        // tc::StageLayout
+  int64_t h_rows;    // rows of the H buffer the tensor map covers; 0: N
 };
 
 // Batches of at most this many tokens stream W from HBM faster than the
@@ -258,7 +259,7 @@ flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, 
   if (!load_encoder()) return FLCE_ERR_CUDA;
   const bool pair = plan.ctas_per_unit == 2;
   CUtensorMap tmH, tmW;
-  if (!encode_bf16_rows(&tmH, op.H, N, op.cols_h, op.ldh, tc::BM) ||
+  if (!encode_bf16_rows(&tmH, op.H, op.h_rows > 0 ? op.h_rows : N, op.cols_h, op.ldh, tc::BM) ||
       !encode_bf16_rows(&tmW, op.W, V, op.cols_w, op.ldw, pair ? tc2::HALF_N : tc::BN))
     return FLCE_ERR_UNSUPPORTED;
   tc::Args a;
@@ -299,11 +300,12 @@ flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, 
 // fp32 inputs: split `src` (rows, D; row stride ld) into its bf16 (rows,
 // nseg Dp) copy at `dst`: lo in segment lo_segment, hi in the others.  With
 // src2 (rows2 rows, row stride ld2, copy at dst2) a second matrix of the same
-// D is split in the same launch.
+// D is split in the same launch.  rows_out > rows: the first copy gets zero
+// rows after the source rows, up to rows_out.
 flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, int64_t Dp,
                          int nseg, int lo_segment, void* dst, int sms, cudaStream_t st,
                          const void* src2 = nullptr, int64_t ld2 = 0, int64_t rows2 = 0,
-                         void* dst2 = nullptr) {
+                         void* dst2 = nullptr, int64_t rows_out = 0) {
   split::Args a;
   a.src = static_cast<const float*>(src);
   a.ld = ld;
@@ -313,14 +315,17 @@ flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, i
   a.nseg = nseg;
   a.lo_segment = lo_segment;
   a.dst = static_cast<__nv_bfloat16*>(dst);
+  a.src_rows = rows;
+  if (rows_out > rows) a.rows = rows_out;  // zero rows after the source rows
   split::Args b = a;
   b.src = static_cast<const float*>(src2);
   b.ld = ld2;
   b.rows = src2 != nullptr ? rows2 : 0;
+  b.src_rows = b.rows;
   b.dst = static_cast<__nv_bfloat16*>(dst2);
   const int64_t warps_per_block = split::NUM_THREADS / 32;
   const int64_t blocks = std::max<int64_t>(
-      1, std::min<int64_t>(cdiv(rows + b.rows, warps_per_block), int64_t(sms) * 8));
+      1, std::min<int64_t>(cdiv(a.rows + b.rows, warps_per_block), int64_t(sms) * 8));
   const bool vec = D % 8 == 0 && ld % 4 == 0 && aligned16(src) &&
                    (b.rows == 0 || (ld2 % 4 == 0 && aligned16(src2)));
   if (vec)
@@ -347,15 +352,29 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
   // their [hi | lo] split copies in the workspace (fp32), each K block's four
   // parts staged together for the three products hi hi + hi lo + lo hi.
   Operands op = bf16_operands(H, ldh, W, ldw, N, D);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
   if (dtype == FLCE_FP32) {
-    uint8_t* wsb = static_cast<uint8_t*>(ws);
     const int64_t Dp = fwd_split_segment(D);
     uint8_t* hs = wsb + state_bytes_for(N, V);
     uint8_t* wsplit = hs + fwd_split_h_bytes(N, D);
-    // H and W in one launch
-    if ((s = launch_split(H, ldh, N, D, Dp, 2, 1, hs, di.sms, st, W, ldw, V, wsplit)) != FLCE_OK)
+    // H (padded with zero rows up to kMinHRows) and W in one launch
+    if ((s = launch_split(H, ldh, N, D, Dp, 2, 1, hs, di.sms, st, W, ldw, V, wsplit,
+                          padded_h_rows(N))) != FLCE_OK)
       return s;
-    op = Operands{hs, 2 * Dp, 2 * Dp, Dp, wsplit, 2 * Dp, 2 * Dp, Dp, Dp / tc::BK, tc::kSplitHW};
+    op = Operands{hs, 2 * Dp, 2 * Dp, Dp, wsplit, 2 * Dp, 2 * Dp, Dp, Dp / tc::BK, tc::kSplitHW,
+                  padded_h_rows(N)};
+  } else if (N < kMinHRows) {
+    // a tiny batch: H read from a copy padded with zero rows (kMinHRows)
+    uint8_t* hp = wsb + state_bytes_for(N, V);
+    const int64_t nvec = kMinHRows * (D / 8);
+    split::flce_pad_rows_kernel<<<unsigned(std::min<int64_t>(cdiv(nvec, 256), 4 * di.sms)), 256, 0,
+                                  st>>>(static_cast<const uint4*>(H), ldh / 8, int32_t(N),
+                                        int32_t(D / 8), int32_t(kMinHRows),
+                                        reinterpret_cast<uint4*>(hp));
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    op.H = hp;
+    op.ldh = D;
+    op.h_rows = kMinHRows;
   }
   return launch_contraction(op, y, y_offset, N, V, plan, out_target, ws, true, st, merged);
 }

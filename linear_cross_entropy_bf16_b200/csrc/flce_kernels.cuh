@@ -941,9 +941,10 @@ namespace split {
 constexpr int NUM_THREADS = 256;   // 8 warps, one row per warp at a time
 
 struct Args {
-  const float* src;       // (rows, D) fp32, row stride ld elements
+  const float* src;       // (src_rows, D) fp32, row stride ld elements
   int64_t ld;
-  int64_t rows;
+  int64_t rows;           // rows written; rows >= src_rows are written as zeros
+  int64_t src_rows;
   int32_t D;
   int32_t Dp;             // one segment: D rounded up (to 64 for the forward, 8 for the backward)
   int32_t nseg;           // segments per row: 3, or 2 for [hi | lo]
@@ -974,13 +975,14 @@ __global__ void __launch_bounds__(NUM_THREADS) flce_split3_kernel(const Args fir
     const bool in_first = rr < first.rows;
     const Args& a = in_first ? first : second;
     const int64_t r = in_first ? rr : rr - first.rows;
-    const float* row = a.src + r * a.ld;
+    const bool pad_row = r >= a.src_rows;   // zero padding below the source rows
+    const float* row = a.src + (pad_row ? 0 : r) * a.ld;
     uint4* out = reinterpret_cast<uint4*>(a.dst + r * a.nseg * int64_t(a.Dp));
     for (int g = lane; g < groups; g += 32) {
       const int k0 = g * 8;
       float x[8];
-      if (k0 >= a.D) {
-        // zero padding from D to the segment length: nothing of the row is read
+      if (k0 >= a.D || pad_row) {
+        // zero padding from D to the segment length (or a padding row): nothing is read
 #pragma unroll
         for (int j = 0; j < 8; ++j) x[j] = 0.f;
       } else if (kVec) {        // D % 8 == 0: all 8 elements lie inside the row
@@ -1008,6 +1010,20 @@ __global__ void __launch_bounds__(NUM_THREADS) flce_split3_kernel(const Args fir
       const uint4 vl = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       for (int seg = 0; seg < a.nseg; ++seg) out[seg * groups + g] = seg == a.lo_segment ? vl : vh;
     }
+  }
+}
+
+// bf16 H padded with zero rows: dst (rows_out, D) = src (N rows, row stride
+// ld) followed by rows_out - N zero rows.  16-byte vectors (D and ld are
+// multiples of 8 and src is 16-byte aligned for bf16 inputs).
+__global__ void __launch_bounds__(256) flce_pad_rows_kernel(const uint4* src, int64_t ld_vec,
+                                                            int32_t N, int32_t d_vec,
+                                                            int32_t rows_out, uint4* dst) {
+  const int64_t total = int64_t(rows_out) * d_vec;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / d_vec, c = i - r * d_vec;
+    dst[i] = r < N ? __ldg(src + r * ld_vec + c) : make_uint4(0u, 0u, 0u, 0u);
   }
 }
 

@@ -60,10 +60,23 @@ int64_t k_extent(int64_t D, flce_dtype dtype) {
   return dtype == FLCE_FP32 ? 2 * fwd_split_segment(D) : D;
 }
 
-// Workspace for the forward's split copies of fp32 inputs: H (N, 2 Dp) and
-// W (V, 2 Dp) bf16, each 256-byte aligned.
+// Batches of fewer than this many tokens read H from a copy padded with zero
+// rows up to it.  All CTAs read the same H rows every K block; with 1 to 8
+// rows those few lines are a hot spot that slowed the whole W stream by 20%
+// on B200 (N = 1 and 8: 254-270 us against 208-212 us at N = 32 and 128, V =
+// 151936, D = 4096), and 32 rows spread the reads enough.
+constexpr int64_t kMinHRows = 32;
+int64_t padded_h_rows(int64_t N) { return std::max<int64_t>(N, kMinHRows); }
+
+// bf16 inputs with N < kMinHRows: the padded copy of H (kMinHRows, D) bf16.
+size_t fwd_pad_h_bytes(int64_t N, int64_t D) {
+  return N < kMinHRows ? align256(size_t(kMinHRows) * size_t(D) * 2) : 0;
+}
+
+// Workspace for the forward's split copies of fp32 inputs: H (padded_h_rows,
+// 2 Dp) and W (V, 2 Dp) bf16, each 256-byte aligned.
 size_t fwd_split_h_bytes(int64_t N, int64_t D) {
-  return align256(size_t(N) * size_t(2 * fwd_split_segment(D)) * 2);
+  return align256(size_t(padded_h_rows(N)) * size_t(2 * fwd_split_segment(D)) * 2);
 }
 size_t fwd_split_w_bytes(int64_t V, int64_t D) {
   return align256(size_t(V) * size_t(2 * fwd_split_segment(D)) * 2);
@@ -77,6 +90,7 @@ size_t bwd_split_bytes_for(int64_t rows, int64_t D) {
 size_t workspace_bytes_for(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
   size_t b = state_bytes_for(N, V);
   if (dtype == FLCE_FP32) b += fwd_split_h_bytes(N, D) + fwd_split_w_bytes(V, D);
+  else b += fwd_pad_h_bytes(N, D);
   return b;
 }
 

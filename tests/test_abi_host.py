@@ -47,26 +47,41 @@ def test_status_strings(lib):
     assert flce.status_string(99) == "unknown status"
 
 
+def r256(b):
+    return (b + 255) // 256 * 256
+
+
+def state_bytes(N, V):
+    """The forward's state: header, one counter per 128-token row block (two per 256
+    tokens), the (m, s) partials per (slab, token), one fp64 per 128-token row block."""
+    rb = 2 * math.ceil(max(N, 1) / 256)
+    slabs = min(math.ceil(V / 256), 512)
+    return 256 + r256(4 * rb) + r256(8 * N * slabs) + r256(8 * max(1, math.ceil(N / 128), rb))
+
+
 def test_workspace_is_O_N_not_O_NV(lib):
     for N, V, D in [(8192, 151936, 4096), (16384, 262144, 2048), (1, 1, 8), (4096, 128256, 4096)]:
         ws = flce.workspace_size(N, V, D)
         slabs = min(math.ceil(V / 256), 512)
         assert ws >= 256 + 8 * N * slabs
-        assert ws <= 256 + 8 * N * 512 + 256 + 8 * (N // 32 + 1) + 512
+        assert ws <= 256 + 8 * N * 512 + 256 + 8 * (N // 32 + 1) + 512 + r256(64 * D)
         if V >= 100000:
             assert ws < 4 * N * V / 50        # the logits it replaces are 4 N V bytes
     assert lib.flce_workspace_size(-1, 10, 8, 0) == 0
     assert lib.flce_workspace_size(4, 0, 8, 0) == 0
     assert lib.flce_workspace_size(4, 10, 0, 0) == 0
     assert lib.flce_workspace_size(4, 10, 8, 7) == 0
-    # bf16: independent of D
+    # bf16: the state, independent of D from 32 tokens on; below, plus H padded to
+    # 32 rows (32 D bf16)
     assert flce.workspace_size(100, 5000, 64) == flce.workspace_size(100, 5000, 4096)
-    # fp32: plus the bf16 hi/lo split copies, H (N, 2 Dp) and W (V, 2 Dp), Dp = ceil64(D)
+    for N, V, D in [(100, 5000, 64), (8192, 151936, 4096), (31, 7, 8), (1, 1, 4096), (32, 3, 16)]:
+        pad = r256(64 * D) if N < 32 else 0
+        assert flce.workspace_size(N, V, D) == state_bytes(N, V) + pad
+    # fp32: plus the bf16 hi/lo split copies, H (max(N, 32), 2 Dp) and W (V, 2 Dp), Dp = ceil64(D)
     for N, V, D in [(100, 5000, 64), (256, 2048, 256), (7, 9, 5), (1, 1, 1), (3, 4, 65)]:
         Dp = (D + 63) // 64 * 64
-        r256 = lambda b: (b + 255) // 256 * 256
-        assert flce.workspace_size(N, V, D, 1) == (flce.workspace_size(N, V, D)
-                                                   + r256(4 * Dp * N) + r256(4 * Dp * V))
+        assert flce.workspace_size(N, V, D, 1) == (state_bytes(N, V) + r256(4 * Dp * max(N, 32))
+                                                   + r256(4 * Dp * V))
 
 
 def unit_order(p):
@@ -226,13 +241,11 @@ def test_forward_ex_argument_checks_need_no_gpu(lib):
 
 def test_quantized_workspace_and_argument_checks_need_no_gpu(lib):
     # size: one chunk's slab state + a float4 per (chunk, token) + one chunk of [hi | lo] rows
-    r256 = lambda b: (b + 255) // 256 * 256
     for N, V, D in [(8192, 151936, 4096), (10, 100, 64), (300, 40000, 192)]:
         C = min(V, 16384)
         chunks = math.ceil(V / C)
         Ds = math.ceil(D / 64) * 64
-        state = flce.workspace_size(N, C, 64)           # bf16 state size depends on (N, V) only
-        want = state + r256(16 * N * chunks) + r256(C * 2 * Ds * 2)
+        want = state_bytes(N, C) + r256(16 * N * chunks) + r256(C * 2 * Ds * 2)
         assert flce.quantized_workspace_size(N, V, D, 4, 64) == want
     # far below the 4 N V bytes of logits at the page's shape
     assert flce.quantized_workspace_size(8192, 151936, 4096, 4, 64) < 4 * 8192 * 151936 / 10

@@ -211,6 +211,22 @@ def test_strided_rows_and_int32_targets(dtype, y32):
     assert torch.equal(ref_gpu[0], loss)
 
 
+@pytest.mark.parametrize("dtype,N", [("bf16", 1), ("bf16", 31), ("fp32", 3), ("bf16", 32)])
+def test_tiny_batches_strided(dtype, N):
+    """Fewer than 32 tokens read H from a copy padded with zero rows (bf16: a copy
+    kernel; fp32: the split kernel writes the zero rows); with strided rows too."""
+    import linear_cross_entropy_bf16_b200 as flce
+    V, D, pad = 5000, 256, 24
+    H, W, y = synth.random_inputs(N, V, D + pad, seed=62 + N, dtype=dtype)
+    Hd, Wd, yd = to_device(H, W, y)
+    Hs = Hd[:, pad:]
+    loss, lse, tgt, mean = flce.forward_strided(Hs, Wd[:, :D], yd, check=True)
+    ref = oracle.forward(np.ascontiguousarray(H[:, pad:]), np.ascontiguousarray(W[:, :D]), y)
+    gpu = {"loss": loss.cpu().double().numpy(), "lse": lse.cpu().double().numpy(),
+           "target": tgt.cpu().double().numpy(), "mean": float(mean.item())}
+    compare(gpu, ref, mean_ref=oracle.mean(ref["loss"]))
+
+
 # ---------------------------------------------------------------- fp32 inputs
 # fp32 H and W are split into bf16 hi = bf16(x), lo = bf16(x - hi) and
 # contracted as hi*hi + hi*lo + lo*hi on the tensor cores.  Per product the
