@@ -508,7 +508,8 @@ def run_ours(args, w, rank, world, local_rank):
     # the optional legs take their own max over ranks: every rank runs them
     extra = {}
     if "backward" in legs and w.dtype == "bf16":
-        extra["backward"] = time_backward(flce, H, W, y, fwd.lse, N, V, D, dev, stream, args, peaks, world)
+        extra["backward"] = time_backward(flce, H, W, y, fwd.lse, N, V, D, dev, stream, args, peaks, world,
+                                          local_rank)
     if "quantized" in legs and w.dtype == "bf16":
         bits, gs = (int(v) for v in args.quantized.split(","))
         extra["quantized"] = time_quantized(flce, H, Wn, y, N, V, D, bits, gs, dev, stream, args, peaks,
@@ -725,8 +726,10 @@ def time_e2e(flce, fwd, H_h, W_h, y_h, w, dev, stream, args, world, mean_loss):
                                  "results out every step, around flce_forward"}}
 
 
-def time_backward(flce, H, W, y, lse, N, V, D, dev, stream, args, peaks, world):
-    """The backward (dH, dW of the mean loss) on the same inputs, timed like the forward."""
+def time_backward(flce, H, W, y, lse, N, V, D, dev, stream, args, peaks, world, gpu_index=0):
+    """The backward (dH, dW of the mean loss) on the same inputs: per-step events over
+    at least --backward-steps steps and about 1.5 s, with the SM clock sampled, so that
+    its rate per MHz compares with the forward's sustained window."""
     import torch
     out = {"dH": torch.empty(N, D, device=dev), "dW": torch.empty(V, D, device=dev)}
     ws = torch.empty(flce.backward_workspace_size(N, V, D, H.dtype), dtype=torch.uint8, device=dev)
@@ -734,31 +737,48 @@ def time_backward(flce, H, W, y, lse, N, V, D, dev, stream, args, peaks, world):
     def step():
         flce.backward(H, W, y, lse, None, 1.0 / N, out=out, workspace=ws, stream=stream)
 
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
-        for _ in range(3):
+        for _ in range(2):
             step()
+        e0.record(stream)
+        step()
+        e1.record(stream)
     stream.synchronize()
     if flce.check(ws, stream) != flce.OK:
         raise flce.FlceError(flce.check(ws, stream), "backward")
-    Kb = max(3, args.backward_steps)
+    Kb = max(3, args.backward_steps, int(1500.0 / max(e0.elapsed_time(e1), 1e-3)))
+    Kb = int(max_over_ranks([Kb], world, device=dev)[0])   # the same step count on every rank
+    sampler = ClockSampler(gpu_index)
+    sampler.start()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Kb)]
+    t0 = time.time()
     with torch.cuda.stream(stream):
         for k in range(Kb):
             ev[k][0].record(stream)
             step()
             ev[k][1].record(stream)
     torch.cuda.synchronize(dev)
+    t1 = time.time()
+    sampler.stop()
     per = [ev[k][0].elapsed_time(ev[k][1]) for k in range(Kb)]
     ms, ms_mean = max_over_ranks([median(per), float(np.mean(per))], world, device=dev)
     flops = 3 * 2 * N * V * D          # logits regenerated, dH, dW
     tflops = flops / (ms * 1e-3) / 1e12
-    return {"ms_per_step": ms, "ms_per_step_mean": ms_mean, "steps": Kb,
-            "tokens_per_s": weak_scaling_tokens_per_s(world, N, ms),
-            "flops_per_step": flops, "tflops": tflops, "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
-            "frac_of_sustained_peak": tflops / peaks["bf16_tflops_sustained"],
-            "workspace_bytes": int(ws.numel()),
-            "what": "dH and dW of the mean loss from the forward's lse (3 contractions per step); "
-                    "median of per-step events"}
+    res = {"ms_per_step": ms, "ms_per_step_mean": ms_mean, "steps": Kb,
+           "tokens_per_s": weak_scaling_tokens_per_s(world, N, ms),
+           "flops_per_step": flops, "tflops": tflops, "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
+           "frac_of_sustained_peak": tflops / peaks["bf16_tflops_sustained"],
+           "workspace_bytes": int(ws.numel()),
+           "what": "dH and dW of the mean loss from the forward's lse (3 contractions per step); "
+                   "median of per-step events"}
+    clocks = sampler.summary(t0, t1)
+    if clocks:
+        res["clocks"] = clocks
+        res["tflops_per_mhz"] = tflops / clocks["sm_mhz"]
+        res["frac_of_per_cycle_peak_at_median_clock"] = tflops / (
+            B200_SMS * FLOP_PER_SM_CYCLE * clocks["sm_mhz"] * 1e6 / 1e12)
+    return res
 
 
 def time_quantized(flce, H, Wn, y, N, V, D, bits, gs, dev, stream, args, peaks, world):
