@@ -48,3 +48,20 @@ def test_bench_line_has_the_contract_keys():
     assert d["config"]["workload"] == "n1024_v32000_d1024" and "flushed" in d["config"]["l2"]
     ref = run_bench(*args[:2], "--impl", "reference", "--steps", "2", "--warmup", "3")
     assert ref["impl"] == "reference" and ref["config"] == d["config"]
+
+
+def test_bench_vocab_parallel_mode_on_one_gpu():
+    """`--parallel vocab` with one rank: the whole vocabulary is its shard, the
+    exchange is empty, and the line reports each stage of the forward and the
+    backward."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    d = run_bench("--workload", "n1024_v32000_d1024", "--parallel", "vocab", "--steps", "4", "--warmup", "3")
+    assert d["scaling"] == "strong" and d["n_gpus"] == 1
+    vp = d["vocab_parallel"]
+    f = vp["forward"]
+    assert f["compute_ms"] > 0 and f["merge_ms"] > 0 and f["exchange_bytes_per_rank"] == 0
+    assert f["ms_per_step"] >= f["compute_ms"]
+    assert vp["backward"]["ms_per_step"] > 0
+    assert d["value"] == pytest.approx(1024 / (d["ms_per_step"] * 1e-3), rel=1e-9)
+    assert 8.0 < d["mean_loss"] < 14.0     # about ln 32000 = 10.4 for logits of unit variance
