@@ -335,6 +335,18 @@ flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, i
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
+// bf16 H of a batch of fewer than kMinHRows tokens, copied with zero rows up to
+// kMinHRows into `dst` (kMinHRows x D, contiguous); see kMinHRows.
+flce_status launch_pad_h(const void* H, int64_t ldh, int64_t N, int64_t D, void* dst, int sms,
+                         cudaStream_t st) {
+  const int64_t nvec = kMinHRows * (D / 8);
+  split::flce_pad_rows_kernel<<<unsigned(std::min<int64_t>(cdiv(nvec, 256), 4 * int64_t(sms))), 256,
+                                0, st>>>(static_cast<const uint4*>(H), ldh / 8, int32_t(N),
+                                         int32_t(D / 8), int32_t(kMinHRows),
+                                         static_cast<uint4*>(dst));
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
 // Stage 1 of the forward for bf16 or fp32 H and W (fp32: split first); with
 // `merged`, the whole forward (the merge runs inside the contraction kernel).
 flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t ldw, Targets y,
@@ -366,12 +378,7 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
   } else if (N < kMinHRows) {
     // a tiny batch: H read from a copy padded with zero rows (kMinHRows)
     uint8_t* hp = wsb + state_bytes_for(N, V);
-    const int64_t nvec = kMinHRows * (D / 8);
-    split::flce_pad_rows_kernel<<<unsigned(std::min<int64_t>(cdiv(nvec, 256), 4 * di.sms)), 256, 0,
-                                  st>>>(static_cast<const uint4*>(H), ldh / 8, int32_t(N),
-                                        int32_t(D / 8), int32_t(kMinHRows),
-                                        reinterpret_cast<uint4*>(hp));
-    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    if ((s = launch_pad_h(H, ldh, N, D, hp, di.sms, st)) != FLCE_OK) return s;
     op.H = hp;
     op.ldh = D;
     op.h_rows = kMinHRows;
@@ -973,7 +980,7 @@ int64_t quant_segment(int64_t D) { return cdiv(D, tc::BK) * tc::BK; }
 // expanded [hi | lo] bf16 rows of one chunk.
 struct QuantLayout {
   int64_t C = 0, chunks = 0;
-  size_t state = 0, states = 0, expanded = 0, total = 0;
+  size_t state = 0, states = 0, expanded = 0, pad = 0, total = 0;
 };
 
 QuantLayout quant_layout(int64_t N, int64_t V, int64_t D) {
@@ -983,7 +990,8 @@ QuantLayout quant_layout(int64_t N, int64_t V, int64_t D) {
   L.state = state_bytes_for(N, L.C);
   L.states = align256(size_t(16) * size_t(N) * size_t(L.chunks));
   L.expanded = align256(size_t(L.C) * size_t(2 * quant_segment(D)) * 2);
-  L.total = L.state + L.states + L.expanded;
+  L.pad = fwd_pad_h_bytes(N, D);   // fewer than kMinHRows tokens: H padded with zero rows
+  L.total = L.state + L.states + L.expanded + L.pad;
   return L;
 }
 
@@ -1057,6 +1065,15 @@ extern "C" flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
   // One header for the whole call: its status word collects every stage's
   // findings, and the final merge's block counter starts at zero.
   if (cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess) return FLCE_ERR_CUDA;
+  // A batch of fewer than kMinHRows tokens reads H from a copy padded with zero rows.
+  const void* h_op = H;
+  int64_t h_rows = 0;
+  if (N < kMinHRows) {
+    void* hp = wsb + L.state + L.states + L.expanded;
+    if ((s = launch_pad_h(H, D, N, D, hp, di.sms, st)) != FLCE_OK) return s;
+    h_op = hp;
+    h_rows = kMinHRows;
+  }
   for (int64_t c = 0; c < L.chunks; ++c) {
     const int64_t c0 = c * L.C;
     const int64_t rows = std::min(L.C, V - c0);
@@ -1066,7 +1083,8 @@ extern "C" flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
     flce_plan_t plan;
     make_plan(N, rows, D, FLCE_BF16, workers, &plan);
     // H against the chunk's [hi | lo] rows: H W_hi^T + H W_lo^T per K block
-    const Operands op{H, D, D, 0, expanded, 2 * Ds, 2 * Ds, Ds, Ds / tc::BK, tc::kSplitW};
+    const Operands op{h_op, D, D, 0, expanded, 2 * Ds, 2 * Ds, Ds, Ds / tc::BK, tc::kSplitW,
+                      h_rows};
     if ((s = launch_contraction(op, Targets{y, 0}, c0, N, rows, plan, out_target_logit, workspace,
                                 false, st)) != FLCE_OK)
       return s;
@@ -1225,7 +1243,7 @@ HostLayout host_layout(int64_t N, int64_t V, int64_t D) {
   L.chunks = cdiv(V, L.C);
   L.state = state_bytes_for(N, L.C);
   L.states = align256(size_t(16) * size_t(N) * size_t(L.chunks));
-  L.h = align256(size_t(N) * size_t(D) * 2);
+  L.h = align256(size_t(padded_h_rows(N)) * size_t(D) * 2);   // H, zero rows up to kMinHRows
   L.y = align256(size_t(N) * 8);
   L.outs = align256(size_t(N) * 12 + 4);
   L.staging = align256(size_t(L.C) * size_t(D) * 2);
@@ -1309,9 +1327,13 @@ extern "C" flce_status flce_forward_host(const void* H_host, const void* W_host,
   if (cs != st && (!ok(cudaEventRecord(start, st)) || !ok(cudaStreamWaitEvent(cs, start, 0))))
     return FLCE_ERR_CUDA;
   if (!ok(cudaMemsetAsync(hdr, 0, kHeaderBytes, st))) return FLCE_ERR_CUDA;
-  // H and y first, on the copy stream, ahead of the W chunks.
+  // H and y first, on the copy stream, ahead of the W chunks (a batch of fewer
+  // than kMinHRows tokens gets zero rows after its own, see kMinHRows).
   if (!ok(cudaMemcpyAsync(Hd, H_host, size_t(N) * row_bytes, cudaMemcpyHostToDevice, cs)) ||
       !ok(cudaMemcpyAsync(yd, y_host, size_t(N) * 8, cudaMemcpyHostToDevice, cs)))
+    return FLCE_ERR_CUDA;
+  if (N < kMinHRows && !ok(cudaMemsetAsync(static_cast<uint8_t*>(Hd) + size_t(N) * row_bytes, 0,
+                                           size_t(kMinHRows - N) * row_bytes, cs)))
     return FLCE_ERR_CUDA;
   for (int64_t c = 0; c < L.chunks; ++c) {
     const int b = int(c & 1);
@@ -1325,7 +1347,8 @@ extern "C" flce_status flce_forward_host(const void* H_host, const void* W_host,
       return FLCE_ERR_CUDA;
     flce_plan_t plan;
     make_plan(N, rows, D, FLCE_BF16, workers, &plan);
-    const Operands op = bf16_operands(Hd, D, staging[b], D, N, D);
+    Operands op = bf16_operands(Hd, D, staging[b], D, N, D);
+    op.h_rows = padded_h_rows(N);
     if ((s = launch_contraction(op, Targets{yd, 0}, c0, N, rows, plan, tgt_d, workspace, false,
                                 st)) != FLCE_OK)
       return s;

@@ -245,7 +245,8 @@ def test_quantized_workspace_and_argument_checks_need_no_gpu(lib):
         C = min(V, 16384)
         chunks = math.ceil(V / C)
         Ds = math.ceil(D / 64) * 64
-        want = state_bytes(N, C) + r256(16 * N * chunks) + r256(C * 2 * Ds * 2)
+        pad = r256(64 * D) if N < 32 else 0          # H padded with zero rows to 32
+        want = state_bytes(N, C) + r256(16 * N * chunks) + r256(C * 2 * Ds * 2) + pad
         assert flce.quantized_workspace_size(N, V, D, 4, 64) == want
     # far below the 4 N V bytes of logits at the page's shape
     assert flce.quantized_workspace_size(8192, 151936, 4096, 4, 64) < 4 * 8192 * 151936 / 10
@@ -269,12 +270,13 @@ def test_quantized_workspace_and_argument_checks_need_no_gpu(lib):
 
 
 def test_forward_host_argument_checks_need_no_gpu(lib):
-    r256 = lambda b: (b + 255) // 256 * 256
+    for N, V, D in [(300, 20000, 128), (5, 9000, 64)]:
+        C = min(V, 8192)
+        chunks = math.ceil(V / C)
+        want = (state_bytes(N, C) + r256(16 * N * chunks) + r256(max(N, 32) * D * 2) + r256(8 * N)
+                + r256(12 * N + 4) + 2 * r256(C * D * 2))
+        assert flce.host_workspace_size(N, V, D) == want
     N, V, D = 300, 20000, 128
-    C = 8192
-    want = (flce.workspace_size(N, C, D) + r256(16 * N * 3) + r256(N * D * 2) + r256(8 * N)
-            + r256(12 * N + 4) + 2 * r256(C * D * 2))
-    assert flce.host_workspace_size(N, V, D) == want
     assert lib.flce_forward_host_workspace_size(N, V, 12, 0) == 0      # D % 8
     assert lib.flce_forward_host_workspace_size(N, V, D, 1) == 0       # fp32: not supported
 

@@ -34,7 +34,7 @@ def as_np(res):
             "target": tgt.double().numpy(), "mean": float(mean.item())}
 
 
-@pytest.mark.parametrize("N,V,D", [(1, 1, 8), (129, 8192, 64), (300, 20000, 128), (700, 16385, 64),
+@pytest.mark.parametrize("N,V,D", [(1, 1, 8), (17, 20000, 64), (129, 8192, 64), (300, 20000, 128), (700, 16385, 64),
                                    (64, 30000, 264)])
 def test_host_forward_every_row(N, V, D):
     """One chunk, exactly one chunk, ragged chunks, a one-row last chunk, ragged D."""
