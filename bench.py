@@ -14,8 +14,9 @@ over ranks; `--parallel vocab` splits W's rows over the ranks instead (one
 all-gather of 16 bytes per token per step; scaling is strong).
 
 Also measured in the default run, each in its own object of the same line:
-  * roofline: the forward is one kernel launch (the contraction with the
-    merge in its epilogue); its median duration (CUDA events on its stream)
+  * roofline: the forward is the contraction kernel with the merge in its
+    epilogue, after a one-block kernel that clears the workspace header (the
+    contraction starts early and overlaps it); the step's median duration (CUDA events on its stream)
     over a sustained window of at least --sustain-seconds, against the
     measured bf16 peaks, with the SM clock sampled during that window (median,
     and the kernel's rate binned by clock); the burst figures of the K steps
@@ -338,9 +339,9 @@ def sync(device):
 
 
 class ForwardTimer:
-    """One forward step: flce_forward, one kernel launch (the contraction with the
-    merge in its epilogue) after a small header reset, between two CUDA events on
-    the launching stream."""
+    """One forward step: flce_forward, two launches (a one-block header clear, and
+    the contraction with the merge in its epilogue, which starts early and overlaps
+    it), between two CUDA events on the launching stream."""
 
     def __init__(self, flce, H, W, y, dev, stream):
         import torch
@@ -397,8 +398,8 @@ def sustained_window(timer: ForwardTimer, seconds: float, chunk_steps: int = 20)
 
 
 def sustained_summary(chunks, flops: float, N: int, peaks: dict, sampler: ClockSampler) -> dict:
-    """Medians of the sustained window's steps (the forward is one kernel launch, so
-    the step time is the kernel's), their rate against the peaks, and by clock."""
+    """Medians of the sustained window's steps (the contraction kernel is all but a
+    microsecond of a step), their rate against the peaks, and by clock."""
     kern = [v for c in chunks for v in c[2]]
     km = median(kern)
     res = {"seconds": chunks[-1][1] - chunks[0][0], "steps": len(kern),
@@ -569,7 +570,7 @@ def run_ours(args, w, rank, world, local_rank):
         "sustained": sustained,
         "e2e": e2e["e2e"],
         "e2e_resident_head": e2e["resident"],
-        "gpu_launches": K,
+        "gpu_launches": 2 * K,  # per step: the header clear and the contraction
         "kernel_ms_stats": {"median": median(part_ms), "min": float(np.min(part_ms)),
                             "max": float(np.max(part_ms)), "mean": float(np.mean(part_ms))},
         "env": run_environment(dev),

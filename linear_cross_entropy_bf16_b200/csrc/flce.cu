@@ -214,12 +214,23 @@ Operands bf16_operands(const void* H, int64_t ldh, const void* W, int64_t ldw, i
 }
 
 template <int L>
-void launch_contraction_kernel(bool pair, unsigned grid, const CUtensorMap& tmH,
-                               const CUtensorMap& tmW, const tc::Args& a, cudaStream_t st) {
-  if (pair)
-    tc2::flce_tc2_kernel<L><<<grid, tc2::NUM_THREADS, tc2::Cfg<L>::SMEM_BYTES, st>>>(tmH, tmW, a);
-  else
-    tc::flce_tc_kernel<L><<<grid, tc::NUM_THREADS, tc::Cfg<L>::SMEM_BYTES, st>>>(tmH, tmW, a);
+cudaError_t launch_contraction_kernel(bool pair, unsigned grid, const CUtensorMap& tmH,
+                                      const CUtensorMap& tmW, const tc::Args& a, bool early,
+                                      cudaStream_t st) {
+  // early: programmatic serialization, so that the kernel's prologue and first
+  // loads overlap the header-clearing kernel launched just before it
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(pair ? tc2::NUM_THREADS : tc::NUM_THREADS);
+  cfg.dynamicSmemBytes = pair ? tc2::Cfg<L>::SMEM_BYTES : tc::Cfg<L>::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = early ? attr : nullptr;
+  cfg.numAttrs = early ? 1 : 0;
+  if (pair) return cudaLaunchKernelEx(&cfg, tc2::flce_tc2_kernel<L>, tmH, tmW, a);
+  return cudaLaunchKernelEx(&cfg, tc::flce_tc_kernel<L>, tmH, tmW, a);
 }
 
 // Outputs of the merge when it runs inside the contraction kernel (the whole
@@ -231,22 +242,32 @@ struct MergeOutputs {
   float* sum;   // may be null
 };
 
+// Who clears the workspace header (status word) and the row-block counters
+// (the first state_layout().part bytes) before the contraction: a one-block
+// kernel launched here, which the contraction overlaps (programmatic launch);
+// a kernel of the same call that ran just before (the fp32 split or the
+// tiny-batch H copy, which do it in their first block); or nobody (a chunk of
+// a chunked call, whose caller cleared the header once).
+enum class HeaderReset { kHere, kDoneBefore, kNone };
+
 // The contraction with the online (m, s) epilogue.  Writes (m, s) per (slab,
 // token) into the workspace's state and the target logits W owns; with
-// `merged` also the merged loss, lse, mean and sum (then y_offset must be 0
-// and V the whole vocabulary).  reset_header: clear the header (status word)
-// and the row-block counters first.
+// `merged` also the merged loss, lse, mean and sum (then y_offset must be 0,
+// V the whole vocabulary, and the header and counters cleared for this call).
 flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, int64_t N,
                                int64_t V, const flce_plan_t& plan, float* out_target, void* ws,
-                               bool reset_header, cudaStream_t st,
+                               HeaderReset reset, cudaStream_t st,
                                const MergeOutputs* merged = nullptr) {
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
   const StateLayout L = state_layout(N, V);
   float2* part = reinterpret_cast<float2*>(wsb + L.part);
-  if (merged != nullptr && (!reset_header || y_offset != 0)) return FLCE_ERR_INVALID_ARG;
-  // the header and the row-block counters
-  if (reset_header && cudaMemsetAsync(hdr, 0, L.part, st) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (merged != nullptr && (reset == HeaderReset::kNone || y_offset != 0)) return FLCE_ERR_INVALID_ARG;
+  if (reset == HeaderReset::kHere) {
+    split::flce_clear_header_kernel<<<1, 128, 0, st>>>(reinterpret_cast<uint32_t*>(hdr),
+                                                       int32_t(L.part / 4));
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  }
 
   Schedule sch;
   sch.token_blocks = int32_t(plan.token_blocks);
@@ -287,14 +308,24 @@ flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, 
     a.fm.row_blocks = int32_t(plan.token_blocks * plan.ctas_per_unit);
   }
   const unsigned grid = unsigned(plan.grid);
+  const bool early = reset == HeaderReset::kHere;
+  cudaError_t e;
   switch (op.layout) {
-    case tc::kPlain: launch_contraction_kernel<tc::kPlain>(pair, grid, tmH, tmW, a, st); break;
-    case tc::kSplitW: launch_contraction_kernel<tc::kSplitW>(pair, grid, tmH, tmW, a, st); break;
-    case tc::kSplitHW: launch_contraction_kernel<tc::kSplitHW>(pair, grid, tmH, tmW, a, st); break;
-    case tc::kPlain1: launch_contraction_kernel<tc::kPlain1>(pair, grid, tmH, tmW, a, st); break;
+    case tc::kPlain:
+      e = launch_contraction_kernel<tc::kPlain>(pair, grid, tmH, tmW, a, early, st);
+      break;
+    case tc::kSplitW:
+      e = launch_contraction_kernel<tc::kSplitW>(pair, grid, tmH, tmW, a, early, st);
+      break;
+    case tc::kSplitHW:
+      e = launch_contraction_kernel<tc::kSplitHW>(pair, grid, tmH, tmW, a, early, st);
+      break;
+    case tc::kPlain1:
+      e = launch_contraction_kernel<tc::kPlain1>(pair, grid, tmH, tmW, a, early, st);
+      break;
     default: return FLCE_ERR_INVALID_ARG;
   }
-  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
 // fp32 inputs: split `src` (rows, D; row stride ld) into its bf16 (rows,
@@ -305,7 +336,8 @@ flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, 
 flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, int64_t Dp,
                          int nseg, int lo_segment, void* dst, int sms, cudaStream_t st,
                          const void* src2 = nullptr, int64_t ld2 = 0, int64_t rows2 = 0,
-                         void* dst2 = nullptr, int64_t rows_out = 0) {
+                         void* dst2 = nullptr, int64_t rows_out = 0, void* zero = nullptr,
+                         size_t zero_bytes = 0) {
   split::Args a;
   a.src = static_cast<const float*>(src);
   a.ld = ld;
@@ -317,12 +349,16 @@ flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, i
   a.dst = static_cast<__nv_bfloat16*>(dst);
   a.src_rows = rows;
   if (rows_out > rows) a.rows = rows_out;  // zero rows after the source rows
+  a.zero = static_cast<uint32_t*>(zero);
+  a.zero_words = int32_t(zero_bytes / 4);
   split::Args b = a;
   b.src = static_cast<const float*>(src2);
   b.ld = ld2;
   b.rows = src2 != nullptr ? rows2 : 0;
   b.src_rows = b.rows;
   b.dst = static_cast<__nv_bfloat16*>(dst2);
+  b.zero = nullptr;
+  b.zero_words = 0;
   const int64_t warps_per_block = split::NUM_THREADS / 32;
   const int64_t blocks = std::max<int64_t>(
       1, std::min<int64_t>(cdiv(a.rows + b.rows, warps_per_block), int64_t(sms) * 8));
@@ -337,13 +373,15 @@ flce_status launch_split(const void* src, int64_t ld, int64_t rows, int64_t D, i
 
 // bf16 H of a batch of fewer than kMinHRows tokens, copied with zero rows up to
 // kMinHRows into `dst` (kMinHRows x D, contiguous); see kMinHRows.
+// `zero` (zero_bytes, a multiple of 4, may be null) is cleared by the same launch.
 flce_status launch_pad_h(const void* H, int64_t ldh, int64_t N, int64_t D, void* dst, int sms,
-                         cudaStream_t st) {
+                         cudaStream_t st, void* zero = nullptr, size_t zero_bytes = 0) {
   const int64_t nvec = kMinHRows * (D / 8);
   split::flce_pad_rows_kernel<<<unsigned(std::min<int64_t>(cdiv(nvec, 256), 4 * int64_t(sms))), 256,
                                 0, st>>>(static_cast<const uint4*>(H), ldh / 8, int32_t(N),
                                          int32_t(D / 8), int32_t(kMinHRows),
-                                         static_cast<uint4*>(dst));
+                                         static_cast<uint4*>(dst), static_cast<uint32_t*>(zero),
+                                         int32_t(zero_bytes / 4));
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
@@ -365,25 +403,30 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
   // parts staged together for the three products hi hi + hi lo + lo hi.
   Operands op = bf16_operands(H, ldh, W, ldw, N, D);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
+  // the header and counters: cleared by the kernel that runs first in this call
+  HeaderReset reset = HeaderReset::kHere;
+  const size_t reset_bytes = state_layout(N, V).part;
   if (dtype == FLCE_FP32) {
     const int64_t Dp = fwd_split_segment(D);
     uint8_t* hs = wsb + state_bytes_for(N, V);
     uint8_t* wsplit = hs + fwd_split_h_bytes(N, D);
     // H (padded with zero rows up to kMinHRows) and W in one launch
     if ((s = launch_split(H, ldh, N, D, Dp, 2, 1, hs, di.sms, st, W, ldw, V, wsplit,
-                          padded_h_rows(N))) != FLCE_OK)
+                          padded_h_rows(N), wsb, reset_bytes)) != FLCE_OK)
       return s;
+    reset = HeaderReset::kDoneBefore;
     op = Operands{hs, 2 * Dp, 2 * Dp, Dp, wsplit, 2 * Dp, 2 * Dp, Dp, Dp / tc::BK, tc::kSplitHW,
                   padded_h_rows(N)};
   } else if (N < kMinHRows) {
     // a tiny batch: H read from a copy padded with zero rows (kMinHRows)
     uint8_t* hp = wsb + state_bytes_for(N, V);
-    if ((s = launch_pad_h(H, ldh, N, D, hp, di.sms, st)) != FLCE_OK) return s;
+    if ((s = launch_pad_h(H, ldh, N, D, hp, di.sms, st, wsb, reset_bytes)) != FLCE_OK) return s;
+    reset = HeaderReset::kDoneBefore;
     op.H = hp;
     op.ldh = D;
     op.h_rows = kMinHRows;
   }
-  return launch_contraction(op, y, y_offset, N, V, plan, out_target, ws, true, st, merged);
+  return launch_contraction(op, y, y_offset, N, V, plan, out_target, ws, reset, st, merged);
 }
 
 flce_status launch_merge(Targets y, int64_t N, int64_t V, float* out_loss, float* out_lse,
@@ -1086,7 +1129,7 @@ extern "C" flce_status flce_forward_quantized(const void* H, const uint32_t* wq,
     const Operands op{h_op, D, D, 0, expanded, 2 * Ds, 2 * Ds, Ds, Ds / tc::BK, tc::kSplitW,
                       h_rows};
     if ((s = launch_contraction(op, Targets{y, 0}, c0, N, rows, plan, out_target_logit, workspace,
-                                false, st)) != FLCE_OK)
+                                HeaderReset::kNone, st)) != FLCE_OK)
       return s;
     flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
         reinterpret_cast<const float2*>(wsb + state_layout(N, rows).part), hdr, y, int32_t(N), c0,
@@ -1349,8 +1392,8 @@ extern "C" flce_status flce_forward_host(const void* H_host, const void* W_host,
     make_plan(N, rows, D, FLCE_BF16, workers, &plan);
     Operands op = bf16_operands(Hd, D, staging[b], D, N, D);
     op.h_rows = padded_h_rows(N);
-    if ((s = launch_contraction(op, Targets{yd, 0}, c0, N, rows, plan, tgt_d, workspace, false,
-                                st)) != FLCE_OK)
+    if ((s = launch_contraction(op, Targets{yd, 0}, c0, N, rows, plan, tgt_d, workspace,
+                                HeaderReset::kNone, st)) != FLCE_OK)
       return s;
     flce_shard_state_kernel<<<unsigned(cdiv(N, kMergeThreads)), kMergeThreads, 0, st>>>(
         reinterpret_cast<const float2*>(wsb + state_layout(N, rows).part), hdr, yd, int32_t(N), c0,

@@ -131,6 +131,7 @@ __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile i
       if (flag != nullptr && *flag) return false;
       if (ptx::globaltimer_ns() - t0 > limit_ns) {
         if (flag != nullptr) *flag = 1;
+        ptx::griddep_wait();  // after the kernel that cleared the status word
         atomicOr(status, kStatTimeout);
         return false;
       }
@@ -496,6 +497,7 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
   if (threadIdx.x == 0 && blockIdx.x == 0) {
+    ptx::griddep_wait();  // the header is cleared by the kernel before this one
     a.hdr->slabs = a.sch.slabs;
     a.hdr->N = a.N;
     a.hdr->V = a.V;
@@ -603,6 +605,10 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // The header and the row-block counters may be cleared by the kernel just
+    // before this one, which lets this one start early (programmatic launch):
+    // wait for it before touching them (or the outputs).
+    ptx::griddep_wait();
     const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
     const int row_in_tile = quad * 32 + lane;  // token row of this thread inside the tile
     const uint32_t lane_addr = uint32_t(quad * 32) << 16;
@@ -749,6 +755,7 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
   if (threadIdx.x == 0 && blockIdx.x == 0) {
+    ptx::griddep_wait();  // the header is cleared by the kernel before this one
     a.hdr->slabs = a.sch.slabs;
     a.hdr->N = a.N;
     a.hdr->V = a.V;
@@ -863,6 +870,7 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    ptx::griddep_wait();  // as in flce_tc_kernel
     const int quad = warp & 3;
     const int row_in_tile = quad * 32 + lane;
     const uint32_t lane_addr = uint32_t(quad * 32) << 16;
@@ -950,6 +958,8 @@ struct Args {
   int32_t nseg;           // segments per row: 3, or 2 for [hi | lo]
   int32_t lo_segment;     // the segment that holds lo; every other one holds hi
   __nv_bfloat16* dst;     // (rows, nseg Dp) bf16, contiguous
+  uint32_t* zero;         // first matrix only: words cleared by block 0 (a forward's
+  int32_t zero_words;     // workspace header and counters), or null
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 a, __nv_bfloat16 b) {
@@ -970,6 +980,8 @@ __global__ void __launch_bounds__(NUM_THREADS) flce_split3_kernel(const Args fir
   const int64_t warps = int64_t(gridDim.x) * (NUM_THREADS / 32);
   const int groups = first.Dp / 8;
   const int64_t total = first.rows + second.rows;
+  if (blockIdx.x == 0 && first.zero != nullptr)
+    for (int i = threadIdx.x; i < first.zero_words; i += NUM_THREADS) first.zero[i] = 0u;
   for (int64_t rr = int64_t(blockIdx.x) * (NUM_THREADS / 32) + (threadIdx.x >> 5); rr < total;
        rr += warps) {
     const bool in_first = rr < first.rows;
@@ -1016,9 +1028,23 @@ __global__ void __launch_bounds__(NUM_THREADS) flce_split3_kernel(const Args fir
 // bf16 H padded with zero rows: dst (rows_out, D) = src (N rows, row stride
 // ld) followed by rows_out - N zero rows.  16-byte vectors (D and ld are
 // multiples of 8 and src is 16-byte aligned for bf16 inputs).
+// Clears `n` words at `p` (a forward's workspace header and row-block
+// counters) in one block, and lets the contraction launched after it with
+// programmatic serialization start at once; the contraction waits for it
+// (griddep_wait) before it touches those words.
+__global__ void __launch_bounds__(128) flce_clear_header_kernel(uint32_t* p, int32_t n) {
+  ptx::griddep_launch_dependents();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) p[i] = 0u;
+}
+
+// Block 0 also clears `zero_words` words at `zero` (a forward's workspace
+// header and counters) when `zero` is not null.
 __global__ void __launch_bounds__(256) flce_pad_rows_kernel(const uint4* src, int64_t ld_vec,
                                                             int32_t N, int32_t d_vec,
-                                                            int32_t rows_out, uint4* dst) {
+                                                            int32_t rows_out, uint4* dst,
+                                                            uint32_t* zero, int32_t zero_words) {
+  if (blockIdx.x == 0 && zero != nullptr)
+    for (int i = threadIdx.x; i < zero_words; i += blockDim.x) zero[i] = 0u;
   const int64_t total = int64_t(rows_out) * d_vec;
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += int64_t(gridDim.x) * blockDim.x) {

@@ -136,6 +136,16 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&u)[32]
       : "memory");
 }
 
+// Programmatic dependent launch.  griddep_wait: block until the grids this
+// one was launched to overlap with have completed and their writes are
+// visible (returns at once when there are none).  griddep_launch_dependents:
+// let the next grid on the stream, launched with programmatic serialization,
+// start before this one ends.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Barrier `id` (1-15) among `nthreads` threads (whole warps) of the CTA.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
