@@ -1091,7 +1091,7 @@ def run_vocab(args, w, rank, world, local_rank):
                 "h2d_bytes_per_step": int(H_h.numel() * 2 + y_h.numel() * 8),
                 "d2h_bytes_per_step": int(w.N * 4 + 4), "ms_per_step": e2e_ms,
                 "what": "W shards resident; H and y copied in and loss, mean out every step (host clock)"},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 4 * args.steps,  # per step: header clear, contraction, shard state, merge
         "mean_loss": float(res["mean"].item()),
         "env": run_environment(dev),
     }

@@ -221,31 +221,51 @@ __device__ __forceinline__ void fold_tile(uint32_t taddr, int ncols, int64_t rel
 // The merge of one token's P slab states part[p * N] (p = 0 .. P-1), the
 // recurrence of section 1 applied to whole slabs in slab order:
 // m = max_p m_p, s = sum_p s_p exp(m_p - m), accumulated in fp64, with a
-// running maximum over batches of 16 slabs (sixteen independent loads in
-// flight, one pass); returns lse = m + log s (log in fp64).  Each factor
+// running maximum over batches of 16 slabs (one pass); returns lse = m + log s (log in fp64).  Each factor
 // exp(m_p - m) is evaluated as 2^((m_p - m) log2 e) on the SFU, as the
 // contraction's own exponentials are: relative error about 2^-22 per term,
 // and the slab holding the maximum contributes exactly s_p.  Every slab holds
 // at least one real column, so m is finite.
+// Loads slab states p0 .. p0 + 15 of a token (past P: empty states).
+__device__ __forceinline__ void load_slab_batch(float2 (&b)[16], const float2* part, int p0, int P,
+                                                int N) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j)
+    b[j] = p0 + j < P ? __ldcg(part + size_t(p0 + j) * size_t(N)) : make_float2(-INFINITY, 0.f);
+}
+
+// Folds one batch of 16 states into the running (M, S).
+__device__ __forceinline__ void fold_slab_batch(const float2 (&b)[16], float& M, double& S) {
+  float mb = b[0].x;
+#pragma unroll
+  for (int j = 1; j < 16; ++j) mb = fmaxf(mb, b[j].x);
+  if (mb > M) {  // rescale the running sum (on the first batch S = 0 and 2^-inf = 0)
+    S *= double(ptx::ex2(__fmul_rn(M - mb, kLog2e)));
+    M = mb;
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) S += double(b[j].y * ptx::ex2(__fmul_rn(b[j].x - M, kLog2e)));
+}
+
 __device__ __forceinline__ double merge_slab_states(const float2* part, int P, int N) {
-  constexpr int kBatch = 16;
+  // Batches of 16 states in three register buffers that take turns: a batch
+  // is loaded two batches ahead of its fold, so that the L2 round trips
+  // overlap the folds (no buffer is copied into another, which would wait
+  // for the loads).  The arithmetic is batch by batch in slab order.
+  float2 b0[16], b1[16], b2[16];
+  load_slab_batch(b0, part, 0, P, N);
+  if (P > 16) load_slab_batch(b1, part, 16, P, N);
   float M = -INFINITY;
   double S = 0.0;
-  for (int p0 = 0; p0 < P; p0 += kBatch) {
-    float2 st[kBatch];
-#pragma unroll
-    for (int j = 0; j < kBatch; ++j)
-      st[j] = p0 + j < P ? __ldcg(part + size_t(p0 + j) * size_t(N)) : make_float2(-INFINITY, 0.f);
-    float mb = st[0].x;
-#pragma unroll
-    for (int j = 1; j < kBatch; ++j) mb = fmaxf(mb, st[j].x);
-    if (mb > M) {  // rescale the running sum (on the first batch S = 0 and 2^-inf = 0)
-      S *= double(ptx::ex2(__fmul_rn(M - mb, kLog2e)));
-      M = mb;
-    }
-#pragma unroll
-    for (int j = 0; j < kBatch; ++j)
-      S += double(st[j].y * ptx::ex2(__fmul_rn(st[j].x - M, kLog2e)));
+  for (int p0 = 0; p0 < P; p0 += 48) {
+    if (p0 + 32 < P) load_slab_batch(b2, part, p0 + 32, P, N);
+    fold_slab_batch(b0, M, S);
+    if (p0 + 16 >= P) break;
+    if (p0 + 48 < P) load_slab_batch(b0, part, p0 + 48, P, N);
+    fold_slab_batch(b1, M, S);
+    if (p0 + 32 >= P) break;
+    if (p0 + 64 < P) load_slab_batch(b1, part, p0 + 64, P, N);
+    fold_slab_batch(b2, M, S);
   }
   return double(M) + log(S);
 }
@@ -265,19 +285,27 @@ __device__ __forceinline__ double sum128(double v, int t, volatile double* red, 
 // Row block `rb` (128 tokens, thread t holding token loss `l`) records its
 // loss sum; the row block that finishes last of `nblocks` adds the block sums
 // (thread t: blocks t, t + 128, ... in order, then sum128) into the mean and
-// the sum, and resets the counter.  The same order for any set of finishing
-// times, so results are bitwise deterministic.
+// the sum, and resets the counter (a single block's sum is the total: no
+// count).  The same order for any set of finishing times, so results are
+// bitwise deterministic.
 template <class Sync>
 __device__ __forceinline__ void rowblock_finish(double l, int t, int rb, int nblocks,
                                                 double* block_sums, uint32_t* counter, float* mean,
                                                 float* sum, int N, volatile double* red,
                                                 volatile int* flag, Sync sync) {
   const double b = sum128(l, t, red, sync);
+  if (nblocks == 1) {  // the only block: its sum is the total (no count, no reload)
+    if (t == 0) {
+      if (mean != nullptr) *mean = float(b / double(N));
+      if (sum != nullptr) *sum = float(b);
+    }
+    return;
+  }
   if (t == 0) {
     block_sums[rb] = b;
-    __threadfence();  // release: this block sum before the count
+    ptx::fence_acq_rel_gpu();  // release: this block sum before the count
     const bool last = atomicAdd(counter, 1u) == uint32_t(nblocks - 1);
-    if (last) __threadfence();  // acquire: every block sum, seen through the count
+    if (last) ptx::fence_acq_rel_gpu();  // acquire: every block sum, seen through the count
     *flag = last;
   }
   sync();  // the other threads read block sums after thread 0's acquire, through L2 only
@@ -421,23 +449,25 @@ __device__ __forceinline__ void fused_merge(const Args& a, int rb, int row, bool
   // block) before its barrier.  The merge reads them through L2 (ld.cg).
   epi_sync();
   if (t == 0) {
-    __threadfence();
+    ptx::fence_acq_rel_gpu();
     const bool last = atomicAdd(&a.fm.arrivals[rb], 1u) == uint32_t(a.sch.slabs - 1);
-    if (last) __threadfence();
+    if (last) ptx::fence_acq_rel_gpu();
     *flag = last;
   }
   epi_sync();
   if (!*flag) return;
   double l = 0.0;
   if (valid) {
+    const bool target_ok = yi >= 0 && yi < a.V;
+    const float zt = target_ok ? __ldcg(a.target_logit + row) : 0.f;  // in flight with the states
     const double lse = merge_slab_states(a.part + row, a.sch.slabs, a.N);
     float loss_f;
-    if (yi < 0 || yi >= a.V) {  // no slab holds the target: invalid input
+    if (!target_ok) {  // no slab holds the target: invalid input
       loss_f = __int_as_float(0x7fc00000);
       a.target_logit[row] = loss_f;
       atomicOr(&a.hdr->status, kStatTarget);
     } else {
-      loss_f = float(lse - double(__ldcg(a.target_logit + row)));
+      loss_f = float(lse - double(zt));
     }
     a.fm.loss[row] = loss_f;
     a.fm.lse[row] = float(lse);
@@ -1292,13 +1322,13 @@ __global__ void __launch_bounds__(kMergeThreads) flce_merge_shards_kernel(
     double b = 0.0;
     for (int w = 0; w < kMergeThreads / 32; ++w) b += warp_sums[w];
     block_sums[blockIdx.x] = b;
-    __threadfence();
+    ptx::fence_acq_rel_gpu();  // release: this block sum before the count
     const uint32_t ticket = atomicAdd(&hdr->counter, 1u);
     is_last = ticket == gridDim.x - 1;
   }
   __syncthreads();
   if (is_last && threadIdx.x == 0) {
-    __threadfence();
+    ptx::fence_acq_rel_gpu();  // acquire: every block sum, seen through the count
     const volatile double* bs = block_sums;
     double total = 0.0;
     for (int b = 0; b < int(gridDim.x); ++b) total += bs[b];

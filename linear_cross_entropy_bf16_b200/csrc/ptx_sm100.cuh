@@ -146,6 +146,12 @@ __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Acquire-release fence at GPU scope (lighter than the sequentially consistent
+// __threadfence, which is all a last-arriver count needs: the writes before
+// it, including those of the CTA's threads ordered before by a barrier, are
+// released to the CTA that counts last, which acquires them with its own).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 // Barrier `id` (1-15) among `nthreads` threads (whole warps) of the CTA.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

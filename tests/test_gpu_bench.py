@@ -33,7 +33,7 @@ def test_bench_line_has_the_contract_keys():
               "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches",
               "clocks", "cpu_baseline", "sustained"):
         assert k in d, k
-    assert d["steps"] == 4 and d["warmup"] == 3 and d["n_gpus"] == 1 and d["gpu_launches"] == 4
+    assert d["steps"] == 4 and d["warmup"] == 3 and d["n_gpus"] == 1 and d["gpu_launches"] == 8
     assert d["value"] == pytest.approx(1024 / (d["ms_per_step"] * 1e-3), rel=1e-9)
     r = d["roofline"]
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["peak"] > 0
