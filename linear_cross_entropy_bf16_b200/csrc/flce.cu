@@ -245,9 +245,10 @@ struct MergeOutputs {
 // Who clears the workspace header (status word) and the row-block counters
 // (the first state_layout().part bytes) before the contraction: a one-block
 // kernel launched here, which the contraction overlaps (programmatic launch);
-// a kernel of the same call that ran just before (the fp32 split or the
-// tiny-batch H copy, which do it in their first block); or nobody (a chunk of
-// a chunked call, whose caller cleared the header once).
+// the kernel launched just before that writes the operands (the fp32 split
+// or the tiny-batch H copy, which clear them in their first block; the
+// contraction overlaps it too and its producer waits for it); or nobody (a
+// chunk of a chunked call, whose caller cleared the header once).
 enum class HeaderReset { kHere, kDoneBefore, kNone };
 
 // The contraction with the online (m, s) epilogue.  Writes (m, s) per (slab,
@@ -308,7 +309,11 @@ flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, 
     a.fm.row_blocks = int32_t(plan.token_blocks * plan.ctas_per_unit);
   }
   const unsigned grid = unsigned(plan.grid);
-  const bool early = reset == HeaderReset::kHere;
+  // Launched to overlap the kernel before it: the header clear (which it
+  // waits for before touching the header), or the split / padded copy of the
+  // operands (which the producer waits for before its first load).
+  const bool early = reset == HeaderReset::kHere || reset == HeaderReset::kDoneBefore;
+  a.wait_operands = reset == HeaderReset::kDoneBefore ? 1 : 0;
   cudaError_t e;
   switch (op.layout) {
     case tc::kPlain:

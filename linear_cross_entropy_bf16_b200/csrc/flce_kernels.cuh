@@ -423,6 +423,8 @@ struct Args {
   Schedule sch;
   uint64_t wait_limit_ns;
   FusedMerge fm;
+  int32_t wait_operands;   // 1: H or W is written by the kernel launched just before this
+                           // one, which this one may overlap: the producer waits for it
 };
 
 // Barrier over the 128 epilogue threads (warps 2-5) of a contraction CTA:
@@ -541,6 +543,7 @@ flce_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      if (a.wait_operands) ptx::griddep_wait();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t used = 0, last_parity = 0;  // per stage: ever issued / parity of last issue
@@ -799,6 +802,7 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
+      if (a.wait_operands) ptx::griddep_wait();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t used = 0, last_parity = 0;
@@ -1010,6 +1014,7 @@ __global__ void __launch_bounds__(NUM_THREADS) flce_split3_kernel(const Args fir
   const int64_t warps = int64_t(gridDim.x) * (NUM_THREADS / 32);
   const int groups = first.Dp / 8;
   const int64_t total = first.rows + second.rows;
+  ptx::griddep_launch_dependents();  // a contraction after this launch may start (and wait)
   if (blockIdx.x == 0 && first.zero != nullptr)
     for (int i = threadIdx.x; i < first.zero_words; i += NUM_THREADS) first.zero[i] = 0u;
   for (int64_t rr = int64_t(blockIdx.x) * (NUM_THREADS / 32) + (threadIdx.x >> 5); rr < total;
@@ -1073,6 +1078,7 @@ __global__ void __launch_bounds__(256) flce_pad_rows_kernel(const uint4* src, in
                                                             int32_t N, int32_t d_vec,
                                                             int32_t rows_out, uint4* dst,
                                                             uint32_t* zero, int32_t zero_words) {
+  ptx::griddep_launch_dependents();  // a contraction after this launch may start (and wait)
   if (blockIdx.x == 0 && zero != nullptr)
     for (int i = threadIdx.x; i < zero_words; i += blockDim.x) zero[i] = 0u;
   const int64_t total = int64_t(rows_out) * d_vec;
