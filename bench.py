@@ -629,6 +629,9 @@ def time_workload(flce, w, dev, stream, args, peaks, flush):
            "kernel_ms": km, "kernel_ms_min": float(np.min(kern)), **roofline_numbers(w.flops, km, peaks),
            "l2": "flushed between steps" if needs_flush else "inputs larger than L2, no flush",
            "mean_loss": float(t.mean.item())}
+    # DRAM bytes per launch from the committed ncu summary of this kernel and workload
+    # (null when there is none, or when the kernel's sources changed since it was taken)
+    res["traffic"] = profiled_traffic(w.name, res["kernel"])
     if w.dtype == "fp32":
         Dp = (w.D + 63) // 64 * 64
         tensor = 2 * w.N * w.V * 3 * Dp
