@@ -340,3 +340,40 @@ def test_loss_sum_output_quantized():
                            torch.from_numpy(bi).view(torch.bfloat16).to(dev),
                            torch.from_numpy(y).to(dev), bits, G, out={"sum": total}, check=True)
     assert abs(float(total.item()) - want) <= MEAN_RTOL * abs(want)
+
+
+# Slab counts P on both sides of every batch edge of the merge (batches of 16
+# slab states, loaded two batches ahead in three buffers that take turns: the
+# merge leaves its loop after the first, second or third buffer of a round).
+# N = 64 runs on the single-CTA kernel, where the planner gives one slab per
+# vocabulary tile up to 148 tiles; N = 300 on CTA pairs.  V = 256 tiles - 37
+# keeps a ragged last tile.
+MERGE_SLAB_COUNTS = [(64, t, t) for t in (1, 15, 16, 17, 32, 33, 48, 49, 64, 65, 97, 148)] + \
+                    [(300, 5, 5), (300, 17, 17), (300, 33, 33), (300, 148, 37)]
+
+
+@pytest.mark.parametrize("N,tiles,P", MERGE_SLAB_COUNTS)
+def test_fused_merge_every_slab_count(N, tiles, P):
+    import linear_cross_entropy_bf16_b200 as flce
+    V, D = 256 * tiles - 37, 64
+    # the planned P on 148 SMs (the pair kernel's P follows the pairs that are
+    # resident on the device, so it is checked for the single-CTA kernel only)
+    assert flce.plan(N, V, D)["slabs"] == P
+    if N == 64:
+        props = torch.cuda.get_device_properties(0)
+        assert flce.plan(N, V, D, sm_count=props.multi_processor_count)["slabs"] == min(P, props.multi_processor_count)
+    H, W, y = synth.random_inputs(N, V, D, seed=1000 + N + tiles)
+    gpu = run(H, W, y)
+    ref = oracle.forward(H, W, y)
+    compare(gpu, ref, mean_ref=oracle.mean(ref["loss"]))
+    # the two-stage forward (flce_merge_kernel) agrees bit for bit
+    Hd, Wd, yd = to_device(H, W, y)
+    one = flce.forward(Hd, Wd, yd)
+    ws = torch.empty(flce.workspace_size(N, V, D), dtype=torch.uint8, device="cuda")
+    loss, lse, tgt = (torch.empty(N, device="cuda") for _ in range(3))
+    mean = torch.empty((), device="cuda")
+    flce.partials(Hd, Wd, yd, tgt, ws)
+    flce.merge(yd, V, loss, lse, tgt, mean, ws)
+    assert flce.check(ws) == flce.OK
+    for x, z in zip(one, (loss, lse, tgt, mean)):
+        assert torch.equal(x, z)
