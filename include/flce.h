@@ -121,11 +121,13 @@ FLCE_API flce_status flce_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype
  *                contents on entry are ignored; it holds the status word that
  *                flce_check() reads until the next call that uses it
  *   stream       cudaStream_t
- * One kernel launch (after a reset of the workspace header, and for fp32
- * inputs the split of H and W): the CTA that writes the last vocab slab's
- * state of a 128-token row block merges that block in the same kernel, and
- * the one that merges the last row block forms the mean.  The results equal
- * those of flce_partials followed by flce_merge bit for bit.
+ * One contraction launch, after a kernel that clears the workspace header:
+ * a one-block clear that the contraction overlaps (programmatic stream
+ * serialization), or for fp32 inputs the split of H and W and for N < 32 the
+ * padded copy of H, which clear it in their first block.  The CTA that writes
+ * the last vocab slab's state of a 128-token row block merges that block in
+ * the same kernel, and the one that merges the last row block forms the mean.
+ * The results equal those of flce_partials followed by flce_merge bit for bit.
  * A row whose target is out of range gets NaN loss and NaN target logit and
  * sets FLCE_ERR_TARGET_OUT_OF_RANGE for flce_check().  N == 0 is a no-op that
  * returns FLCE_OK and writes nothing (out_mean untouched).
