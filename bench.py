@@ -108,6 +108,11 @@ def run_environment(dev) -> dict:
     import torch
     env = {"kernel_sources_sha256": kernel_sources_sha256(), "gpu": torch.cuda.get_device_name(dev),
            "torch": torch.__version__, "cuda_runtime": torch.version.cuda}
+    # CTA pairs on the two L2 partitions, as mapped by the first large forward
+    # (the pair kernel's partition-aware order), or None if it was not taken
+    import linear_cross_entropy_bf16_b200 as flce
+    pm = flce.partition_map(dev)
+    env["l2_partition_pairs"] = list(pm) if pm is not None else None
     try:
         h = hashlib.sha256()
         with open(os.path.abspath(__file__), "rb") as f:

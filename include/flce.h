@@ -106,6 +106,44 @@ FLCE_API size_t flce_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype 
 FLCE_API flce_status flce_plan(int64_t N, int64_t V, int64_t D, flce_dtype dtype, int32_t sm_count,
                       flce_plan_t* plan);
 
+/* The partition-aware order of the pair kernel's work units (host only, no
+ * GPU call).  B200's L2 is two partitions, each caching what its own SMs
+ * read.  When a forward has at least 16 units per CTA pair and more token
+ * blocks than one raster group (flce_plan_t group_blocks), the pairs on
+ * partition 0 take the first side0_units units of the token-block-major
+ * order and the pairs on partition 1 the rest, each side slab-major over its
+ * own token blocks (the units and their arithmetic are those of the plain
+ * order; only which pair computes which unit changes, so results are bitwise
+ * the same).  The first such forward on a device maps the partitions with two
+ * small kernels on the caller's stream and waits for them (once per device;
+ * not while the stream is being captured into a CUDA graph, where the plain
+ * order is used until a forward runs outside a capture).
+ *
+ * flce_partition_order writes, for token_blocks TB and slabs P, the (slab,
+ * token block) of each unit of partition 0's list and then of partition 1's:
+ * 2 TB P int32 values to out.  FLCE_ERR_INVALID_ARG if TB < 1, P < 1,
+ * TB P >= 2^30, side0_units outside [0, TB P] or out NULL.
+ *
+ * flce_partition_take: the (partition, rank) a pair takes when it arrives as
+ * number `arrival` (from 0) on partition `side`, with pairs0 and pairs1 pairs
+ * planned on the two partitions and pairs0 + pairs1 pairs launched: its own
+ * rank while the side has fewer than planned, else the highest rank of the
+ * other side that no pair of that side can reach.  FLCE_ERR_INVALID_ARG if a
+ * count is < 1, side is not 0 or 1, arrival is outside [0, pairs0 + pairs1)
+ * or an output is NULL. */
+FLCE_API flce_status flce_partition_order(int32_t token_blocks, int32_t slabs,
+                                          int32_t side0_units, int32_t* out);
+FLCE_API flce_status flce_partition_take(int32_t pairs0, int32_t pairs1, int32_t side,
+                                         int32_t arrival, int32_t* out_side, int32_t* out_rank);
+
+/* The current device's partition map, if a forward has taken it: the CTA
+ * pairs found resident on partitions 0 and 1 (out_pairs[2]).  Returns
+ * FLCE_ERR_UNSUPPORTED while there is none (no forward large enough has run
+ * on the device, or the latencies did not split into two clear groups, in
+ * which case every forward uses the plain order), FLCE_ERR_INVALID_ARG for a
+ * NULL pointer.  Host only: reads what the library recorded. */
+FLCE_API flce_status flce_partition_map(int32_t* out_pairs);
+
 /*
  * The full forward: per-token loss, log-sum-exp and target logit, and the
  * mean loss.  Section 1 of the page: loss_i = logsumexp(Z_i) - Z_{i, y_i}.

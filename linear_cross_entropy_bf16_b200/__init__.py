@@ -118,6 +118,13 @@ def load_library():
         lib.flce_workspace_size.restype = sz
         lib.flce_plan.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int32, ctypes.POINTER(Plan)]
         lib.flce_plan.restype = st
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        lib.flce_partition_order.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, i32p]
+        lib.flce_partition_order.restype = st
+        lib.flce_partition_take.argtypes = [ctypes.c_int32] * 4 + [i32p, i32p]
+        lib.flce_partition_take.restype = st
+        lib.flce_partition_map.argtypes = [i32p]
+        lib.flce_partition_map.restype = st
         lib.flce_forward.argtypes = [vp, vp, vp, i64, i64, i64, ctypes.c_int, vp, vp, vp, vp, vp, sz, vp]
         lib.flce_forward.restype = st
         lib.flce_partials.argtypes = [vp, vp, vp, i64, i64, i64, ctypes.c_int, vp, vp, sz, vp]
@@ -571,6 +578,17 @@ def merge(y, V, loss, lse, target_logit, mean, workspace, stream=None):
                                         workspace.data_ptr(),
                                         workspace.numel() * workspace.element_size(), sp),
               "flce_merge")
+
+
+def partition_map(device=None):
+    """CTA pairs on the two L2 partitions of the device, as mapped by the first
+    forward large enough for the partition-aware order, or None (see
+    flce_partition_map)."""
+    lib = load_library()
+    if device is not None:
+        torch.cuda.set_device(device)
+    out = (ctypes.c_int32 * 2)()
+    return (out[0], out[1]) if lib.flce_partition_map(out) == OK else None
 
 
 def check(workspace: torch.Tensor, stream=None) -> int:

@@ -233,6 +233,180 @@ cudaError_t launch_contraction_kernel(bool pair, unsigned grid, const CUtensorMa
   return cudaLaunchKernelEx(&cfg, tc::flce_tc_kernel<L>, tmH, tmW, a);
 }
 
+// ---- The partition-aware order of the pair kernel (tc::PartArgs) ----
+//
+// Which L2 partition each SM reads through is found once per device by two
+// small kernels on the caller's stream, whose results the host waits for:
+// dependent atomic adds from every SM to lines spread over memory (an add
+// completes at the slice that homes its line, so each line shows a short
+// latency from the SMs of its partition and a long one from the others), and
+// a launch of as many CTA pairs as can be resident that records where they
+// land.  Measured on B200: 266-272 against 708-773 cycles, SMs in two groups
+// of 70 and 78 (74 and 74 on another GPU); N=8192 V=151936 D=4096 read 1.70
+// GB from DRAM per launch in this order against 3.38 GB (same box, same
+// call), and the results are bitwise those of the plain order.
+constexpr int kPartLines = 64;
+constexpr int kPartLineWords = 4096;  // lines 16 KiB apart
+constexpr size_t kPartLinesBytes = size_t(kPartLines) * kPartLineWords * 4;
+constexpr int kPartMaxSms = 256;
+constexpr size_t kPartCalBytes =
+    kPartLinesBytes + size_t(kPartMaxSms) * kPartLines * 4 + size_t(2 * kPartMaxSms + 2) * 4;
+// Units per pair below which the order is not used: each side's share of the
+// units is rounded, so a side may run one unit more per pair than the plain
+// order (N=2048 V=32000 D=1024, one unit per pair, ran 66% slower).
+constexpr int64_t kPartMinUnitsPerPair = 16;
+// Each partition's rows of H (bf16 bytes) must stay well inside its half of
+// the L2 beside the W tiles in flight.
+constexpr int64_t kPartHBytes = 40ll << 20;
+// The order's two pair counters sit in the workspace header, after WsHeader.
+constexpr size_t kPartRegOffset = 128;
+static_assert(sizeof(WsHeader) <= kPartRegOffset && kPartRegOffset + 8 <= kHeaderBytes, "header");
+
+struct PartMap {
+  bool tried = false, ok = false;
+  int32_t npairs = 0;       // pairs resident when the map was taken
+  int32_t pairs[2] = {0, 0};
+  uint8_t side[kPartMaxSms] = {};
+};
+std::mutex g_part_mu;
+PartMap g_part_map[64];
+
+// Takes the map of the current device (first kPartCalBytes of `ws` as
+// scratch, on `st`, waiting for the result).  Leaves m.ok false when the
+// latencies do not fall into two clear groups.
+void calibrate_partitions(int sms, int npairs, uint8_t* ws, cudaStream_t st, PartMap& m) {
+  m.tried = true;
+  if (sms > kPartMaxSms || npairs < 2) return;
+  const int smem = tc2::Cfg<tc::kPlain>::SMEM_BYTES;
+  if (ensure_smem_limit(reinterpret_cast<const void*>(tc2::flce_part_latency_kernel), smem) !=
+          FLCE_OK ||
+      ensure_smem_limit(reinterpret_cast<const void*>(tc2::flce_part_cluster_kernel), smem) != FLCE_OK)
+    return;
+  uint32_t* lines = reinterpret_cast<uint32_t*>(ws);
+  uint32_t* lat = reinterpret_cast<uint32_t*>(ws + kPartLinesBytes);
+  int32_t* smid_blk = reinterpret_cast<int32_t*>(lat + size_t(kPartMaxSms) * kPartLines);
+  int32_t* smid_pair = smid_blk + kPartMaxSms;
+  uint32_t* ctr = reinterpret_cast<uint32_t*>(smid_pair + kPartMaxSms);  // arrived, timed out
+  if (cudaMemsetAsync(ws, 0, kPartCalBytes, st) != cudaSuccess) return;
+  tc2::flce_part_latency_kernel<<<unsigned(sms), 32, smem, st>>>(lines, kPartLines, kPartLineWords,
+                                                                  lat, smid_blk);
+  tc2::flce_part_cluster_kernel<<<unsigned(2 * npairs), 32, smem, st>>>(smid_pair, ctr, ctr + 1);
+  std::vector<uint32_t> hl;
+  std::vector<int32_t> hb, hp;
+  hl.resize(size_t(sms) * kPartLines);
+  hb.resize(size_t(sms));
+  hp.resize(size_t(npairs));
+  uint32_t hc[2] = {0, 0};
+  if (cudaGetLastError() != cudaSuccess ||
+      cudaMemcpyAsync(hl.data(), lat, hl.size() * 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(hb.data(), smid_blk, hb.size() * 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(hp.data(), smid_pair, hp.size() * 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(hc, ctr, 8, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return;
+  }
+  if (hc[1] != 0) return;  // not every pair could be resident at once
+  // near (0) or far (1) per block and line, for the lines whose latencies split
+  // clearly (the longest at least 1.5 x the shortest)
+  std::vector<int> usable;
+  std::vector<uint8_t> far(hl.size());
+  for (int l = 0; l < kPartLines; ++l) {
+    uint32_t lo = ~0u, hi = 0;
+    for (int b = 0; b < sms; ++b) {
+      lo = std::min(lo, hl[size_t(b) * kPartLines + l]);
+      hi = std::max(hi, hl[size_t(b) * kPartLines + l]);
+    }
+    if (lo == 0 || uint64_t(hi) * 2 < uint64_t(lo) * 3) continue;
+    usable.push_back(l);
+    for (int b = 0; b < sms; ++b)
+      far[size_t(b) * kPartLines + l] = uint64_t(hl[size_t(b) * kPartLines + l]) * 2 > uint64_t(lo) + hi;
+  }
+  if (usable.size() < 16) return;
+  uint8_t side[kPartMaxSms] = {};
+  bool seen[kPartMaxSms] = {};
+  for (int b = 0; b < sms; ++b) {
+    int agree = 0;
+    for (int l : usable) agree += far[size_t(b) * kPartLines + l] == far[l];
+    const int n = int(usable.size());
+    if (agree * 10 > n && agree * 10 < 9 * n) return;  // neither side clearly
+    const int sm = hb[size_t(b)];
+    if (sm < 0 || sm >= kPartMaxSms) return;
+    const uint8_t sd = agree * 2 > n ? 0 : 1;
+    if (seen[sm] && side[sm] != sd) return;
+    side[sm] = sd;
+    seen[sm] = true;
+  }
+  int32_t pairs[2] = {0, 0};
+  for (int p = 0; p < npairs; ++p) {
+    const int sm = hp[size_t(p)];
+    if (sm < 0 || sm >= kPartMaxSms) return;
+    ++pairs[side[sm]];
+  }
+  if (pairs[0] == 0 || pairs[1] == 0) return;
+  std::memcpy(m.side, side, sizeof(side));
+  m.pairs[0] = pairs[0];
+  m.pairs[1] = pairs[1];
+  m.npairs = npairs;
+  m.ok = true;
+}
+
+// Whether a forward with this plan gains from the partition order: the pair
+// kernel with kPartMinUnitsPerPair units per pair, and more token blocks than
+// one raster group holds, so that the plain order streams W more than once
+// (N=8192 V=40000 D=128, a single group, ran 4% slower in the partition
+// order).
+bool part_order_sized(const flce_plan_t& plan) {
+  const int64_t npairs = plan.grid / 2;
+  return plan.ctas_per_unit == 2 && npairs >= 2 && plan.units >= kPartMinUnitsPerPair * npairs &&
+         plan.token_blocks > plan.group_blocks;
+}
+
+// Takes the current device's map at the first forward sized for the order,
+// unless `st` is being captured into a graph (then that forward and the ones
+// after it use the plain order until one runs outside a capture).
+void maybe_calibrate(const flce_plan_t& plan, int sms, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!part_order_sized(plan) || ws_bytes < kPartCalBytes) return;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return;
+  std::lock_guard<std::mutex> lock(g_part_mu);
+  if (g_part_map[dev].tried) return;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+    (void)cudaGetLastError();
+    return;
+  }
+  calibrate_partitions(sms, int(plan.grid / 2), static_cast<uint8_t*>(ws), st, g_part_map[dev]);
+}
+
+// The partition order for this launch, if the device's map allows it: the
+// split (q, r) gives partition 0 its pairs' share of the units.
+bool part_order(const flce_plan_t& plan, int64_t D, uint32_t* reg, tc::PartArgs& pa) {
+  if (!part_order_sized(plan)) return false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  PartMap m;
+  {
+    std::lock_guard<std::mutex> lock(g_part_mu);
+    m = g_part_map[dev];
+  }
+  const int64_t npairs = plan.grid / 2;
+  if (!m.ok || m.npairs != npairs) return false;
+  const int64_t U = plan.units, P = plan.slabs, TB = plan.token_blocks;
+  const int64_t u0 = (U * m.pairs[0] + npairs / 2) / npairs;
+  if (u0 <= 0 || u0 >= U) return false;
+  const int64_t q = u0 / P, r = u0 % P;
+  const int64_t blocks = std::max<int64_t>(q + (r > 0 ? 1 : 0), TB - q);
+  if (blocks * plan.block_rows * D * 2 > kPartHBytes) return false;
+  pa.reg = reg;
+  pa.pairs[0] = m.pairs[0];
+  pa.pairs[1] = m.pairs[1];
+  pa.q = int32_t(q);
+  pa.r = int32_t(r);
+  std::memcpy(pa.side, m.side, sizeof(pa.side));
+  return true;
+}
+
 // Outputs of the merge when it runs inside the contraction kernel (the whole
 // forward in one launch); see tc::fused_merge.
 struct MergeOutputs {
@@ -299,6 +473,11 @@ flce_status launch_contraction(const Operands& op, Targets y, int64_t y_offset, 
   a.sch = sch;
   a.wait_limit_ns = kDefaultWaitLimitNs;
   a.fm = tc::FusedMerge{};
+  a.porder.reg = nullptr;
+  // the partition order needs its pair counters cleared by this call
+  if (reset != HeaderReset::kNone &&
+      !part_order(plan, op.cols_h, reinterpret_cast<uint32_t*>(wsb + kPartRegOffset), a.porder))
+    a.porder.reg = nullptr;
   if (merged != nullptr) {
     a.fm.arrivals = reinterpret_cast<uint32_t*>(wsb + L.counters);
     a.fm.loss = merged->loss;
@@ -402,6 +581,8 @@ flce_status launch_partials(const void* H, int64_t ldh, const void* W, int64_t l
   if (s != FLCE_OK) return s;
   flce_plan_t plan;
   make_plan(N, V, D, dtype, workers, &plan);
+  // the first forward of this size on the device maps its L2 partitions
+  maybe_calibrate(plan, di.sms, ws, state_layout(N, V).total, st);
 
   // The operands the tensor-core kernels read: H and W themselves (bf16), or
   // their [hi | lo] split copies in the workspace (fp32), each K block's four
@@ -734,6 +915,55 @@ flce_status launch_gemm(const CUtensorMap& A, const CUtensorMap& B, const bwd::G
 }
 
 }  // namespace
+
+extern "C" flce_status flce_partition_order(int32_t token_blocks, int32_t slabs,
+                                            int32_t side0_units, int32_t* out) {
+  if (token_blocks < 1 || slabs < 1 || out == nullptr ||
+      int64_t(token_blocks) * slabs >= (int64_t(1) << 30) || side0_units < 0 ||
+      side0_units > token_blocks * slabs)
+    return FLCE_ERR_INVALID_ARG;
+  Schedule s{};
+  s.token_blocks = token_blocks;
+  s.slabs = slabs;
+  s.units = token_blocks * slabs;
+  const int32_t q = side0_units / slabs, r = side0_units % slabs;
+  int64_t o = 0;
+  for (int side = 0; side < 2; ++side)
+    for (int k = 0; k < part_units(s, q, r, side); ++k) {
+      int slab = 0, tb = 0;
+      part_unit(s, q, r, side, k, slab, tb);
+      out[o++] = slab;
+      out[o++] = tb;
+    }
+  return FLCE_OK;
+}
+
+extern "C" flce_status flce_partition_map(int32_t* out_pairs) {
+  if (out_pairs == nullptr) return FLCE_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return FLCE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_part_mu);
+  const PartMap& m = g_part_map[dev];
+  if (!m.ok) return FLCE_ERR_UNSUPPORTED;
+  out_pairs[0] = m.pairs[0];
+  out_pairs[1] = m.pairs[1];
+  return FLCE_OK;
+}
+
+extern "C" flce_status flce_partition_take(int32_t pairs0, int32_t pairs1, int32_t side,
+                                           int32_t arrival, int32_t* out_side,
+                                           int32_t* out_rank) {
+  if (pairs0 < 1 || pairs1 < 1 || (side != 0 && side != 1) || arrival < 0 ||
+      arrival >= pairs0 + pairs1 || out_side == nullptr || out_rank == nullptr)
+    return FLCE_ERR_INVALID_ARG;
+  const int32_t pairs[2] = {pairs0, pairs1};
+  int sd = side, rank = arrival;
+  part_take(pairs, sd, rank);
+  *out_side = sd;
+  *out_rank = rank;
+  return FLCE_OK;
+}
 
 extern "C" size_t flce_backward_workspace_size(int64_t N, int64_t V, int64_t D, flce_dtype dtype) {
   if (!sizes_ok(N, V, D, dtype) || N < 1) return 0;

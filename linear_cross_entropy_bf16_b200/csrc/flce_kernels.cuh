@@ -112,6 +112,66 @@ __device__ __forceinline__ void unit_coords(const Schedule& s, int u, int& slab,
   ntiles = s.slab_base + (slab < s.slab_rem ? 1 : 0);
 }
 
+// Partition-aware order of the pair kernel.  The B200's L2 is two partitions,
+// each caching what its own SMs read, so data that every SM reads gets about
+// half of the L2.  In this order the CTA pairs on partition 0 take the first
+// U0 units of the token-block-major order (token blocks [0, q) and slabs
+// [0, r) of block q, U0 = q P + r) and the pairs on partition 1 the rest,
+// each side slab-major over its own blocks: each partition's L2 holds only
+// its own rows of H, and the two sides stream the same W tiles at the same
+// time.  The split (q, r) makes U0 / U the share of the pairs on partition 0.
+__host__ __device__ inline int32_t part_units(const Schedule& s, int32_t q, int32_t r, int side) {
+  const int32_t u0 = q * s.slabs + r;
+  return side == 0 ? u0 : s.units - u0;
+}
+
+// Slab and token block of unit k (< part_units) of partition `side`.
+__host__ __device__ inline void part_unit(const Schedule& s, int32_t q, int32_t r, int side, int k,
+                                          int& slab, int& tblock) {
+  if (side == 0) {
+    // slabs [0, r) hold blocks [0, q]; slabs [r, P) blocks [0, q)
+    const int head = r * (q + 1);
+    if (k < head) {
+      slab = k / (q + 1);
+      tblock = k - slab * (q + 1);
+    } else {
+      const int k2 = k - head;  // q > 0 whenever a unit lies here
+      slab = r + k2 / q;
+      tblock = k2 - (slab - r) * q;
+    }
+  } else {
+    // slabs [0, r) hold blocks [q + 1, TB); slabs [r, P) blocks [q, TB)
+    const int c = s.token_blocks - q - 1;
+    const int head = r * c;
+    if (k < head) {  // c > 0 whenever a unit lies here
+      slab = k / c;
+      tblock = q + 1 + (k - slab * c);
+    } else {
+      const int k2 = k - head;
+      slab = r + k2 / (c + 1);
+      tblock = q + (k2 - (slab - r) * (c + 1));
+    }
+  }
+}
+
+// A pair that arrived as number `arrival` on partition `side` (counted from
+// 0 by the header counter) takes rank `arrival` there, unless the side
+// already has its planned `pairs[side]`: then it takes the highest rank of
+// the other side that no pair can reach.  With pairs[0] + pairs[1] pairs in
+// all, every planned (side, rank) is taken exactly once, however the pairs
+// land.
+__host__ __device__ inline void part_take(const int32_t (&pairs)[2], int& side, int& rank) {
+  if (rank >= pairs[side]) {
+    rank = pairs[side ^ 1] - 1 - (rank - pairs[side]);
+    side ^= 1;
+  }
+}
+
+__host__ __device__ inline void slab_tiles(const Schedule& s, int slab, int& tile0, int& ntiles) {
+  tile0 = slab * s.slab_base + (slab < s.slab_rem ? slab : s.slab_rem);
+  ntiles = s.slab_base + (slab < s.slab_rem ? 1 : 0);
+}
+
 // ----------------------------------------------------------------- bounded waits
 
 // Bounded mbarrier waits.  `flag` is the CTA's shared abort flag: once any
@@ -378,7 +438,8 @@ struct Cfg {
   static constexpr int STAGE_BYTES = Layout<L>::NA * A_BYTES + Layout<L>::NB * B_BYTES;
   static constexpr int STAGES = stages_for(STAGE_BYTES);
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-  static_assert(STAGES >= 2 && 2 * STAGES + 11 <= 32, "stage ring, barriers and merge scratch");
+  static_assert(STAGES >= 2 && 2 * STAGES + 12 <= 32,
+                "stage ring, barriers, merge scratch and the pair's work");
 };
 
 // Instruction descriptor of tcgen05.mma kind::f16: D fp32 (bits 4-5 = 1),
@@ -410,6 +471,22 @@ struct FusedMerge {
   int32_t row_blocks;   // token blocks x CTAs per unit: 128 tokens each
 };
 
+// The partition-aware order (part_unit) of the pair kernel's units.  Each
+// pair learns its partition from its SM id and its rank in that partition
+// from a counter in the workspace header (cleared before every call), and
+// takes every pairs[side]-th unit of its side's list from its rank on.  The
+// host launches exactly pairs[0] + pairs[1] pairs; a pair whose rank is at or
+// beyond its side's planned count (the map was wrong, or the hardware placed
+// the pairs otherwise) takes the highest rank of the other side instead,
+// which is then missing there, so every unit of both lists is computed once
+// however the pairs land.
+struct PartArgs {
+  uint32_t* reg;         // [2] pairs seen per partition; null: plain round-robin order
+  int32_t pairs[2];      // pairs the order plans on each partition
+  int32_t q, r;          // partition 0 takes U0 = q P + r units
+  uint8_t side[256];     // partition of each SM id
+};
+
 struct Args {
   Targets y;
   int64_t y_offset;        // first vocabulary id of W's rows (a vocabulary shard); 0 otherwise
@@ -425,6 +502,7 @@ struct Args {
   FusedMerge fm;
   int32_t wait_operands;   // 1: H or W is written by the kernel launched just before this
                            // one, which this one may overlap: the producer waits for it
+  PartArgs porder;         // pair kernel: the partition-aware order, or plain round-robin
 };
 
 // Barrier over the 128 epilogue threads (warps 2-5) of a contraction CTA:
@@ -432,6 +510,18 @@ struct Args {
 struct EpiSync {
   __device__ __forceinline__ void operator()() const { ptx::named_bar_sync(1, 128); }
 };
+
+// Unit k of a pair's work: of the plain order (side < 0) or of partition
+// side's list.
+__device__ __forceinline__ void work_coords(const Args& a, int side, int k, int& slab, int& tblock,
+                                            int& tile0, int& ntiles) {
+  if (side < 0) {
+    unit_coords(a.sch, k, slab, tblock, tile0, ntiles);
+    return;
+  }
+  part_unit(a.sch, a.porder.q, a.porder.r, side, k, slab, tblock);
+  slab_tiles(a.sch, slab, tile0, ntiles);
+}
 
 // Called by all 128 epilogue threads after the CTA wrote its (m, s) states
 // of one vocab slab for the 128 tokens of row block `rb` (thread t owns token
@@ -729,7 +819,8 @@ struct Cfg {
   static constexpr int STAGES = tc::stages_for(STAGE_BYTES);
   static constexpr uint32_t PAIR_TX_BYTES = 2 * STAGE_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
-  static_assert(STAGES >= 2 && 2 * STAGES + 11 <= 32, "stage ring, barriers and merge scratch");
+  static_assert(STAGES >= 2 && 2 * STAGES + 12 <= 32,
+                "stage ring, barriers, merge scratch and the pair's work");
 };
 
 // kind::f16 descriptor as in the single-CTA kernel, with M = 256 (bits 24-28).
@@ -783,9 +874,29 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
     ptx::tmem_alloc_pair(ptx::smem_addr(tmem_slot), TMEM_COLS);
     ptx::tmem_relinquish_pair();
   }
+  // This pair's work: plain round-robin over all units (side -1), or every
+  // pairs[side]-th unit of its partition's list from its rank on (PartArgs).
+  int* work = reinterpret_cast<int*>(bars + 2 * STAGES + 11);  // [2] side, first unit
+  if (threadIdx.x == 0 && rank == 0) {
+    int side = -1, first = pair;
+    if (a.porder.reg != nullptr) {
+      ptx::griddep_wait();  // the counters are cleared by the kernel before this one
+      side = a.porder.side[ptx::smid() & 255u];
+      first = int(atomicAdd(&a.porder.reg[side], 1u));
+      part_take(a.porder.pairs, side, first);
+    }
+    work[0] = side;
+    work[1] = first;
+    ptx::st_shared_cluster_u32(ptx::map_to_cta(ptx::smem_addr(&work[0]), 1), uint32_t(side));
+    ptx::st_shared_cluster_u32(ptx::map_to_cta(ptx::smem_addr(&work[1]), 1), uint32_t(first));
+  }
   ptx::tc_fence_before_sync();
   ptx::cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
   ptx::tc_fence_after_sync();
+  const int work_side = work[0], work_first = work[1];
+  const int work_stride = work_side < 0 ? npairs : a.porder.pairs[work_side];
+  const int work_count =
+      work_side < 0 ? a.sch.units : part_units(a.sch, a.porder.q, a.porder.r, work_side);
   const uint32_t tmem_base = *tmem_slot;
   if (threadIdx.x == 0 && blockIdx.x == 0) {
     ptx::griddep_wait();  // the header is cleared by the kernel before this one
@@ -797,7 +908,6 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
 
   uint32_t* status = &a.hdr->status;
   const uint64_t lim = a.wait_limit_ns;
-  const Schedule& sch = a.sch;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -807,9 +917,9 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
       uint32_t phase = 0;
       uint32_t used = 0, last_parity = 0;
       bool ok = true;
-      for (int u = pair; ok && u < sch.units; u += npairs) {
+      for (int u = work_first; ok && u < work_count; u += work_stride) {
         int slab, tb, t0, nt;
-        unit_coords(sch, u, slab, tb, t0, nt);
+        work_coords(a, work_side, u, slab, tb, t0, nt);
         const int hrow = tb * PAIR_M + int(rank) * BM;
         for (int t = t0; ok && t < t0 + nt; ++t) {
           const int wrow = t * BN + int(rank) * HALF_N;
@@ -856,9 +966,9 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int u = pair; ok && u < sch.units; u += npairs) {
+      for (int u = work_first; ok && u < work_count; u += work_stride) {
         int slab, tb, t0, nt;
-        unit_coords(sch, u, slab, tb, t0, nt);
+        work_coords(a, work_side, u, slab, tb, t0, nt);
         for (int t = 0; ok && t < nt; ++t) {
           if (!wait_bounded(ptx::smem_addr(&tempty_bar[acc]), acc_phase ^ 1u, abort_flag, status,
                             lim)) {
@@ -911,9 +1021,9 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int u = pair; ok && u < sch.units; u += npairs) {
+    for (int u = work_first; ok && u < work_count; u += work_stride) {
       int slab, tb, t0, nt;
-      unit_coords(sch, u, slab, tb, t0, nt);
+      work_coords(a, work_side, u, slab, tb, t0, nt);
       const int row = tb * PAIR_M + int(rank) * BM + row_in_tile;
       const bool valid = row < a.N;
       const int64_t yi = valid ? a.y[row] - a.y_offset : -1;  // target column within W
@@ -959,6 +1069,52 @@ flce_tc2_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__
   if (warp == 1) {
     ptx::tc_fence_after_sync();
     ptx::tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+// Calibration of the partition-aware order, once per device (host side:
+// calibrate_partitions in flce.cu).  Both kernels take the pair kernel's dynamic
+// shared memory, so that each CTA has an SM to itself.
+//
+// Latency of dependent atomic adds, which complete at the L2 slice that
+// homes the line, from each CTA's SM to each of `nlines` zeroed lines (the
+// lines stay zero: each add adds 0, and each address depends on the value
+// before it).  CTAs start on different lines so that they do not queue on
+// one slice.
+__global__ void __launch_bounds__(32, 1)
+flce_part_latency_kernel(uint32_t* lines, int32_t nlines, int32_t stride_words, uint32_t* lat,
+                         int32_t* smid_of_block) {
+  if (threadIdx.x != 0) return;
+  smid_of_block[blockIdx.x] = int32_t(ptx::smid());
+  uint32_t v = 0;
+  for (int k = 0; k < nlines; ++k) {
+    const int l = (k + int(blockIdx.x)) % nlines;
+    uint32_t* p = lines + size_t(l) * size_t(stride_words);
+    v = atomicAdd(p + (v >> 31), 0u);
+    const long long t0 = clock64();
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i) v = atomicAdd(p + (v >> 31), 0u);
+    const long long t1 = clock64() + (long long)(v >> 31);
+    lat[size_t(blockIdx.x) * size_t(nlines) + size_t(l)] = uint32_t((t1 - t0) / 16);
+  }
+}
+
+// Where the pairs land when as many as can be resident are launched at once:
+// each records the SM of its even CTA, then waits (at most 1 s) until all have
+// arrived, so that none leaves its SMs to a later one.  `arrived` starts at
+// zero; *timed_out is set if the wait ran out.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(32, 1)
+flce_part_cluster_kernel(int32_t* smid_of_pair, uint32_t* arrived, uint32_t* timed_out) {
+  if (threadIdx.x != 0) return;
+  if (ptx::cluster_ctarank() == 0) smid_of_pair[ptx::cluster_id_x()] = int32_t(ptx::smid());
+  atomicAdd(arrived, 1u);
+  const uint32_t all = 2u * ptx::cluster_count_x();
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (*reinterpret_cast<volatile uint32_t*>(arrived) < all) {
+    if (ptx::globaltimer_ns() - t0 > 1000000000ull) {
+      atomicOr(timed_out, 1u);
+      break;
+    }
   }
 }
 

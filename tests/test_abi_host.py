@@ -331,3 +331,64 @@ def test_backward_shard_checks_need_no_gpu(lib):
     assert call(v_offset=950) == flce.ERR_INVALID_ARG        # shard runs past V_total
     assert call(V_shard=0) == flce.ERR_INVALID_ARG
     assert call(N=0) == flce.OK
+
+
+# ---- the partition-aware order of the pair kernel (host-only queries) ----
+
+def partition_lists(lib, TB, P, u0):
+    out = (ctypes.c_int32 * (2 * TB * P))()
+    assert lib.flce_partition_order(TB, P, u0, out) == flce.OK
+    units = [(out[2 * i], out[2 * i + 1]) for i in range(TB * P)]
+    return units[:u0], units[u0:]
+
+
+@pytest.mark.parametrize("TB,P,u0", [
+    (32, 99, 1584), (32, 99, 1498), (32, 99, 1), (32, 99, 98), (32, 99, 99), (32, 99, 3167),
+    (2, 3, 1), (2, 3, 3), (2, 3, 5), (1, 7, 4), (64, 128, 4027), (17, 5, 0), (17, 5, 85)])
+def test_partition_order_covers_every_unit_once(lib, TB, P, u0):
+    side0, side1 = partition_lists(lib, TB, P, u0)
+    assert sorted(side0 + side1) == [(p, t) for p in range(P) for t in range(TB)]
+    q, r = divmod(u0, P)
+    # partition 0: token blocks [0, q) and slabs [0, r) of block q; partition 1 the rest
+    assert set(side0) == {(p, t) for p in range(P) for t in range(TB)
+                          if t < q or (t == q and p < r)}
+    # each side walks its units slab by slab
+    for units in (side0, side1):
+        slabs = [p for p, _ in units]
+        assert slabs == sorted(slabs)
+        for p in set(slabs):
+            blocks = [t for s, t in units if s == p]
+            assert blocks == sorted(blocks)
+
+
+def test_partition_order_rejects_bad_arguments(lib):
+    out = (ctypes.c_int32 * 64)()
+    for args in ((0, 4, 0), (4, 0, 0), (4, 4, -1), (4, 4, 17)):
+        assert lib.flce_partition_order(*args, out) == flce.ERR_INVALID_ARG
+    assert lib.flce_partition_order(4, 4, 3, None) == flce.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("n0,n1", [(37, 37), (35, 39), (1, 5), (5, 1), (2, 2)])
+def test_partition_take_gives_every_rank_once_however_pairs_land(lib, n0, n1):
+    """Whatever number a0 of the n0 + n1 pairs lands on partition 0, the pairs'
+    (partition, rank) are exactly the planned ones."""
+    s, r = ctypes.c_int32(), ctypes.c_int32()
+    for a0 in range(n0 + n1 + 1):
+        taken = []
+        for side, count in ((0, a0), (1, n0 + n1 - a0)):
+            for arrival in range(count):
+                assert lib.flce_partition_take(n0, n1, side, arrival, ctypes.byref(s),
+                                               ctypes.byref(r)) == flce.OK
+                taken.append((s.value, r.value))
+        assert sorted(taken) == [(0, k) for k in range(n0)] + [(1, k) for k in range(n1)]
+
+
+def test_partition_take_rejects_bad_arguments(lib):
+    s, r = ctypes.c_int32(), ctypes.c_int32()
+    for args in ((0, 3, 0, 0), (3, 0, 0, 0), (3, 3, 2, 0), (3, 3, 0, 6), (3, 3, 0, -1)):
+        assert lib.flce_partition_take(*args, ctypes.byref(s), ctypes.byref(r)) == flce.ERR_INVALID_ARG
+    assert lib.flce_partition_take(3, 3, 0, 0, None, ctypes.byref(r)) == flce.ERR_INVALID_ARG
+
+
+def test_partition_map_rejects_null(lib):
+    assert lib.flce_partition_map(None) == flce.ERR_INVALID_ARG
