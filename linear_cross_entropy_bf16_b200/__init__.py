@@ -585,10 +585,13 @@ def partition_map(device=None):
     forward large enough for the partition-aware order, or None (see
     flce_partition_map)."""
     lib = load_library()
-    if device is not None:
-        torch.cuda.set_device(device)
     out = (ctypes.c_int32 * 2)()
-    return (out[0], out[1]) if lib.flce_partition_map(out) == OK else None
+    if device is None:
+        st = lib.flce_partition_map(out)
+    else:
+        with torch.cuda.device(device):
+            st = lib.flce_partition_map(out)
+    return (out[0], out[1]) if st == OK else None
 
 
 def check(workspace: torch.Tensor, stream=None) -> int:
